@@ -1,0 +1,168 @@
+"""fp64 CPU oracle for the selective scan and the decode state update.
+
+TEST INFRASTRUCTURE ONLY: the tests, the package smoke check and the
+benchmark's CPU-baseline leg are the only callers.  The CUDA library never
+imports, links or runs anything here, and this package imports nothing from
+it.  The arithmetic lives in ``oracle.c`` (plain C, fp64, OpenMP over rows);
+this module only builds that file with gcc and marshals numpy arrays.
+
+Every function here is pinned by ``tests/test_oracle_pins.py``; no function is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``liboracle.so`` (gcc, -O2, IEEE semantics, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-fopenmp", "-shared", "-fPIC",
+                               "-std=c11", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        lib.oracle_scan_f64.argtypes = [I64, I64, I64, I64, P, P, P, P, P, P, P, P,
+                                        ctypes.c_int, P, P, P]
+        lib.oracle_scan_f64.restype = None
+        lib.oracle_state_update_f64.argtypes = [I64, I64, I64, P, P, P, P, P, P, P, P, P,
+                                                ctypes.c_int, P]
+        lib.oracle_state_update_f64.restype = None
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+         h0=None) -> Tuple[np.ndarray, np.ndarray]:
+    """Selective scan in fp64.
+
+    Shapes: ``u, delta, z`` [Bt, D, L]; ``B, C`` [Bt, N, L]; ``A`` [D, N];
+    ``D, delta_bias`` [D]; ``h0`` [Bt, D, N] (zero when omitted).
+    Returns ``(y [Bt, D, L], last_state [Bt, D, N])`` as float64.
+    """
+    u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
+    D, z, delta_bias, h0 = map(_f64, (D, z, delta_bias, h0))
+    Bt, Dd, L = u.shape
+    N = A.shape[1]
+    if N > 64:
+        raise ValueError("oracle supports N <= 64")
+    assert delta.shape == u.shape and B.shape == (Bt, N, L) and C.shape == (Bt, N, L)
+    assert A.shape == (Dd, N)
+    for v, shp in ((D, (Dd,)), (delta_bias, (Dd,)), (z, u.shape), (h0, (Bt, Dd, N))):
+        assert v is None or v.shape == shp
+    out = np.empty((Bt, Dd, L), np.float64)
+    last = np.empty((Bt, Dd, N), np.float64)
+    _load().oracle_scan_f64(Bt, Dd, L, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                            _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
+                            _ptr(h0), _ptr(out), _ptr(last))
+    return out, last
+
+
+def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
+                 softplus=True) -> Tuple[np.ndarray, np.ndarray]:
+    """One decode step in fp64 on a copy of ``state``.
+
+    Shapes: ``state`` [Bt, D, N]; ``x, dt, z`` [Bt, D]; ``B, C`` [Bt, N]; ``A`` [D, N].
+    Returns ``(new_state [Bt, D, N], y [Bt, D])``.
+    """
+    st = np.array(state, dtype=np.float64, copy=True, order="C")
+    x, dt, A, B, C = map(_f64, (x, dt, A, B, C))
+    D, z, dt_bias = map(_f64, (D, z, dt_bias))
+    Bt, Dd, N = st.shape
+    if N > 64:
+        raise ValueError("oracle supports N <= 64")
+    assert x.shape == (Bt, Dd) and dt.shape == (Bt, Dd) and A.shape == (Dd, N)
+    assert B.shape == (Bt, N) and C.shape == (Bt, N)
+    out = np.empty((Bt, Dd), np.float64)
+    _load().oracle_state_update_f64(Bt, Dd, N, _ptr(st), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                                    _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+                                    int(bool(softplus)), _ptr(out))
+    return st, out
+
+
+# --------------------------------------------------------------------------
+# convenience over synth.ScanInputs / synth.DecodeInputs
+# --------------------------------------------------------------------------
+
+
+def scan_inputs(inp, h0=None):
+    """Oracle scan of a whole ``synth.ScanInputs`` problem."""
+    return scan(inp.f64("u"), inp.f64("delta"), inp.f64("A"), inp.f64("B"), inp.f64("C"),
+                inp.f64("D"), inp.f64("z"), inp.f64("delta_bias"), inp.softplus, h0=h0)
+
+
+def scan_rows(inp, rows: Sequence[Tuple[int, int]]):
+    """Oracle scan of selected rows ``(b, d)`` of a ``synth.ScanInputs`` problem.
+
+    Returns ``(y [len(rows), L], last_state [len(rows), N])``.  Used to check
+    full-size outputs at sampled rows without running the whole problem.
+    """
+    ys, hs = [], []
+    for b, d in rows:
+        u = _widen_slice(inp, "u", b, d)
+        dl = _widen_slice(inp, "delta", b, d)
+        z = _widen_slice(inp, "z", b, d)
+        Bm = _widen_batch(inp, "B", b)
+        Cm = _widen_batch(inp, "C", b)
+        A = np.asarray(inp.A[d:d + 1], np.float64)
+        D = None if inp.D is None else np.asarray(inp.D[d:d + 1], np.float64)
+        bias = None if inp.delta_bias is None else np.asarray(inp.delta_bias[d:d + 1], np.float64)
+        y, h = scan(u, dl, A, Bm, Cm, D, z, bias, inp.softplus)
+        ys.append(y[0, 0])
+        hs.append(h[0, 0])
+    return np.stack(ys), np.stack(hs)
+
+
+def _widen_slice(inp, name, b, d):
+    a = getattr(inp, name)
+    if a is None:
+        return None
+    sl = a[b:b + 1, d:d + 1]
+    from synth import to_f64  # input widening only (bit manipulation)
+    return to_f64(sl, inp.io_dtype)
+
+
+def _widen_batch(inp, name, b):
+    a = getattr(inp, name)
+    from synth import to_f64
+    return to_f64(a[b:b + 1], inp.io_dtype)
+
+
+def state_update_inputs(inp, state=None):
+    """Oracle decode step of a ``synth.DecodeInputs`` batch (``state`` overrides ``inp.state``)."""
+    st = inp.state if state is None else state
+    return state_update(st, inp.f64("x"), inp.f64("dt"), inp.f64("A"), inp.f64("B"),
+                        inp.f64("C"), inp.f64("D"), inp.f64("z"), inp.f64("dt_bias"),
+                        inp.softplus)

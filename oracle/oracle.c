@@ -1,0 +1,164 @@
+/*
+ * fp64 CPU oracle for the Mamba-1 selective scan and its one-token state update.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only the tests, the package's smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header or constant with the
+ * CUDA library.
+ *
+ * What it computes (plain definition, no blocking, no reordering):
+ *
+ *   for every row (b, d), with h[n] = 0 at the start (or a given h0):
+ *     for t = 0 .. L-1:
+ *       delta = delta_raw[b,d,t] + bias[d]               (bias optional)
+ *       delta = softplus(delta) = log(1 + exp(delta))    (if softplus_flag)
+ *       for n:  h[n] = exp(delta * A[d,n]) * h[n] + delta * B[b,n,t] * u[b,d,t]
+ *       y = sum_n C[b,n,t] * h[n] + D[d] * u[b,d,t]      (D optional)
+ *       y = y * z / (1 + exp(-z))   with z = z[b,d,t]    (gate optional)
+ *       out[b,d,t] = y
+ *     last_state[b,d,:] = h
+ *
+ * Sources (web pages, by title and section):
+ *  - "Linear Attention vs Softmax Attention: Can RWKV or Mamba Replace
+ *    Transformers?", section Implementation, the forward pass of the listed
+ *    SelectiveSSMLayer: the step size is softplus of a projection that carries a
+ *    bias; A = -exp(A_log); the sequential discretisation loop (A_bar = exp(dt*A),
+ *    B_bar = dt*B, h = A_bar*h + B_bar*x, y = h.C + D*x) starts from a zero state;
+ *    its output is multiplied by silu of the gate branch.
+ *  - "State Space Models in Large Language Models: How Mamba, S4, and Selective
+ *    Recurrence Challenge Transformer Attention", section "Mamba: Selective State
+ *    Spaces and Hardware-Aware Scans", Dynamic Parameterization: the step is
+ *    Softplus(Parameter + Linear(x)), read here as softplus(delta_raw + bias).
+ *  - same page, section Discretization, Recurrent View: one recurrence step is
+ *    exactly the decode update (oracle_state_update_f64 below).
+ *
+ * Readings where the pages leave a choice open:
+ *  - B_bar = delta*B (the page's code), not the zero-order-hold form printed in
+ *    the pages' equations.
+ *  - softplus is the exact log(1 + exp(x)) with no threshold (the listing calls
+ *    F.softplus with defaults; the threshold-20 shortcut differs by < 2.1e-9).
+ *  - bias absent means 0; D absent means no skip; z absent means no gate.
+ *
+ * Parity pins (tests/test_oracle_pins.py) tie this file to closed forms and
+ * brute force: A = 0 prefix sums, the LTI convolution identity, the fully
+ * unrolled sum on tiny inputs, the delta -> 0 and delta -> inf limits,
+ * decode-chaining == scan, split-scan == scan, linearity in u, spot values
+ * of softplus and silu, and a hand-derived worked example.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Exact softplus in double: log(1 + exp(x)), evaluated without overflow. */
+static double sp_exact(double x)
+{
+    if (x > 0.0)
+        return x + log1p(exp(-x));
+    return log1p(exp(x));
+}
+
+/* silu(z) = z * sigmoid(z) = z / (1 + exp(-z)). */
+static double silu(double z)
+{
+    return z / (1.0 + exp(-z));
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Selective scan over a batch of rows.  All arrays are dense, C order:
+ *   u, delta, z, out : [Bt, D, L]
+ *   B, C             : [Bt, N, L]
+ *   A                : [D, N]
+ *   Dskip, bias      : [D]
+ *   h0, last_state   : [Bt, D, N]
+ * Nullable: Dskip, z, bias, h0, last_state.
+ */
+void oracle_scan_f64(int64_t Bt, int64_t D, int64_t L, int64_t N,
+                     const double *u, const double *delta, const double *A,
+                     const double *B, const double *C, const double *Dskip,
+                     const double *z, const double *bias, int softplus_flag,
+                     const double *h0, double *out, double *last_state)
+{
+    int64_t rows = Bt * D;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t b = r / D, d = r % D;
+        double h[64];
+        for (int64_t n = 0; n < N; ++n)
+            h[n] = h0 ? h0[r * N + n] : 0.0;
+        const double *ur = u + r * L;
+        const double *dr = delta + r * L;
+        const double *zr = z ? z + r * L : NULL;
+        const double *Bb = B + b * N * L;
+        const double *Cb = C + b * N * L;
+        const double *Ad = A + d * N;
+        double *yr = out + r * L;
+        for (int64_t t = 0; t < L; ++t) {
+            double dt = dr[t] + (bias ? bias[d] : 0.0);
+            if (softplus_flag)
+                dt = sp_exact(dt);
+            double x = ur[t];
+            double y = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                double a_bar = exp(dt * Ad[n]);
+                double b_bar = dt * Bb[n * L + t];
+                h[n] = a_bar * h[n] + b_bar * x;
+                y += Cb[n * L + t] * h[n];
+            }
+            if (Dskip)
+                y += Dskip[d] * x;
+            if (zr)
+                y *= silu(zr[t]);
+            yr[t] = y;
+        }
+        if (last_state)
+            for (int64_t n = 0; n < N; ++n)
+                last_state[r * N + n] = h[n];
+    }
+}
+
+/*
+ * One decode step (the recurrence applied to a single token), state updated in place.
+ *   state : [Bt, D, N]      x, dt, z, out : [Bt, D]
+ *   A     : [D, N]          B, C          : [Bt, N]
+ *   Dskip, bias : [D]       Nullable: Dskip, z, bias.
+ */
+void oracle_state_update_f64(int64_t Bt, int64_t D, int64_t N, double *state,
+                             const double *x, const double *dt_in, const double *A,
+                             const double *B, const double *C, const double *Dskip,
+                             const double *z, const double *bias, int softplus_flag,
+                             double *out)
+{
+    int64_t rows = Bt * D;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t b = r / D, d = r % D;
+        double dt = dt_in[r] + (bias ? bias[d] : 0.0);
+        if (softplus_flag)
+            dt = sp_exact(dt);
+        double xv = x[r];
+        double *h = state + r * N;
+        double y = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            h[n] = exp(dt * A[d * N + n]) * h[n] + dt * B[b * N + n] * xv;
+            y += C[b * N + n] * h[n];
+        }
+        if (Dskip)
+            y += Dskip[d] * xv;
+        if (z)
+            y *= silu(z[r]);
+        out[r] = y;
+    }
+}

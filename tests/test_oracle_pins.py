@@ -1,0 +1,407 @@
+"""Pins for the fp64 oracle: closed forms, limits, brute force and invariants.
+
+Each test ties the oracle to something other than itself, so that a plausible
+mistake in it (a dropped term, a wrong sign or index, a transposed operand,
+an off-by-one in when the input enters the state) fails at least one of them.
+``test_mutants_are_caught`` checks exactly that by compiling deliberately
+wrong variants of the oracle and running the pins against them.
+
+The method is the Mamba-1 selective scan as the pages define it:
+"Linear Attention vs Softmax Attention: Can RWKV or Mamba Replace
+Transformers?" (section Implementation: the sequential loop of the listed
+SelectiveSSMLayer) and "State Space Models in Large Language Models ..."
+(sections Discretization and Dynamic Parameterization).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+N = 16
+
+
+def softplus_ref(x):
+    # independent routine: log(exp(0) + exp(x))
+    return np.logaddexp(0.0, x)
+
+
+def sigmoid_ref(x):
+    # independent formulation: 0.5 * (1 + tanh(x / 2))
+    return 0.5 * (1.0 + np.tanh(0.5 * x))
+
+
+def rand_problem(rng, Bt, D, L, *, structured=False, with_z=True, with_D=True,
+                 with_bias=True):
+    u = rng.standard_normal((Bt, D, L))
+    delta = rng.standard_normal((Bt, D, L))
+    if structured:
+        A = -np.tile(np.arange(1, N + 1, dtype=np.float64), (D, 1))
+    else:
+        A = -np.exp(rng.uniform(-1.0, 1.5, size=(D, N)))
+    B = rng.standard_normal((Bt, N, L))
+    C = rng.standard_normal((Bt, N, L))
+    Dv = rng.standard_normal(D) if with_D else None
+    z = rng.standard_normal((Bt, D, L)) if with_z else None
+    bias = rng.uniform(-4.0, -1.0, size=D) if with_bias else None
+    return dict(u=u, delta=delta, A=A, B=B, C=C, D=Dv, z=z, delta_bias=bias)
+
+
+def eff_delta(p, softplus=True):
+    d = p["delta"] + (0.0 if p["delta_bias"] is None else p["delta_bias"][None, :, None])
+    return softplus_ref(d) if softplus else d
+
+
+def gate(y, z):
+    return y if z is None else y * z * sigmoid_ref(z)
+
+
+# ---------------------------------------------------------------------------
+# 1. A = 0: A_bar = 1, the state is a running sum of dt * B * u
+# ---------------------------------------------------------------------------
+
+def test_A_zero_is_prefix_sum():
+    rng = np.random.default_rng(1)
+    p = rand_problem(rng, 2, 3, 37)
+    p["A"] = np.zeros_like(p["A"])
+    y, last = oracle.scan(**p, softplus=True)
+    dt = eff_delta(p)
+    # h[b, d, n, t] = cumsum_t dt[b,d,t] * B[b,n,t] * u[b,d,t]
+    incr = dt[:, :, None, :] * p["B"][:, None, :, :] * p["u"][:, :, None, :]
+    h = np.cumsum(incr, axis=-1)
+    y_ref = np.einsum("bdnt,bnt->bdt", h, p["C"]) + p["D"][None, :, None] * p["u"]
+    y_ref = gate(y_ref, p["z"])
+    np.testing.assert_allclose(y, y_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(last, h[..., -1], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# 2. LTI case: constant dt, B, C -> causal convolution with K_k = sum_n C_n a_n^k dt B_n
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("softplus", [True, False])
+def test_lti_equals_convolution(softplus):
+    rng = np.random.default_rng(2)
+    D, L = 3, 50
+    u = rng.standard_normal((1, D, L))
+    A = -np.exp(rng.uniform(-2.0, 1.0, size=(D, N)))
+    raw = rng.uniform(-3.0, 0.5, size=D)
+    delta = np.repeat(raw[None, :, None], L, axis=2)
+    b = rng.standard_normal(N)
+    c = rng.standard_normal(N)
+    B = np.repeat(b[None, :, None], L, axis=2)
+    C = np.repeat(c[None, :, None], L, axis=2)
+    Dv = rng.standard_normal(D)
+    y, _ = oracle.scan(u, delta, A, B, C, Dv, None, None, softplus)
+    dt = softplus_ref(raw) if softplus else raw
+    for d in range(D):
+        k = np.arange(L)
+        a = np.exp(dt[d] * A[d])                       # [N]
+        K = (c[None, :] * a[None, :] ** k[:, None] * dt[d] * b[None, :]).sum(1)
+        y_ref = np.convolve(u[0, d], K)[:L] + Dv[d] * u[0, d]
+        np.testing.assert_allclose(y[0, d], y_ref, rtol=1e-11, atol=1e-12)
+
+
+def test_lti_step_input_closed_form():
+    # u = 1 for all t: y_t = sum_n C_n dt B_n (1 - a_n^(t+1)) / (1 - a_n) + D
+    D, L = 2, 40
+    A = -np.tile(np.arange(1, N + 1, dtype=np.float64), (D, 1))
+    dt = np.array([0.05, 0.7])
+    b = np.linspace(-1, 1, N)
+    c = np.cos(np.arange(N))
+    u = np.ones((1, D, L))
+    delta = np.repeat(dt[None, :, None], L, axis=2)
+    B = np.repeat(b[None, :, None], L, axis=2)
+    C = np.repeat(c[None, :, None], L, axis=2)
+    y, last = oracle.scan(u, delta, A, B, C, np.full(D, 0.5), None, None, False)
+    for d in range(D):
+        a = np.exp(dt[d] * A[d])
+        t = np.arange(L)[:, None]
+        y_ref = (c * dt[d] * b * (1 - a ** (t + 1)) / (1 - a)).sum(1) + 0.5
+        np.testing.assert_allclose(y[0, d], y_ref, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(last[0, d], dt[d] * b * (1 - a ** L) / (1 - a), rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# 3. tiny inputs: the fully unrolled sum
+#    y_t = sum_{s<=t} sum_n C_{t,n} (prod_{s<r<=t} A_bar_{r,n}) dt_s B_{s,n} u_s + D u_t
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed,L,D", [(3, 1, 1), (4, 5, 2), (5, 12, 3)])
+def test_tiny_unrolled_sum(seed, L, D):
+    rng = np.random.default_rng(seed)
+    p = rand_problem(rng, 2, D, L)
+    y, last = oracle.scan(**p, softplus=True)
+    dt = eff_delta(p)
+    for b in range(2):
+        for d in range(D):
+            abar = [[math.exp(dt[b, d, r] * p["A"][d, n]) for n in range(N)] for r in range(L)]
+            for t in range(L):
+                acc = 0.0
+                for s in range(t + 1):
+                    for n in range(N):
+                        prod = 1.0
+                        for r in range(s + 1, t + 1):
+                            prod *= abar[r][n]
+                        acc += p["C"][b, n, t] * prod * dt[b, d, s] * p["B"][b, n, s] * p["u"][b, d, s]
+                acc += p["D"][d] * p["u"][b, d, t]
+                z = p["z"][b, d, t]
+                acc *= z * sigmoid_ref(z)
+                assert abs(y[b, d, t] - acc) <= 1e-12 * (1 + abs(acc))
+            for n in range(N):
+                hs = 0.0
+                for s in range(L):
+                    prod = 1.0
+                    for r in range(s + 1, L):
+                        prod *= abar[r][n]
+                    hs += prod * dt[b, d, s] * p["B"][b, n, s] * p["u"][b, d, s]
+                assert abs(last[b, d, n] - hs) <= 1e-12 * (1 + abs(hs))
+
+
+# ---------------------------------------------------------------------------
+# 4. limits of the step size
+# ---------------------------------------------------------------------------
+
+def test_delta_to_zero_preserves_state():
+    rng = np.random.default_rng(6)
+    p = rand_problem(rng, 1, 4, 30, with_z=False, with_bias=False)
+    p["delta"] = np.full_like(p["delta"], -60.0)     # softplus(-60) ~ 8.8e-27
+    h0 = rng.standard_normal((1, 4, N))
+    y, last = oracle.scan(**p, softplus=True, h0=h0)
+    np.testing.assert_allclose(last, h0, rtol=1e-20, atol=1e-22)
+    y_ref = np.einsum("bdn,bnt->bdt", h0, p["C"]) + p["D"][None, :, None] * p["u"]
+    np.testing.assert_allclose(y, y_ref, rtol=1e-20, atol=1e-20)
+    # from a zero state nothing enters
+    y0, last0 = oracle.scan(**p, softplus=True)
+    assert np.abs(last0).max() < 1e-24
+    np.testing.assert_allclose(y0, p["D"][None, :, None] * p["u"], rtol=0, atol=1e-24)
+
+
+def test_large_delta_resets_state():
+    rng = np.random.default_rng(7)
+    p = rand_problem(rng, 2, 3, 25, with_bias=False)
+    p["delta"] = np.full_like(p["delta"], 1.0e3)     # exp(-1e3 * |A|) == 0 in fp64
+    y, last = oracle.scan(**p, softplus=False)
+    h = 1.0e3 * p["B"][:, None, :, :] * p["u"][:, :, None, :]   # [b, d, n, t]
+    y_ref = np.einsum("bdnt,bnt->bdt", h, p["C"]) + p["D"][None, :, None] * p["u"]
+    np.testing.assert_allclose(y, gate(y_ref, p["z"]), rtol=1e-13, atol=1e-10)
+    np.testing.assert_allclose(last, h[..., -1], rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# 5. recurrent view == scan;  split scan == scan  (associativity of the
+#    composition of the per-step affine maps h -> A_bar h + B_bar x)
+# ---------------------------------------------------------------------------
+
+def test_decode_steps_reproduce_scan():
+    rng = np.random.default_rng(8)
+    p = rand_problem(rng, 2, 5, 20)
+    y, last = oracle.scan(**p, softplus=True)
+    state = np.zeros((2, 5, N))
+    for t in range(20):
+        state, yt = oracle.state_update(state, p["u"][..., t], p["delta"][..., t], p["A"],
+                                        p["B"][..., t], p["C"][..., t], p["D"], p["z"][..., t],
+                                        p["delta_bias"], True)
+        np.testing.assert_allclose(yt, y[..., t], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(state, last, rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("split", [1, 7, 19])
+def test_split_scan_equals_scan(split):
+    rng = np.random.default_rng(9)
+    p = rand_problem(rng, 1, 3, 20)
+    y, last = oracle.scan(**p, softplus=True)
+    first = {k: (v[..., :split] if k in ("u", "delta", "B", "C", "z") else v) for k, v in p.items()}
+    second = {k: (v[..., split:] if k in ("u", "delta", "B", "C", "z") else v) for k, v in p.items()}
+    y1, h1 = oracle.scan(**first, softplus=True)
+    y2, h2 = oracle.scan(**second, softplus=True, h0=h1)
+    np.testing.assert_allclose(np.concatenate([y1, y2], -1), y, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(h2, last, rtol=1e-13, atol=1e-14)
+
+
+def test_affine_composition_is_associative():
+    # the per-step map (a, b): h -> a*h + b composes as (a1,b1) then (a2,b2) = (a2 a1, a2 b1 + b2)
+    rng = np.random.default_rng(10)
+
+    def comp(p, q):
+        return (q[0] * p[0], q[0] * p[1] + q[1])
+
+    for _ in range(100):
+        p, q, r = [(rng.uniform(0, 1), rng.standard_normal()) for _ in range(3)]
+        lhs = comp(comp(p, q), r)
+        rhs = comp(p, comp(q, r))
+        assert abs(lhs[0] - rhs[0]) < 1e-15 and abs(lhs[1] - rhs[1]) < 1e-14
+    # and the oracle's one-row state after L steps equals the composed map applied to 0
+    D, L = 1, 9
+    p = rand_problem(rng, 1, D, L, with_z=False, with_bias=False)
+    _, last = oracle.scan(**p, softplus=False)
+    for n in range(N):
+        acc = (1.0, 0.0)
+        for t in range(L):
+            dt = p["delta"][0, 0, t]
+            acc = comp(acc, (math.exp(dt * p["A"][0, n]), dt * p["B"][0, n, t] * p["u"][0, 0, t]))
+        assert abs(acc[1] - last[0, 0, n]) <= 1e-12 * (1 + abs(acc[1]))
+
+
+# ---------------------------------------------------------------------------
+# 6. linearity in u (fixed dt, B, C, no gate), constant state size
+# ---------------------------------------------------------------------------
+
+def test_linear_in_u():
+    rng = np.random.default_rng(11)
+    p = rand_problem(rng, 2, 3, 33, with_z=False)
+    u1, u2 = rng.standard_normal(p["u"].shape), rng.standard_normal(p["u"].shape)
+    ys = []
+    for u in (u1, u2, 2.5 * u1 - 0.75 * u2):
+        q = dict(p)
+        q["u"] = u
+        ys.append(oracle.scan(**q, softplus=True))
+    np.testing.assert_allclose(ys[2][0], 2.5 * ys[0][0] - 0.75 * ys[1][0], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(ys[2][1], 2.5 * ys[0][1] - 0.75 * ys[1][1], rtol=1e-11, atol=1e-12)
+
+
+def test_state_size_independent_of_length():
+    rng = np.random.default_rng(12)
+    for L in (1, 10, 100):
+        p = rand_problem(rng, 2, 3, L)
+        y, last = oracle.scan(**p, softplus=True)
+        assert last.shape == (2, 3, N) and y.shape == (2, 3, L)
+
+
+# ---------------------------------------------------------------------------
+# 7. spot values of softplus and silu
+# ---------------------------------------------------------------------------
+
+def test_softplus_and_silu_spot_values():
+    one = np.ones((1, 1, 1))
+    A = -np.ones((1, N))
+    B = np.full((1, N, 1), 0.5)
+    C = np.full((1, N, 1), 2.0)
+    u = 3.0 * one
+    # softplus(0) = ln 2: y = sum_n C * (ln2 * B * u) = 16 * 2 * ln2 * 0.5 * 3
+    y, last = oracle.scan(u, 0 * one, A, B, C, None, None, None, True)
+    assert abs(y[0, 0, 0] - 48 * math.log(2)) < 1e-13
+    assert np.allclose(last, 1.5 * math.log(2), rtol=1e-15)
+    # silu(0) = 0
+    y, _ = oracle.scan(u, 0 * one, A, B, C, None, 0 * one, None, True)
+    assert y[0, 0, 0] == 0.0
+    # silu(40) = 40 / (1 + e^-40) ~ 40
+    y, _ = oracle.scan(u, 0 * one, A, B, C, None, 40 * one, None, True)
+    assert abs(y[0, 0, 0] - 40 * 48 * math.log(2)) < 1e-9
+    # bias enters before the softplus: raw -1 + bias 1 == raw 0
+    y2, _ = oracle.scan(u, -one, A, B, C, None, None, np.ones(1), True)
+    assert abs(y2[0, 0, 0] - 48 * math.log(2)) < 1e-13
+    # softplus of a large argument does not overflow: softplus(800) = 800
+    y3, _ = oracle.scan(u, 800 * one, A, B, C, None, None, None, True)
+    assert abs(y3[0, 0, 0] - 16 * 2 * 800 * 0.5 * 3) < 1e-9
+
+
+# ---------------------------------------------------------------------------
+# 8. hand-derived worked example (tests/golden/halving_decay.txt)
+# ---------------------------------------------------------------------------
+
+def test_golden_halving_decay():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "halving_decay.txt"))
+            if l.strip() and not l.startswith("#")]
+    L = len(rows)
+    u = np.array([float(r[1]) for r in rows]).reshape(1, 1, L)
+    y_exp = np.array([float(r[2]) for r in rows])
+    A = -np.arange(1, N + 1, dtype=np.float64).reshape(1, N)
+    delta = np.full((1, 1, L), math.log(2))
+    Bm = np.ones((1, N, L))
+    Cm = np.ones((1, N, L))
+    y, last = oracle.scan(u, delta, A, Bm, Cm, None, None, None, False)
+    np.testing.assert_allclose(y[0, 0], y_exp, rtol=1e-14)
+    ln2 = math.log(2)
+    np.testing.assert_allclose(last[0, 0], 8.0 ** -(np.arange(N) + 1) * ln2 + 2 * ln2, rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# 9. the pins catch plausible mistakes: compile wrong variants of oracle.c
+#    (mutations applied here, on the CPU, to a temporary copy) and require
+#    every variant to fail at least one pin.
+# ---------------------------------------------------------------------------
+
+MUTANTS = {
+    "dropped_u_in_input_term": ("h[n] = a_bar * h[n] + b_bar * x;", "h[n] = a_bar * h[n] + b_bar;"),
+    "decay_sign_flipped": ("double a_bar = exp(dt * Ad[n]);", "double a_bar = exp(-dt * Ad[n]);"),
+    "decay_without_dt": ("double a_bar = exp(dt * Ad[n]);", "double a_bar = exp(Ad[n]);"),
+    "B_and_C_swapped": ("double b_bar = dt * Bb[n * L + t];", "double b_bar = dt * Cb[n * L + t];"),
+    "B_bar_without_dt": ("double b_bar = dt * Bb[n * L + t];", "double b_bar = Bb[n * L + t];"),
+    "B_time_index_off_by_one": ("double b_bar = dt * Bb[n * L + t];",
+                                "double b_bar = dt * Bb[n * L + (t > 0 ? t - 1 : 0)];"),
+    "readout_before_update": ("                h[n] = a_bar * h[n] + b_bar * x;\n"
+                              "                y += Cb[n * L + t] * h[n];",
+                              "                y += Cb[n * L + t] * h[n];\n"
+                              "                h[n] = a_bar * h[n] + b_bar * x;"),
+    "skip_uses_dt": ("y += Dskip[d] * x;", "y += Dskip[d] * dt;"),
+    "gate_is_sigmoid": ("y *= silu(zr[t]);", "y *= 1.0 / (1.0 + exp(-zr[t]));"),
+    "bias_dropped": ("double dt = dr[t] + (bias ? bias[d] : 0.0);", "double dt = dr[t];"),
+    "softplus_is_exp": ("dt = sp_exact(dt);\n            double x = ur[t];",
+                        "dt = exp(dt);\n            double x = ur[t];"),
+    "A_channel_ignored": ("const double *Ad = A + d * N;", "const double *Ad = A;"),
+    "decode_dropped_dt_on_input": ("+ dt * B[b * N + n] * xv;", "+ B[b * N + n] * xv;"),
+    "decode_bias_dropped": ("double dt = dt_in[r] + (bias ? bias[d] : 0.0);", "double dt = dt_in[r];"),
+    "decode_gate_dropped": ("            y *= silu(z[r]);\n        out[r] = y;", "        out[r] = y;"),
+}
+
+PIN_CALLS = [
+    test_A_zero_is_prefix_sum,
+    lambda: test_lti_equals_convolution(True),
+    lambda: test_lti_equals_convolution(False),
+    test_lti_step_input_closed_form,
+    lambda: test_tiny_unrolled_sum(4, 5, 2),
+    test_delta_to_zero_preserves_state,
+    test_large_delta_resets_state,
+    test_decode_steps_reproduce_scan,
+    lambda: test_split_scan_equals_scan(7),
+    test_affine_composition_is_associative,
+    test_linear_in_u,
+    test_softplus_and_silu_spot_values,
+    test_golden_halving_decay,
+]
+
+
+def _compile_variant(src_text, out_dir, tag):
+    import subprocess
+    c = os.path.join(out_dir, f"m_{tag}.c")
+    so = os.path.join(out_dir, f"m_{tag}.so")
+    with open(c, "w") as f:
+        f.write(src_text)
+    subprocess.check_call(["gcc", "-O1", "-fopenmp", "-shared", "-fPIC", "-std=c11", c, "-o", so, "-lm"])
+    return so
+
+
+def _count_failures(lib_path):
+    import ctypes
+    lib = ctypes.CDLL(lib_path)
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    lib.oracle_scan_f64.argtypes = [I64, I64, I64, I64, P, P, P, P, P, P, P, P, ctypes.c_int, P, P, P]
+    lib.oracle_state_update_f64.argtypes = [I64, I64, I64, P, P, P, P, P, P, P, P, P, ctypes.c_int, P]
+    lib.oracle_num_threads.restype = ctypes.c_int
+    saved = oracle._lib
+    oracle._lib = lib
+    fails = 0
+    try:
+        with np.errstate(all="ignore"):
+            for call in PIN_CALLS:
+                try:
+                    call()
+                except AssertionError:
+                    fails += 1
+    finally:
+        oracle._lib = saved
+    return fails
+
+
+def test_mutants_are_caught(tmp_path):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "oracle.c")).read()
+    # the unmutated copy passes every pin
+    assert _count_failures(_compile_variant(src, str(tmp_path), "orig")) == 0
+    for tag, (old, new) in MUTANTS.items():
+        assert src.count(old) == 1, f"mutation site for {tag} not unique"
+        so = _compile_variant(src.replace(old, new), str(tmp_path), tag)
+        assert _count_failures(so) > 0, f"mutant {tag} passed every pin"
