@@ -1,0 +1,525 @@
+"""Benchmark of the B200 selective scan (and its decode step) through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl mssm|reference]
+
+One step is one pass of the hot path over one batch of synthetic input:
+for the scan workloads, one mssm_selective_scan_fwd call (softplus,
+discretisation, recurrence, readout, D skip, gate, store, final state); for the
+decode workload, one mssm_state_update call.  Inputs are resident in HBM when
+the timed region starts; the L2 is flushed (a 256 MiB write) before every timed
+step, outside the step's event bracket.  The K timed steps are captured into one
+CUDA graph (flush, start event, step, end event per step) so host launch
+overhead cannot leak into a step's device time.
+
+Multi-GPU (``torchrun --nproc-per-node N bench.py --gpus N``): rows of the scan
+are independent, so every rank runs its own batch of the same shape (weak
+scaling, no collective on the data path); the step time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "selective-scan B·D·L elems/s and achieved HBM GB/s vs ~8 TB/s B200 peak"
+DECODE_METRIC = "selective state update rows/s and achieved HBM GB/s vs ~8 TB/s B200 peak"
+DEFAULT_WORKLOAD = "scan_bf16_2x1536x2048"
+L2_FLUSH_BYTES = 256 << 20
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+N_STATE = 16
+
+
+# --------------------------------------------------------------------------
+# host-side helpers (also exercised by the multi-rank CPU tests)
+# --------------------------------------------------------------------------
+
+def rank_seed(rank: int, base: int = 0) -> int:
+    """Each rank draws its own batch: seed = base + rank."""
+    return base + rank
+
+
+def reduce_max(value: float, dist=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    if dist is None or not dist.is_available() or not dist.is_initialized():
+        return value
+    import torch
+    backend = dist.get_backend()
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def scan_algorithmic_bytes(batch, dim, length, io_bytes, has_z=True, has_D=True, has_bias=True,
+                           last_state=True) -> int:
+    """Bytes the scan must move once: u, delta, z, y per element; B, C per (batch, step);
+    A, D, bias per channel; the final fp32 state per row."""
+    elems = batch * dim * length
+    b = elems * io_bytes * (3 + (1 if has_z else 0))            # u, delta, out (+ z)
+    b += 2 * batch * N_STATE * length * io_bytes                 # B, C
+    b += dim * (N_STATE * 4 + (4 if has_D else 0) + (4 if has_bias else 0))
+    if last_state:
+        b += batch * dim * N_STATE * 4
+    return b
+
+
+def decode_algorithmic_bytes(batch, dim, io_bytes, has_z=True, has_D=True) -> int:
+    """Per decode step: state read + write (fp32), x, dt, (z), y per row; B, C per batch; A, D per channel."""
+    rows = batch * dim
+    b = rows * N_STATE * 4 * 2
+    b += rows * io_bytes * (3 + (1 if has_z else 0))
+    b += 2 * batch * N_STATE * io_bytes
+    b += dim * (N_STATE * 4 + (4 if has_D else 0))
+    return b
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_46_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current sources."""
+    p = os.path.join(ROOT, "profiles", f"traffic_{kernel}_{workload}.txt")
+    if not os.path.exists(p):
+        return None, None
+    text = open(p).read()
+    m_b = re.search(r"dram_bytes_per_launch\s*=\s*([0-9.eE+]+)", text)
+    m_h = re.search(r"source_hash\s*=\s*([0-9a-f]+)", text)
+    if not m_b or not m_h:
+        return None, None
+    if m_h.group(1) != kernel_source_hash():
+        return None, "stale"
+    scale = re.search(r"scale_to_full\s*=\s*([0-9.eE+]+)", text)
+    val = float(m_b.group(1)) * (float(scale.group(1)) if scale else 1.0)
+    return val, os.path.relpath(p, ROOT)
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return self
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# reference arm: the fp64 CPU oracle on the host cores
+# --------------------------------------------------------------------------
+
+def oracle_sample(workload: str, rows: int):
+    """A bounded sample of the workload for the CPU oracle: the first ``rows`` channels of batch 0."""
+    import oracle
+    inp = synth.workload_inputs(workload)
+    if isinstance(inp, synth.ScanInputs):
+        d = min(rows, inp.dim)
+        args = dict(u=inp.f64("u")[:1, :d], delta=inp.f64("delta")[:1, :d], A=inp.f64("A")[:d],
+                    B=inp.f64("B")[:1], C=inp.f64("C")[:1], D=None if inp.D is None else inp.f64("D")[:d],
+                    z=None if inp.z is None else inp.f64("z")[:1, :d],
+                    delta_bias=None if inp.delta_bias is None else inp.f64("delta_bias")[:d],
+                    softplus=inp.softplus)
+        units = d * inp.length
+        desc = f"batch 0, channels 0..{d - 1}, all {inp.length} steps ({units} elements)"
+        return (lambda: oracle.scan(**args)), units, desc
+    b = max(1, min(inp.batch, rows // inp.dim if rows >= inp.dim else 1))
+    args = dict(state=inp.state[:b], x=inp.f64("x")[:b], dt=inp.f64("dt")[:b], A=inp.f64("A"),
+                B=inp.f64("B")[:b], C=inp.f64("C")[:b], D=inp.f64("D"), z=inp.f64("z")[:b],
+                dt_bias=None, softplus=inp.softplus)
+    units = b * inp.dim
+    return (lambda: oracle.state_update(**args)), units, f"batches 0..{b - 1} ({units} rows)"
+
+
+def cpu_baseline(workload: str, budget_s: float = 10.0):
+    import oracle
+    is_scan = WORKLOADS_KIND[workload] == "scan"
+    rows = 512 if is_scan else 256 * 5120
+    fn, units, desc = oracle_sample(workload, rows)
+    fn()  # build + warm
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        fn()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 10000:
+            break
+    return {"value": units * n / el, "unit": "elems/s" if is_scan else "rows/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{desc}, repeated {n}x over {el:.1f} s (fp64, OpenMP over rows)"}
+
+
+WORKLOADS_KIND = {k: v["kind"] for k, v in synth.WORKLOADS.items()}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    is_scan = WORKLOADS_KIND[args.workload] == "scan"
+    fn, units, desc = oracle_sample(args.workload, 256 if is_scan else 256 * 5120)
+    for _ in range(max(args.warmup, 0)):
+        fn()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        fn()
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * statistics.mean(times)
+    value = units / (ms / 1e3)
+    unit = "elems/s" if is_scan else "rows/s"
+    line = {
+        "impl": "reference", "metric": METRIC if is_scan else DECODE_METRIC, "value": value, "unit": unit,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": {"workload": args.workload, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# the GPU arm
+# --------------------------------------------------------------------------
+
+def run_mssm(args):
+    import torch
+    import torch.distributed as dist
+    import selective_state_space_46_b200 as m
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    kind = WORKLOADS_KIND[args.workload]
+    spec = synth.WORKLOADS[args.workload]
+    io_bytes = 2 if spec["io_dtype"] == "bf16" else 4
+
+    def to_dev(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+
+    def pinned(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+        else:
+            t = torch.from_numpy(np.ascontiguousarray(a, np.float32))
+        return t.pin_memory()
+
+    seed = rank_seed(rank)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    if kind == "scan":
+        inp = synth.workload_inputs(args.workload, seed=seed)
+        host = {k: getattr(inp, k) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+        d = {k: to_dev(v) for k, v in host.items()}
+        out = torch.empty_like(d["u"])
+        last = torch.empty(inp.batch, inp.dim, N_STATE, device=dev)
+        units = inp.batch * inp.dim * inp.length
+        alg_bytes = scan_algorithmic_bytes(inp.batch, inp.dim, inp.length, io_bytes, inp.z is not None,
+                                           inp.D is not None, inp.delta_bias is not None)
+
+        def step():
+            m.mssm_selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
+                                      d["delta_bias"], inp.softplus, out, last)
+        config = {"workload": args.workload, "batch": inp.batch, "channels": inp.dim, "length": inp.length,
+                  "state": N_STATE, "io_dtype": inp.io_dtype, "gate": inp.z is not None,
+                  "softplus_bias": inp.delta_bias is not None, "D_skip": inp.D is not None}
+        metric, unit = METRIC, "elems/s"
+        dom_kernel = "scan_out"
+    else:
+        ring = [synth.workload_inputs(args.workload, seed=seed, step_stream=k) for k in range(8)]
+        inp = ring[0]
+        state = to_dev(inp.state)
+        A_d, D_d = to_dev(inp.A), to_dev(inp.D)
+        dring = [{k: to_dev(getattr(r, k)) for k in ("x", "dt", "B", "C", "z")} for r in ring]
+        out = torch.empty_like(dring[0]["x"])
+        units = inp.batch * inp.dim
+        alg_bytes = decode_algorithmic_bytes(inp.batch, inp.dim, io_bytes, inp.z is not None, inp.D is not None)
+        counter = [0]
+
+        def step():
+            r = dring[counter[0] % 8]
+            counter[0] += 1
+            m.mssm_state_update(state, r["x"], r["dt"], A_d, r["B"], r["C"], D_d, r["z"], out)
+        config = {"workload": args.workload, "batch": inp.batch, "channels": inp.dim, "state": N_STATE,
+                  "io_dtype": inp.io_dtype, "input_ring": 8, "state_in_place": True}
+        metric, unit = DECODE_METRIC, "rows/s"
+        dom_kernel = "state_update"
+
+    # ---- warm-up (also allocates the library's carry workspace before capture)
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    m.mssm_get_error()
+
+    # ---- capture the K timed steps into one graph
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    before = m.mssm_kernel_stats()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record()
+            step()
+            ends[k].record()
+    after = m.mssm_kernel_stats()
+    launches = sum(after[k]["launches"] - before[k]["launches"] for k in after)
+
+    sampler = ClockSampler(local).start()
+    # soak: keep the GPU at its loaded clocks for a while before the timed replay
+    t_soak = time.perf_counter()
+    while time.perf_counter() - t_soak < args.soak:
+        g.replay()
+        torch.cuda.synchronize(dev)
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    m.mssm_get_error()
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = reduce_max(sum(per_step), dist if world > 1 else None)
+    ms_per_step = total_ms / args.steps
+    value = units * world / (ms_per_step / 1e3)
+
+    # ---- per-kernel durations (same launches, events bracketing each kernel)
+    m.mssm_set_option(m.MSSM_OPT_KERNEL_TIMING, 1)
+    m.mssm_kernel_stats(reset=True)
+    for _ in range(args.steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    ks = m.mssm_kernel_stats(reset=True)
+    m.mssm_set_option(m.MSSM_OPT_KERNEL_TIMING, 0)
+    kern = {k: {"launches_per_step": v["timed"] / args.steps,
+                "ms_per_launch": (v["ms"] / v["timed"]) if v["timed"] else None}
+            for k, v in ks.items() if v["timed"]}
+    dom = kern.get(dom_kernel)
+    peak, peak_kind = measured_peaks()
+    dom_ms = dom["ms_per_launch"] if dom else None
+    achieved = alg_bytes / (dom_ms / 1e3) / 1e9 if dom_ms else None
+    traffic, traffic_src = recorded_traffic(dom_kernel, args.workload)
+    roofline = {"bound": "hbm", "kernel": dom_kernel, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": (achieved / peak) if achieved else None, "peak_source": peak_kind,
+                "algorithmic_bytes_per_launch": alg_bytes,
+                "traffic": traffic, "traffic_source": traffic_src}
+
+    # ---- end to end: host buffers in pinned memory, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, kind, inp, d if kind == "scan" else None, dev, m, units, world)
+
+    step_gbs = alg_bytes / (ms_per_step / 1e3) / 1e9
+    line = {
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; no datasets or weights)",
+        "config": {**config, "l2": "flushed before every timed step (256 MiB write)",
+                   "parallelism": f"replicas x{world} (independent rows, no collective)",
+                   "timing": "CUDA events per step inside one captured graph"},
+        "hbm_gbs": step_gbs * world, "hbm_gbs_per_gpu": step_gbs,
+        "hbm_frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS, "hbm_frac_of_measured": step_gbs / peak,
+        "kernels": kern, "roofline": roofline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+        "source_hash": kernel_source_hash(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        del g
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_e2e(args, kind, inp, d, dev, m, units, world):
+    import torch
+    import torch.distributed as dist
+    steps = max(1, min(args.steps, 20))
+
+    def pin(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+        else:
+            t = torch.from_numpy(np.ascontiguousarray(a, np.float32))
+        return t.pin_memory()
+
+    if kind == "scan":
+        names = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
+        h = {k: pin(getattr(inp, k)) for k in names}
+        dd = {k: (None if v is None else torch.empty(v.shape, dtype=v.dtype, device=dev)) for k, v in h.items()}
+        out = torch.empty_like(dd["u"])
+        last = torch.empty(inp.batch, inp.dim, N_STATE, device=dev)
+        y_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        s_host = torch.empty(last.shape, dtype=last.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in h.values() if v is not None)
+        d2h = y_host.numel() * y_host.element_size() + s_host.numel() * s_host.element_size()
+
+        def one():
+            for k in names:
+                if h[k] is not None:
+                    dd[k].copy_(h[k], non_blocking=True)
+            m.mssm_selective_scan_fwd(dd["u"], dd["delta"], dd["A"], dd["B"], dd["C"], dd["D"], dd["z"],
+                                      dd["delta_bias"], inp.softplus, out, last)
+            y_host.copy_(out, non_blocking=True)
+            s_host.copy_(last, non_blocking=True)
+    else:
+        names = ("state", "x", "dt", "A", "B", "C", "D", "z")
+        h = {k: pin(getattr(inp, k)) for k in names}
+        dd = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in h.items()}
+        out = torch.empty_like(dd["x"])
+        y_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        s_host = torch.empty(dd["state"].shape, dtype=torch.float32).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in h.values())
+        d2h = y_host.numel() * y_host.element_size() + s_host.numel() * s_host.element_size()
+
+        def one():
+            for k in names:
+                dd[k].copy_(h[k], non_blocking=True)
+            m.mssm_state_update(dd["state"], dd["x"], dd["dt"], dd["A"], dd["B"], dd["C"], dd["D"], dd["z"], out)
+            y_host.copy_(out, non_blocking=True)
+            s_host.copy_(dd["state"], non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        one()
+    t1.record()
+    torch.cuda.synchronize(dev)
+    ms = reduce_max(t0.elapsed_time(t1), dist if world > 1 else None) / steps
+    return {"value": units * world / (ms / 1e3), "unit": "elems/s" if kind == "scan" else "rows/s",
+            "ms_per_step": ms, "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "path": "pinned host buffers -> H2D copies -> C-ABI call -> D2H of y and final state"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mssm", "reference"], default="mssm")
+    ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--soak", type=float, default=1.5, help="seconds of untimed graph replays before timing")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_mssm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

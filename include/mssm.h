@@ -1,0 +1,205 @@
+/*
+ * mssm.h - C ABI of the B200 (sm_100a) Mamba-1 selective scan library (libmssm.so).
+ *
+ * The library computes, on one GPU, the forward selective scan of a Mamba-1
+ * layer and its one-token decode counterpart:
+ *
+ *   delta_t   = softplus(delta_raw_t + bias_d)          (softplus and bias optional)
+ *   A_bar_tn  = exp(delta_t * A_dn)
+ *   h_tn      = A_bar_tn * h_(t-1)n + delta_t * B_tn * u_t          (h_(-1) = 0)
+ *   y_t       = sum_n C_tn * h_tn + D_d * u_t                       (D optional)
+ *   out_t     = y_t * silu(z_t)                                     (z optional)
+ *
+ * Sources (web pages, by title and section):
+ *  - "Linear Attention vs Softmax Attention: Can RWKV or Mamba Replace
+ *    Transformers?": section Core Concepts, item 3 (Selective State Space
+ *    Models: the continuous system and its discretisation A_bar = exp(Delta A));
+ *    section Implementation (the listed SelectiveSSMLayer: softplus step size,
+ *    A = -exp(A_log), the sequential loop with B_bar = Delta B from a zero state,
+ *    readout C.h + D x, output multiplied by silu of the gate branch); section
+ *    How It Works (the fused scan: inputs read once, only y written back).
+ *  - "State Space Models in Large Language Models: How Mamba, S4, and Selective
+ *    Recurrence Challenge Transformer Attention": sections Discretization
+ *    (recurrent view, one O(1) step per token) and Dynamic Parameterization
+ *    (Delta_t = Softplus(Parameter + Linear(x_t))).
+ *  - "Mamba selective state space" (chenyuan1125.github.io), section
+ *    "Selectivity Removes the Convolution Shortcut; Scan Restores Parallelism":
+ *    each position is the affine map (A_bar_t, B_bar_t x_t); neighbouring maps
+ *    compose associatively, which is what lets the length be split into chunks
+ *    whose carries are combined.
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are described by mssm_tensor: a DEVICE pointer plus shape and
+ *    strides in ELEMENTS.  The caller owns all memory; the library never frees
+ *    or retains a caller pointer beyond the call.
+ *  - Supported dtype mixes: everything fp32; or bf16 for u/delta/B/C/z/out
+ *    (x/dt/B/C/z/out for decode) with fp32 A, D, bias and state.
+ *  - The state size N must be 16 (MSSM_ERR_UNSUPPORTED otherwise).
+ *  - The innermost (length) dimension of u/delta/z/out/B/C must have stride 1.
+ *  - All calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Argument errors are reported synchronously, before
+ *    anything is launched; launch failures map to MSSM_ERR_CUDA.  A detailed
+ *    message for the last error on the calling thread is available from
+ *    mssm_last_error().
+ *  - Outputs must not alias inputs; decode `state` is the only in-place tensor.
+ *  - The current CUDA device must be the device that holds the tensors.
+ */
+#ifndef MSSM_H
+#define MSSM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MSSM_F32 = 0,
+    MSSM_BF16 = 1
+} mssm_dtype;
+
+typedef enum {
+    MSSM_OK = 0,
+    MSSM_ERR_INVALID_ARG = 1, /* null required pointer, bad shape/stride/dtype combination */
+    MSSM_ERR_UNSUPPORTED = 2, /* valid but not implemented here (N != 16, misaligned rows, ...) */
+    MSSM_ERR_CUDA = 3         /* a CUDA runtime call or a kernel launch failed */
+} mssm_status;
+
+typedef struct {
+    void *data;         /* device pointer; must be 16-byte aligned for the vector paths */
+    int32_t dtype;      /* mssm_dtype */
+    int32_t ndim;       /* 1..4 */
+    int64_t shape[4];   /* sizes, outermost first */
+    int64_t stride[4];  /* strides in elements, outermost first */
+} mssm_tensor;
+
+/*
+ * Forward selective scan (prefill / training forward), fused:
+ * softplus + discretisation + recurrence + readout + D skip + silu(z) gate +
+ * store, plus the final state.  The B x D x L x N state never touches memory.
+ *
+ *   u          [Bt, D, L]  bf16|f32      the scan input (the conv branch output)
+ *   delta      [Bt, D, L]  dtype of u    the step before softplus (delta_raw)
+ *   A          [D, N]      f32           state matrix (diagonal per channel)
+ *   B, C       [Bt, N, L]  dtype of u    input/readout projections, shared by channels
+ *   D          [D]         f32 or NULL   skip weight (NULL: no skip)
+ *   z          [Bt, D, L]  dtype of u, or NULL (NULL: no gate)
+ *   delta_bias [D]         f32 or NULL   added to delta before softplus
+ *   softplus_flag          1: delta = softplus(delta + bias); 0: delta = delta + bias
+ *   out        [Bt, D, L]  dtype of u    written
+ *   last_state [Bt, D, N]  f32 or NULL   h after the last step, written (n stride 1)
+ *   stream                 cudaStream_t
+ *
+ * Initial state is zero.  Bt*D == 0 is a no-op; L == 0 writes a zero
+ * last_state.  Long sequences are split into chunks: a first kernel summarises
+ * every chunk but the last (its total step and its end state from zero), the
+ * last CTA of each row tile to finish folds those summaries into carried
+ * states, and a second kernel runs each chunk from its carried state.  No CTA
+ * ever waits on another.  The summaries live in a per-device workspace owned
+ * by the library: allocated with cudaMalloc on the first call that needs it
+ * (grown when a larger problem needs more, which synchronises the device) and
+ * freed by mssm_shutdown().  Calls that use the workspace must not overlap on
+ * the GPU (different streams of one device); run them on one stream or order
+ * them with events.  A first call of the largest size before any stream
+ * capture keeps allocation out of captured work.
+ */
+mssm_status mssm_selective_scan_fwd(const mssm_tensor *u, const mssm_tensor *delta,
+                                    const mssm_tensor *A, const mssm_tensor *B,
+                                    const mssm_tensor *C, const mssm_tensor *D,
+                                    const mssm_tensor *z, const mssm_tensor *delta_bias,
+                                    int softplus_flag, mssm_tensor *out,
+                                    mssm_tensor *last_state, void *stream);
+
+/*
+ * One-token selective state update (decode), state updated IN PLACE:
+ *
+ *   state [Bt, D, N] f32   read and written (n stride 1)
+ *   x, dt [Bt, D]          bf16|f32; dt is the step before softplus (delta_raw)
+ *   A     [D, N] f32
+ *   B, C  [Bt, N]          dtype of x
+ *   D     [D] f32 or NULL; z [Bt, D] dtype of x or NULL
+ *   out   [Bt, D]          dtype of x, written
+ *
+ * This entry point applies delta = softplus(dt) (no bias).  The same step as
+ * one iteration of mssm_selective_scan_fwd's recurrence ("State Space Models
+ * in Large Language Models ...", section Discretization, recurrent view).
+ */
+mssm_status mssm_state_update(mssm_tensor *state, const mssm_tensor *x, const mssm_tensor *dt,
+                              const mssm_tensor *A, const mssm_tensor *B, const mssm_tensor *C,
+                              const mssm_tensor *D, const mssm_tensor *z, mssm_tensor *out,
+                              void *stream);
+
+/*
+ * As mssm_state_update, with an optional per-channel dt_bias [D] f32 (NULL: none)
+ * and an explicit softplus flag, so that a sequence of decode steps reproduces
+ * mssm_selective_scan_fwd called with the same bias and flag.
+ */
+mssm_status mssm_state_update_ex(mssm_tensor *state, const mssm_tensor *x,
+                                 const mssm_tensor *dt, const mssm_tensor *A,
+                                 const mssm_tensor *B, const mssm_tensor *C,
+                                 const mssm_tensor *D, const mssm_tensor *z,
+                                 const mssm_tensor *dt_bias, int softplus_flag,
+                                 mssm_tensor *out, void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *mssm_status_string(mssm_status status);
+
+/* Detailed message of the last non-OK status returned on the calling thread ("" if none). */
+const char *mssm_last_error(void);
+
+/*
+ * Synchronises `stream` and reports an asynchronous failure of the work queued
+ * on it (MSSM_ERR_CUDA, with the CUDA error text in mssm_last_error()), or
+ * MSSM_OK.  The kernels contain no waits on other CTAs or on the host, so a
+ * call cannot stall on the device.
+ */
+mssm_status mssm_get_error(void *stream);
+
+/*
+ * Tuning / diagnostic options (process-wide; take effect on the next call):
+ *   MSSM_OPT_FORCE_GENERAL_A (value 0/1): when 1, never use the structured-A
+ *     path (A[d,n] == (n+1) * A[d,0] exactly, which computes exp(delta*A[d,n])
+ *     as powers of one exponential); every state then takes its own exponential.
+ *   MSSM_OPT_CHUNK_LEN (value 0, or a positive multiple of 64): length of the
+ *     chunks a sequence is split into (a value >= L means no split); 0 restores
+ *     the automatic choice.
+ *   MSSM_OPT_KERNEL_TIMING (value 0/1): when 1, every kernel launch is bracketed
+ *     by two CUDA events recorded on the caller's stream (see mssm_kernel_stats).
+ * Unknown options or invalid values return MSSM_ERR_INVALID_ARG.
+ */
+typedef enum {
+    MSSM_OPT_FORCE_GENERAL_A = 1,
+    MSSM_OPT_CHUNK_LEN = 2,
+    MSSM_OPT_KERNEL_TIMING = 3
+} mssm_option;
+mssm_status mssm_set_option(int option, int64_t value);
+
+/* Kernel kinds counted by mssm_kernel_stats. */
+typedef enum {
+    MSSM_KERNEL_SCAN_CHUNK_STATE = 0, /* chunk summaries + carry fold (split scans only) */
+    MSSM_KERNEL_SCAN_OUT = 1,         /* forward sweep with fused epilogue */
+    MSSM_KERNEL_STATE_UPDATE = 2,     /* decode step */
+    MSSM_KERNEL_KINDS = 3
+} mssm_kernel_kind;
+
+/*
+ * Diagnostics: per kernel kind, the number of launches issued so far
+ * (`launches`), and, for launches made while MSSM_OPT_KERNEL_TIMING was on, how
+ * many were timed (`timed`) and their summed device duration in ms (`ms`).
+ * Waits for the pending timing events.  Any output pointer may be NULL (each
+ * non-NULL one is an array of MSSM_KERNEL_KINDS).  reset != 0 zeroes the
+ * counters afterwards.
+ */
+mssm_status mssm_kernel_stats(int64_t *launches, int64_t *timed, double *ms, int reset);
+
+/* Frees the library's per-device workspaces (call with no work in flight). */
+mssm_status mssm_shutdown(void);
+
+/* Library version, "major.minor.patch". */
+const char *mssm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSSM_H */

@@ -1,0 +1,193 @@
+"""B200-native (sm_100a) Mamba-1 selective scan: Python binding of libmssm.so.
+
+This module only marshals arguments: it turns torch tensors into the C ABI's
+``mssm_tensor`` descriptors (pointer, dtype, shape, strides) and calls the
+entry points declared in ``include/mssm.h`` with the same names.  Every step of
+the computation runs in the library's CUDA kernels; there is no CPU or PyTorch
+fallback, and importing fails loudly when the library has not been built.
+
+Build the library with ``python -m selective_state_space_46_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "MssmError", "mssm_selective_scan_fwd", "mssm_state_update", "mssm_state_update_ex",
+    "mssm_get_error", "mssm_set_option", "mssm_shutdown", "mssm_version", "mssm_status_string",
+    "mssm_last_error", "selective_scan_fwd", "state_update", "lib_path",
+    "MSSM_OPT_FORCE_GENERAL_A", "MSSM_OPT_CHUNK_LEN", "MSSM_OPT_KERNEL_TIMING", "mssm_kernel_stats",
+    "KERNEL_KINDS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libmssm.so")
+if not os.path.exists(lib_path):
+    raise ImportError(f"{lib_path} is missing: build it with `python -m selective_state_space_46_b200.build` "
+                      "(nvcc, sm_100a); there is no fallback implementation")
+_lib = ctypes.CDLL(lib_path)
+
+MSSM_F32, MSSM_BF16 = 0, 1
+MSSM_OK, MSSM_ERR_INVALID_ARG, MSSM_ERR_UNSUPPORTED, MSSM_ERR_CUDA = 0, 1, 2, 3
+MSSM_OPT_FORCE_GENERAL_A, MSSM_OPT_CHUNK_LEN, MSSM_OPT_KERNEL_TIMING = 1, 2, 3
+KERNEL_KINDS = ("scan_chunk_state", "scan_out", "state_update")
+
+
+class mssm_tensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+_P = ctypes.POINTER(mssm_tensor)
+_V = ctypes.c_void_p
+_lib.mssm_selective_scan_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, _V]
+_lib.mssm_selective_scan_fwd.restype = ctypes.c_int
+_lib.mssm_state_update.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _V]
+_lib.mssm_state_update.restype = ctypes.c_int
+_lib.mssm_state_update_ex.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _V]
+_lib.mssm_state_update_ex.restype = ctypes.c_int
+_lib.mssm_status_string.argtypes = [ctypes.c_int]
+_lib.mssm_status_string.restype = ctypes.c_char_p
+_lib.mssm_last_error.restype = ctypes.c_char_p
+_lib.mssm_get_error.argtypes = [_V]
+_lib.mssm_get_error.restype = ctypes.c_int
+_lib.mssm_set_option.argtypes = [ctypes.c_int, ctypes.c_int64]
+_lib.mssm_set_option.restype = ctypes.c_int
+_lib.mssm_shutdown.restype = ctypes.c_int
+_lib.mssm_version.restype = ctypes.c_char_p
+_lib.mssm_kernel_stats.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
+                                   ctypes.POINTER(ctypes.c_double), ctypes.c_int]
+_lib.mssm_kernel_stats.restype = ctypes.c_int
+
+
+class MssmError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{mssm_status_string(status)}: {message}")
+        self.status = status
+
+
+_DT = {torch.float32: MSSM_F32, torch.bfloat16: MSSM_BF16}
+
+
+def _desc(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if t.dim() > 4:
+        raise ValueError("tensors have at most 4 dims")
+    d = mssm_tensor()
+    d.data = t.data_ptr() if t.numel() > 0 else None
+    d.dtype = _DT.get(t.dtype, -1)
+    d.ndim = t.dim()
+    for i, (s, st) in enumerate(zip(t.shape, t.stride())):
+        d.shape[i] = s
+        d.stride[i] = st
+    return ctypes.byref(d), d
+
+
+def _ref(x):
+    return None if x is None else x[0]
+
+
+def _stream(stream, ref: torch.Tensor):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream(ref.device).cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(status: int):
+    if status != MSSM_OK:
+        raise MssmError(status, mssm_last_error())
+
+
+def mssm_status_string(status: int) -> str:
+    return _lib.mssm_status_string(status).decode()
+
+
+def mssm_last_error() -> str:
+    return _lib.mssm_last_error().decode()
+
+
+def mssm_version() -> str:
+    return _lib.mssm_version().decode()
+
+
+def mssm_set_option(option: int, value: int) -> None:
+    _check(_lib.mssm_set_option(option, value))
+
+
+def mssm_shutdown() -> None:
+    _check(_lib.mssm_shutdown())
+
+
+def mssm_kernel_stats(reset: bool = False) -> dict:
+    """Launch counts and (when MSSM_OPT_KERNEL_TIMING is on) timed launches and summed ms, per kernel kind."""
+    n = len(KERNEL_KINDS)
+    launches = (ctypes.c_int64 * n)()
+    timed = (ctypes.c_int64 * n)()
+    ms = (ctypes.c_double * n)()
+    _check(_lib.mssm_kernel_stats(launches, timed, ms, int(reset)))
+    return {k: {"launches": launches[i], "timed": timed[i], "ms": ms[i]} for i, k in enumerate(KERNEL_KINDS)}
+
+
+def mssm_get_error(stream=None) -> None:
+    s = ctypes.c_void_p(None) if stream is None else (
+        ctypes.c_void_p(stream.cuda_stream) if isinstance(stream, torch.cuda.Stream) else ctypes.c_void_p(int(stream)))
+    _check(_lib.mssm_get_error(s))
+
+
+def mssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state,
+                            stream=None) -> None:
+    """Marshal torch tensors into ``mssm_selective_scan_fwd`` (see include/mssm.h)."""
+    ds = [_desc(t) for t in (u, delta, A, B, C, D, z, delta_bias, out, last_state)]
+    _check(_lib.mssm_selective_scan_fwd(*[_ref(x) for x in ds[:8]], int(softplus_flag),
+                                        _ref(ds[8]), _ref(ds[9]), _stream(stream, u)))
+
+
+def mssm_state_update(state, x, dt, A, B, C, D, z, out, stream=None) -> None:
+    """Marshal torch tensors into ``mssm_state_update`` (state updated in place)."""
+    ds = [_desc(t) for t in (state, x, dt, A, B, C, D, z, out)]
+    _check(_lib.mssm_state_update(*[_ref(v) for v in ds], _stream(stream, x)))
+
+
+def mssm_state_update_ex(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, out,
+                         stream=None) -> None:
+    """Marshal torch tensors into ``mssm_state_update_ex`` (state updated in place)."""
+    ds = [_desc(t) for t in (state, x, dt, A, B, C, D, z, dt_bias)]
+    do = _desc(out)
+    _check(_lib.mssm_state_update_ex(*[_ref(v) for v in ds], int(softplus_flag), _ref(do),
+                                     _stream(stream, x)))
+
+
+# --------------------------------------------------------------------------
+# allocation conveniences (torch allocates; the library computes)
+# --------------------------------------------------------------------------
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
+                       out=None, last_state=None, return_last_state=True,
+                       stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Allocate ``out`` (and ``last_state``) with torch and run the scan on the GPU."""
+    if not u.is_cuda:
+        raise ValueError("selective_scan_fwd runs on CUDA tensors only")
+    if out is None:
+        out = torch.empty_like(u, memory_format=torch.contiguous_format)
+    if last_state is None and return_last_state:
+        last_state = torch.empty(u.shape[0], u.shape[1], A.shape[1], device=u.device, dtype=torch.float32)
+    mssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, out, last_state, stream)
+    return out, last_state
+
+
+def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True, out=None,
+                 stream=None) -> torch.Tensor:
+    """Run one decode step on the GPU (``state`` updated in place); returns ``out``."""
+    if not x.is_cuda:
+        raise ValueError("state_update runs on CUDA tensors only")
+    if out is None:
+        out = torch.empty_like(x, memory_format=torch.contiguous_format)
+    mssm_state_update_ex(state, x, dt, A, B, C, D, z, dt_bias, softplus, out, stream)
+    return out

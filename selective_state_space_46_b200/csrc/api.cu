@@ -1,0 +1,430 @@
+// C ABI of libmssm.so: argument validation, dtype/shape dispatch, the carry
+// workspace, status codes.  Every compute step runs in the kernels of scan.cu
+// and decode.cu; nothing here touches tensor contents on the host.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "../../include/mssm.h"
+#include "launch.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+mssm_status fail(mssm_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+mssm_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(MSSM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+std::mutex g_mu;
+int g_force_general = 0;
+int64_t g_chunk_len = 0;
+
+// ---- launch accounting and optional per-kernel event timing (diagnostics)
+int64_t g_launches[MSSM_KERNEL_KINDS] = {0, 0, 0};
+int g_timing = 0;
+struct TimedLaunch {
+  int kind;
+  cudaEvent_t a, b;
+};
+std::vector<TimedLaunch> g_pending;
+std::vector<cudaEvent_t> g_event_pool;
+double g_time_ms[MSSM_KERNEL_KINDS] = {0, 0, 0};
+int64_t g_timed[MSSM_KERNEL_KINDS] = {0, 0, 0};
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Launch through `fn`, counting it and, when timing is on, bracketing it with
+// events recorded on the same stream.  Caller holds g_mu.
+template <typename F>
+cudaError_t tracked(int kind, cudaStream_t s, F&& fn) {
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (g_timing) {
+    a = take_event();
+    b = take_event();
+    if (a && b && cudaEventRecord(a, s) != cudaSuccess) a = nullptr;
+  }
+  cudaError_t e = fn();
+  if (e != cudaSuccess) return e;
+  ++g_launches[kind];
+  if (g_timing && a && b && cudaEventRecord(b, s) == cudaSuccess) g_pending.push_back({kind, a, b});
+  return cudaSuccess;
+}
+
+struct DeviceState {
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  int sm_count = 0;
+};
+std::vector<DeviceState> g_dev;
+
+DeviceState* device_state(int dev) {
+  if (dev < 0) return nullptr;
+  if (int(g_dev.size()) <= dev) g_dev.resize(dev + 1);
+  DeviceState& s = g_dev[dev];
+  if (s.sm_count == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    s.sm_count = v;
+  }
+  return &s;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t esize(int dtype) { return dtype == MSSM_BF16 ? 2 : 4; }
+
+const char* dname(int dtype) { return dtype == MSSM_BF16 ? "bf16" : dtype == MSSM_F32 ? "f32" : "?"; }
+
+// Shape/dtype check of one tensor.  shape entries < 0 are not checked.
+mssm_status check(const mssm_tensor* t, const char* name, int ndim, const int64_t* shape,
+                  int dtype, bool inner_contig) {
+  if (!t) return fail(MSSM_ERR_INVALID_ARG, "%s: null tensor descriptor", name);
+  if (t->ndim != ndim) return fail(MSSM_ERR_INVALID_ARG, "%s: expected %d dims, got %d", name, ndim, t->ndim);
+  int64_t numel = 1;
+  for (int i = 0; i < ndim; ++i) {
+    if (t->shape[i] < 0) return fail(MSSM_ERR_INVALID_ARG, "%s: negative size in dim %d", name, i);
+    if (shape[i] >= 0 && t->shape[i] != shape[i])
+      return fail(MSSM_ERR_INVALID_ARG, "%s: dim %d is %lld, expected %lld", name, i,
+                  (long long)t->shape[i], (long long)shape[i]);
+    numel *= t->shape[i];
+  }
+  if (t->dtype != dtype)
+    return fail(MSSM_ERR_INVALID_ARG, "%s: dtype %s, expected %s", name, dname(t->dtype), dname(dtype));
+  if (numel > 0 && !t->data) return fail(MSSM_ERR_INVALID_ARG, "%s: null data pointer", name);
+  if (inner_contig && t->shape[ndim - 1] > 1 && t->stride[ndim - 1] != 1)
+    return fail(MSSM_ERR_UNSUPPORTED, "%s: innermost stride must be 1", name);
+  if (!aligned16(t->data) && (reinterpret_cast<uintptr_t>(t->data) % esize(dtype)) != 0)
+    return fail(MSSM_ERR_INVALID_ARG, "%s: data pointer not aligned to its element size", name);
+  return MSSM_OK;
+}
+
+// rows of a [.., .., L] tensor start on 16-byte boundaries
+bool rows_vec(const mssm_tensor* t) {
+  const int64_t es = int64_t(esize(t->dtype));
+  return aligned16(t->data) && (t->stride[0] * es) % 16 == 0 && (t->stride[1] * es) % 16 == 0;
+}
+
+bool same_ptr(const mssm_tensor* a, const mssm_tensor* b) {
+  return a && b && a->data && a->data == b->data;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mssm_version(void) { return "0.1.0"; }
+
+const char* mssm_status_string(mssm_status s) {
+  switch (s) {
+    case MSSM_OK: return "MSSM_OK";
+    case MSSM_ERR_INVALID_ARG: return "MSSM_ERR_INVALID_ARG";
+    case MSSM_ERR_UNSUPPORTED: return "MSSM_ERR_UNSUPPORTED";
+    case MSSM_ERR_CUDA: return "MSSM_ERR_CUDA";
+  }
+  return "MSSM_ERR_UNKNOWN";
+}
+
+const char* mssm_last_error(void) { return g_last_error.c_str(); }
+
+mssm_status mssm_set_option(int option, int64_t value) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  switch (option) {
+    case MSSM_OPT_FORCE_GENERAL_A:
+      if (value != 0 && value != 1) return fail(MSSM_ERR_INVALID_ARG, "FORCE_GENERAL_A takes 0 or 1");
+      g_force_general = int(value);
+      return MSSM_OK;
+    case MSSM_OPT_CHUNK_LEN:
+      if (value < 0 || value % mssm::kSegQuant != 0 || value > (int64_t(1) << 30))
+        return fail(MSSM_ERR_INVALID_ARG, "CHUNK_LEN must be 0 or a positive multiple of %d", mssm::kSegQuant);
+      g_chunk_len = value;
+      return MSSM_OK;
+    case MSSM_OPT_KERNEL_TIMING:
+      if (value != 0 && value != 1) return fail(MSSM_ERR_INVALID_ARG, "KERNEL_TIMING takes 0 or 1");
+      g_timing = int(value);
+      return MSSM_OK;
+  }
+  return fail(MSSM_ERR_INVALID_ARG, "unknown option %d", option);
+}
+
+mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* delta,
+                                    const mssm_tensor* A, const mssm_tensor* B,
+                                    const mssm_tensor* C, const mssm_tensor* D,
+                                    const mssm_tensor* z, const mssm_tensor* delta_bias,
+                                    int softplus_flag, mssm_tensor* out, mssm_tensor* last_state,
+                                    void* stream) {
+  if (!u) return fail(MSSM_ERR_INVALID_ARG, "u: null tensor descriptor");
+  if (u->ndim != 3) return fail(MSSM_ERR_INVALID_ARG, "u: expected 3 dims [Bt, D, L]");
+  const int dt = u->dtype;
+  if (dt != MSSM_F32 && dt != MSSM_BF16) return fail(MSSM_ERR_INVALID_ARG, "u: dtype must be f32 or bf16");
+  if (!A || A->ndim != 2) return fail(MSSM_ERR_INVALID_ARG, "A: expected 2 dims [D, N]");
+  const int64_t Bt = u->shape[0], Dd = u->shape[1], L = u->shape[2], N = A->shape[1];
+  if (N != mssm::kN)
+    return fail(MSSM_ERR_UNSUPPORTED, "state size N = %lld; this build supports N = %d", (long long)N, mssm::kN);
+  const int64_t s_bdl[3] = {Bt, Dd, L}, s_bnl[3] = {Bt, N, L}, s_dn[2] = {Dd, N}, s_d[1] = {Dd},
+                s_bdn[3] = {Bt, Dd, N};
+  mssm_status st;
+  if ((st = check(u, "u", 3, s_bdl, dt, true)) != MSSM_OK) return st;
+  if ((st = check(delta, "delta", 3, s_bdl, dt, true)) != MSSM_OK) return st;
+  if ((st = check(A, "A", 2, s_dn, MSSM_F32, false)) != MSSM_OK) return st;
+  if ((st = check(B, "B", 3, s_bnl, dt, true)) != MSSM_OK) return st;
+  if ((st = check(C, "C", 3, s_bnl, dt, true)) != MSSM_OK) return st;
+  if (D && (st = check(D, "D", 1, s_d, MSSM_F32, false)) != MSSM_OK) return st;
+  if (z && (st = check(z, "z", 3, s_bdl, dt, true)) != MSSM_OK) return st;
+  if (delta_bias && (st = check(delta_bias, "delta_bias", 1, s_d, MSSM_F32, false)) != MSSM_OK) return st;
+  if ((st = check(out, "out", 3, s_bdl, dt, true)) != MSSM_OK) return st;
+  if (last_state && (st = check(last_state, "last_state", 3, s_bdn, MSSM_F32, true)) != MSSM_OK) return st;
+  if (Bt > INT32_MAX || Dd > INT32_MAX || L > INT32_MAX - 2 * mssm::kSegQuant)
+    return fail(MSSM_ERR_UNSUPPORTED, "Bt, D and L must each fit in 31 bits");
+  const mssm_tensor* ins[] = {u, delta, B, C, z, A, D, delta_bias};
+  for (const mssm_tensor* t : ins)
+    if (same_ptr(out, t)) return fail(MSSM_ERR_INVALID_ARG, "out must not alias an input");
+  if (last_state)
+    for (const mssm_tensor* t : ins)
+      if (same_ptr(last_state, t)) return fail(MSSM_ERR_INVALID_ARG, "last_state must not alias an input");
+  if (Bt == 0 || Dd == 0) return MSSM_OK;
+
+  mssm::ScanArgs a{};
+  a.u = u->data; a.delta = delta->data; a.z = z ? z->data : nullptr; a.out = out->data;
+  a.u_sb = u->stride[0]; a.u_sd = u->stride[1];
+  a.dl_sb = delta->stride[0]; a.dl_sd = delta->stride[1];
+  a.z_sb = z ? z->stride[0] : 0; a.z_sd = z ? z->stride[1] : 0;
+  a.o_sb = out->stride[0]; a.o_sd = out->stride[1];
+  a.B = B->data; a.C = C->data;
+  a.B_sb = B->stride[0]; a.B_sn = B->stride[1]; a.C_sb = C->stride[0]; a.C_sn = C->stride[1];
+  a.A = static_cast<const float*>(A->data); a.A_sd = A->stride[0]; a.A_sn = A->stride[1];
+  a.Dskip = D ? static_cast<const float*>(D->data) : nullptr; a.D_s = D ? D->stride[0] : 0;
+  a.bias = delta_bias ? static_cast<const float*>(delta_bias->data) : nullptr;
+  a.bias_s = delta_bias ? delta_bias->stride[0] : 0;
+  a.last_state = last_state ? static_cast<float*>(last_state->data) : nullptr;
+  a.ls_sb = last_state ? last_state->stride[0] : 0; a.ls_sd = last_state ? last_state->stride[1] : 0;
+  a.Bt = int(Bt); a.D = int(Dd); a.L = int(L);
+  a.tiles_per_batch = int((Dd + mssm::kRows - 1) / mssm::kRows);
+  a.vec_rows = rows_vec(u) && rows_vec(delta) && rows_vec(out) && (!z || rows_vec(z));
+  a.vec_bc = rows_vec(B) && rows_vec(C);
+
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  std::lock_guard<std::mutex> lk(g_mu);
+  a.force_general = g_force_general;
+  DeviceState* ds = device_state(dev);
+  const int64_t tiles = Bt * a.tiles_per_batch;
+  // Chunk length: enough (row tile, chunk) CTAs for about 4 per SM, in
+  // multiples of kSegQuant; no split when the rows alone fill the GPU.
+  int64_t seg = L;
+  if (g_chunk_len > 0) {
+    seg = g_chunk_len;
+  } else {
+    const int64_t want = 4 * int64_t(ds->sm_count);
+    if (tiles < want && L > mssm::kSegQuant) {
+      const int64_t nseg = (want + tiles - 1) / tiles;
+      seg = (L + nseg - 1) / nseg;
+    }
+  }
+  seg = ((seg + mssm::kSegQuant - 1) / mssm::kSegQuant) * mssm::kSegQuant;
+  if (seg < mssm::kSegQuant) seg = mssm::kSegQuant;
+  int64_t nseg = L > 0 ? (L + seg - 1) / seg : 1;
+  while (nseg > 65535) {  // grid.y limit
+    seg *= 2;
+    nseg = (L + seg - 1) / seg;
+  }
+  a.seg_len = int(seg);
+  a.nseg = int(nseg);
+
+  if (nseg > 1) {
+    const int64_t rows_total = tiles * mssm::kRows;
+    const size_t count_bytes = ((size_t(tiles) * 4 + 255) / 256) * 256;
+    const size_t s_bytes = ((size_t(nseg - 1) * rows_total * 4 + 255) / 256) * 256;
+    const size_t h_bytes = size_t(nseg - 1) * rows_total * mssm::kN * 4;
+    const size_t need = count_bytes + s_bytes + h_bytes;
+    if (ds->ws_bytes < need) {
+      if (ds->ws) {
+        e = cudaFree(ds->ws);  // synchronises the device
+        ds->ws = nullptr;
+        ds->ws_bytes = 0;
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFree(workspace)");
+      }
+      e = cudaMalloc(&ds->ws, need);
+      if (e != cudaSuccess) {
+        ds->ws = nullptr;
+        return cuda_fail(e, "cudaMalloc(workspace)");
+      }
+      ds->ws_bytes = need;
+      // arrival counters start at zero; every complete call leaves them at zero
+      e = cudaMemsetAsync(ds->ws, 0, need, s);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+    }
+    char* base = static_cast<char*>(ds->ws);
+    a.ws_count = reinterpret_cast<unsigned*>(base);
+    a.ws_S = reinterpret_cast<float*>(base + count_bytes);
+    a.ws_H = reinterpret_cast<float*>(base + count_bytes + s_bytes);
+  }
+
+  if (nseg > 1) {
+    e = tracked(MSSM_KERNEL_SCAN_CHUNK_STATE, s,
+                [&] { return mssm::launch_scan_chunk_state(a, dt, softplus_flag != 0, s); });
+    if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel launch");
+  }
+  e = tracked(MSSM_KERNEL_SCAN_OUT, s,
+              [&] { return mssm::launch_scan_out(a, dt, z != nullptr, softplus_flag != 0, s); });
+  if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
+  return MSSM_OK;
+}
+
+static mssm_status state_update_impl(mssm_tensor* state, const mssm_tensor* x, const mssm_tensor* dt_t,
+                                     const mssm_tensor* A, const mssm_tensor* B, const mssm_tensor* C,
+                                     const mssm_tensor* D, const mssm_tensor* z, const mssm_tensor* bias,
+                                     int softplus_flag, mssm_tensor* out, void* stream) {
+  if (!x) return fail(MSSM_ERR_INVALID_ARG, "x: null tensor descriptor");
+  if (x->ndim != 2) return fail(MSSM_ERR_INVALID_ARG, "x: expected 2 dims [Bt, D]");
+  const int dt = x->dtype;
+  if (dt != MSSM_F32 && dt != MSSM_BF16) return fail(MSSM_ERR_INVALID_ARG, "x: dtype must be f32 or bf16");
+  if (!A || A->ndim != 2) return fail(MSSM_ERR_INVALID_ARG, "A: expected 2 dims [D, N]");
+  const int64_t Bt = x->shape[0], Dd = x->shape[1], N = A->shape[1];
+  if (N != mssm::kN)
+    return fail(MSSM_ERR_UNSUPPORTED, "state size N = %lld; this build supports N = %d", (long long)N, mssm::kN);
+  const int64_t s_bd[2] = {Bt, Dd}, s_bn[2] = {Bt, N}, s_dn[2] = {Dd, N}, s_d[1] = {Dd}, s_bdn[3] = {Bt, Dd, N};
+  mssm_status st;
+  if ((st = check(state, "state", 3, s_bdn, MSSM_F32, true)) != MSSM_OK) return st;
+  if ((st = check(x, "x", 2, s_bd, dt, false)) != MSSM_OK) return st;
+  if ((st = check(dt_t, "dt", 2, s_bd, dt, false)) != MSSM_OK) return st;
+  if ((st = check(A, "A", 2, s_dn, MSSM_F32, false)) != MSSM_OK) return st;
+  if ((st = check(B, "B", 2, s_bn, dt, false)) != MSSM_OK) return st;
+  if ((st = check(C, "C", 2, s_bn, dt, false)) != MSSM_OK) return st;
+  if (D && (st = check(D, "D", 1, s_d, MSSM_F32, false)) != MSSM_OK) return st;
+  if (z && (st = check(z, "z", 2, s_bd, dt, false)) != MSSM_OK) return st;
+  if (bias && (st = check(bias, "dt_bias", 1, s_d, MSSM_F32, false)) != MSSM_OK) return st;
+  if ((st = check(out, "out", 2, s_bd, dt, false)) != MSSM_OK) return st;
+  if (Bt > INT32_MAX || Dd > INT32_MAX) return fail(MSSM_ERR_UNSUPPORTED, "Bt and D must fit in 31 bits");
+  const mssm_tensor* ins[] = {x, dt_t, A, B, C, D, z, bias};
+  for (const mssm_tensor* t : ins) {
+    if (same_ptr(out, t)) return fail(MSSM_ERR_INVALID_ARG, "out must not alias an input");
+    if (same_ptr(state, t)) return fail(MSSM_ERR_INVALID_ARG, "state must not alias an input");
+  }
+  if (same_ptr(out, state)) return fail(MSSM_ERR_INVALID_ARG, "out must not alias state");
+  if (Bt == 0 || Dd == 0) return MSSM_OK;
+  if (Bt * Dd * 4 / 256 + 1 > int64_t(INT32_MAX)) return fail(MSSM_ERR_UNSUPPORTED, "too many rows for one launch");
+
+  mssm::DecodeArgs a{};
+  a.state = static_cast<float*>(state->data);
+  a.st_sb = state->stride[0]; a.st_sd = state->stride[1];
+  a.x = x->data; a.dt = dt_t->data; a.z = z ? z->data : nullptr; a.out = out->data;
+  a.x_sb = x->stride[0]; a.x_sd = x->stride[1];
+  a.dt_sb = dt_t->stride[0]; a.dt_sd = dt_t->stride[1];
+  a.z_sb = z ? z->stride[0] : 0; a.z_sd = z ? z->stride[1] : 0;
+  a.o_sb = out->stride[0]; a.o_sd = out->stride[1];
+  a.A = static_cast<const float*>(A->data); a.A_sd = A->stride[0]; a.A_sn = A->stride[1];
+  a.B = B->data; a.C = C->data;
+  a.B_sb = B->stride[0]; a.B_sn = B->stride[1]; a.C_sb = C->stride[0]; a.C_sn = C->stride[1];
+  a.Dskip = D ? static_cast<const float*>(D->data) : nullptr; a.D_s = D ? D->stride[0] : 0;
+  a.bias = bias ? static_cast<const float*>(bias->data) : nullptr; a.bias_s = bias ? bias->stride[0] : 0;
+  a.Bt = int(Bt); a.D = int(Dd);
+  a.softplus = softplus_flag != 0;
+  a.vec_state = aligned16(state->data) && (state->stride[0] * 4) % 16 == 0 && (state->stride[1] * 4) % 16 == 0;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lk(g_mu);
+  cudaError_t e = tracked(MSSM_KERNEL_STATE_UPDATE, s,
+                          [&] { return mssm::launch_state_update(a, dt, z != nullptr, s); });
+  if (e != cudaSuccess) return cuda_fail(e, "state update launch");
+  return MSSM_OK;
+}
+
+mssm_status mssm_state_update(mssm_tensor* state, const mssm_tensor* x, const mssm_tensor* dt,
+                              const mssm_tensor* A, const mssm_tensor* B, const mssm_tensor* C,
+                              const mssm_tensor* D, const mssm_tensor* z, mssm_tensor* out,
+                              void* stream) {
+  return state_update_impl(state, x, dt, A, B, C, D, z, nullptr, 1, out, stream);
+}
+
+mssm_status mssm_state_update_ex(mssm_tensor* state, const mssm_tensor* x, const mssm_tensor* dt,
+                                 const mssm_tensor* A, const mssm_tensor* B, const mssm_tensor* C,
+                                 const mssm_tensor* D, const mssm_tensor* z, const mssm_tensor* dt_bias,
+                                 int softplus_flag, mssm_tensor* out, void* stream) {
+  return state_update_impl(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, out, stream);
+}
+
+mssm_status mssm_kernel_stats(int64_t launches[MSSM_KERNEL_KINDS], int64_t timed[MSSM_KERNEL_KINDS],
+                              double ms[MSSM_KERNEL_KINDS], int reset) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  mssm_status st = MSSM_OK;
+  for (const TimedLaunch& t : g_pending) {
+    float v = 0.0f;
+    cudaError_t e = cudaEventSynchronize(t.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&v, t.a, t.b);
+    if (e != cudaSuccess) {
+      st = cuda_fail(e, "kernel timing events");
+    } else {
+      g_time_ms[t.kind] += v;
+      g_timed[t.kind] += 1;
+    }
+    g_event_pool.push_back(t.a);
+    g_event_pool.push_back(t.b);
+  }
+  g_pending.clear();
+  for (int k = 0; k < MSSM_KERNEL_KINDS; ++k) {
+    if (launches) launches[k] = g_launches[k];
+    if (timed) timed[k] = g_timed[k];
+    if (ms) ms[k] = g_time_ms[k];
+    if (reset) {
+      g_launches[k] = 0;
+      g_timed[k] = 0;
+      g_time_ms[k] = 0.0;
+    }
+  }
+  return st;
+}
+
+mssm_status mssm_get_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "asynchronous kernel error");
+  return MSSM_OK;
+}
+
+mssm_status mssm_shutdown(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  mssm_status st = MSSM_OK;
+  int prev = -1;
+  if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+  for (size_t i = 0; i < g_dev.size(); ++i) {
+    if (!g_dev[i].ws) continue;
+    cudaSetDevice(int(i));
+    cudaError_t e = cudaFree(g_dev[i].ws);
+    if (e != cudaSuccess) st = cuda_fail(e, "cudaFree(workspace)");
+    g_dev[i].ws = nullptr;
+    g_dev[i].ws_bytes = 0;
+  }
+  if (prev >= 0) cudaSetDevice(prev);
+  return st;
+}
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+"""Helpers for the GPU parity tests: move synth inputs to the device, run the
+library through its C ABI, compare with the oracle under the stated tolerance.
+
+Tolerance: |gpu - ref| <= tol * (1 + |ref|) elementwise, with tol = 1e-4 for
+fp32 I/O and 2e-2 for bf16 I/O, on both y and the final state.
+"""
+import numpy as np
+import torch
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def to_dev(a, io_dtype=None):
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def to_f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def check_close(gpu, ref, io_dtype, what="y"):
+    tol = TOL[io_dtype]
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
+    assert np.isfinite(gpu).all(), f"{what}: non-finite values from the GPU"
+    err = np.abs(gpu - ref) / (1.0 + np.abs(ref))
+    worst = float(err.max()) if err.size else 0.0
+    if worst > tol:
+        idx = np.unravel_index(int(err.argmax()), err.shape)
+        raise AssertionError(f"{what}: worst scaled error {worst:.3e} > {tol:g} at {idx}: "
+                             f"gpu={gpu[idx]!r} ref={ref[idx]!r}")
+    return worst
+
+
+def dev_scan_inputs(inp):
+    """Device tensors of a synth.ScanInputs problem."""
+    return dict(u=to_dev(inp.u), delta=to_dev(inp.delta), A=to_dev(inp.A), B=to_dev(inp.B),
+                C=to_dev(inp.C), D=to_dev(inp.D), z=to_dev(inp.z), delta_bias=to_dev(inp.delta_bias))
+
+
+def run_scan(inp, dev=None, **kw):
+    import selective_state_space_46_b200 as m
+    dev = dev or dev_scan_inputs(inp)
+    out, last = m.selective_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dev["D"],
+                                     dev["z"], dev["delta_bias"], inp.softplus, **kw)
+    torch.cuda.synchronize()
+    return out, last

@@ -1,0 +1,169 @@
+"""Host-side checks of the C ABI, no GPU needed.
+
+* libmssm.so loads and exports every function include/mssm.h declares;
+* argument validation returns the documented status before anything touches
+  the device (descriptors carry fake, never-dereferenced device pointers).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from selective_state_space_46_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(mssm_[a-z0-9_]+)\s*\(", text):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"mssm_selective_scan_fwd", "mssm_state_update"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+# ---------------------------------------------------------------------------
+# validation (fake pointers; every case below fails before any CUDA call)
+# ---------------------------------------------------------------------------
+
+class T(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+_fake = [0x10000]
+
+
+def mk(shape, dtype=1, stride=None):
+    t = T()
+    _fake[0] += 1 << 30
+    t.data = _fake[0]
+    t.dtype = dtype
+    t.ndim = len(shape)
+    if stride is None:
+        stride, acc = [], 1
+        for s in reversed(shape):
+            stride.insert(0, acc)
+            acc *= s
+    for i, (s, st) in enumerate(zip(shape, stride)):
+        t.shape[i] = s
+        t.stride[i] = st
+    return t
+
+
+def scan_args(Bt=2, D=8, L=32, N=16, dt=1, **over):
+    a = dict(u=mk([Bt, D, L], dt), delta=mk([Bt, D, L], dt), A=mk([D, N], 0), B=mk([Bt, N, L], dt),
+             C=mk([Bt, N, L], dt), D=mk([D], 0), z=mk([Bt, D, L], dt), delta_bias=mk([D], 0),
+             out=mk([Bt, D, L], dt), last_state=mk([Bt, D, N], 0))
+    a.update(over)
+    return a
+
+
+def call_scan(lib, a, softplus=1):
+    P = lambda t: None if t is None else ctypes.byref(t)  # noqa: E731
+    f = lib.mssm_selective_scan_fwd
+    f.restype = ctypes.c_int
+    return f(P(a["u"]), P(a["delta"]), P(a["A"]), P(a["B"]), P(a["C"]), P(a["D"]), P(a["z"]),
+             P(a["delta_bias"]), softplus, P(a["out"]), P(a["last_state"]), None)
+
+
+def last_error(lib):
+    lib.mssm_last_error.restype = ctypes.c_char_p
+    return lib.mssm_last_error().decode()
+
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("null_u", INVALID),
+    ("null_out", INVALID),
+    ("N8", UNSUPPORTED),
+    ("delta_dtype", INVALID),
+    ("A_bf16", INVALID),
+    ("B_shape", INVALID),
+    ("z_shape", INVALID),
+    ("out_aliases_u", INVALID),
+    ("inner_stride", UNSUPPORTED),
+    ("last_state_dtype", INVALID),
+    ("null_data", INVALID),
+    ("bad_u_dtype", INVALID),
+])
+def test_scan_validation(lib, case, expect):
+    a = scan_args()
+    if case == "null_u":
+        a["u"] = None
+    elif case == "null_out":
+        a["out"] = None
+    elif case == "N8":
+        a = scan_args(N=8)
+    elif case == "delta_dtype":
+        a["delta"] = mk([2, 8, 32], 0)
+    elif case == "A_bf16":
+        a["A"] = mk([8, 16], 1)
+    elif case == "B_shape":
+        a["B"] = mk([2, 16, 31], 1)
+    elif case == "z_shape":
+        a["z"] = mk([2, 7, 32], 1)
+    elif case == "out_aliases_u":
+        a["out"].data = a["u"].data
+    elif case == "inner_stride":
+        a["u"] = mk([2, 8, 32], 1, stride=[512, 64, 2])
+    elif case == "last_state_dtype":
+        a["last_state"] = mk([2, 8, 16], 1)
+    elif case == "null_data":
+        a["C"].data = None
+    elif case == "bad_u_dtype":
+        a["u"].dtype = 7
+    assert call_scan(lib, a) == expect
+    assert last_error(lib)
+
+
+def test_empty_problem_is_noop(lib):
+    # Bt == 0 returns OK without touching the device
+    a = scan_args(Bt=0)
+    assert call_scan(lib, a) == 0
+
+
+def test_decode_validation(lib):
+    P = ctypes.byref
+    f = lib.mssm_state_update
+    f.restype = ctypes.c_int
+    st, x, dt = mk([4, 8, 16], 0), mk([4, 8], 1), mk([4, 8], 1)
+    A, B, C, D, z, out = mk([8, 16], 0), mk([4, 16], 1), mk([4, 16], 1), mk([8], 0), mk([4, 8], 1), mk([4, 8], 1)
+    bad_state = mk([4, 8, 16], 1)
+    assert f(P(bad_state), P(x), P(dt), P(A), P(B), P(C), P(D), P(z), P(out), None) == INVALID
+    bad_A = mk([8, 32], 0)
+    assert f(P(st), P(x), P(dt), P(bad_A), P(B), P(C), P(D), P(z), P(out), None) == UNSUPPORTED
+    out.data = x.data
+    assert f(P(st), P(x), P(dt), P(A), P(B), P(C), P(D), P(z), P(out), None) == INVALID
+    assert f(None, P(x), P(dt), P(A), P(B), P(C), P(D), P(z), P(out), None) == INVALID
+
+
+def test_options_and_strings(lib):
+    lib.mssm_set_option.argtypes = [ctypes.c_int, ctypes.c_int64]
+    assert lib.mssm_set_option(1, 2) == INVALID
+    assert lib.mssm_set_option(2, 100) == INVALID      # not a multiple of 64
+    assert lib.mssm_set_option(99, 0) == INVALID
+    assert lib.mssm_set_option(2, 128) == 0
+    assert lib.mssm_set_option(2, 0) == 0
+    lib.mssm_status_string.restype = ctypes.c_char_p
+    assert lib.mssm_status_string(2) == b"MSSM_ERR_UNSUPPORTED"
+    lib.mssm_version.restype = ctypes.c_char_p
+    assert re.match(rb"^\d+\.\d+\.\d+$", lib.mssm_version())

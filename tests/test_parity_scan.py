@@ -1,0 +1,247 @@
+"""GPU parity of mssm_selective_scan_fwd against the fp64 oracle.
+
+Small and medium problems are compared element by element; the full-size
+prefill shapes are run whole on the GPU in the launch configuration the
+benchmark uses and checked on sampled rows that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import check_close, dev_scan_inputs, run_scan, to_dev, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _defaults(cuda_device):
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 0)
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
+    yield
+    m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 0)
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
+
+
+def compare_full(inp, **kw):
+    out, last = run_scan(inp, **kw)
+    y_ref, h_ref = oracle.scan_inputs(inp)
+    check_close(to_f64(out), y_ref, inp.io_dtype, "y")
+    check_close(to_f64(last), h_ref, inp.io_dtype, "last_state")
+
+
+def random_A(dim, seed):
+    rng = np.random.default_rng(seed)
+    return (-np.exp(rng.uniform(-1.0, 1.5, size=(dim, 16)))).astype(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# the named workloads
+# ---------------------------------------------------------------------------
+
+def test_workload_f32_1x64x256():
+    compare_full(synth.workload_inputs("scan_f32_1x64x256"))
+
+
+def test_workload_bf16_2x1536x2048():
+    compare_full(synth.workload_inputs("scan_bf16_2x1536x2048"))
+
+
+def test_workload_bf16_2x1536x2048_general_A_path():
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 1)
+    compare_full(synth.workload_inputs("scan_bf16_2x1536x2048"))
+
+
+def _sampled(name, rows_per_batch=6, seed=0):
+    inp = synth.workload_inputs(name)
+    out, last = run_scan(inp)
+    rng = np.random.default_rng(seed)
+    rows = []
+    for b in range(inp.batch):
+        ds = set(rng.choice(inp.dim, size=rows_per_batch, replace=False).tolist())
+        ds |= {0, inp.dim - 1}
+        rows += [(b, int(d)) for d in sorted(ds)]
+    y_ref, h_ref = oracle.scan_rows(inp, rows)
+    bi = torch.tensor([r[0] for r in rows], device=out.device)
+    di = torch.tensor([r[1] for r in rows], device=out.device)
+    check_close(to_f64(out[bi, di]), y_ref, inp.io_dtype, "y")
+    check_close(to_f64(last[bi, di]), h_ref, inp.io_dtype, "last_state")
+
+
+@pytest.mark.slow
+def test_workload_bf16_8x5120x4096_sampled():
+    _sampled("scan_bf16_8x5120x4096", rows_per_batch=4)
+
+
+@pytest.mark.slow
+def test_workload_bf16_1x2048x131072_sampled():
+    _sampled("scan_bf16_1x2048x131072", rows_per_batch=10)
+
+
+# ---------------------------------------------------------------------------
+# shapes: ragged lengths and channel counts, options on and off
+# ---------------------------------------------------------------------------
+
+SHAPES = [
+    (1, 1, 1), (1, 3, 2), (2, 5, 7), (1, 64, 15), (1, 65, 16), (2, 63, 17), (1, 1, 31),
+    (1, 130, 33), (2, 64, 64), (1, 7, 100), (3, 129, 257), (1, 64, 1000), (2, 200, 777),
+]
+
+
+@pytest.mark.parametrize("Bt,D,L", SHAPES)
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_shapes(Bt, D, L, io):
+    inp = synth.make_scan_inputs(Bt, D, L, io_dtype=io, seed=L * 7 + D)
+    compare_full(inp)
+
+
+@pytest.mark.parametrize("with_z,with_D,with_bias,softplus", [
+    (False, False, False, True), (True, False, True, False), (False, True, False, False),
+    (True, True, True, True),
+])
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_optional_inputs(with_z, with_D, with_bias, softplus, io):
+    inp = synth.make_scan_inputs(2, 70, 300, io_dtype=io, seed=3, with_z=with_z, with_D=with_D,
+                                 with_bias=with_bias, softplus=softplus)
+    if not softplus:
+        # keep the step positive and small without softplus: delta = |raw| * 0.05
+        raw = synth.bf16_bits_to_f32(inp.delta) if io == "bf16" else inp.delta
+        pos = np.abs(raw) * 0.05
+        inp.delta = synth.f32_to_bf16_bits(pos) if io == "bf16" else pos.astype(np.float32)
+        inp.delta_bias = None
+    compare_full(inp)
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_general_A_values(io):
+    inp = synth.make_scan_inputs(2, 96, 500, io_dtype=io, seed=11)
+    inp.A = random_A(96, 5)
+    compare_full(inp)
+
+
+# ---------------------------------------------------------------------------
+# the length split and its carry
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("chunk", [64, 128, 192, 320])
+@pytest.mark.parametrize("structured", [True, False])
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_chunked_carry(chunk, structured, io):
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, chunk)
+    inp = synth.make_scan_inputs(2, 80, 1000, io_dtype=io, seed=chunk, delta_range=(1e-4, 1e-2))
+    if not structured:
+        inp.A = random_A(80, chunk)
+    compare_full(inp)
+
+
+def test_chunked_equals_unchunked_closely():
+    # the split changes only the association order of fp32 sums
+    import selective_state_space_46_b200 as m
+    inp = synth.make_scan_inputs(1, 64, 2048, io_dtype="f32", seed=21, delta_range=(1e-4, 1e-2))
+    dev = dev_scan_inputs(inp)
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 4096)
+    y1, h1 = run_scan(inp, dev)
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 128)
+    y2, h2 = run_scan(inp, dev)
+    scale = 1 + y1.abs()
+    assert float(((y1 - y2).abs() / scale).max()) < 1e-5
+    assert float(((h1 - h2).abs() / (1 + h1.abs())).max()) < 1e-5
+
+
+def test_long_slow_decay_many_chunks():
+    inp = synth.make_scan_inputs(1, 64, 16384, io_dtype="bf16", seed=5, delta_range=(1e-4, 1e-2))
+    compare_full(inp)
+
+
+# ---------------------------------------------------------------------------
+# layouts: strided and unaligned rows take the scalar path
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_strided_unaligned_rows(io):
+    Bt, D, L = 2, 70, 203
+    inp = synth.make_scan_inputs(Bt, D, L, io_dtype=io, seed=9)
+    dev = dev_scan_inputs(inp)
+
+    def padded(t, pad):
+        big = torch.zeros(*t.shape[:-1], t.shape[-1] + pad, dtype=t.dtype, device=t.device)
+        big[..., 1:1 + t.shape[-1]] = t
+        return big[..., 1:1 + t.shape[-1]]
+
+    for k in ("u", "delta", "z", "B", "C"):
+        dev[k] = padded(dev[k], 5)
+        assert not dev[k].is_contiguous()
+    out_big = torch.zeros(Bt, D, L + 3, dtype=dev["u"].dtype, device="cuda")
+    out = out_big[..., :L]
+    last = torch.empty(Bt, D, 16, device="cuda")
+    import selective_state_space_46_b200 as m
+    m.mssm_selective_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dev["D"], dev["z"],
+                              dev["delta_bias"], True, out, last)
+    torch.cuda.synchronize()
+    y_ref, h_ref = oracle.scan_inputs(inp)
+    check_close(to_f64(out), y_ref, io, "y")
+    check_close(to_f64(last), h_ref, io, "last_state")
+    assert float(out_big[..., L:].abs().max()) == 0.0   # nothing written past the view
+
+
+# ---------------------------------------------------------------------------
+# edge cases and API behaviour
+# ---------------------------------------------------------------------------
+
+def test_empty_and_zero_length():
+    import selective_state_space_46_b200 as m
+    inp = synth.make_scan_inputs(2, 9, 0, io_dtype="bf16", seed=1)
+    dev = dev_scan_inputs(inp)
+    last = torch.full((2, 9, 16), 7.0, device="cuda")
+    out = torch.empty(2, 9, 0, dtype=torch.bfloat16, device="cuda")
+    m.mssm_selective_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dev["D"], dev["z"],
+                              dev["delta_bias"], True, out, last)
+    torch.cuda.synchronize()
+    assert float(last.abs().max()) == 0.0
+    inp0 = synth.make_scan_inputs(0, 9, 10, io_dtype="bf16", seed=1)
+    y, h = run_scan(inp0)
+    assert y.numel() == 0 and h.numel() == 0
+
+
+def test_output_only_no_last_state_and_determinism():
+    inp = synth.make_scan_inputs(2, 100, 900, io_dtype="bf16", seed=4)
+    dev = dev_scan_inputs(inp)
+    y1, _ = run_scan(inp, dev, return_last_state=False)
+    y2, _ = run_scan(inp, dev, return_last_state=False)
+    assert torch.equal(y1, y2)
+    y_ref, _ = oracle.scan_inputs(inp)
+    check_close(to_f64(y1), y_ref, "bf16")
+
+
+def test_side_stream():
+    import selective_state_space_46_b200 as m
+    inp = synth.make_scan_inputs(1, 64, 512, io_dtype="bf16", seed=8)
+    dev = dev_scan_inputs(inp)
+    s = torch.cuda.Stream()
+    out = torch.empty_like(dev["u"])
+    last = torch.empty(1, 64, 16, device="cuda")
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        m.mssm_selective_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dev["D"],
+                                  dev["z"], dev["delta_bias"], True, out, last, stream=s)
+    m.mssm_get_error(s)
+    y_ref, h_ref = oracle.scan_inputs(inp)
+    check_close(to_f64(out), y_ref, "bf16")
+    check_close(to_f64(last), h_ref, "bf16")
+
+
+def test_invalid_arguments_raise():
+    import selective_state_space_46_b200 as m
+    inp = synth.make_scan_inputs(1, 8, 16, io_dtype="bf16", seed=2)
+    dev = dev_scan_inputs(inp)
+    with pytest.raises(m.MssmError) as e:
+        m.selective_scan_fwd(dev["u"], dev["delta"].float(), dev["A"], dev["B"], dev["C"])
+    assert e.value.status == m.MSSM_ERR_INVALID_ARG
+    with pytest.raises(m.MssmError) as e:
+        m.selective_scan_fwd(dev["u"], dev["delta"], dev["A"][:, :8].contiguous(), dev["B"][:, :8],
+                             dev["C"][:, :8])
+    assert e.value.status == m.MSSM_ERR_UNSUPPORTED
