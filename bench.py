@@ -301,6 +301,8 @@ def run_mssm(args):
         return t.pin_memory()
 
     seed = rank_seed(rank)
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, args.chunk_len)
+    m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 1 if args.general_a else 0)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -319,7 +321,11 @@ def run_mssm(args):
                                       d["delta_bias"], inp.softplus, out, last)
         config = {"workload": args.workload, "batch": inp.batch, "channels": inp.dim, "length": inp.length,
                   "state": N_STATE, "io_dtype": inp.io_dtype, "gate": inp.z is not None,
-                  "softplus_bias": inp.delta_bias is not None, "D_skip": inp.D is not None}
+                  "softplus_bias": inp.delta_bias is not None, "D_skip": inp.D is not None,
+                  "exp_path": "general (one exponential per state)" if args.general_a
+                  else "structured A (powers of one exponential)",
+                  "chunk_len": args.chunk_len or "auto",
+                  "plan": m.mssm_scan_plan(inp.batch, inp.dim, inp.length)}
         metric, unit = METRIC, "elems/s"
         dom_kernel = "scan_out"
     else:
@@ -350,8 +356,9 @@ def run_mssm(args):
     m.mssm_get_error()
 
     # ---- capture the K timed steps into one graph
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    # external=True: the records become event nodes of the graph, so every replay re-records them
+    starts = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(args.steps)]
     before = m.mssm_kernel_stats()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
@@ -513,6 +520,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--chunk-len", type=int, default=0, help="length split (0: automatic; multiple of 64)")
+    ap.add_argument("--general-a", action="store_true",
+                    help="disable the structured-A path (one exponential per state)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -62,7 +62,8 @@ typedef enum {
     MSSM_OK = 0,
     MSSM_ERR_INVALID_ARG = 1, /* null required pointer, bad shape/stride/dtype combination */
     MSSM_ERR_UNSUPPORTED = 2, /* valid but not implemented here (N != 16, misaligned rows, ...) */
-    MSSM_ERR_CUDA = 3         /* a CUDA runtime call or a kernel launch failed */
+    MSSM_ERR_CUDA = 3,        /* a CUDA runtime call or a kernel launch failed */
+    MSSM_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (see mssm_get_error) */
 } mssm_status;
 
 typedef struct {
@@ -123,6 +124,8 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor *u, const mssm_tensor *del
  * This entry point applies delta = softplus(dt) (no bias).  The same step as
  * one iteration of mssm_selective_scan_fwd's recurrence ("State Space Models
  * in Large Language Models ...", section Discretization, recurrent view).
+ * When `state` is one contiguous 16-byte-aligned [Bt*D][16] range, each CTA
+ * moves its 16 KB tile with a bulk copy in and out of shared memory.
  */
 mssm_status mssm_state_update(mssm_tensor *state, const mssm_tensor *x, const mssm_tensor *dt,
                               const mssm_tensor *A, const mssm_tensor *B, const mssm_tensor *C,
@@ -149,9 +152,11 @@ const char *mssm_last_error(void);
 
 /*
  * Synchronises `stream` and reports an asynchronous failure of the work queued
- * on it (MSSM_ERR_CUDA, with the CUDA error text in mssm_last_error()), or
- * MSSM_OK.  The kernels contain no waits on other CTAs or on the host, so a
- * call cannot stall on the device.
+ * on it: MSSM_ERR_CUDA (with the CUDA error text in mssm_last_error()), or
+ * MSSM_ERR_TIMEOUT when a bounded device-side wait gave up since the last call
+ * (the decode kernel waits, with an iteration limit, for its own bulk copy; on
+ * giving up it leaves that tile's state rows unchanged).  Clears the device
+ * error word.  No kernel waits on another CTA or on the host.
  */
 mssm_status mssm_get_error(void *stream);
 
@@ -173,6 +178,16 @@ typedef enum {
     MSSM_OPT_KERNEL_TIMING = 3
 } mssm_option;
 mssm_status mssm_set_option(int option, int64_t value);
+
+/*
+ * Host-only query of the launch plan mssm_selective_scan_fwd would use for a
+ * [Bt, D, L] problem on a GPU with sm_count SMs (sm_count <= 0: the current
+ * device, or 148 when there is none): channels per CTA (32 or 64), chunk length
+ * and number of chunks (1 = no split).  Honours MSSM_OPT_CHUNK_LEN.  Launches
+ * nothing; any output pointer may be NULL.
+ */
+mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int *rows_per_cta,
+                           int64_t *chunk_len, int64_t *n_chunks);
 
 /* Kernel kinds counted by mssm_kernel_stats. */
 typedef enum {

@@ -6,7 +6,7 @@ entry points declared in ``include/mssm.h`` with the same names.  Every step of
 the computation runs in the library's CUDA kernels; there is no CPU or PyTorch
 fallback, and importing fails loudly when the library has not been built.
 
-Build the library with ``python -m selective_state_space_46_b200.build``.
+Build the library with ``python selective_state_space_46_b200/build.py``.
 """
 from __future__ import annotations
 
@@ -20,19 +20,19 @@ __all__ = [
     "MssmError", "mssm_selective_scan_fwd", "mssm_state_update", "mssm_state_update_ex",
     "mssm_get_error", "mssm_set_option", "mssm_shutdown", "mssm_version", "mssm_status_string",
     "mssm_last_error", "selective_scan_fwd", "state_update", "lib_path",
-    "MSSM_OPT_FORCE_GENERAL_A", "MSSM_OPT_CHUNK_LEN", "MSSM_OPT_KERNEL_TIMING", "mssm_kernel_stats",
+    "MSSM_OPT_FORCE_GENERAL_A", "MSSM_OPT_CHUNK_LEN", "MSSM_OPT_KERNEL_TIMING", "mssm_kernel_stats", "mssm_scan_plan",
     "KERNEL_KINDS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libmssm.so")
 if not os.path.exists(lib_path):
-    raise ImportError(f"{lib_path} is missing: build it with `python -m selective_state_space_46_b200.build` "
+    raise ImportError(f"{lib_path} is missing: build it with `python selective_state_space_46_b200/build.py` "
                       "(nvcc, sm_100a); there is no fallback implementation")
 _lib = ctypes.CDLL(lib_path)
 
 MSSM_F32, MSSM_BF16 = 0, 1
-MSSM_OK, MSSM_ERR_INVALID_ARG, MSSM_ERR_UNSUPPORTED, MSSM_ERR_CUDA = 0, 1, 2, 3
+MSSM_OK, MSSM_ERR_INVALID_ARG, MSSM_ERR_UNSUPPORTED, MSSM_ERR_CUDA, MSSM_ERR_TIMEOUT = 0, 1, 2, 3, 4
 MSSM_OPT_FORCE_GENERAL_A, MSSM_OPT_CHUNK_LEN, MSSM_OPT_KERNEL_TIMING = 1, 2, 3
 KERNEL_KINDS = ("scan_chunk_state", "scan_out", "state_update")
 
@@ -62,6 +62,10 @@ _lib.mssm_version.restype = ctypes.c_char_p
 _lib.mssm_kernel_stats.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
                                    ctypes.POINTER(ctypes.c_double), ctypes.c_int]
 _lib.mssm_kernel_stats.restype = ctypes.c_int
+_lib.mssm_scan_plan.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int64),
+                                ctypes.POINTER(ctypes.c_int64)]
+_lib.mssm_scan_plan.restype = ctypes.c_int
 
 
 class MssmError(RuntimeError):
@@ -133,6 +137,13 @@ def mssm_kernel_stats(reset: bool = False) -> dict:
     ms = (ctypes.c_double * n)()
     _check(_lib.mssm_kernel_stats(launches, timed, ms, int(reset)))
     return {k: {"launches": launches[i], "timed": timed[i], "ms": ms[i]} for i, k in enumerate(KERNEL_KINDS)}
+
+
+def mssm_scan_plan(Bt: int, D: int, L: int, sm_count: int = 0) -> dict:
+    """Launch plan of the scan for a [Bt, D, L] problem (host only, launches nothing)."""
+    rows, seg, nseg = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int64()
+    _check(_lib.mssm_scan_plan(Bt, D, L, sm_count, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg)))
+    return {"rows_per_cta": rows.value, "chunk_len": seg.value, "n_chunks": nseg.value}
 
 
 def mssm_get_error(stream=None) -> None:

@@ -1,6 +1,9 @@
 """Build libmssm.so in-tree with nvcc for sm_100a.
 
-    python -m selective_state_space_46_b200.build [--force] [--verbose]
+    python selective_state_space_46_b200/build.py [--force] [--verbose] [extra nvcc flags]
+
+Run this file directly (or load it by path): importing it through the package
+would load the library it is meant to build.
 
 Each .cu file is compiled to an object in parallel, then linked into a shared
 library next to this file.  The CUDA runtime is linked statically, so loading
@@ -86,3 +89,4 @@ if __name__ == "__main__":
     args = sys.argv[1:]
     extra = [a for a in args if a not in ("--force", "--verbose")]
     print(build(force="--force" in args, verbose="--verbose" in args, extra_flags=extra))
+

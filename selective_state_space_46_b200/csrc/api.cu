@@ -116,7 +116,7 @@ mssm_status check(const mssm_tensor* t, const char* name, int ndim, const int64_
   if (t->dtype != dtype)
     return fail(MSSM_ERR_INVALID_ARG, "%s: dtype %s, expected %s", name, dname(t->dtype), dname(dtype));
   if (numel > 0 && !t->data) return fail(MSSM_ERR_INVALID_ARG, "%s: null data pointer", name);
-  if (inner_contig && t->shape[ndim - 1] > 1 && t->stride[ndim - 1] != 1)
+  if (inner_contig && numel > 0 && t->shape[ndim - 1] > 1 && t->stride[ndim - 1] != 1)
     return fail(MSSM_ERR_UNSUPPORTED, "%s: innermost stride must be 1", name);
   if (!aligned16(t->data) && (reinterpret_cast<uintptr_t>(t->data) % esize(dtype)) != 0)
     return fail(MSSM_ERR_INVALID_ARG, "%s: data pointer not aligned to its element size", name);
@@ -133,6 +133,60 @@ bool same_ptr(const mssm_tensor* a, const mssm_tensor* b) {
   return a && b && a->data && a->data == b->data;
 }
 
+// Launch shape of the scan: channels per CTA and the length split.
+struct LaunchShape {
+  int rows;
+  int64_t seg, nseg;
+};
+
+int64_t round_seg(int64_t v) {
+  v = ((v + mssm::kSegQuant - 1) / mssm::kSegQuant) * mssm::kSegQuant;
+  return v < mssm::kSegQuant ? mssm::kSegQuant : v;
+}
+
+// Cost model (in FP32-pipe cycles of the busiest SM, up to a constant): the
+// CTAs of a kernel run in waves of at most kMaxCta[rows] per SM (register
+// limited) and carry equal work; an SM needs kSat threads to keep its pipes
+// busy, below which its time is set by one thread's serial work.  Per element
+// the forward kernel costs kOut and the chunk-summary kernel kSum; each launch
+// adds kLaunch.  Candidates: 32 or 64 channels per CTA (32 first: its kernel
+// has the larger register budget, so it wins ties), 1..64 chunks (lengths in
+// multiples of kSegQuant).
+LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forced_seg) {
+  constexpr double kSat = 512.0, kOut = 80.0, kSum = 45.0, kLaunch = 3.0e5;
+  LaunchShape best{32, L > 0 ? L : 1, 1};
+  double best_cost = -1.0;
+  for (int rows : {32, 64}) {
+    const int64_t max_cta = rows == 32 ? 12 : 8;
+    const int64_t tiles = Bt * ((D + rows - 1) / rows);
+    auto sm_time = [&](int64_t ctas, double per_elem, double seg) {
+      const int64_t on_sm = (ctas + sms - 1) / sms;
+      const int64_t waves = (on_sm + max_cta - 1) / max_cta;
+      const int64_t resident = on_sm < max_cta ? on_sm : max_cta;
+      const double threads = double(resident * rows);
+      const double work = threads * seg * per_elem / 128.0;
+      const double serial = threads < kSat ? seg * per_elem * kSat / 128.0 : 0.0;
+      return double(waves) * (work > serial ? work : serial) + kLaunch;
+    };
+    for (int64_t want = 1; want <= 64; ++want) {
+      int64_t seg = forced_seg > 0 ? forced_seg : round_seg((L + want - 1) / want);
+      int64_t nseg = L > 0 ? (L + seg - 1) / seg : 1;
+      while (nseg > 65535) {
+        seg *= 2;
+        nseg = (L + seg - 1) / seg;
+      }
+      double cost = sm_time(tiles * nseg, kOut, double(seg));
+      if (nseg > 1) cost += sm_time(tiles * (nseg - 1), kSum, double(seg));
+      if (best_cost < 0.0 || cost < best_cost * 0.999) {
+        best_cost = cost;
+        best = LaunchShape{rows, seg, nseg};
+      }
+      if (forced_seg > 0 || L <= mssm::kSegQuant) break;
+    }
+  }
+  return best;
+}
+
 }  // namespace
 
 extern "C" {
@@ -145,6 +199,7 @@ const char* mssm_status_string(mssm_status s) {
     case MSSM_ERR_INVALID_ARG: return "MSSM_ERR_INVALID_ARG";
     case MSSM_ERR_UNSUPPORTED: return "MSSM_ERR_UNSUPPORTED";
     case MSSM_ERR_CUDA: return "MSSM_ERR_CUDA";
+    case MSSM_ERR_TIMEOUT: return "MSSM_ERR_TIMEOUT";
   }
   return "MSSM_ERR_UNKNOWN";
 }
@@ -223,9 +278,10 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* del
   a.last_state = last_state ? static_cast<float*>(last_state->data) : nullptr;
   a.ls_sb = last_state ? last_state->stride[0] : 0; a.ls_sd = last_state ? last_state->stride[1] : 0;
   a.Bt = int(Bt); a.D = int(Dd); a.L = int(L);
-  a.tiles_per_batch = int((Dd + mssm::kRows - 1) / mssm::kRows);
   a.vec_rows = rows_vec(u) && rows_vec(delta) && rows_vec(out) && (!z || rows_vec(z));
   a.vec_bc = rows_vec(B) && rows_vec(C);
+  a.vec_ls = last_state && aligned16(last_state->data) && (last_state->stride[0] * 4) % 16 == 0 &&
+             (last_state->stride[1] * 4) % 16 == 0;
 
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -235,31 +291,16 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* del
   std::lock_guard<std::mutex> lk(g_mu);
   a.force_general = g_force_general;
   DeviceState* ds = device_state(dev);
+  const LaunchShape shape = choose_shape(Bt, Dd, L, ds->sm_count, g_chunk_len);
+  const int64_t seg = shape.seg, nseg = shape.nseg;
+  const int rows_per_cta = shape.rows;
+  a.tiles_per_batch = int((Dd + rows_per_cta - 1) / rows_per_cta);
   const int64_t tiles = Bt * a.tiles_per_batch;
-  // Chunk length: enough (row tile, chunk) CTAs for about 4 per SM, in
-  // multiples of kSegQuant; no split when the rows alone fill the GPU.
-  int64_t seg = L;
-  if (g_chunk_len > 0) {
-    seg = g_chunk_len;
-  } else {
-    const int64_t want = 4 * int64_t(ds->sm_count);
-    if (tiles < want && L > mssm::kSegQuant) {
-      const int64_t nseg = (want + tiles - 1) / tiles;
-      seg = (L + nseg - 1) / nseg;
-    }
-  }
-  seg = ((seg + mssm::kSegQuant - 1) / mssm::kSegQuant) * mssm::kSegQuant;
-  if (seg < mssm::kSegQuant) seg = mssm::kSegQuant;
-  int64_t nseg = L > 0 ? (L + seg - 1) / seg : 1;
-  while (nseg > 65535) {  // grid.y limit
-    seg *= 2;
-    nseg = (L + seg - 1) / seg;
-  }
   a.seg_len = int(seg);
   a.nseg = int(nseg);
 
   if (nseg > 1) {
-    const int64_t rows_total = tiles * mssm::kRows;
+    const int64_t rows_total = tiles * rows_per_cta;
     const size_t count_bytes = ((size_t(tiles) * 4 + 255) / 256) * 256;
     const size_t s_bytes = ((size_t(nseg - 1) * rows_total * 4 + 255) / 256) * 256;
     const size_t h_bytes = size_t(nseg - 1) * rows_total * mssm::kN * 4;
@@ -289,11 +330,11 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* del
 
   if (nseg > 1) {
     e = tracked(MSSM_KERNEL_SCAN_CHUNK_STATE, s,
-                [&] { return mssm::launch_scan_chunk_state(a, dt, softplus_flag != 0, s); });
+                [&] { return mssm::launch_scan_chunk_state(a, rows_per_cta, dt, softplus_flag != 0, s); });
     if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel launch");
   }
   e = tracked(MSSM_KERNEL_SCAN_OUT, s,
-              [&] { return mssm::launch_scan_out(a, dt, z != nullptr, softplus_flag != 0, s); });
+              [&] { return mssm::launch_scan_out(a, rows_per_cta, dt, z != nullptr, softplus_flag != 0, s); });
   if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
   return MSSM_OK;
 }
@@ -330,7 +371,7 @@ static mssm_status state_update_impl(mssm_tensor* state, const mssm_tensor* x, c
   }
   if (same_ptr(out, state)) return fail(MSSM_ERR_INVALID_ARG, "out must not alias state");
   if (Bt == 0 || Dd == 0) return MSSM_OK;
-  if (Bt * Dd * 4 / 256 + 1 > int64_t(INT32_MAX)) return fail(MSSM_ERR_UNSUPPORTED, "too many rows for one launch");
+  if (Bt * Dd / 256 + 1 > int64_t(INT32_MAX)) return fail(MSSM_ERR_UNSUPPORTED, "too many rows for one launch");
 
   mssm::DecodeArgs a{};
   a.state = static_cast<float*>(state->data);
@@ -348,11 +389,17 @@ static mssm_status state_update_impl(mssm_tensor* state, const mssm_tensor* x, c
   a.Bt = int(Bt); a.D = int(Dd);
   a.softplus = softplus_flag != 0;
   a.vec_state = aligned16(state->data) && (state->stride[0] * 4) % 16 == 0 && (state->stride[1] * 4) % 16 == 0;
+  a.vec_A = aligned16(A->data) && A->stride[1] == 1 && (A->stride[0] * 4) % 16 == 0;
+  const int64_t es = int64_t(esize(dt));
+  a.vec_BC = aligned16(B->data) && aligned16(C->data) && B->stride[1] == 1 && C->stride[1] == 1 &&
+             (B->stride[0] * es) % 16 == 0 && (C->stride[0] * es) % 16 == 0;
 
+  // one contiguous [rows][16] state range, 16-byte aligned: the bulk-copy kernel
+  const bool bulk = aligned16(state->data) && state->stride[1] == mssm::kN && state->stride[0] == Dd * mssm::kN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lk(g_mu);
   cudaError_t e = tracked(MSSM_KERNEL_STATE_UPDATE, s,
-                          [&] { return mssm::launch_state_update(a, dt, z != nullptr, s); });
+                          [&] { return mssm::launch_state_update(a, dt, z != nullptr, bulk, s); });
   if (e != cudaSuccess) return cuda_fail(e, "state update launch");
   return MSSM_OK;
 }
@@ -369,6 +416,28 @@ mssm_status mssm_state_update_ex(mssm_tensor* state, const mssm_tensor* x, const
                                  const mssm_tensor* D, const mssm_tensor* z, const mssm_tensor* dt_bias,
                                  int softplus_flag, mssm_tensor* out, void* stream) {
   return state_update_impl(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, out, stream);
+}
+
+mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int* rows_per_cta,
+                           int64_t* chunk_len, int64_t* n_chunks) {
+  if (Bt < 0 || D < 0 || L < 0) return fail(MSSM_ERR_INVALID_ARG, "negative size");
+  if (sm_count <= 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    sm_count = v;
+  }
+  int64_t forced;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    forced = g_chunk_len;
+  }
+  const LaunchShape sh = choose_shape(Bt, D, L, sm_count, forced);
+  if (rows_per_cta) *rows_per_cta = sh.rows;
+  if (chunk_len) *chunk_len = sh.seg;
+  if (n_chunks) *n_chunks = sh.nseg;
+  return MSSM_OK;
 }
 
 mssm_status mssm_kernel_stats(int64_t launches[MSSM_KERNEL_KINDS], int64_t timed[MSSM_KERNEL_KINDS],
@@ -407,6 +476,12 @@ mssm_status mssm_get_error(void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "asynchronous kernel error");
+  unsigned int word = 0u;
+  e = mssm::read_device_error(&word, true);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (word & 1u)
+    return fail(MSSM_ERR_TIMEOUT, "a decode bulk copy did not complete within its bounded wait; "
+                "the state rows of that tile were left unchanged");
   return MSSM_OK;
 }
 

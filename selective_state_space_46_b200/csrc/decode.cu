@@ -1,19 +1,49 @@
-// Instantiation and launch of the decode state-update kernel.
+// Instantiation and launch of the decode state-update kernels; the device error word.
 #include "launch.h"
 
 namespace mssm {
 
+__device__ unsigned int g_device_error = 0u;
+
+// Address of this device's copy of the error word, looked up once per device
+// (the caller serialises launches, so the cache needs no lock of its own).
+static cudaError_t error_word(unsigned int** out) {
+  static void* cache[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!cache[dev]) {
+    e = cudaGetSymbolAddress(&cache[dev], g_device_error);
+    if (e != cudaSuccess) return e;
+  }
+  *out = static_cast<unsigned int*>(cache[dev]);
+  return cudaSuccess;
+}
+
 template <typename T, bool HAS_Z>
-static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
-  const int64_t threads = int64_t(a.Bt) * a.D * 4;
-  const int64_t blocks = (threads + kDecodeThreads - 1) / kDecodeThreads;
-  state_update_kernel<T, HAS_Z><<<unsigned(blocks), kDecodeThreads, 0, s>>>(a);
+static cudaError_t launch_decode_t(DecodeArgs a, bool bulk, cudaStream_t s) {
+  cudaError_t e = error_word(&a.err);
+  if (e != cudaSuccess) return e;
+  const int64_t rows = int64_t(a.Bt) * a.D;
+  const int64_t blocks = (rows + kDecodeThreads - 1) / kDecodeThreads;
+  if (bulk)
+    state_update_bulk_kernel<T, HAS_Z><<<unsigned(blocks), kDecodeThreads, 0, s>>>(a);
+  else
+    state_update_kernel<T, HAS_Z><<<unsigned(blocks), kDecodeThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, cudaStream_t s) {
-  if (dtype == 1) return has_z ? launch_decode_t<uint16_t, true>(a, s) : launch_decode_t<uint16_t, false>(a, s);
-  return has_z ? launch_decode_t<float, true>(a, s) : launch_decode_t<float, false>(a, s);
+cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, bool bulk, cudaStream_t s) {
+  if (dtype == 1) return has_z ? launch_decode_t<uint16_t, true>(a, bulk, s) : launch_decode_t<uint16_t, false>(a, bulk, s);
+  return has_z ? launch_decode_t<float, true>(a, bulk, s) : launch_decode_t<float, false>(a, bulk, s);
+}
+
+cudaError_t read_device_error(unsigned int* value, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(unsigned int));
+  if (e != cudaSuccess || !clear || *value == 0u) return e;
+  const unsigned int zero = 0u;
+  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
 }
 
 }  // namespace mssm

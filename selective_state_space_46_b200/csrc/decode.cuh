@@ -7,10 +7,18 @@
 // y = C . h + D x, times silu(z); h is read and written in place.
 //
 // The step moves 64 + 64 bytes of fp32 state per row against 16 exponentials,
-// so it is HBM-bound.  Four threads own one row, one 16-byte quarter of its
-// state each: a warp reads and writes eight rows' states as 512 contiguous
-// bytes, with one 128-bit load and one 128-bit store per thread.  The partial
-// readouts of the four quarters are summed with two butterfly shuffles.
+// so it is HBM-bound and the design goal is bytes in flight.
+//  * Contiguous state (the usual [Bt, D, 16] layout): a CTA owns 256 rows, whose
+//    16 KB of state is one contiguous range.  One thread issues a single bulk
+//    copy (cp.async.bulk, completion counted on an mbarrier) into shared memory,
+//    so every resident CTA keeps 16 KB in flight from one instruction, while
+//    all threads load their x/dt/z and A/B/C.  Each thread then updates its row
+//    in shared memory (the four 16-byte quarters are visited in a lane-rotated
+//    order, which makes the accesses bank-conflict free) and one thread writes
+//    the tile back with a bulk store.  The mbarrier wait is bounded: if it gives
+//    up, the CTA records an error in a device word (read by mssm_get_error),
+//    waits a bounded time more for its copy, and leaves its rows untouched.
+//  * Any other layout: one thread per row with 128-bit loads where aligned.
 #pragma once
 
 #include <cstdint>
@@ -20,7 +28,8 @@
 
 namespace mssm {
 
-constexpr int kDecodeThreads = 256;  // 64 rows per CTA
+constexpr int kDecodeThreads = 256;            // rows per CTA
+constexpr int kDecodeSpinLimit = 1 << 22;      // bounded mbarrier polls
 
 struct DecodeArgs {
   float* state;
@@ -42,6 +51,9 @@ struct DecodeArgs {
   int Bt, D;
   int softplus;
   int vec_state;  // every row's state starts 16-byte aligned
+  int vec_A;      // A rows 16-byte aligned with unit n stride
+  int vec_BC;     // B and C rows 16-byte aligned with unit n stride
+  unsigned int* err;  // device error word: bit 0 = a bulk copy did not complete in time
 };
 
 template <typename T>
@@ -49,65 +61,169 @@ __device__ __forceinline__ float ld_elem(const void* base, int64_t off) {
   return Elem<T>::load(static_cast<const T*>(base) + off);
 }
 
-template <typename T, bool HAS_Z>
-__global__ void __launch_bounds__(kDecodeThreads) state_update_kernel(const DecodeArgs p) {
-  const int64_t gid = int64_t(blockIdx.x) * kDecodeThreads + threadIdx.x;
-  const int64_t row = gid >> 2;
-  const int q = int(gid & 3);
-  const int64_t rows = int64_t(p.Bt) * p.D;
-  // Lanes past the last row compute on a clamped row and store nothing, so the
-  // whole warp stays converged for the shuffles below.
-  const bool live = row < rows;
-  const int64_t rr = live ? row : rows - 1;
-  const int b = int(rr / p.D);
-  const int d = int(rr - int64_t(b) * p.D);
-
-  float* st = p.state + int64_t(b) * p.st_sb + int64_t(d) * p.st_sd + 4 * q;
-  float4 h;
-  if (p.vec_state) {
-    h = __ldcs(reinterpret_cast<const float4*>(st));
-  } else {
-    h = make_float4(st[0], st[1], st[2], st[3]);
-  }
-  const float xv = ld_elem<T>(p.x, int64_t(b) * p.x_sb + int64_t(d) * p.x_sd);
-  float dt = ld_elem<T>(p.dt, int64_t(b) * p.dt_sb + int64_t(d) * p.dt_sd);
-  if (p.bias) dt += p.bias[int64_t(d) * p.bias_s];
-  if (p.softplus) dt = softplus_f(dt);
-  const float* Ar = p.A + int64_t(d) * p.A_sd + int64_t(4 * q) * p.A_sn;
-  const float a0 = Ar[0], a1 = Ar[p.A_sn], a2 = Ar[2 * p.A_sn], a3 = Ar[3 * p.A_sn];
-  const int64_t bo = int64_t(b) * p.B_sb + int64_t(4 * q) * p.B_sn;
-  const int64_t co = int64_t(b) * p.C_sb + int64_t(4 * q) * p.C_sn;
-  const float b0 = ld_elem<T>(p.B, bo), b1 = ld_elem<T>(p.B, bo + p.B_sn);
-  const float b2 = ld_elem<T>(p.B, bo + 2 * p.B_sn), b3 = ld_elem<T>(p.B, bo + 3 * p.B_sn);
-  const float c0 = ld_elem<T>(p.C, co), c1 = ld_elem<T>(p.C, co + p.C_sn);
-  const float c2 = ld_elem<T>(p.C, co + 2 * p.C_sn), c3 = ld_elem<T>(p.C, co + 3 * p.C_sn);
-
-  const float w = dt * xv;
-  const float dl2 = dt * kLog2e;
-  h.x = fmaf(ex2f(dl2 * a0), h.x, w * b0);
-  h.y = fmaf(ex2f(dl2 * a1), h.y, w * b1);
-  h.z = fmaf(ex2f(dl2 * a2), h.z, w * b2);
-  h.w = fmaf(ex2f(dl2 * a3), h.w, w * b3);
-  float y = fmaf(c0, h.x, fmaf(c1, h.y, fmaf(c2, h.z, c3 * h.w)));
-  y += __shfl_xor_sync(0xffffffffu, y, 1);
-  y += __shfl_xor_sync(0xffffffffu, y, 2);
-
-  if (!live) return;
-  if (p.vec_state) {
-    __stcs(reinterpret_cast<float4*>(st), h);
-  } else {
-    st[0] = h.x; st[1] = h.y; st[2] = h.z; st[3] = h.w;
-  }
-  if (q == 0) {
-    if (p.Dskip) y = fmaf(p.Dskip[int64_t(d) * p.D_s], xv, y);
-    if constexpr (HAS_Z) y *= silu_f(ld_elem<T>(p.z, int64_t(b) * p.z_sb + int64_t(d) * p.z_sd));
-    T* o = static_cast<T*>(p.out) + int64_t(b) * p.o_sb + int64_t(d) * p.o_sd;
+// 4 consecutive values (n stride 1, aligned) or strided scalars
+template <typename T>
+__device__ __forceinline__ float4 load4(const void* base, int64_t off, int64_t stride, bool vec) {
+  const T* p = static_cast<const T*>(base) + off;
+  if (vec) {
     if constexpr (sizeof(T) == 2) {
-      *o = f_to_bf16(y);
+      const uint2 w = __ldg(reinterpret_cast<const uint2*>(p));
+      return make_float4(bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y));
     } else {
-      *o = y;
+      return __ldg(reinterpret_cast<const float4*>(p));
     }
   }
+  return make_float4(Elem<T>::load(p), Elem<T>::load(p + stride), Elem<T>::load(p + 2 * stride),
+                     Elem<T>::load(p + 3 * stride));
+}
+
+// Per-row scalars of the update.
+struct DecodeRow {
+  int b, d;
+  float x, dt, w, dl2;
+};
+
+template <typename T>
+__device__ __forceinline__ DecodeRow decode_row_scalars(const DecodeArgs& p, int64_t row) {
+  DecodeRow r;
+  r.b = int(row / p.D);
+  r.d = int(row - int64_t(r.b) * p.D);
+  r.x = ld_elem<T>(p.x, int64_t(r.b) * p.x_sb + int64_t(r.d) * p.x_sd);
+  float dt = ld_elem<T>(p.dt, int64_t(r.b) * p.dt_sb + int64_t(r.d) * p.dt_sd);
+  if (p.bias) dt += p.bias[int64_t(r.d) * p.bias_s];
+  if (p.softplus) dt = softplus_f(dt);
+  r.dt = dt;
+  r.w = dt * r.x;
+  r.dl2 = dt * kLog2e;
+  return r;
+}
+
+// Update one 16-byte quarter q (states 4q..4q+3); returns the partial readout.
+template <typename T>
+__device__ __forceinline__ float decode_quarter(const DecodeArgs& p, const DecodeRow& r, int q, float4& h) {
+  const float4 a = load4<float>(p.A, int64_t(r.d) * p.A_sd + int64_t(4 * q) * p.A_sn, p.A_sn, p.vec_A != 0);
+  const float4 bv = load4<T>(p.B, int64_t(r.b) * p.B_sb + int64_t(4 * q) * p.B_sn, p.B_sn, p.vec_BC != 0);
+  const float4 cv = load4<T>(p.C, int64_t(r.b) * p.C_sb + int64_t(4 * q) * p.C_sn, p.C_sn, p.vec_BC != 0);
+  h.x = fmaf(ex2f(r.dl2 * a.x), h.x, r.w * bv.x);
+  h.y = fmaf(ex2f(r.dl2 * a.y), h.y, r.w * bv.y);
+  h.z = fmaf(ex2f(r.dl2 * a.z), h.z, r.w * bv.z);
+  h.w = fmaf(ex2f(r.dl2 * a.w), h.w, r.w * bv.w);
+  return fmaf(cv.x, h.x, fmaf(cv.y, h.y, fmaf(cv.z, h.z, cv.w * h.w)));
+}
+
+template <typename T, bool HAS_Z>
+__device__ __forceinline__ void decode_finish(const DecodeArgs& p, const DecodeRow& r, float y) {
+  if (p.Dskip) y = fmaf(p.Dskip[int64_t(r.d) * p.D_s], r.x, y);
+  if constexpr (HAS_Z) y *= gate_f<T>(ld_elem<T>(p.z, int64_t(r.b) * p.z_sb + int64_t(r.d) * p.z_sd));
+  T* o = static_cast<T*>(p.out) + int64_t(r.b) * p.o_sb + int64_t(r.d) * p.o_sd;
+  if constexpr (sizeof(T) == 2) {
+    *o = f_to_bf16(y);
+  } else {
+    *o = y;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// contiguous state: bulk copy in, update in shared memory, bulk copy out
+// ---------------------------------------------------------------------------
+template <typename T, bool HAS_Z>
+__global__ void __launch_bounds__(kDecodeThreads) state_update_bulk_kernel(const DecodeArgs p) {
+  __shared__ __align__(128) float st_s[kDecodeThreads * kN];
+  __shared__ __align__(8) unsigned long long mbar;
+  const int tid = threadIdx.x;
+  const int64_t rows = int64_t(p.Bt) * p.D;
+  const int64_t r0 = int64_t(blockIdx.x) * kDecodeThreads;
+  const int nrows = int(rows - r0 < kDecodeThreads ? rows - r0 : kDecodeThreads);
+  const uint32_t bytes = uint32_t(nrows) * kN * 4;
+  float* gtile = p.state + r0 * kN;  // contiguous layout: row r starts at r * 16
+  const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(st_s));
+  const uint32_t mb = static_cast<uint32_t>(__cvta_generic_to_shared(&mbar));
+
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mb) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (tid == 0) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(sbase), "l"(gtile), "r"(bytes), "r"(mb) : "memory");
+  }
+
+  const bool live = tid < nrows;
+  DecodeRow r{};
+  if (live) r = decode_row_scalars<T>(p, r0 + tid);
+
+  uint32_t done = 0;
+  for (int it = 0; it < kDecodeSpinLimit && !done; ++it) {
+    asm volatile("{\n .reg .pred pr;\n mbarrier.try_wait.parity.shared::cta.b64 pr, [%1], 0;\n selp.u32 %0, 1, 0, pr;\n}"
+                 : "=r"(done) : "r"(mb) : "memory");
+  }
+  if (!__syncthreads_and(done)) {
+    // give up: record the error, give the copy a bounded time more, leave the rows untouched
+    if (tid == 0) atomicOr(p.err, 1u);
+    for (int it = 0; it < kDecodeSpinLimit && !done; ++it) {
+      asm volatile("{\n .reg .pred pr;\n mbarrier.try_wait.parity.shared::cta.b64 pr, [%1], 0;\n selp.u32 %0, 1, 0, pr;\n}"
+                   : "=r"(done) : "r"(mb) : "memory");
+    }
+    return;
+  }
+
+  if (live) {
+    float4* hs = reinterpret_cast<float4*>(st_s + tid * kN);
+    float y = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int q = (k + (tid >> 1)) & 3;  // lane-rotated quarter order: conflict-free
+      float4 h = hs[q];
+      y += decode_quarter<T>(p, r, q, h);
+      hs[q] = h;
+    }
+    decode_finish<T, HAS_Z>(p, r, y);
+  }
+  // make the generic-proxy shared-memory writes visible to the bulk copy, then store
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncthreads();
+  if (tid == 0) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gtile), "r"(sbase), "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// any layout: one thread per row
+// ---------------------------------------------------------------------------
+template <typename T, bool HAS_Z>
+__global__ void __launch_bounds__(kDecodeThreads) state_update_kernel(const DecodeArgs p) {
+  const int64_t row = int64_t(blockIdx.x) * kDecodeThreads + threadIdx.x;
+  const int64_t rows = int64_t(p.Bt) * p.D;
+  if (row >= rows) return;
+  const int b = int(row / p.D);
+  const int d = int(row - int64_t(b) * p.D);
+  float* st = p.state + int64_t(b) * p.st_sb + int64_t(d) * p.st_sd;
+  float4 h[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (p.vec_state) {
+      h[q] = __ldcs(reinterpret_cast<const float4*>(st) + q);
+    } else {
+      h[q] = make_float4(st[4 * q], st[4 * q + 1], st[4 * q + 2], st[4 * q + 3]);
+    }
+  }
+  const DecodeRow r = decode_row_scalars<T>(p, row);
+  float y = 0.0f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    y += decode_quarter<T>(p, r, q, h[q]);
+    if (p.vec_state) {
+      __stcs(reinterpret_cast<float4*>(st) + q, h[q]);
+    } else {
+      st[4 * q] = h[q].x; st[4 * q + 1] = h[q].y; st[4 * q + 2] = h[q].z; st[4 * q + 3] = h[q].w;
+    }
+  }
+  decode_finish<T, HAS_Z>(p, r, y);
 }
 
 }  // namespace mssm

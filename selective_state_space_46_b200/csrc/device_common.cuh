@@ -52,6 +52,26 @@ __device__ __forceinline__ float silu_f(float z) {
   return z * rcpf(1.0f + ex2f(-z * kLog2e));
 }
 
+// silu(z) = (z/2)(1 + tanh(z/2)) with the SFU tanh (relative error about 2^-11).
+// The result's error is at most |z| 2^-12 relative to |silu(z)|'s scale, below
+// the rounding of a bf16 output for |z| < 8; used only where the output is bf16.
+__device__ __forceinline__ float silu_tanh(float z) {
+  const float hz = 0.5f * z;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hz));
+  return fmaf(hz, t, hz);
+}
+
+// the gate used for an output stored as T: exact for fp32, SFU tanh for bf16
+template <typename T>
+__device__ __forceinline__ float gate_f(float z) {
+  if constexpr (sizeof(T) == 2) {
+    return silu_tanh(z);
+  } else {
+    return silu_f(z);
+  }
+}
+
 // ---------------------------------------------------------------- bf16 storage
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }

@@ -9,8 +9,12 @@
 namespace mssm {
 
 // dtype: 0 = fp32 storage, 1 = bf16 storage.  Return the launch error, if any.
-cudaError_t launch_scan_chunk_state(const ScanArgs& a, int dtype, bool softplus, cudaStream_t s);
-cudaError_t launch_scan_out(const ScanArgs& a, int dtype, bool has_z, bool softplus, cudaStream_t s);
-cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, cudaStream_t s);
+// rows: channels per CTA (32 or 64); the grid is (Bt * tiles_per_batch, nseg [- 1]).
+cudaError_t launch_scan_chunk_state(const ScanArgs& a, int rows, int dtype, bool softplus, cudaStream_t s);
+cudaError_t launch_scan_out(const ScanArgs& a, int rows, int dtype, bool has_z, bool softplus, cudaStream_t s);
+// bulk: the state is one contiguous [rows][16] range (bulk-copy kernel), else one thread per row.
+cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, bool bulk, cudaStream_t s);
+// Reads (and optionally clears) the current device's error word.
+cudaError_t read_device_error(unsigned int* value, bool clear);
 
 }  // namespace mssm

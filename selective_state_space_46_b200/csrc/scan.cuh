@@ -1,4 +1,4 @@
-// Selective scan forward kernels and their launcher (sm_100a).
+// Selective scan forward kernels (sm_100a).
 //
 // The scan is the Mamba-1 selective state space recurrence: per row (b, d) and
 // state n, h_t = exp(delta_t A_dn) h_(t-1) + delta_t B_tn u_t, y_t = C_t . h_t +
@@ -8,26 +8,32 @@
 // delta = softplus(parameter + linear)).
 //
 // Work decomposition
-//  * One thread owns one row (b, d) and keeps its 16-wide state in registers
-//    as eight packed fp32 pairs; rows of one CTA are 64 consecutive channels
-//    of the same batch, so the CTA stages B and C of that batch once per
-//    32-step chunk in shared memory (converted to fp32, laid out [t][B0..15,
-//    C0..15]) and every row reads them as warp-wide broadcasts.
-//  * u / delta / z are streamed per row along L with 16-byte vector loads and
-//    one 16-step block of prefetch; y is written with 16-byte vector stores.
+//  * One thread owns one row (b, d) and keeps its 16-wide state in registers as
+//    eight packed fp32 pairs (fma.rn.f32x2).  A CTA is ROWS (32 or 64)
+//    consecutive channels of one batch; it stages that batch's B and C once per
+//    32-step chunk in shared memory (fp32, [t][B0..15, C0..15]) and every row
+//    reads them as warp-wide broadcasts.
+//  * u / delta_raw / z are streamed per row in 16-byte blocks (8 bf16 or 4 fp32
+//    steps) by cp.async into a per-thread shared-memory slot ring four blocks
+//    deep; each thread reads only its own slots, so the stream needs no barrier
+//    and holds no registers while in flight.  y leaves as one 16-byte store per
+//    block.
+//  * Arithmetic runs in base 2: s = delta / ln 2 comes straight out of the
+//    softplus (bias folded into one FMA), exp(delta A) = 2^(s A), and the ln 2
+//    that s lacks is folded into B when B is staged, so delta*B*u = s*u*(ln2 B).
 //  * Long sequences are split into chunks of seg_len steps.  The per-position
 //    affine maps (A_bar_t, B_bar_t u_t) compose associatively ("Mamba selective
 //    state space", section "Selectivity Removes the Convolution Shortcut; Scan
-//    Restores Parallelism"), so a chunk is summarised by (S, H): S = sum of
-//    delta over the chunk (the chunk's decay is exp(A_n S)) and H = the chunk's
-//    end state from a zero start.  Kernel 1 computes (S, H) for every chunk but
-//    the last with a backward sweep (2 flops per state and step instead of 3),
-//    and the last CTA of a row tile to finish folds the summaries into carried
-//    states (no CTA ever waits on another).  Kernel 2 re-runs every chunk
-//    forward from its carried state and writes y and the final state.
+//    Restores Parallelism"), so a chunk is summarised by (S, H): S = sum of s
+//    over the chunk (its decay is 2^(A_n S)) and H = its end state from zero.
+//    Kernel 1 computes (S, H) for every chunk but the last with a backward sweep
+//    (H_n = sum_t s_t u_t ln2 B_tn 2^(A_n sum_{r>t} s_r): two FP32 operations per
+//    state and step), and the last CTA of a row tile to finish folds the
+//    summaries into carried states; no CTA ever waits on another.  Kernel 2 runs
+//    every chunk forward from its carried state and writes y and the final state.
 //  * Structured A (A_dn == (n+1) A_d0 exactly, the S4D-real initialisation the
-//    pages use) computes exp(delta A_dn) as powers of one exponential; any
-//    other A takes one SFU exponential per state.  The choice is uniform per CTA.
+//    pages use) computes 2^(s A_dn) as powers of one exponential; any other A
+//    takes one SFU exponential per state.  The choice is uniform per CTA.
 #pragma once
 
 #include <cstdint>
@@ -37,9 +43,9 @@
 
 namespace mssm {
 
-constexpr int kRows = 64;   // rows (threads) per CTA
-constexpr int kTC = 32;     // steps per staged B/C chunk
-constexpr int kSegQuant = 64;  // chunk lengths of the length split are multiples of this
+constexpr int kTC = 32;         // steps per staged B/C chunk
+constexpr int kSegQuant = 64;   // chunk lengths of the length split are multiples of this
+constexpr int kStages = 4;      // depth of the per-thread cp.async ring (16-byte blocks)
 
 struct ScanArgs {
   const void* u;
@@ -61,97 +67,77 @@ struct ScanArgs {
   int Bt, D, L;
   int force_general;
   int nseg, seg_len;
-  int tiles_per_batch;
-  int vec_rows;  // u/delta/z/out row starts are 16-byte aligned
-  int vec_bc;    // B/C row starts are 16-byte aligned
-  // carry workspace, used when nseg > 1
-  float* ws_H;          // [nseg-1][ntiles*kRows][16]: chunk end state, then carried state
-  float* ws_S;          // [nseg-1][ntiles*kRows]: sum of delta over the chunk
-  unsigned* ws_count;   // [ntiles]: arrivals of kernel-1 CTAs, reset by the last one
+  int tiles_per_batch;   // ceil(D / ROWS)
+  int vec_rows;          // u/delta/z/out row starts are 16-byte aligned
+  int vec_bc;            // B/C row starts are 16-byte aligned
+  int vec_ls;            // last_state rows are 16-byte aligned
+  // carry workspace, used when nseg > 1 (rows_total = Bt * tiles_per_batch * ROWS)
+  float* ws_H;           // [nseg-1][rows_total][16]: chunk end state, then carried state
+  float* ws_S;           // [nseg-1][rows_total]: sum of delta / ln2 over the chunk
+  unsigned* ws_count;    // [Bt * tiles_per_batch]: kernel-1 arrivals, reset by the last one
 };
 
 // ---------------------------------------------------------------------------
-// per-row 16-step (bf16) / 8-step (fp32) blocks of u, delta, z: 32 bytes each
+// small device helpers
 // ---------------------------------------------------------------------------
-template <typename T> struct Blk {
-  static constexpr int kSteps = 32 / int(sizeof(T));
-  uint32_t w[8];
-  __device__ __forceinline__ float at(int j) const {
-    if constexpr (sizeof(T) == 2) {
-      return (j & 1) ? bf16hi(w[j >> 1]) : bf16lo(w[j >> 1]);
-    } else {
-      return __uint_as_float(w[j]);
-    }
-  }
-  __device__ __forceinline__ void zero() {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = 0u;
-  }
-  // Load steps [t, t + kSteps) of a row; steps at or past t_end read as 0.
-  __device__ __forceinline__ void load(const T* row, int t, int t_end, bool vec) {
-    if (vec && t + kSteps <= t_end) {
-      const uint4* p = reinterpret_cast<const uint4*>(row + t);
-      const uint4 a = __ldg(p), b = __ldg(p + 1);
-      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-      w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-    } else {
-      if constexpr (sizeof(T) == 2) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t lo = (t + 2 * i < t_end) ? uint32_t(__ldg(row + t + 2 * i)) : 0u;
-          const uint32_t hi = (t + 2 * i + 1 < t_end) ? uint32_t(__ldg(row + t + 2 * i + 1)) : 0u;
-          w[i] = lo | (hi << 16);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          w[i] = (t + i < t_end) ? __float_as_uint(__ldg(row + t + i)) : 0u;
-      }
-    }
-  }
-};
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
 
-// Store steps [t, t + kSteps) of y (fp32 values), clipped at t_end.
+// bf16 halves of a 32-bit word widened to fp32 with a byte permute (ALU pipe)
+__device__ __forceinline__ float bf_lo(uint32_t w) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, 0x1044;" : "=r"(r) : "r"(w));
+  return __uint_as_float(r);
+}
+__device__ __forceinline__ float bf_hi(uint32_t w) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, 0x3244;" : "=r"(r) : "r"(w));
+  return __uint_as_float(r);
+}
+
+// element j of a 16-byte block
 template <typename T>
-__device__ __forceinline__ void store_block(T* row, int t, int t_end, bool vec, const float* y) {
-  constexpr int S = Blk<T>::kSteps;
+__device__ __forceinline__ float blk_at(const uint4& v, int j) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   if constexpr (sizeof(T) == 2) {
-    uint32_t w[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
-    if (vec && t + S <= t_end) {
-      uint4* p = reinterpret_cast<uint4*>(row + t);
-      p[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      p[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (t + 2 * i < t_end) row[t + 2 * i] = uint16_t(w[i] & 0xffffu);
-        if (t + 2 * i + 1 < t_end) row[t + 2 * i + 1] = uint16_t(w[i] >> 16);
-      }
-    }
+    return (j & 1) ? bf_hi(w[j >> 1]) : bf_lo(w[j >> 1]);
   } else {
-    if (vec && t + S <= t_end) {
-      float4* p = reinterpret_cast<float4*>(row + t);
-      p[0] = make_float4(y[0], y[1], y[2], y[3]);
-      p[1] = make_float4(y[4], y[5], y[6], y[7]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (t + i < t_end) row[t + i] = y[i];
-    }
+    return __uint_as_float(w[j]);
   }
 }
 
+// softplus in base 2: returns softplus(v) / ln2 given v2 = v * log2(e).
+//  * v > 20: v (remainder below 2.1e-9, PyTorch's softplus threshold).
+//  * e = e^v < 2^-6: the series e - e^2/2 + e^3/3 (scaled by log2 e), whose
+//    truncation error is below e^4/4 (relative < 2^-20); avoids forming 1 + e.
+//  * otherwise log2(1 + e), within the SFU's 2^-22 absolute error of a result
+//    >= log2(1 + 2^-6), i.e. < 2e-5 relative.
+__device__ __forceinline__ float softplus2(float v2) {
+  const float e = ex2f(v2);
+  const float big = lg2f(1.0f + e);
+  const float small = e * fmaf(e, fmaf(e, 0.48089834696298783f, -0.72134752044448170f), 1.4426950408889634f);
+  const float r = (e < 0.015625f) ? small : big;
+  return (v2 > 28.853900817779268f) ? v2 : r;
+}
+
 // ---------------------------------------------------------------------------
-// B/C staging: a kTC-step chunk of NR rows (B rows 0..15 then C rows 0..15)
-// loaded by the CTA's 64 threads into registers, then written transposed to
-// shared memory as fp32 [t][row].
+// B/C staging: a kTC-step chunk of B rows 0..15 and C rows 0..15 loaded by the
+// CTA's ROWS threads into registers, then written transposed to shared memory
+// as fp32 [t][32] with B pre-multiplied by ln 2.
 // ---------------------------------------------------------------------------
-template <typename T, int NR> struct BCStage {
-  static constexpr int kVals = NR * kTC / kRows;     // values per thread (16 or 8)
+template <typename T, int ROWS> struct BCStage {
+  static constexpr int kVals = 32 * kTC / ROWS;        // values per thread: 16 or 32
   static constexpr int kWords = kVals * int(sizeof(T)) / 4;
-  static constexpr int kThreadsPerRow = kTC / kVals;  // 2 or 4
+  static constexpr int kThreadsPerRow = kTC / kVals;   // 2 or 1
   uint32_t w[kWords];
 
   __device__ __forceinline__ void load(const ScanArgs& p, int b, int cs, int t_end) {
@@ -183,51 +169,109 @@ template <typename T, int NR> struct BCStage {
     }
   }
 
-  __device__ __forceinline__ void store(float* s) const {  // s: [kTC][32] floats
+  __device__ __forceinline__ void store(float* s) const {  // s: [kTC][32]
     const int tid = threadIdx.x;
     const int r = tid / kThreadsPerRow;
     const int t = (tid % kThreadsPerRow) * kVals;
+    const float scale = (r < 16) ? kLn2 : 1.0f;
 #pragma unroll
     for (int j = 0; j < kVals; ++j) {
       float v;
       if constexpr (sizeof(T) == 2) {
-        v = (j & 1) ? bf16hi(w[j >> 1]) : bf16lo(w[j >> 1]);
+        v = (j & 1) ? bf_hi(w[j >> 1]) : bf_lo(w[j >> 1]);
       } else {
         v = __uint_as_float(w[j]);
       }
-      s[(t + j) * 32 + r] = v;
+      s[(t + j) * 32 + r] = v * scale;
     }
   }
 };
 
-// ---------------------------------------------------------------------------
-// exp(delta * A_dn) for the row's 16 states, as 8 packed pairs
-// ---------------------------------------------------------------------------
-template <bool STRUCT>
-__device__ __forceinline__ void decay_pairs(float dt, float a2_0, const f2_t (&A2p)[8], f2_t (&dA)[8]) {
-  if constexpr (STRUCT) {
-    // exp(dt (n+1) A_0) = a^(n+1), a = exp(dt A_0): one SFU op, 15 multiplies, depth 4
-    const float a = ex2f(dt * a2_0);
-    const float a2 = a * a;
-    dA[0] = f2(a, a2);
-    const f2_t s2 = f2(a2, a2);
-    dA[1] = mul2(dA[0], s2);
-    const float a4 = f2hi(dA[1]);
-    const f2_t s4 = f2(a4, a4);
-    dA[2] = mul2(dA[0], s4);
-    dA[3] = mul2(dA[1], s4);
-    const float a8 = f2hi(dA[3]);
-    const f2_t s8 = f2(a8, a8);
-    dA[4] = mul2(dA[0], s8);
-    dA[5] = mul2(dA[1], s8);
-    dA[6] = mul2(dA[2], s8);
-    dA[7] = mul2(dA[3], s8);
+// Fetch the 16-byte block of a row starting at step t into a shared slot:
+// cp.async when aligned and complete, else synchronous element loads (zero past t_end).
+template <typename T>
+__device__ __forceinline__ void fetch_block(uint4* slot, const T* row, int t, int t_end, bool vec) {
+  constexpr int S = 16 / int(sizeof(T));
+  if (vec && t + S <= t_end) {
+    cp_async16(smem_u32(slot), row + t);
   } else {
-    const f2_t d2 = f2(dt, dt);
+    uint32_t w[4];
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = (t + 2 * i < t_end) ? uint32_t(__ldg(row + t + 2 * i)) : 0u;
+        const uint32_t hi = (t + 2 * i + 1 < t_end) ? uint32_t(__ldg(row + t + 2 * i + 1)) : 0u;
+        w[i] = lo | (hi << 16);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w[i] = (t + i < t_end) ? __float_as_uint(__ldg(row + t + i)) : 0u;
+    }
+    *slot = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Store a block of y (S steps of fp32 values) at step t, clipped at t_end.
+template <typename T>
+__device__ __forceinline__ void store_block(T* row, int t, int t_end, bool vec, const float* y) {
+  constexpr int S = 16 / int(sizeof(T));
+  if constexpr (sizeof(T) == 2) {
+    const uint32_t w0 = pack_bf16x2(y[0], y[1]), w1 = pack_bf16x2(y[2], y[3]);
+    const uint32_t w2 = pack_bf16x2(y[4], y[5]), w3 = pack_bf16x2(y[6], y[7]);
+    if (vec && t + S <= t_end) {
+      *reinterpret_cast<uint4*>(row + t) = make_uint4(w0, w1, w2, w3);
+    } else {
+      const uint32_t w[4] = {w0, w1, w2, w3};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (t + 2 * i < t_end) row[t + 2 * i] = uint16_t(w[i] & 0xffffu);
+        if (t + 2 * i + 1 < t_end) row[t + 2 * i + 1] = uint16_t(w[i] >> 16);
+      }
+    }
+  } else {
+    if (vec && t + S <= t_end) {
+      *reinterpret_cast<float4*>(row + t) = make_float4(y[0], y[1], y[2], y[3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (t + i < t_end) row[t + i] = y[i];
+    }
+  }
+}
+
+// Powers a^1 .. a^16 as eight pairs (a^(2k+1), a^(2k+2)); 15 multiplies, depth 4.
+__device__ __forceinline__ void powers16(float a, f2_t (&dA)[8]) {
+  const float a2 = a * a;
+  const float a3 = a2 * a, a4 = a2 * a2;
+  const float a5 = a4 * a, a6 = a4 * a2, a7 = a4 * a3, a8 = a4 * a4;
+  dA[0] = f2(a, a2);
+  dA[1] = f2(a3, a4);
+  dA[2] = f2(a5, a6);
+  dA[3] = f2(a7, a8);
+  dA[4] = f2(a8 * a, a8 * a2);
+  dA[5] = f2(a8 * a3, a8 * a4);
+  dA[6] = f2(a8 * a5, a8 * a6);
+  dA[7] = f2(a8 * a7, a8 * a8);
+}
+
+// Per-row constants of the scan.
+struct RowParams {
+  float bias2;   // bias * log2(e)
+  float Dd;      // skip weight
+  float A0;      // A[d, 0]
+  f2_t Ap[8];    // A[d, n] pairs (general path)
+};
+
+template <bool STRUCT>
+__device__ __forceinline__ void decay(float s, const RowParams& rp, f2_t (&dA)[8]) {
+  if constexpr (STRUCT) {
+    powers16(ex2f(s * rp.A0), dA);
+  } else {
+    const f2_t s2 = f2(s, s);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       float lo, hi;
-      f2split(mul2(d2, A2p[k]), lo, hi);
+      f2split(mul2(s2, rp.Ap[k]), lo, hi);
       dA[k] = f2(ex2f(lo), ex2f(hi));
     }
   }
@@ -235,114 +279,187 @@ __device__ __forceinline__ void decay_pairs(float dt, float a2_0, const f2_t (&A
 
 // ---------------------------------------------------------------------------
 // Kernel 2: forward sweep of one chunk from its carried state, fused epilogue.
+//
+// Software-pipelined over 16-byte blocks of S steps: while block k runs its
+// recurrence (FMA pipe), block k+1's per-step scalars (softplus, decay base,
+// s*u: SFU-heavy) are computed in the same loop body, so the two overlap.
 // ---------------------------------------------------------------------------
-// One block of S steps.  PARTIAL: the block runs past t1; the steps past the
-// end become identity steps (delta = 0 gives A_bar = 1 and no input), so the
-// state is exactly the state at t1 - 1.
-template <typename T, bool HAS_Z, bool SOFTPLUS, bool STRUCT, bool PARTIAL>
-__device__ __forceinline__ void forward_block(const float* bcrow, int valid, const Blk<T>& cu,
-                                              const Blk<T>& cd, const Blk<T>& cz, float bias,
-                                              float Dd, float a2_0, const f2_t (&A2p)[8],
-                                              f2_t (&h2)[8], float* ybuf) {
-  constexpr int S = Blk<T>::kSteps;
+
+// Per-step scalars of one block: x = decay base 2^(s A_0) (structured A) or s
+// (general A), w = s * u.  PARTIAL: steps at or past `valid` become identity
+// steps (s = 0: A_bar = 1 and no input).
+template <typename T, bool SOFTPLUS, bool STRUCT, bool PARTIAL>
+__device__ __forceinline__ void block_scalars(const uint4& ru, const uint4& rd, int valid, const RowParams& rp,
+                                              float* x, float* w) {
+  constexpr int S = 16 / int(sizeof(T));
 #pragma unroll
   for (int j = 0; j < S; ++j) {
-    float uu = cu.at(j);
-    float dt = cd.at(j) + bias;
-    if constexpr (SOFTPLUS) dt = softplus_f(dt);
+    const float v2 = fmaf(blk_at<T>(rd, j), kLog2e, rp.bias2);
+    float s = SOFTPLUS ? softplus2(v2) : v2;
+    float uu = blk_at<T>(ru, j);
     if constexpr (PARTIAL) {
-      if (j >= valid) {
-        dt = 0.0f;
-        uu = 0.0f;
-      }
+      s = (j < valid) ? s : 0.0f;
+      uu = (j < valid) ? uu : 0.0f;
     }
-    f2_t dA[8];
-    decay_pairs<STRUCT>(dt, a2_0, A2p, dA);
-    const float w = dt * uu;
-    const f2_t w2 = f2(w, w);
-    const ulonglong2* q = reinterpret_cast<const ulonglong2*>(bcrow + j * 32);
-    f2_t yA = 0ull, yB = 0ull;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const ulonglong2 bb = q[k];      // B pairs (2k, 2k+1) of states 4k..4k+3
-      const ulonglong2 cc = q[4 + k];  // C pairs
-      h2[2 * k] = fma2(dA[2 * k], h2[2 * k], mul2(w2, bb.x));
-      h2[2 * k + 1] = fma2(dA[2 * k + 1], h2[2 * k + 1], mul2(w2, bb.y));
-      yA = (k == 0) ? mul2(cc.x, h2[0]) : fma2(cc.x, h2[2 * k], yA);
-      yB = (k == 0) ? mul2(cc.y, h2[1]) : fma2(cc.y, h2[2 * k + 1], yB);
-    }
-    float y0, y1, y2, y3;
-    f2split(yA, y0, y1);
-    f2split(yB, y2, y3);
-    float y = ((y0 + y1) + (y2 + y3)) + Dd * uu;
-    if constexpr (HAS_Z) y *= silu_f(cz.at(j));
-    ybuf[j] = y;
+    x[j] = STRUCT ? ex2f(s * rp.A0) : s;
+    w[j] = s * uu;
   }
 }
 
-template <typename T, bool HAS_Z, bool SOFTPLUS, bool STRUCT>
-__device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[kTC * 32], int b,
-                                              int t0, int t1, const T* urow, const T* dlrow,
-                                              const T* zrow, T* orow, bool row_ok, float bias,
-                                              float Dd, float a2_0, const f2_t (&A2p)[8],
+// Recurrence and readout of one block; yout[j] = C_t . h_t (before skip and gate).
+template <typename T, bool STRUCT>
+__device__ __forceinline__ void block_recurrence(const float* bcrow, const float* x, const float* w,
+                                                 const RowParams& rp, f2_t (&h2)[8], float* yout) {
+  constexpr int S = 16 / int(sizeof(T));
+#pragma unroll
+  for (int j = 0; j < S; ++j) {
+    f2_t dA[8];
+    if constexpr (STRUCT) {
+      powers16(x[j], dA);
+    } else {
+      const f2_t s2 = f2(x[j], x[j]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        float lo, hi;
+        f2split(mul2(s2, rp.Ap[k]), lo, hi);
+        dA[k] = f2(ex2f(lo), ex2f(hi));
+      }
+    }
+    const f2_t w2 = f2(w[j], w[j]);
+    const ulonglong2* q = reinterpret_cast<const ulonglong2*>(bcrow + j * 32);
+    f2_t ya = 0ull;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const ulonglong2 bb = q[k];      // ln2 * B, pairs (4k, 4k+1), (4k+2, 4k+3)
+      const ulonglong2 cc = q[4 + k];  // C pairs
+      h2[2 * k] = fma2(dA[2 * k], h2[2 * k], mul2(w2, bb.x));
+      h2[2 * k + 1] = fma2(dA[2 * k + 1], h2[2 * k + 1], mul2(w2, bb.y));
+      ya = (k == 0) ? mul2(cc.x, h2[0]) : fma2(cc.x, h2[2 * k], ya);
+      ya = fma2(cc.y, h2[2 * k + 1], ya);
+    }
+    float a0, a1;
+    f2split(ya, a0, a1);
+    yout[j] = a0 + a1;
+  }
+}
+
+template <typename T, int ROWS, bool HAS_Z, bool SOFTPLUS, bool STRUCT>
+__device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[kTC * 32], uint4* slots,
+                                              int b, int t0, int t1, const T* urow, const T* dlrow,
+                                              const T* zrow, T* orow, bool row_ok, const RowParams& rp,
                                               f2_t (&h2)[8]) {
-  constexpr int S = Blk<T>::kSteps;
+  constexpr int S = 16 / int(sizeof(T));
+  constexpr int kBlkPerChunk = kTC / S;
+  const int tid = threadIdx.x;
   const bool vec = p.vec_rows != 0;
-  BCStage<T, 32> stage;
+  const int nblk = (t1 - t0 + S - 1) / S;
   const int nchunks = (t1 - t0 + kTC - 1) / kTC;
   if (nchunks <= 0) return;
+
+  auto slot = [&](int stage, int tensor) { return slots + (stage * 3 + tensor) * ROWS + tid; };
+  auto issue = [&](int k) {
+    const int t = t0 + k * S;
+    const int st = k % kStages;
+    fetch_block<T>(slot(st, 0), urow, t, t1, vec);
+    fetch_block<T>(slot(st, 1), dlrow, t, t1, vec);
+    if constexpr (HAS_Z) fetch_block<T>(slot(st, 2), zrow, t, t1, vec);
+  };
+  auto scalars = [&](int k, const uint4& ru, const uint4& rd, float* x, float* w) {
+    const int valid = t1 - (t0 + k * S);
+    if (valid >= S)
+      block_scalars<T, SOFTPLUS, STRUCT, false>(ru, rd, S, rp, x, w);
+    else
+      block_scalars<T, SOFTPLUS, STRUCT, true>(ru, rd, valid, rp, x, w);
+  };
+#pragma unroll
+  for (int k = 0; k < kStages - 1; ++k) {
+    if (k < nblk) issue(k);
+    cp_commit();
+  }
+
+  BCStage<T, ROWS> stage;
   stage.load(p, b, t0, t1);
   stage.store(bc_s[0]);
+
+  // block 0's scalars
+  cp_wait<kStages - 2>();
+  uint4 ru = *slot(0, 0);
+  uint4 rz = HAS_Z ? *slot(0, 2) : make_uint4(0u, 0u, 0u, 0u);
+  float xc[S], wc[S];
+  scalars(0, ru, *slot(0, 1), xc, wc);
   __syncthreads();
 
-  Blk<T> cu, cd, cz;
-  cu.load(urow, t0, t1, vec);
-  cd.load(dlrow, t0, t1, vec);
-  if constexpr (HAS_Z) cz.load(zrow, t0, t1, vec);
-  else cz.zero();
-
+  int k = 0;
   for (int c = 0; c < nchunks; ++c) {
     const int cs = t0 + c * kTC;
-    const int ce = min(t1, cs + kTC);
     if (c + 1 < nchunks) stage.load(p, b, cs + kTC, t1);
     const float* bcb = bc_s[c & 1];
-    for (int tb = cs; tb < ce; tb += S) {
-      Blk<T> nu, nd, nz;
-      const int tn = tb + S;
-      if (tn < t1) {
-        nu.load(urow, tn, t1, vec);
-        nd.load(dlrow, tn, t1, vec);
-        if constexpr (HAS_Z) nz.load(zrow, tn, t1, vec);
-        else nz.zero();
-      } else {
-        nu.zero();
-        nd.zero();
-        nz.zero();
+#pragma unroll 1
+    for (int kb = 0; kb < kBlkPerChunk && k < nblk; ++kb, ++k) {
+      // next block: fetch further ahead, then its scalars (independent of this block's recurrence)
+      if (k + kStages - 1 < nblk) issue(k + kStages - 1);
+      cp_commit();
+      float xn[S], wn[S];
+      uint4 run = make_uint4(0u, 0u, 0u, 0u), rzn = make_uint4(0u, 0u, 0u, 0u);
+      if (k + 1 < nblk) {
+        cp_wait<kStages - 2>();
+        const int st = (k + 1) % kStages;
+        run = *slot(st, 0);
+        if constexpr (HAS_Z) rzn = *slot(st, 2);
+        scalars(k + 1, run, *slot(st, 1), xn, wn);
       }
-      float ybuf[S];
-      const float* bcrow = bcb + (tb - cs) * 32;
-      if (tb + S <= t1)
-        forward_block<T, HAS_Z, SOFTPLUS, STRUCT, false>(bcrow, S, cu, cd, cz, bias, Dd, a2_0, A2p, h2, ybuf);
-      else
-        forward_block<T, HAS_Z, SOFTPLUS, STRUCT, true>(bcrow, t1 - tb, cu, cd, cz, bias, Dd, a2_0, A2p, h2, ybuf);
-      if (row_ok) store_block<T>(orow, tb, t1, vec, ybuf);
-      cu = nu;
-      cd = nd;
-      cz = nz;
+      // this block: recurrence, readout, skip, gate, store
+      float y[S];
+      block_recurrence<T, STRUCT>(bcb + kb * S * 32, xc, wc, rp, h2, y);
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        float v = fmaf(rp.Dd, blk_at<T>(ru, j), y[j]);
+        if constexpr (HAS_Z) v *= gate_f<T>(blk_at<T>(rz, j));
+        y[j] = v;
+      }
+      if (row_ok) store_block<T>(orow, t0 + k * S, t1, vec, y);
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        xc[j] = xn[j];
+        wc[j] = wn[j];
+      }
+      ru = run;
+      rz = rzn;
     }
     if (c + 1 < nchunks) stage.store(bc_s[(c + 1) & 1]);
     __syncthreads();
   }
+  cp_wait<0>();
 }
 
-template <typename T, bool HAS_Z, bool SOFTPLUS>
-__global__ void __launch_bounds__(kRows) scan_out_kernel(const ScanArgs p) {
+template <int ROWS>
+__device__ __forceinline__ bool load_row_params(const ScanArgs& p, int dc, RowParams& rp) {
+  const float bias = p.bias ? p.bias[int64_t(dc) * p.bias_s] : 0.0f;
+  rp.bias2 = bias * kLog2e;
+  rp.Dd = p.Dskip ? p.Dskip[int64_t(dc) * p.D_s] : 0.0f;
+  const float* Ar = p.A + int64_t(dc) * p.A_sd;
+  rp.A0 = Ar[0];
+  bool st = true;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float lo = Ar[int64_t(2 * k) * p.A_sn], hi = Ar[int64_t(2 * k + 1) * p.A_sn];
+    st = st && (lo == float(2 * k + 1) * rp.A0) && (hi == float(2 * k + 2) * rp.A0);
+    rp.Ap[k] = f2(lo, hi);
+  }
+  return st;
+}
+
+// 64-row CTAs are used when the grid must fill 16 warps per SM (128 registers);
+// 32-row CTAs when the rows alone limit occupancy, so they may use up to 224.
+template <typename T, int ROWS, bool HAS_Z, bool SOFTPLUS>
+__global__ void __launch_bounds__(ROWS, ROWS == 32 ? 9 : 8) scan_out_kernel(const ScanArgs p) {
   __shared__ __align__(16) float bc_s[2][kTC * 32];
+  __shared__ __align__(16) uint4 slots[kStages * 3 * ROWS];
   const int tid = threadIdx.x;
   const int tile = blockIdx.x;
   const int seg = blockIdx.y;
   const int b = tile / p.tiles_per_batch;
-  const int d = (tile - b * p.tiles_per_batch) * kRows + tid;
+  const int d = (tile - b * p.tiles_per_batch) * ROWS + tid;
   const bool row_ok = d < p.D;
   const int dc = row_ok ? d : p.D - 1;
   const int t0 = seg * p.seg_len;
@@ -353,25 +470,15 @@ __global__ void __launch_bounds__(kRows) scan_out_kernel(const ScanArgs p) {
   const T* zrow = HAS_Z ? static_cast<const T*>(p.z) + int64_t(b) * p.z_sb + int64_t(dc) * p.z_sd : nullptr;
   T* orow = static_cast<T*>(p.out) + int64_t(b) * p.o_sb + int64_t(dc) * p.o_sd;
 
-  const float bias = p.bias ? p.bias[int64_t(dc) * p.bias_s] : 0.0f;
-  const float Dd = p.Dskip ? p.Dskip[int64_t(dc) * p.D_s] : 0.0f;
-  const float* Ar = p.A + int64_t(dc) * p.A_sd;
-  f2_t A2p[8];
-  bool st = true;
-  const float A0 = Ar[0];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float lo = Ar[int64_t(2 * k) * p.A_sn], hi = Ar[int64_t(2 * k + 1) * p.A_sn];
-    st = st && (lo == float(2 * k + 1) * A0) && (hi == float(2 * k + 2) * A0);
-    A2p[k] = f2(lo * kLog2e, hi * kLog2e);
-  }
+  RowParams rp;
+  const bool st = load_row_params<ROWS>(p, dc, rp);
   const bool structured = __syncthreads_and(st) && !p.force_general;
-  const float a2_0 = A0 * kLog2e;
 
   f2_t h2[8];
   if (seg > 0) {
-    const int64_t rowg = int64_t(tile) * kRows + tid;
-    const float4* src = reinterpret_cast<const float4*>(p.ws_H + (int64_t(seg - 1) * p.Bt * p.tiles_per_batch * kRows + rowg) * kN);
+    const int64_t rows_total = int64_t(p.Bt) * p.tiles_per_batch * ROWS;
+    const int64_t rowg = int64_t(tile) * ROWS + tid;
+    const float4* src = reinterpret_cast<const float4*>(p.ws_H + (int64_t(seg - 1) * rows_total + rowg) * kN);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float4 v = __ldcg(src + i);
@@ -384,144 +491,177 @@ __global__ void __launch_bounds__(kRows) scan_out_kernel(const ScanArgs p) {
   }
 
   if (structured)
-    forward_chunk<T, HAS_Z, SOFTPLUS, true>(p, bc_s, b, t0, t1, urow, dlrow, zrow, orow, row_ok,
-                                            bias, Dd, a2_0, A2p, h2);
+    forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, true>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
+                                                  row_ok, rp, h2);
   else
-    forward_chunk<T, HAS_Z, SOFTPLUS, false>(p, bc_s, b, t0, t1, urow, dlrow, zrow, orow, row_ok,
-                                             bias, Dd, a2_0, A2p, h2);
+    forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, false>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
+                                                   row_ok, rp, h2);
 
   if (seg == p.nseg - 1 && row_ok && p.last_state) {
     float* dst = p.last_state + int64_t(b) * p.ls_sb + int64_t(d) * p.ls_sd;
+    float v[16];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      float lo, hi;
-      f2split(h2[k], lo, hi);
-      dst[2 * k] = lo;
-      dst[2 * k + 1] = hi;
+    for (int k = 0; k < 8; ++k) f2split(h2[k], v[2 * k], v[2 * k + 1]);
+    if (p.vec_ls) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int n = 0; n < 16; ++n) dst[n] = v[n];
     }
   }
 }
 
 // ---------------------------------------------------------------------------
 // Kernel 1: chunk summaries (S, H) by a backward sweep, then the carry fold.
-//   H_n = sum_s delta_s u_s B_sn exp(A_n sum_{s<r<=end} delta_r),  S = sum_s delta_s
 // ---------------------------------------------------------------------------
-template <typename T, bool SOFTPLUS, bool STRUCT>
-__device__ __forceinline__ void backward_chunk(const ScanArgs& p, float (*bc_s)[kTC * 32], int b,
-                                               int t0, int t1, const T* urow, const T* dlrow,
-                                               float bias, float a2_0, const f2_t (&A2p)[8],
-                                               f2_t (&H2)[8], float& S) {
-  constexpr int SB = Blk<T>::kSteps;
+// Per-step scalars of a block for the backward sweep: s and w = s * u.
+template <typename T, bool SOFTPLUS>
+__device__ __forceinline__ void block_scalars_bwd(const uint4& ru, const uint4& rd, const RowParams& rp,
+                                                  float* sv, float* wv) {
+  constexpr int S = 16 / int(sizeof(T));
+#pragma unroll
+  for (int j = 0; j < S; ++j) {
+    const float v2 = fmaf(blk_at<T>(rd, j), kLog2e, rp.bias2);
+    const float s = SOFTPLUS ? softplus2(v2) : v2;
+    sv[j] = s;
+    wv[j] = s * blk_at<T>(ru, j);
+  }
+}
+
+template <typename T, int ROWS, bool SOFTPLUS, bool STRUCT>
+__device__ __forceinline__ void backward_chunk(const ScanArgs& p, float (*bc_s)[kTC * 32], uint4* slots,
+                                               int b, int t0, int t1, const T* urow, const T* dlrow,
+                                               const RowParams& rp, f2_t (&H2)[8], float& Ssum) {
+  constexpr int S = 16 / int(sizeof(T));
+  constexpr int kBlkPerChunk = kTC / S;
+  const int tid = threadIdx.x;
   const bool vec = p.vec_rows != 0;
-  BCStage<T, 32> stage;  // rows 16..31 (C) are staged but unused here
-  const int nchunks = (t1 - t0) / kTC;  // chunks of kernel 1 are always full
-  float Tacc = 0.0f;                    // sum of delta over steps after the current one
+  const int nblk = (t1 - t0) / S;          // chunks of kernel 1 are always full
+  const int nchunks = (t1 - t0) / kTC;
+  auto slot = [&](int stage, int tensor) { return slots + (stage * 3 + tensor) * ROWS + tid; };
+  // the i-th block issued is block nblk-1-i (backwards), into stage i % kStages
+  auto issue = [&](int i) {
+    const int t = t0 + (nblk - 1 - i) * S;
+    const int st = i % kStages;
+    fetch_block<T>(slot(st, 0), urow, t, t1, vec);
+    fetch_block<T>(slot(st, 1), dlrow, t, t1, vec);
+  };
+#pragma unroll
+  for (int i = 0; i < kStages - 1; ++i) {
+    if (i < nblk) issue(i);
+    cp_commit();
+  }
+  BCStage<T, ROWS> stage;  // C rows are staged too but unused here
   stage.load(p, b, t0 + (nchunks - 1) * kTC, t1);
   stage.store(bc_s[0]);
+  cp_wait<kStages - 2>();
+  float sc[S], wc[S];
+  block_scalars_bwd<T, SOFTPLUS>(*slot(0, 0), *slot(0, 1), rp, sc, wc);
   __syncthreads();
-  Blk<T> cu, cd;
-  {
-    const int tl = t1 - SB;
-    cu.load(urow, tl, t1, vec);
-    cd.load(dlrow, tl, t1, vec);
-  }
+
+  float Tacc = 0.0f;  // sum of s over the steps after the current one
+  int i = 0;
   for (int ci = 0; ci < nchunks; ++ci) {
     const int c = nchunks - 1 - ci;
     const int cs = t0 + c * kTC;
     if (c > 0) stage.load(p, b, cs - kTC, t1);
     const float* bcb = bc_s[ci & 1];
-    for (int tb = cs + kTC - SB; tb >= cs; tb -= SB) {
-      Blk<T> nu, nd;
-      const int tn = tb - SB;
-      if (tn >= t0) {
-        nu.load(urow, tn, t1, vec);
-        nd.load(dlrow, tn, t1, vec);
-      } else {
-        nu.zero();
-        nd.zero();
+#pragma unroll 1
+    for (int kb = kBlkPerChunk - 1; kb >= 0; --kb, ++i) {
+      if (i + kStages - 1 < nblk) issue(i + kStages - 1);
+      cp_commit();
+      float sn[S], wn[S];
+      if (i + 1 < nblk) {
+        cp_wait<kStages - 2>();
+        const int st = (i + 1) % kStages;
+        block_scalars_bwd<T, SOFTPLUS>(*slot(st, 0), *slot(st, 1), rp, sn, wn);
       }
+      // suffix sums: T_j = Tacc + sum_{j < r < S} s_r (independent exponent inputs)
+      float Tj[S];
+      Tj[S - 1] = Tacc;
 #pragma unroll
-      for (int jj = 0; jj < SB; ++jj) {
-        const int j = SB - 1 - jj;
-        float dt = cd.at(j) + bias;
-        if constexpr (SOFTPLUS) dt = softplus_f(dt);
-        const float w = dt * cu.at(j);
-        const ulonglong2* q = reinterpret_cast<const ulonglong2*>(bcb + (tb + j - cs) * 32);
+      for (int j = S - 2; j >= 0; --j) Tj[j] = Tj[j + 1] + sc[j + 1];
+      Tacc = Tj[0] + sc[0];
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        const ulonglong2* q = reinterpret_cast<const ulonglong2*>(bcb + (kb * S + j) * 32);
+        const float w = wc[j];
         f2_t v[8];
         if constexpr (STRUCT) {
-          const float pi = ex2f(a2_0 * Tacc);   // prod_{r>t} A_bar_r,0
+          // v_n = w pi^(n+1), pi = 2^(A_0 T_j) = prod_{r>t} A_bar_r,0
+          const float pi = ex2f(rp.A0 * Tj[j]);
           const float pi2 = pi * pi;
-          v[0] = mul2(f2(w, w), f2(pi, pi2));   // (w pi, w pi^2)
-          const f2_t s2 = f2(pi2, pi2);
+          float c0 = w * pi, c1 = w * pi2;
+          v[0] = f2(c0, c1);
 #pragma unroll
-          for (int k = 1; k < 8; ++k) v[k] = mul2(v[k - 1], s2);
+          for (int kk = 1; kk < 8; ++kk) {
+            c0 *= pi2;
+            c1 *= pi2;
+            v[kk] = f2(c0, c1);
+          }
         } else {
-          const f2_t T2 = f2(Tacc, Tacc);
+          const f2_t T2 = f2(Tj[j], Tj[j]);
           const f2_t w2 = f2(w, w);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
+          for (int kk = 0; kk < 8; ++kk) {
             float lo, hi;
-            f2split(mul2(T2, A2p[k]), lo, hi);
-            v[k] = mul2(w2, f2(ex2f(lo), ex2f(hi)));
+            f2split(mul2(T2, rp.Ap[kk]), lo, hi);
+            v[kk] = mul2(w2, f2(ex2f(lo), ex2f(hi)));
           }
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const ulonglong2 bb = q[k];
-          H2[2 * k] = fma2(v[2 * k], bb.x, H2[2 * k]);
-          H2[2 * k + 1] = fma2(v[2 * k + 1], bb.y, H2[2 * k + 1]);
+        for (int kk = 0; kk < 4; ++kk) {
+          const ulonglong2 bb = q[kk];
+          H2[2 * kk] = fma2(v[2 * kk], bb.x, H2[2 * kk]);
+          H2[2 * kk + 1] = fma2(v[2 * kk + 1], bb.y, H2[2 * kk + 1]);
         }
-        Tacc += dt;
       }
-      cu = nu;
-      cd = nd;
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        sc[j] = sn[j];
+        wc[j] = wn[j];
+      }
     }
     if (c > 0) stage.store(bc_s[(ci + 1) & 1]);
     __syncthreads();
   }
-  S = Tacc;
+  cp_wait<0>();
+  Ssum = Tacc;
 }
 
-template <typename T, bool SOFTPLUS>
-__global__ void __launch_bounds__(kRows) scan_chunk_state_kernel(const ScanArgs p) {
+template <typename T, int ROWS, bool SOFTPLUS>
+__global__ void __launch_bounds__(ROWS, 512 / ROWS) scan_chunk_state_kernel(const ScanArgs p) {
   __shared__ __align__(16) float bc_s[2][kTC * 32];
+  __shared__ __align__(16) uint4 slots[kStages * 3 * ROWS];
   __shared__ int s_last;
   const int tid = threadIdx.x;
   const int tile = blockIdx.x;
   const int seg = blockIdx.y;  // 0 .. nseg-2
   const int b = tile / p.tiles_per_batch;
-  const int d = (tile - b * p.tiles_per_batch) * kRows + tid;
+  const int d = (tile - b * p.tiles_per_batch) * ROWS + tid;
   const int dc = d < p.D ? d : p.D - 1;
   const int t0 = seg * p.seg_len;
   const int t1 = t0 + p.seg_len;
 
   const T* urow = static_cast<const T*>(p.u) + int64_t(b) * p.u_sb + int64_t(dc) * p.u_sd;
   const T* dlrow = static_cast<const T*>(p.delta) + int64_t(b) * p.dl_sb + int64_t(dc) * p.dl_sd;
-  const float bias = p.bias ? p.bias[int64_t(dc) * p.bias_s] : 0.0f;
-  const float* Ar = p.A + int64_t(dc) * p.A_sd;
-  f2_t A2p[8];
-  bool st = true;
-  const float A0 = Ar[0];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float lo = Ar[int64_t(2 * k) * p.A_sn], hi = Ar[int64_t(2 * k + 1) * p.A_sn];
-    st = st && (lo == float(2 * k + 1) * A0) && (hi == float(2 * k + 2) * A0);
-    A2p[k] = f2(lo * kLog2e, hi * kLog2e);
-  }
+  RowParams rp;
+  const bool st = load_row_params<ROWS>(p, dc, rp);
   const bool structured = __syncthreads_and(st) && !p.force_general;
-  const float a2_0 = A0 * kLog2e;
 
   f2_t H2[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) H2[k] = 0ull;
-  float S = 0.0f;
+  float Ssum = 0.0f;
   if (structured)
-    backward_chunk<T, SOFTPLUS, true>(p, bc_s, b, t0, t1, urow, dlrow, bias, a2_0, A2p, H2, S);
+    backward_chunk<T, ROWS, SOFTPLUS, true>(p, bc_s, slots, b, t0, t1, urow, dlrow, rp, H2, Ssum);
   else
-    backward_chunk<T, SOFTPLUS, false>(p, bc_s, b, t0, t1, urow, dlrow, bias, a2_0, A2p, H2, S);
+    backward_chunk<T, ROWS, SOFTPLUS, false>(p, bc_s, slots, b, t0, t1, urow, dlrow, rp, H2, Ssum);
 
-  const int64_t rows_total = int64_t(p.Bt) * p.tiles_per_batch * kRows;
-  const int64_t rowg = int64_t(tile) * kRows + tid;
+  const int64_t rows_total = int64_t(p.Bt) * p.tiles_per_batch * ROWS;
+  const int64_t rowg = int64_t(tile) * ROWS + tid;
   {
     float4* dst = reinterpret_cast<float4*>(p.ws_H + (int64_t(seg) * rows_total + rowg) * kN);
 #pragma unroll
@@ -531,11 +671,11 @@ __global__ void __launch_bounds__(kRows) scan_chunk_state_kernel(const ScanArgs 
       f2split(H2[2 * i + 1], c, dd);
       __stcg(dst + i, make_float4(a, bq, c, dd));
     }
-    __stcg(p.ws_S + int64_t(seg) * rows_total + rowg, S);
+    __stcg(p.ws_S + int64_t(seg) * rows_total + rowg, Ssum);
   }
 
   // The last kernel-1 CTA of this row tile folds the chunk summaries, in chunk
-  // order, into carried states: prefix_k = exp(A S_k) prefix_(k-1) + H_k, stored
+  // order, into carried states: prefix_k = 2^(A S_k) prefix_(k-1) + H_k, stored
   // over H_k.  Nobody waits: the fold runs in whichever CTA arrives last.
   __threadfence();
   __syncthreads();
@@ -546,18 +686,36 @@ __global__ void __launch_bounds__(kRows) scan_chunk_state_kernel(const ScanArgs 
   f2_t h[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) h[k] = 0ull;
-  for (int k = 0; k < p.nseg - 1; ++k) {
+  const int nrec = p.nseg - 1;
+  // records are prefetched one ahead so the serial walk waits on arithmetic, not on L2
+  float4 nv[4];
+  float nS = 0.0f;
+  {
+    const float4* rec = reinterpret_cast<const float4*>(p.ws_H + rowg * kN);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) nv[i] = __ldcg(rec + i);
+    nS = __ldcg(p.ws_S + rowg);
+  }
+  for (int k = 0; k < nrec; ++k) {
+    float4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = nv[i];
+    const float Sk = nS;
+    if (k + 1 < nrec) {
+      const float4* nrec_p = reinterpret_cast<const float4*>(p.ws_H + (int64_t(k + 1) * rows_total + rowg) * kN);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) nv[i] = __ldcg(nrec_p + i);
+      nS = __ldcg(p.ws_S + int64_t(k + 1) * rows_total + rowg);
+    }
     float4* rec = reinterpret_cast<float4*>(p.ws_H + (int64_t(k) * rows_total + rowg) * kN);
-    const float Sk = __ldcg(p.ws_S + int64_t(k) * rows_total + rowg);
     const f2_t S2 = f2(Sk, Sk);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 v = __ldcg(rec + i);
       float e0, e1, e2, e3;
-      f2split(mul2(S2, A2p[2 * i]), e0, e1);
-      f2split(mul2(S2, A2p[2 * i + 1]), e2, e3);
-      h[2 * i] = fma2(f2(ex2f(e0), ex2f(e1)), h[2 * i], f2(v.x, v.y));
-      h[2 * i + 1] = fma2(f2(ex2f(e2), ex2f(e3)), h[2 * i + 1], f2(v.z, v.w));
+      f2split(mul2(S2, rp.Ap[2 * i]), e0, e1);
+      f2split(mul2(S2, rp.Ap[2 * i + 1]), e2, e3);
+      h[2 * i] = fma2(f2(ex2f(e0), ex2f(e1)), h[2 * i], f2(v[i].x, v[i].y));
+      h[2 * i + 1] = fma2(f2(ex2f(e2), ex2f(e3)), h[2 * i + 1], f2(v[i].z, v[i].w));
       float a, bq, c, dd;
       f2split(h[2 * i], a, bq);
       f2split(h[2 * i + 1], c, dd);
@@ -566,5 +724,6 @@ __global__ void __launch_bounds__(kRows) scan_chunk_state_kernel(const ScanArgs 
   }
   if (tid == 0) p.ws_count[tile] = 0u;
 }
+
 
 }  // namespace mssm

@@ -16,9 +16,12 @@ HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROO
 
 @pytest.fixture(scope="module")
 def lib():
-    from selective_state_space_46_b200 import build
-    path = build.build()
-    return ctypes.CDLL(path)
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_mssm_build", os.path.join(ROOT, "selective_state_space_46_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
+    return ctypes.CDLL(build.build())
 
 
 def declared_functions():
@@ -161,9 +164,40 @@ def test_options_and_strings(lib):
     assert lib.mssm_set_option(1, 2) == INVALID
     assert lib.mssm_set_option(2, 100) == INVALID      # not a multiple of 64
     assert lib.mssm_set_option(99, 0) == INVALID
+    assert lib.mssm_set_option(4, 1) == INVALID
     assert lib.mssm_set_option(2, 128) == 0
     assert lib.mssm_set_option(2, 0) == 0
     lib.mssm_status_string.restype = ctypes.c_char_p
     assert lib.mssm_status_string(2) == b"MSSM_ERR_UNSUPPORTED"
     lib.mssm_version.restype = ctypes.c_char_p
     assert re.match(rb"^\d+\.\d+\.\d+$", lib.mssm_version())
+
+
+def test_scan_plan_host_only(lib):
+    """The launch plan is host logic: check its invariants without a GPU."""
+    f = lib.mssm_scan_plan
+    f.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                  ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)]
+    rows, seg, nseg = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int64()
+    for Bt, D, L in [(1, 64, 256), (2, 1536, 2048), (8, 5120, 4096), (1, 2048, 131072), (3, 7, 1), (1, 1, 0),
+                     (64, 8192, 100), (1, 16, 1 << 24)]:
+        assert f(Bt, D, L, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg)) == 0
+        assert rows.value in (32, 64)
+        assert seg.value % 64 == 0 and seg.value >= 64
+        assert nseg.value >= 1 and nseg.value <= 65535
+        if L > 0:
+            # the chunks cover the sequence exactly: every chunk but the last is full
+            assert (nseg.value - 1) * seg.value < L <= nseg.value * seg.value
+    # a shape whose rows fill the GPU is not split
+    assert f(8, 5120, 4096, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg)) == 0
+    assert nseg.value == 1
+    # few rows and a long sequence are split
+    assert f(1, 2048, 131072, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg)) == 0
+    assert nseg.value > 1
+    # an explicit chunk length is honoured
+    lib.mssm_set_option.argtypes = [ctypes.c_int, ctypes.c_int64]
+    assert lib.mssm_set_option(2, 128) == 0
+    assert f(1, 64, 1000, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg)) == 0
+    assert (seg.value, nseg.value) == (128, 8)
+    assert lib.mssm_set_option(2, 0) == 0
+    assert f(-1, 64, 1000, 148, None, None, None) == INVALID

@@ -15,14 +15,17 @@ from gpu_util import check_close, dev_scan_inputs, run_scan, to_dev, to_f64
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True)
-def _defaults(cuda_device):
+def _reset_options():
     import selective_state_space_46_b200 as m
     m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 0)
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
+
+
+@pytest.fixture(autouse=True)
+def _defaults(cuda_device):
+    _reset_options()
     yield
-    m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 0)
-    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
+    _reset_options()
 
 
 def compare_full(inp, **kw):
@@ -129,7 +132,7 @@ def test_general_A_values(io):
 @pytest.mark.parametrize("chunk", [64, 128, 192, 320])
 @pytest.mark.parametrize("structured", [True, False])
 @pytest.mark.parametrize("io", ["bf16", "f32"])
-def test_chunked_carry(chunk, structured, io):
+def test_chunked_carry(chunk, structured, io,):
     import selective_state_space_46_b200 as m
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, chunk)
     inp = synth.make_scan_inputs(2, 80, 1000, io_dtype=io, seed=chunk, delta_range=(1e-4, 1e-2))
