@@ -78,6 +78,7 @@ cudaError_t tracked(int kind, cudaStream_t s, F&& fn) {
 struct DeviceState {
   void* ws = nullptr;
   size_t ws_bytes = 0;
+  int64_t count_cap = 0;  // arrival counters at the start of ws (a region only counters ever use)
   int sm_count = 0;
 };
 std::vector<DeviceState> g_dev;
@@ -226,12 +227,24 @@ mssm_status mssm_set_option(int option, int64_t value) {
   return fail(MSSM_ERR_INVALID_ARG, "unknown option %d", option);
 }
 
-mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* delta,
-                                    const mssm_tensor* A, const mssm_tensor* B,
-                                    const mssm_tensor* C, const mssm_tensor* D,
-                                    const mssm_tensor* z, const mssm_tensor* delta_bias,
-                                    int softplus_flag, mssm_tensor* out, mssm_tensor* last_state,
-                                    void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Validation and kernel arguments of a scan call, shared by both scan entry points.
+struct ScanCall {
+  mssm::ScanArgs a{};
+  int dtype = 0;
+  bool has_z = false;
+  bool softplus = false;
+  bool noop = false;       // Bt * D == 0: nothing to launch
+  int64_t Bt = 0, D = 0, L = 0;
+};
+
+mssm_status scan_prepare(const mssm_tensor* u, const mssm_tensor* delta, const mssm_tensor* A,
+                         const mssm_tensor* B, const mssm_tensor* C, const mssm_tensor* D,
+                         const mssm_tensor* z, const mssm_tensor* delta_bias, int softplus_flag,
+                         mssm_tensor* out, mssm_tensor* last_state, ScanCall& call) {
   if (!u) return fail(MSSM_ERR_INVALID_ARG, "u: null tensor descriptor");
   if (u->ndim != 3) return fail(MSSM_ERR_INVALID_ARG, "u: expected 3 dims [Bt, D, L]");
   const int dt = u->dtype;
@@ -261,9 +274,16 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* del
   if (last_state)
     for (const mssm_tensor* t : ins)
       if (same_ptr(last_state, t)) return fail(MSSM_ERR_INVALID_ARG, "last_state must not alias an input");
-  if (Bt == 0 || Dd == 0) return MSSM_OK;
+  call.dtype = dt;
+  call.has_z = z != nullptr;
+  call.softplus = softplus_flag != 0;
+  call.Bt = Bt;
+  call.D = Dd;
+  call.L = L;
+  call.noop = (Bt == 0 || Dd == 0);
+  if (call.noop) return MSSM_OK;
 
-  mssm::ScanArgs a{};
+  mssm::ScanArgs& a = call.a;
   a.u = u->data; a.delta = delta->data; a.z = z ? z->data : nullptr; a.out = out->data;
   a.u_sb = u->stride[0]; a.u_sd = u->stride[1];
   a.dl_sb = delta->stride[0]; a.dl_sd = delta->stride[1];
@@ -282,6 +302,73 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* del
   a.vec_bc = rows_vec(B) && rows_vec(C);
   a.vec_ls = last_state && aligned16(last_state->data) && (last_state->stride[0] * 4) % 16 == 0 &&
              (last_state->stride[1] * 4) % 16 == 0;
+  return MSSM_OK;
+}
+
+// Plans the launch (caller holds g_mu) and returns the carry workspace layout.
+struct ScanPlan {
+  int rows_per_cta = 64;
+  int64_t nseg = 1;
+  size_t count_bytes = 0, s_bytes = 0, h_bytes = 0;
+  size_t need() const { return nseg > 1 ? count_bytes + s_bytes + h_bytes : 0; }
+};
+
+ScanPlan scan_plan(ScanCall& call, int sm_count) {
+  mssm::ScanArgs& a = call.a;
+  a.force_general = g_force_general;
+  const LaunchShape shape = choose_shape(call.Bt, call.D, call.L, sm_count, g_chunk_len);
+  ScanPlan plan;
+  plan.rows_per_cta = shape.rows;
+  plan.nseg = shape.nseg;
+  a.tiles_per_batch = int((call.D + shape.rows - 1) / shape.rows);
+  const int64_t tiles = call.Bt * a.tiles_per_batch;
+  a.seg_len = int(shape.seg);
+  a.nseg = int(shape.nseg);
+  if (shape.nseg > 1) {
+    const int64_t rows_total = tiles * shape.rows;
+    plan.count_bytes = ((size_t(tiles) * 4 + 255) / 256) * 256;
+    plan.s_bytes = ((size_t(shape.nseg - 1) * rows_total * 4 + 255) / 256) * 256;
+    plan.h_bytes = size_t(shape.nseg - 1) * rows_total * mssm::kN * 4;
+  }
+  return plan;
+}
+
+void scan_bind_workspace(mssm::ScanArgs& a, const ScanPlan& plan, void* ws) {
+  char* base = static_cast<char*>(ws);
+  a.ws_count = reinterpret_cast<unsigned*>(base);
+  a.ws_S = reinterpret_cast<float*>(base + plan.count_bytes);
+  a.ws_H = reinterpret_cast<float*>(base + plan.count_bytes + plan.s_bytes);
+}
+
+// The kernel launches of a planned call (caller holds g_mu).
+mssm_status scan_launch(const ScanCall& call, const ScanPlan& plan, cudaStream_t s) {
+  cudaError_t e;
+  if (plan.nseg > 1) {
+    e = tracked(MSSM_KERNEL_SCAN_CHUNK_STATE, s, [&] {
+      return mssm::launch_scan_chunk_state(call.a, plan.rows_per_cta, call.dtype, call.softplus, s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel launch");
+  }
+  e = tracked(MSSM_KERNEL_SCAN_OUT, s, [&] {
+    return mssm::launch_scan_out(call.a, plan.rows_per_cta, call.dtype, call.has_z, call.softplus, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
+  return MSSM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* delta,
+                                    const mssm_tensor* A, const mssm_tensor* B,
+                                    const mssm_tensor* C, const mssm_tensor* D,
+                                    const mssm_tensor* z, const mssm_tensor* delta_bias,
+                                    int softplus_flag, mssm_tensor* out, mssm_tensor* last_state,
+                                    void* stream) {
+  ScanCall call;
+  mssm_status st = scan_prepare(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state, call);
+  if (st != MSSM_OK || call.noop) return st;
 
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -289,27 +376,25 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* del
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   std::lock_guard<std::mutex> lk(g_mu);
-  a.force_general = g_force_general;
   DeviceState* ds = device_state(dev);
-  const LaunchShape shape = choose_shape(Bt, Dd, L, ds->sm_count, g_chunk_len);
-  const int64_t seg = shape.seg, nseg = shape.nseg;
-  const int rows_per_cta = shape.rows;
-  a.tiles_per_batch = int((Dd + rows_per_cta - 1) / rows_per_cta);
-  const int64_t tiles = Bt * a.tiles_per_batch;
-  a.seg_len = int(seg);
-  a.nseg = int(nseg);
-
-  if (nseg > 1) {
-    const int64_t rows_total = tiles * rows_per_cta;
-    const size_t count_bytes = ((size_t(tiles) * 4 + 255) / 256) * 256;
-    const size_t s_bytes = ((size_t(nseg - 1) * rows_total * 4 + 255) / 256) * 256;
-    const size_t h_bytes = size_t(nseg - 1) * rows_total * mssm::kN * 4;
-    const size_t need = count_bytes + s_bytes + h_bytes;
-    if (ds->ws_bytes < need) {
+  const ScanPlan plan = scan_plan(call, ds->sm_count);
+  if (plan.nseg > 1) {
+    // The arrival counters keep a region of their own at the start of the
+    // workspace, sized for the most row tiles seen so far: they start at zero
+    // and every complete call leaves them at zero, so they are never cleared
+    // per call.  (Sharing the counters' bytes with the summaries of a call with
+    // more tiles would leave non-zero counters behind.)
+    const int64_t tiles = plan.count_bytes / 4;
+    const int64_t cap = tiles > ds->count_cap ? tiles : ds->count_cap;
+    ScanPlan layout = plan;
+    layout.count_bytes = ((size_t(cap) * 4 + 255) / 256) * 256;
+    const size_t need = layout.need();
+    if (ds->ws_bytes < need || cap > ds->count_cap) {
       if (ds->ws) {
         e = cudaFree(ds->ws);  // synchronises the device
         ds->ws = nullptr;
         ds->ws_bytes = 0;
+        ds->count_cap = 0;
         if (e != cudaSuccess) return cuda_fail(e, "cudaFree(workspace)");
       }
       e = cudaMalloc(&ds->ws, need);
@@ -318,25 +403,14 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* del
         return cuda_fail(e, "cudaMalloc(workspace)");
       }
       ds->ws_bytes = need;
-      // arrival counters start at zero; every complete call leaves them at zero
+      ds->count_cap = int64_t(layout.count_bytes / 4);
       e = cudaMemsetAsync(ds->ws, 0, need, s);
       if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
     }
-    char* base = static_cast<char*>(ds->ws);
-    a.ws_count = reinterpret_cast<unsigned*>(base);
-    a.ws_S = reinterpret_cast<float*>(base + count_bytes);
-    a.ws_H = reinterpret_cast<float*>(base + count_bytes + s_bytes);
+    layout.count_bytes = size_t(ds->count_cap) * 4;
+    scan_bind_workspace(call.a, layout, ds->ws);
   }
-
-  if (nseg > 1) {
-    e = tracked(MSSM_KERNEL_SCAN_CHUNK_STATE, s,
-                [&] { return mssm::launch_scan_chunk_state(a, rows_per_cta, dt, softplus_flag != 0, s); });
-    if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel launch");
-  }
-  e = tracked(MSSM_KERNEL_SCAN_OUT, s,
-              [&] { return mssm::launch_scan_out(a, rows_per_cta, dt, z != nullptr, softplus_flag != 0, s); });
-  if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
-  return MSSM_OK;
+  return scan_launch(call, plan, s);
 }
 
 static mssm_status state_update_impl(mssm_tensor* state, const mssm_tensor* x, const mssm_tensor* dt_t,

@@ -155,6 +155,19 @@ def test_chunked_equals_unchunked_closely():
     assert float(((h1 - h2).abs() / (1 + h1.abs())).max()) < 1e-5
 
 
+def test_workspace_reuse_across_tile_counts():
+    """Split calls with different row-tile counts share the library's carry
+    workspace: a call with few tiles writes chunk sums where a later call with
+    more tiles keeps arrival counters, unless the counters have a region of
+    their own.  Sequence: size the workspace, split 1 tile, split 96 tiles."""
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 64)
+    big = synth.make_scan_inputs(2, 1536, 4096, io_dtype="bf16", seed=30)
+    run_scan(big)
+    for Bt, D, L, seed in [(1, 32, 4096, 31), (2, 1536, 2048, 32)]:
+        compare_full(synth.make_scan_inputs(Bt, D, L, io_dtype="bf16", seed=seed))
+
+
 def test_long_slow_decay_many_chunks():
     inp = synth.make_scan_inputs(1, 64, 16384, io_dtype="bf16", seed=5, delta_range=(1e-4, 1e-2))
     compare_full(inp)
