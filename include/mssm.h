@@ -112,6 +112,36 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor *u, const mssm_tensor *del
                                     mssm_tensor *last_state, void *stream);
 
 /*
+ * mssm_selective_scan_fwd_noalloc: the same scan, same arguments and results,
+ * for callers that cannot allocate device memory during the call.  Examples: a
+ * host application whose device memory is entirely owned by its own allocator
+ * or a pre-reserved pool, or a loop that cannot afford cudaMalloc's implicit
+ * device-wide synchronisation.  (The pages describe no such entry point; it is
+ * a property of this library's boundary, not of the method.)
+ *
+ * It never calls cudaMalloc, cudaFree or any allocating routine.  When a long
+ * sequence is split into chunks, the chunk summaries go to a fixed 8 MiB array
+ * compiled into the library's device image, present on every GPU that loads
+ * the library until the process exits.  A problem whose summaries need more
+ * than 8 MiB (about (chunks - 1) x Bt x D x 68 bytes) is rejected with
+ * MSSM_ERR_UNSUPPORTED and a message naming the size; problems that are not
+ * split use no scratch at all.
+ *
+ * The first call on each device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  Every call shares the one array and finds in it what the previous
+ * call left: each call zeroes the arrival counters it needs (one small
+ * cudaMemsetAsync on `stream`).  Calls that overlap on the GPU race on the
+ * array; issue them on one stream or order them with events.
+ */
+mssm_status mssm_selective_scan_fwd_noalloc(const mssm_tensor *u, const mssm_tensor *delta,
+                                            const mssm_tensor *A, const mssm_tensor *B,
+                                            const mssm_tensor *C, const mssm_tensor *D,
+                                            const mssm_tensor *z, const mssm_tensor *delta_bias,
+                                            int softplus_flag, mssm_tensor *out,
+                                            mssm_tensor *last_state, void *stream);
+
+/*
  * One-token selective state update (decode), state updated IN PLACE:
  *
  *   state [Bt, D, N] f32   read and written (n stride 1)

@@ -17,7 +17,8 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = [
-    "MssmError", "mssm_selective_scan_fwd", "mssm_state_update", "mssm_state_update_ex",
+    "MssmError", "mssm_selective_scan_fwd", "mssm_selective_scan_fwd_noalloc", "mssm_state_update",
+    "mssm_state_update_ex",
     "mssm_get_error", "mssm_set_option", "mssm_shutdown", "mssm_version", "mssm_status_string",
     "mssm_last_error", "selective_scan_fwd", "state_update", "lib_path",
     "MSSM_OPT_FORCE_GENERAL_A", "MSSM_OPT_CHUNK_LEN", "MSSM_OPT_KERNEL_TIMING", "mssm_kernel_stats", "mssm_scan_plan",
@@ -46,6 +47,8 @@ _P = ctypes.POINTER(mssm_tensor)
 _V = ctypes.c_void_p
 _lib.mssm_selective_scan_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, _V]
 _lib.mssm_selective_scan_fwd.restype = ctypes.c_int
+_lib.mssm_selective_scan_fwd_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, _V]
+_lib.mssm_selective_scan_fwd_noalloc.restype = ctypes.c_int
 _lib.mssm_state_update.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _V]
 _lib.mssm_state_update.restype = ctypes.c_int
 _lib.mssm_state_update_ex.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _V]
@@ -158,6 +161,15 @@ def mssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, 
     ds = [_desc(t) for t in (u, delta, A, B, C, D, z, delta_bias, out, last_state)]
     _check(_lib.mssm_selective_scan_fwd(*[_ref(x) for x in ds[:8]], int(softplus_flag),
                                         _ref(ds[8]), _ref(ds[9]), _stream(stream, u)))
+
+
+def mssm_selective_scan_fwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state,
+                                    stream=None) -> None:
+    """Marshal torch tensors into ``mssm_selective_scan_fwd_noalloc``: the same scan for
+    callers that cannot allocate device memory during the call (see include/mssm.h)."""
+    ds = [_desc(t) for t in (u, delta, A, B, C, D, z, delta_bias, out, last_state)]
+    _check(_lib.mssm_selective_scan_fwd_noalloc(*[_ref(x) for x in ds[:8]], int(softplus_flag),
+                                                _ref(ds[8]), _ref(ds[9]), _stream(stream, u)))
 
 
 def mssm_state_update(state, x, dt, A, B, C, D, z, out, stream=None) -> None:

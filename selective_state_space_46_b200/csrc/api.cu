@@ -413,6 +413,70 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* del
   return scan_launch(call, plan, s);
 }
 
+// ---------------------------------------------------------------------------
+// Scan without any allocation.  Its carry scratch is a fixed array in the
+// library's device image instead of a cudaMalloc'd workspace.  The array lives
+// on every GPU that loads this library, from module load until process exit.
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[64] = {};  // per-device address of g_noalloc_scratch, set up on first use
+int g_noalloc_sms[64] = {};    // per-device SM count, set up on first use
+
+}  // namespace
+
+extern "C" {
+
+mssm_status mssm_selective_scan_fwd_noalloc(const mssm_tensor* u, const mssm_tensor* delta,
+                                            const mssm_tensor* A, const mssm_tensor* B,
+                                            const mssm_tensor* C, const mssm_tensor* D,
+                                            const mssm_tensor* z, const mssm_tensor* delta_bias,
+                                            int softplus_flag, mssm_tensor* out,
+                                            mssm_tensor* last_state, void* stream) {
+  ScanCall call;
+  mssm_status st = scan_prepare(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state, call);
+  if (st != MSSM_OK || call.noop) return st;
+
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MSSM_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_sms[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    g_noalloc_sms[dev] = v;
+  }
+  const ScanPlan plan = scan_plan(call, g_noalloc_sms[dev]);
+  if (plan.nseg > 1) {
+    const size_t need = plan.need();
+    if (need > kNoAllocScratchBytes)
+      return fail(MSSM_ERR_UNSUPPORTED,
+                  "this problem needs %zu bytes of carry scratch; the no-allocation scan has a fixed "
+                  "%zu-byte array (use mssm_selective_scan_fwd, or a longer MSSM_OPT_CHUNK_LEN)",
+                  need, kNoAllocScratchBytes);
+    // First use on this device: look up the array's device address with this
+    // device current.  Host code must never pass &g_noalloc_scratch itself.
+    if (!g_noalloc_ptr[dev]) {
+      void* ptr = nullptr;
+      e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+      g_noalloc_ptr[dev] = ptr;
+    }
+    // The array keeps whatever the previous call left: zero the arrival counters.
+    e = cudaMemsetAsync(g_noalloc_ptr[dev], 0, plan.count_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-allocation scratch counters)");
+    scan_bind_workspace(call.a, plan, g_noalloc_ptr[dev]);
+  }
+  return scan_launch(call, plan, s);
+}
+
 static mssm_status state_update_impl(mssm_tensor* state, const mssm_tensor* x, const mssm_tensor* dt_t,
                                      const mssm_tensor* A, const mssm_tensor* B, const mssm_tensor* C,
                                      const mssm_tensor* D, const mssm_tensor* z, const mssm_tensor* bias,
