@@ -102,7 +102,9 @@ typedef struct {
  * freed by mssm_shutdown().  Calls that use the workspace must not overlap on
  * the GPU (different streams of one device); run them on one stream or order
  * them with events.  A first call of the largest size before any stream
- * capture keeps allocation out of captured work.
+ * capture keeps allocation out of captured work.  Shapes with many row tiles
+ * instead use a persistent kernel that runs each tile's chunks in order
+ * (MSSM_ERR_TIMEOUT from mssm_get_error if one of its bounded waits gave up).
  */
 mssm_status mssm_selective_scan_fwd(const mssm_tensor *u, const mssm_tensor *delta,
                                     const mssm_tensor *A, const mssm_tensor *B,
@@ -212,12 +214,15 @@ mssm_status mssm_set_option(int option, int64_t value);
 /*
  * Host-only query of the launch plan mssm_selective_scan_fwd would use for a
  * [Bt, D, L] problem on a GPU with sm_count SMs (sm_count <= 0: the current
- * device, or 148 when there is none): channels per CTA (32 or 64), chunk length
- * and number of chunks (1 = no split).  Honours MSSM_OPT_CHUNK_LEN.  Launches
- * nothing; any output pointer may be NULL.
+ * device, or 148 when there is none): channels per CTA (32 or 64), chunk length,
+ * number of chunks (1 = no split) and schedule: 0 = one forward kernel,
+ * 1 = chunk-summary kernel + forward kernel, 2 = persistent chained forward
+ * kernel (chunks of a tile run in order, each starting from the state the
+ * previous one published).  Honours MSSM_OPT_CHUNK_LEN.  Launches nothing; any
+ * output pointer may be NULL.
  */
 mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int *rows_per_cta,
-                           int64_t *chunk_len, int64_t *n_chunks);
+                           int64_t *chunk_len, int64_t *n_chunks, int *schedule);
 
 /* Kernel kinds counted by mssm_kernel_stats. */
 typedef enum {

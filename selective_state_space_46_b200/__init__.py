@@ -67,7 +67,7 @@ _lib.mssm_kernel_stats.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.POINTE
 _lib.mssm_kernel_stats.restype = ctypes.c_int
 _lib.mssm_scan_plan.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                 ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int64),
-                                ctypes.POINTER(ctypes.c_int64)]
+                                ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int)]
 _lib.mssm_scan_plan.restype = ctypes.c_int
 
 
@@ -144,9 +144,11 @@ def mssm_kernel_stats(reset: bool = False) -> dict:
 
 def mssm_scan_plan(Bt: int, D: int, L: int, sm_count: int = 0) -> dict:
     """Launch plan of the scan for a [Bt, D, L] problem (host only, launches nothing)."""
-    rows, seg, nseg = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int64()
-    _check(_lib.mssm_scan_plan(Bt, D, L, sm_count, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg)))
-    return {"rows_per_cta": rows.value, "chunk_len": seg.value, "n_chunks": nseg.value}
+    rows, seg, nseg, sched = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int()
+    _check(_lib.mssm_scan_plan(Bt, D, L, sm_count, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg),
+                               ctypes.byref(sched)))
+    return {"rows_per_cta": rows.value, "chunk_len": seg.value, "n_chunks": nseg.value,
+            "schedule": ("forward", "summaries+forward", "chained")[sched.value]}
 
 
 def mssm_get_error(stream=None) -> None:

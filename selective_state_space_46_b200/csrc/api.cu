@@ -134,10 +134,15 @@ bool same_ptr(const mssm_tensor* a, const mssm_tensor* b) {
   return a && b && a->data && a->data == b->data;
 }
 
-// Launch shape of the scan: channels per CTA and the length split.
+// Launch shape of the scan.
+//   mode 0: one forward kernel over whole sequences (nseg == 1)
+//   mode 1: chunk-summary kernel + forward kernel over nseg chunks
+//   mode 2: persistent chained forward kernel (32-row tiles, `grid` CTAs)
 struct LaunchShape {
+  int mode;
   int rows;
   int64_t seg, nseg;
+  int grid;
 };
 
 int64_t round_seg(int64_t v) {
@@ -145,30 +150,36 @@ int64_t round_seg(int64_t v) {
   return v < mssm::kSegQuant ? mssm::kSegQuant : v;
 }
 
-// Cost model (in FP32-pipe cycles of the busiest SM, up to a constant): the
-// CTAs of a kernel run in waves of at most kMaxCta[rows] per SM (register
-// limited) and carry equal work; an SM needs kSat threads to keep its pipes
-// busy, below which its time is set by one thread's serial work.  Per element
-// the forward kernel costs kOut and the chunk-summary kernel kSum; each launch
-// adds kLaunch.  Candidates: 32 or 64 channels per CTA (32 first: its kernel
-// has the larger register budget, so it wins ties), 1..64 chunks (lengths in
-// multiples of kSegQuant).
+// Cost model, in cycles of the busiest SM sub-partition (SMSP).  Measured on
+// B200: a warp-step of the forward kernel issues about kOut instructions and
+// of the summary kernel kSum; an SMSP sustains kIpc1 instructions per cycle
+// with one warp and kIpc2 with two or more (more warps do not raise it).  A
+// CTA costs kStart cycles of start-up latency per wave, a launch kLaunch, a
+// chained work item kItem, and the carry fold kFold per chunk.  Grid kernels
+// run their CTAs in waves of at most kMaxCta per SM (register limited) and
+// put ceil(warps / 4) warps on the busiest SMSP.
 LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forced_seg) {
-  constexpr double kSat = 512.0, kOut = 80.0, kSum = 45.0, kLaunch = 3.0e5;
-  LaunchShape best{32, L > 0 ? L : 1, 1};
-  double best_cost = -1.0;
-  for (int rows : {32, 64}) {
+  constexpr double kOut = 96.0, kSum = 55.0, kIpc1 = 0.6, kIpc2 = 0.7;
+  constexpr double kStart = 4000.0, kLaunch = 6000.0, kItem = 4000.0, kFold = 200.0;
+  auto ipc = [&](int64_t k) { return k <= 1 ? kIpc1 : kIpc2; };
+  auto grid_time = [&](int64_t ctas, int rows, double steps, double instr) {
     const int64_t max_cta = rows == 32 ? 12 : 8;
+    const int64_t on_sm = (ctas + sms - 1) / sms;
+    const int64_t waves = (on_sm + max_cta - 1) / max_cta;
+    const int64_t resident = on_sm < max_cta ? on_sm : max_cta;
+    const int64_t k = (resident * (rows / 32) + 3) / 4;
+    return double(waves) * (double(k) * steps * instr / ipc(k) + kStart) + kLaunch;
+  };
+  LaunchShape best{0, 32, L > 0 ? L : 1, 1, 0};
+  double best_cost = -1.0;
+  auto consider = [&](const LaunchShape& sh, double cost) {
+    if (best_cost < 0.0 || cost < best_cost * 0.999) {
+      best_cost = cost;
+      best = sh;
+    }
+  };
+  for (int rows : {32, 64}) {
     const int64_t tiles = Bt * ((D + rows - 1) / rows);
-    auto sm_time = [&](int64_t ctas, double per_elem, double seg) {
-      const int64_t on_sm = (ctas + sms - 1) / sms;
-      const int64_t waves = (on_sm + max_cta - 1) / max_cta;
-      const int64_t resident = on_sm < max_cta ? on_sm : max_cta;
-      const double threads = double(resident * rows);
-      const double work = threads * seg * per_elem / 128.0;
-      const double serial = threads < kSat ? seg * per_elem * kSat / 128.0 : 0.0;
-      return double(waves) * (work > serial ? work : serial) + kLaunch;
-    };
     for (int64_t want = 1; want <= 64; ++want) {
       int64_t seg = forced_seg > 0 ? forced_seg : round_seg((L + want - 1) / want);
       int64_t nseg = L > 0 ? (L + seg - 1) / seg : 1;
@@ -176,11 +187,20 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
         seg *= 2;
         nseg = (L + seg - 1) / seg;
       }
-      double cost = sm_time(tiles * nseg, kOut, double(seg));
-      if (nseg > 1) cost += sm_time(tiles * (nseg - 1), kSum, double(seg));
-      if (best_cost < 0.0 || cost < best_cost * 0.999) {
-        best_cost = cost;
-        best = LaunchShape{rows, seg, nseg};
+      double cost = grid_time(tiles * nseg, rows, double(seg), kOut);
+      if (nseg > 1) cost += grid_time(tiles * (nseg - 1), rows, double(seg), kSum) + kFold * double(nseg);
+      consider(LaunchShape{nseg > 1 ? 1 : 0, rows, seg, nseg, 0}, cost);
+      // chained: 32-row tiles, at most 8 one-warp CTAs per SM and never more CTAs than tiles
+      if (rows == 32 && nseg > 1) {
+        const int64_t per_sm = tiles / sms < 8 ? tiles / sms : 8;
+        if (per_sm >= 4) {
+          // each CTA takes whole items; k warps share an SMSP's issue
+          const int64_t grid = per_sm * sms;
+          const int64_t k = (per_sm + 3) / 4;
+          const int64_t rounds = (tiles * nseg + grid - 1) / grid;
+          const double item = double(seg) * kOut * double(k) / ipc(k) + kItem;
+          consider(LaunchShape{2, 32, seg, nseg, int(grid)}, double(rounds) * item + kLaunch);
+        }
       }
       if (forced_seg > 0 || L <= mssm::kSegQuant) break;
     }
@@ -307,10 +327,14 @@ mssm_status scan_prepare(const mssm_tensor* u, const mssm_tensor* delta, const m
 
 // Plans the launch (caller holds g_mu) and returns the carry workspace layout.
 struct ScanPlan {
+  int mode = 0;
   int rows_per_cta = 64;
+  int grid = 0;
   int64_t nseg = 1;
+  // mode 1: arrival counters, chunk sums, chunk end states
+  // mode 2: ticket + per-tile flags (count_bytes, zeroed per call), carried states (h_bytes)
   size_t count_bytes = 0, s_bytes = 0, h_bytes = 0;
-  size_t need() const { return nseg > 1 ? count_bytes + s_bytes + h_bytes : 0; }
+  size_t need() const { return mode != 0 ? count_bytes + s_bytes + h_bytes : 0; }
 };
 
 ScanPlan scan_plan(ScanCall& call, int sm_count) {
@@ -318,31 +342,54 @@ ScanPlan scan_plan(ScanCall& call, int sm_count) {
   a.force_general = g_force_general;
   const LaunchShape shape = choose_shape(call.Bt, call.D, call.L, sm_count, g_chunk_len);
   ScanPlan plan;
+  plan.mode = shape.mode;
   plan.rows_per_cta = shape.rows;
+  plan.grid = shape.grid;
   plan.nseg = shape.nseg;
   a.tiles_per_batch = int((call.D + shape.rows - 1) / shape.rows);
   const int64_t tiles = call.Bt * a.tiles_per_batch;
   a.seg_len = int(shape.seg);
   a.nseg = int(shape.nseg);
-  if (shape.nseg > 1) {
+  if (shape.mode == 1) {
     const int64_t rows_total = tiles * shape.rows;
     plan.count_bytes = ((size_t(tiles) * 4 + 255) / 256) * 256;
     plan.s_bytes = ((size_t(shape.nseg - 1) * rows_total * 4 + 255) / 256) * 256;
     plan.h_bytes = size_t(shape.nseg - 1) * rows_total * mssm::kN * 4;
+  } else if (shape.mode == 2) {
+    plan.count_bytes = ((size_t(tiles + 1) * 4 + 255) / 256) * 256;
+    plan.h_bytes = size_t(tiles) * 32 * mssm::kN * 4;
   }
   return plan;
 }
 
 void scan_bind_workspace(mssm::ScanArgs& a, const ScanPlan& plan, void* ws) {
   char* base = static_cast<char*>(ws);
+  if (plan.mode == 2) {
+    a.ch_ticket = reinterpret_cast<unsigned*>(base);
+    a.ch_flags = reinterpret_cast<unsigned*>(base) + 1;
+    a.ch_carry = reinterpret_cast<float*>(base + plan.count_bytes);
+    return;
+  }
   a.ws_count = reinterpret_cast<unsigned*>(base);
   a.ws_S = reinterpret_cast<float*>(base + plan.count_bytes);
   a.ws_H = reinterpret_cast<float*>(base + plan.count_bytes + plan.s_bytes);
 }
 
-// The kernel launches of a planned call (caller holds g_mu).
-mssm_status scan_launch(const ScanCall& call, const ScanPlan& plan, cudaStream_t s) {
+// The kernel launches of a planned call (caller holds g_mu).  `ws` is the
+// workspace base the plan was bound to (mode 2 zeroes its ticket and flags).
+mssm_status scan_launch(ScanCall& call, const ScanPlan& plan, void* ws, cudaStream_t s) {
   cudaError_t e;
+  if (plan.mode == 2) {
+    e = mssm::device_error_word(&call.a.err);
+    if (e != cudaSuccess) return cuda_fail(e, "device error word");
+    e = cudaMemsetAsync(ws, 0, plan.count_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(chained schedule flags)");
+    e = tracked(MSSM_KERNEL_SCAN_OUT, s, [&] {
+      return mssm::launch_scan_chained(call.a, plan.grid, call.dtype, call.has_z, call.softplus, s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "chained scan kernel launch");
+    return MSSM_OK;
+  }
   if (plan.nseg > 1) {
     e = tracked(MSSM_KERNEL_SCAN_CHUNK_STATE, s, [&] {
       return mssm::launch_scan_chunk_state(call.a, plan.rows_per_cta, call.dtype, call.softplus, s);
@@ -378,6 +425,31 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* del
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceState* ds = device_state(dev);
   const ScanPlan plan = scan_plan(call, ds->sm_count);
+  if (plan.mode == 2) {
+    // ticket, flags and carried states: zeroed by scan_launch where they must be
+    const size_t need = plan.need() + size_t(ds->count_cap) * 4;
+    if (ds->ws_bytes < need) {
+      if (ds->ws) {
+        e = cudaFree(ds->ws);  // synchronises the device
+        ds->ws = nullptr;
+        ds->ws_bytes = 0;
+        ds->count_cap = 0;
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFree(workspace)");
+      }
+      e = cudaMalloc(&ds->ws, need);
+      if (e != cudaSuccess) {
+        ds->ws = nullptr;
+        return cuda_fail(e, "cudaMalloc(workspace)");
+      }
+      ds->ws_bytes = need;
+      e = cudaMemsetAsync(ds->ws, 0, need, s);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+    }
+    // after the arrival counters of mode 1, which must keep their zeros
+    void* base = static_cast<char*>(ds->ws) + size_t(ds->count_cap) * 4;
+    scan_bind_workspace(call.a, plan, base);
+    return scan_launch(call, plan, base, s);
+  }
   if (plan.nseg > 1) {
     // The arrival counters keep a region of their own at the start of the
     // workspace, sized for the most row tiles seen so far: they start at zero
@@ -410,7 +482,7 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* del
     layout.count_bytes = size_t(ds->count_cap) * 4;
     scan_bind_workspace(call.a, layout, ds->ws);
   }
-  return scan_launch(call, plan, s);
+  return scan_launch(call, plan, ds->ws, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -454,7 +526,7 @@ mssm_status mssm_selective_scan_fwd_noalloc(const mssm_tensor* u, const mssm_ten
     g_noalloc_sms[dev] = v;
   }
   const ScanPlan plan = scan_plan(call, g_noalloc_sms[dev]);
-  if (plan.nseg > 1) {
+  if (plan.mode != 0) {
     const size_t need = plan.need();
     if (need > kNoAllocScratchBytes)
       return fail(MSSM_ERR_UNSUPPORTED,
@@ -469,12 +541,15 @@ mssm_status mssm_selective_scan_fwd_noalloc(const mssm_tensor* u, const mssm_ten
       if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
       g_noalloc_ptr[dev] = ptr;
     }
-    // The array keeps whatever the previous call left: zero the arrival counters.
-    e = cudaMemsetAsync(g_noalloc_ptr[dev], 0, plan.count_bytes, s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-allocation scratch counters)");
+    // The array keeps whatever the previous call left: zero the arrival
+    // counters (the chained schedule zeroes its own ticket and flags).
+    if (plan.mode == 1) {
+      e = cudaMemsetAsync(g_noalloc_ptr[dev], 0, plan.count_bytes, s);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-allocation scratch counters)");
+    }
     scan_bind_workspace(call.a, plan, g_noalloc_ptr[dev]);
   }
-  return scan_launch(call, plan, s);
+  return scan_launch(call, plan, g_noalloc_ptr[dev], s);
 }
 
 static mssm_status state_update_impl(mssm_tensor* state, const mssm_tensor* x, const mssm_tensor* dt_t,
@@ -557,7 +632,7 @@ mssm_status mssm_state_update_ex(mssm_tensor* state, const mssm_tensor* x, const
 }
 
 mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int* rows_per_cta,
-                           int64_t* chunk_len, int64_t* n_chunks) {
+                           int64_t* chunk_len, int64_t* n_chunks, int* schedule) {
   if (Bt < 0 || D < 0 || L < 0) return fail(MSSM_ERR_INVALID_ARG, "negative size");
   if (sm_count <= 0) {
     int dev = 0, v = 0;
@@ -575,6 +650,7 @@ mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int* 
   if (rows_per_cta) *rows_per_cta = sh.rows;
   if (chunk_len) *chunk_len = sh.seg;
   if (n_chunks) *n_chunks = sh.nseg;
+  if (schedule) *schedule = sh.mode;
   return MSSM_OK;
 }
 

@@ -7,7 +7,7 @@ __device__ unsigned int g_device_error = 0u;
 
 // Address of this device's copy of the error word, looked up once per device
 // (the caller serialises launches, so the cache needs no lock of its own).
-static cudaError_t error_word(unsigned int** out) {
+cudaError_t device_error_word(unsigned int** out) {
   static void* cache[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -23,7 +23,7 @@ static cudaError_t error_word(unsigned int** out) {
 
 template <typename T, bool HAS_Z>
 static cudaError_t launch_decode_t(DecodeArgs a, bool bulk, cudaStream_t s) {
-  cudaError_t e = error_word(&a.err);
+  cudaError_t e = device_error_word(&a.err);
   if (e != cudaSuccess) return e;
   const int64_t rows = int64_t(a.Bt) * a.D;
   const int64_t blocks = (rows + kDecodeThreads - 1) / kDecodeThreads;

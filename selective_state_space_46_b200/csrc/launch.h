@@ -12,6 +12,10 @@ namespace mssm {
 // rows: channels per CTA (32 or 64); the grid is (Bt * tiles_per_batch, nseg [- 1]).
 cudaError_t launch_scan_chunk_state(const ScanArgs& a, int rows, int dtype, bool softplus, cudaStream_t s);
 cudaError_t launch_scan_out(const ScanArgs& a, int rows, int dtype, bool has_z, bool softplus, cudaStream_t s);
+// Persistent chained forward kernel (32-row tiles), `grid` one-warp CTAs.
+cudaError_t launch_scan_chained(const ScanArgs& a, int grid, int dtype, bool has_z, bool softplus, cudaStream_t s);
+// Device address of this device's error word (cached per device).
+cudaError_t device_error_word(unsigned int** out);
 // bulk: the state is one contiguous [rows][16] range (bulk-copy kernel), else one thread per row.
 cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, bool bulk, cudaStream_t s);
 // Reads (and optionally clears) the current device's error word.

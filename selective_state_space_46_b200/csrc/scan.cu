@@ -17,6 +17,22 @@ static cudaError_t out_t(const ScanArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <typename T, bool HAS_Z, bool SP>
+static cudaError_t chained_t(const ScanArgs& a, int grid, cudaStream_t s) {
+  scan_out_chained_kernel<T, HAS_Z, SP><<<grid, 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t chained_d(const ScanArgs& a, int grid, bool has_z, bool sp, cudaStream_t s) {
+  if (has_z) return sp ? chained_t<T, true, true>(a, grid, s) : chained_t<T, true, false>(a, grid, s);
+  return sp ? chained_t<T, false, true>(a, grid, s) : chained_t<T, false, false>(a, grid, s);
+}
+
+cudaError_t launch_scan_chained(const ScanArgs& a, int grid, int dtype, bool has_z, bool sp, cudaStream_t s) {
+  return dtype == 1 ? chained_d<uint16_t>(a, grid, has_z, sp, s) : chained_d<float>(a, grid, has_z, sp, s);
+}
+
 template <typename T, int ROWS>
 static cudaError_t chunk_state_d(const ScanArgs& a, bool sp, cudaStream_t s) {
   return sp ? chunk_state_t<T, ROWS, true>(a, s) : chunk_state_t<T, ROWS, false>(a, s);

@@ -75,6 +75,11 @@ struct ScanArgs {
   float* ws_H;           // [nseg-1][rows_total][16]: chunk end state, then carried state
   float* ws_S;           // [nseg-1][rows_total]: sum of delta / ln2 over the chunk
   unsigned* ws_count;    // [Bt * tiles_per_batch]: kernel-1 arrivals, reset by the last one
+  // chained schedule (scan_out_chained_kernel), zeroed before each launch
+  unsigned* ch_ticket;   // work-item counter
+  unsigned* ch_flags;    // [tiles]: chunks of the tile whose carried state is published
+  float* ch_carry;       // [tiles * 32][16]: carried state between consecutive chunks
+  unsigned* err;         // device error word: bit 1 = a chained wait gave up
 };
 
 // ---------------------------------------------------------------------------
@@ -510,6 +515,121 @@ __global__ void __launch_bounds__(ROWS, ROWS == 32 ? 9 : 8) scan_out_kernel(cons
 #pragma unroll
       for (int n = 0; n < 16; ++n) dst[n] = v[n];
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Chained persistent forward kernel.
+//
+// For shapes with many row tiles, splitting L only to balance the work is
+// cheaper done by hand-over than by chunk summaries: work items are (tile,
+// chunk) pairs taken in chunk-major order from an atomic ticket by a grid of
+// persistent one-warp CTAs; an item starts from the state its tile's previous
+// chunk published (st.release / ld.acquire on a per-tile flag) and publishes
+// its own end state.  The grid is never larger than the number of tiles, so an
+// item's predecessor was taken at least a full grid's worth of items earlier
+// and has finished: the wait is a bound that is not expected to be reached.
+// If it is (kChainSpinLimit polls with nanosleep back-off), the item sets bit 1
+// of the device error word (mssm_get_error reports MSSM_ERR_TIMEOUT) and runs
+// from a zero state.  Every SM sub-partition then does the same amount of work
+// instead of the 3-versus-2 warps a fixed grid leaves on some of them.
+// ---------------------------------------------------------------------------
+constexpr int kChainSpinLimit = 1 << 20;
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+template <typename T, bool HAS_Z, bool SOFTPLUS>
+__global__ void __launch_bounds__(32, 8) scan_out_chained_kernel(const ScanArgs p) {
+  constexpr int ROWS = 32;
+  __shared__ __align__(16) float bc_s[2][kTC * 32];
+  __shared__ __align__(16) uint4 slots[kStages * 3 * ROWS];
+  __shared__ int s_item;
+  __shared__ int s_ok;
+  const int tid = threadIdx.x;
+  const int ntiles = p.Bt * p.tiles_per_batch;
+  const int nitems = ntiles * p.nseg;
+  for (;;) {
+    if (tid == 0) s_item = int(atomicAdd(p.ch_ticket, 1u));
+    __syncthreads();
+    const int item = s_item;
+    if (item >= nitems) break;
+    const int c = item / ntiles;
+    const int tile = item - c * ntiles;
+    const int b = tile / p.tiles_per_batch;
+    const int d = (tile - b * p.tiles_per_batch) * ROWS + tid;
+    const bool row_ok = d < p.D;
+    const int dc = row_ok ? d : p.D - 1;
+    const int t0 = c * p.seg_len;
+    const int t1 = min(p.L, t0 + p.seg_len);
+    const T* urow = static_cast<const T*>(p.u) + int64_t(b) * p.u_sb + int64_t(dc) * p.u_sd;
+    const T* dlrow = static_cast<const T*>(p.delta) + int64_t(b) * p.dl_sb + int64_t(dc) * p.dl_sd;
+    const T* zrow = HAS_Z ? static_cast<const T*>(p.z) + int64_t(b) * p.z_sb + int64_t(dc) * p.z_sd : nullptr;
+    T* orow = static_cast<T*>(p.out) + int64_t(b) * p.o_sb + int64_t(dc) * p.o_sd;
+    RowParams rp;
+    const bool st = load_row_params<ROWS>(p, dc, rp);
+
+    f2_t h2[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) h2[k] = 0ull;
+    if (c > 0) {
+      if (tid == 0) {
+        unsigned v = ld_acquire_u32(p.ch_flags + tile);
+        for (int it = 0; v < unsigned(c) && it < kChainSpinLimit; ++it) {
+          __nanosleep(64);
+          v = ld_acquire_u32(p.ch_flags + tile);
+        }
+        s_ok = v >= unsigned(c);
+        if (!s_ok) atomicOr(p.err, 2u);
+      }
+      __syncthreads();
+      if (s_ok) {
+        const float4* src = reinterpret_cast<const float4*>(p.ch_carry + (int64_t(tile) * ROWS + tid) * kN);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 v = __ldcg(src + i);
+          h2[2 * i] = f2(v.x, v.y);
+          h2[2 * i + 1] = f2(v.z, v.w);
+        }
+      }
+    }
+    const bool structured = __syncthreads_and(st) && !p.force_general;
+    if (structured)
+      forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, true>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
+                                                    row_ok, rp, h2);
+    else
+      forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, false>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
+                                                     row_ok, rp, h2);
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) f2split(h2[k], v[2 * k], v[2 * k + 1]);
+    if (c == p.nseg - 1) {
+      if (row_ok && p.last_state) {
+        float* dst = p.last_state + int64_t(b) * p.ls_sb + int64_t(d) * p.ls_sd;
+        if (p.vec_ls) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        } else {
+#pragma unroll
+          for (int n = 0; n < 16; ++n) dst[n] = v[n];
+        }
+      }
+    } else {
+      float4* dst = reinterpret_cast<float4*>(p.ch_carry + (int64_t(tile) * ROWS + tid) * kN);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) __stcg(dst + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) st_release_u32(p.ch_flags + tile, unsigned(c + 1));
+    }
+    __syncthreads();
   }
 }
 

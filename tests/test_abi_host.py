@@ -177,27 +177,28 @@ def test_scan_plan_host_only(lib):
     """The launch plan is host logic: check its invariants without a GPU."""
     f = lib.mssm_scan_plan
     f.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
-                  ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)]
-    rows, seg, nseg = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int64()
+                  ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int)]
+    rows, seg, nseg, sched = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int()
     for Bt, D, L in [(1, 64, 256), (2, 1536, 2048), (8, 5120, 4096), (1, 2048, 131072), (3, 7, 1), (1, 1, 0),
                      (64, 8192, 100), (1, 16, 1 << 24)]:
-        assert f(Bt, D, L, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg)) == 0
+        assert f(Bt, D, L, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg), ctypes.byref(sched)) == 0
         assert rows.value in (32, 64)
         assert seg.value % 64 == 0 and seg.value >= 64
         assert nseg.value >= 1 and nseg.value <= 65535
+        assert sched.value in (0, 1, 2) and (sched.value == 0) == (nseg.value == 1)
         if L > 0:
             # the chunks cover the sequence exactly: every chunk but the last is full
             assert (nseg.value - 1) * seg.value < L <= nseg.value * seg.value
-    # a shape whose rows fill the GPU is not split
-    assert f(8, 5120, 4096, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg)) == 0
-    assert nseg.value == 1
+    # a shape with many row tiles runs its chunks chained, without summaries
+    assert f(8, 5120, 4096, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg), ctypes.byref(sched)) == 0
+    assert sched.value == 2 and rows.value == 32
     # few rows and a long sequence are split
-    assert f(1, 2048, 131072, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg)) == 0
-    assert nseg.value > 1
+    assert f(1, 2048, 131072, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg), ctypes.byref(sched)) == 0
+    assert nseg.value > 1 and sched.value == 1
     # an explicit chunk length is honoured
     lib.mssm_set_option.argtypes = [ctypes.c_int, ctypes.c_int64]
     assert lib.mssm_set_option(2, 128) == 0
-    assert f(1, 64, 1000, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg)) == 0
+    assert f(1, 64, 1000, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg), ctypes.byref(sched)) == 0
     assert (seg.value, nseg.value) == (128, 8)
     assert lib.mssm_set_option(2, 0) == 0
-    assert f(-1, 64, 1000, 148, None, None, None) == INVALID
+    assert f(-1, 64, 1000, 148, None, None, None, None) == INVALID

@@ -168,6 +168,23 @@ def test_workspace_reuse_across_tile_counts():
         compare_full(synth.make_scan_inputs(Bt, D, L, io_dtype="bf16", seed=seed))
 
 
+@pytest.mark.parametrize("io,chunk,structured,L", [
+    ("bf16", 0, True, 1000), ("bf16", 64, True, 777), ("f32", 128, False, 640), ("bf16", 256, False, 1024),
+])
+def test_chained_schedule(io, chunk, structured, L):
+    """Many row tiles: the persistent kernel hands each tile's state from chunk to chunk."""
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, chunk)
+    Bt, D = 2, 9600                      # 600 tiles of 32 rows
+    plan = m.mssm_scan_plan(Bt, D, L)
+    assert plan["schedule"] == "chained", plan
+    inp = synth.make_scan_inputs(Bt, D, L, io_dtype=io, seed=L + chunk, delta_range=(1e-4, 1e-2))
+    if not structured:
+        inp.A = random_A(D, 3)
+    compare_full(inp)
+    m.mssm_get_error()                   # no bounded wait gave up
+
+
 def test_long_slow_decay_many_chunks():
     inp = synth.make_scan_inputs(1, 64, 16384, io_dtype="bf16", seed=5, delta_range=(1e-4, 1e-2))
     compare_full(inp)

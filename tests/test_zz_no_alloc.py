@@ -72,3 +72,16 @@ def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
         assert "scratch" in str(e.value)
     finally:
         m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
+
+
+def test_noalloc_chained_schedule_matches(cuda_device):
+    """A shape with many row tiles uses the chained schedule; its hand-over state
+    also lives in the fixed scratch."""
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
+    inp = synth.make_scan_inputs(2, 9600, 1000, io_dtype="bf16", seed=6)
+    assert m.mssm_scan_plan(inp.batch, inp.dim, inp.length)["schedule"] == "chained"
+    for _ in range(2):
+        (y_ref, h_ref), (y_na, h_na) = _scan_both(inp, m)
+        _close(y_na, y_ref, inp.io_dtype)
+        _close(h_na, h_ref, inp.io_dtype)
