@@ -6,10 +6,14 @@ One step is one pass of the hot path over one batch of synthetic input:
 for the scan workloads, one mssm_selective_scan_fwd call (softplus,
 discretisation, recurrence, readout, D skip, gate, store, final state); for the
 decode workload, one mssm_state_update call.  Inputs are resident in HBM when
-the timed region starts; the L2 is flushed (a 256 MiB write) before every timed
-step, outside the step's event bracket.  The K timed steps are captured into one
-CUDA graph (flush, start event, step, end event per step) so host launch
-overhead cannot leak into a step's device time.
+the timed region starts.  The timed steps rotate through enough copies of the
+workload's buffers to cover 4x the L2 (one copy when a single set is that
+large), so no step finds its inputs in L2 and the write-back of one step's
+dirty lines is paid inside the steps that follow; only a workload too small for
+that (over 16 copies) flushes the L2 (a 256 MiB write) before each step
+instead, outside the step's event bracket.  The K timed steps are captured into
+one CUDA graph (start event, step, end event per step) so host launch overhead
+cannot leak into a step's device time.
 
 Multi-GPU (``torchrun --nproc-per-node N bench.py --gpus N``): rows of the scan
 are independent, so every rank runs its own batch of the same shape (weak
@@ -82,6 +86,48 @@ def scan_algorithmic_bytes(batch, dim, length, io_bytes, has_z=True, has_D=True,
     return b
 
 
+FP32_LANES_PER_SM = 128      # FP32 FMA lanes per SM (4 sub-partitions x 32)
+FLOP_PER_STATE = 6           # per (element, state): decay multiply, (delta u) B_n multiply,
+                             # FMA of the state update, FMA of the readout (an FMA = 2 flop)
+
+
+def algorithmic_flops(units: int) -> int:
+    """FP32 flops the method needs per scan element or decode row: 16 states x 6
+    (transcendentals, which run on the SFU, are not counted)."""
+    return units * N_STATE * FLOP_PER_STATE
+
+
+def fp32_peak_tflops(sm_count: int, sm_mhz: float) -> float:
+    """FP32 FMA-pipe peak from unit counts and clock: SMs x 128 lanes x 2 flop x clock."""
+    return sm_count * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+
+
+def binding_roofline(alg_bytes: float, alg_flops: float, ms: float, hbm_gbs: float, alu_tflops: float) -> dict:
+    """Roofline of one launch: the bound is whichever of HBM bytes / peak bandwidth and
+    FP32 flops / peak FLOP rate takes longer; achieved and frac are against that bound,
+    the other bound's fraction is kept beside it."""
+    t_hbm = alg_bytes / (hbm_gbs * 1e9)
+    t_alu = alg_flops / (alu_tflops * 1e12)
+    gbs = alg_bytes / (ms / 1e3) / 1e9
+    tfl = alg_flops / (ms / 1e3) / 1e12
+    hbm = {"achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs}
+    alu = {"achieved": tfl, "peak": alu_tflops, "unit": "TFLOP/s", "frac": tfl / alu_tflops}
+    if t_alu > t_hbm:
+        return {"bound": "alu", **alu, "other": {"bound": "hbm", **hbm}}
+    return {"bound": "hbm", **hbm, "other": {"bound": "alu", **alu}}
+
+
+def ring_size(set_bytes: int, l2_bytes: int, max_sets: int = 16) -> int:
+    """Number of input/output buffer sets the timed steps rotate through so that no
+    step finds its data in L2: one set when a set alone is 4x the L2, else enough sets
+    to cover 4x the L2; 0 (flush the L2 between steps instead) if that needs more than
+    max_sets."""
+    if set_bytes >= 4 * l2_bytes:
+        return 1
+    r = -(-4 * l2_bytes // max(set_bytes, 1))
+    return r if r <= max_sets else 0
+
+
 def decode_algorithmic_bytes(batch, dim, io_bytes, has_z=True, has_D=True) -> int:
     """Per decode step: state read + write (fp32), x, dt, (z), y per row; B, C per batch; A, D per channel."""
     rows = batch * dim
@@ -102,18 +148,37 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def max_sm_mhz(default: float = 1965.0) -> float:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["sm_max_mhz"])
+    except Exception:
+        return default
+
+
+KERNEL_SOURCES = {
+    "scan_out": ("device_common.cuh", "scan.cuh", "scan.cu"),
+    "scan_chunk_state": ("device_common.cuh", "scan.cuh", "scan.cu"),
+    "state_update": ("device_common.cuh", "decode.cuh", "decode.cu"),
+}
+
+
+def kernel_source_hash(kernel: str | None = None) -> str:
+    """Hash of the device sources a kernel is built from (all of csrc/ when kernel is None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_46_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    names = KERNEL_SOURCES.get(kernel) if kernel else None
+    for name in sorted(names or os.listdir(csrc)):
         if name.endswith((".cu", ".cuh", ".h")):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current sources."""
+def recorded_traffic(kernel: str, workload: str, plan: str | None = None):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    kernel's current sources (and, for a scan, the same launch plan)."""
     p = os.path.join(ROOT, "profiles", f"traffic_{kernel}_{workload}.txt")
     if not os.path.exists(p):
         return None, None
@@ -122,11 +187,21 @@ def recorded_traffic(kernel: str, workload: str):
     m_h = re.search(r"source_hash\s*=\s*([0-9a-f]+)", text)
     if not m_b or not m_h:
         return None, None
-    if m_h.group(1) != kernel_source_hash():
-        return None, "stale"
+    if m_h.group(1) != kernel_source_hash(kernel):
+        return None, "stale: kernel sources changed since the capture"
+    m_p = re.search(r"plan\s*=\s*(.+)", text)
+    if plan is not None and (not m_p or m_p.group(1).strip() != plan):
+        return None, "stale: launch plan changed since the capture"
     scale = re.search(r"scale_to_full\s*=\s*([0-9.eE+]+)", text)
     val = float(m_b.group(1)) * (float(scale.group(1)) if scale else 1.0)
     return val, os.path.relpath(p, ROOT)
+
+
+def plan_string(plan: dict | None) -> str | None:
+    if not plan:
+        return None
+    return (f"{plan['schedule']} rows_per_cta={plan['rows_per_cta']} chunk_len={plan['chunk_len']} "
+            f"n_chunks={plan['n_chunks']}")
 
 
 class ClockSampler:
@@ -303,22 +378,29 @@ def run_mssm(args):
     seed = rank_seed(rank)
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, args.chunk_len)
     m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 1 if args.general_a else 0)
+    m.mssm_set_option(m.MSSM_OPT_DECODE_PATH, m.DECODE_PATHS.get(args.decode_path, 0))
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    props = torch.cuda.get_device_properties(dev)
+    l2_bytes = int(getattr(props, "L2_cache_size", 0) or (126 << 20))
     if kind == "scan":
         inp = synth.workload_inputs(args.workload, seed=seed)
         host = {k: getattr(inp, k) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
-        d = {k: to_dev(v) for k, v in host.items()}
-        out = torch.empty_like(d["u"])
-        last = torch.empty(inp.batch, inp.dim, N_STATE, device=dev)
         units = inp.batch * inp.dim * inp.length
         alg_bytes = scan_algorithmic_bytes(inp.batch, inp.dim, inp.length, io_bytes, inp.z is not None,
                                            inp.D is not None, inp.delta_bias is not None)
+        nsets = ring_size(alg_bytes, l2_bytes)
+        d = {k: to_dev(v) for k, v in host.items()}
+        sets = []
+        for k in range(max(nsets, 1)):
+            dk = d if k == 0 else {**d, **{n: d[n].clone() for n in ("u", "delta", "B", "C", "z") if d[n] is not None}}
+            sets.append((dk, torch.empty_like(d["u"]), torch.empty(inp.batch, inp.dim, N_STATE, device=dev)))
 
-        def step():
-            m.mssm_selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
-                                      d["delta_bias"], inp.softplus, out, last)
+        def step(k=0):
+            dk, out_k, last_k = sets[k % len(sets)]
+            m.mssm_selective_scan_fwd(dk["u"], dk["delta"], dk["A"], dk["B"], dk["C"], dk["D"], dk["z"],
+                                      dk["delta_bias"], inp.softplus, out_k, last_k)
         config = {"workload": args.workload, "batch": inp.batch, "channels": inp.dim, "length": inp.length,
                   "state": N_STATE, "io_dtype": inp.io_dtype, "gate": inp.z is not None,
                   "softplus_bias": inp.delta_bias is not None, "D_skip": inp.D is not None,
@@ -328,30 +410,44 @@ def run_mssm(args):
                   "plan": m.mssm_scan_plan(inp.batch, inp.dim, inp.length)}
         metric, unit = METRIC, "elems/s"
         dom_kernel = "scan_out"
+        set_bytes = alg_bytes
     else:
         ring = [synth.workload_inputs(args.workload, seed=seed, step_stream=k) for k in range(8)]
         inp = ring[0]
-        state = to_dev(inp.state)
-        A_d, D_d = to_dev(inp.A), to_dev(inp.D)
-        dring = [{k: to_dev(getattr(r, k)) for k in ("x", "dt", "B", "C", "z")} for r in ring]
-        out = torch.empty_like(dring[0]["x"])
         units = inp.batch * inp.dim
         alg_bytes = decode_algorithmic_bytes(inp.batch, inp.dim, io_bytes, inp.z is not None, inp.D is not None)
-        counter = [0]
+        # footprint of one step: the state once (read and written in place), the per-row inputs and y
+        set_bytes = units * N_STATE * 4 + units * io_bytes * (4 if inp.z is not None else 3)
+        nsets = ring_size(set_bytes, l2_bytes)
+        state0 = to_dev(inp.state)
+        states = [state0] + [state0.clone() for _ in range(max(nsets, 1) - 1)]
+        A_d, D_d = to_dev(inp.A), to_dev(inp.D)
+        dring = [{k: to_dev(getattr(r, k)) for k in ("x", "dt", "B", "C", "z")} for r in ring]
+        outs = [torch.empty_like(dring[0]["x"]) for _ in states]
 
-        def step():
-            r = dring[counter[0] % 8]
-            counter[0] += 1
-            m.mssm_state_update(state, r["x"], r["dt"], A_d, r["B"], r["C"], D_d, r["z"], out)
+        def step(k=0):
+            r = dring[k % len(dring)]
+            j = k % len(states)
+            m.mssm_state_update(states[j], r["x"], r["dt"], A_d, r["B"], r["C"], D_d, r["z"], outs[j])
         config = {"workload": args.workload, "batch": inp.batch, "channels": inp.dim, "state": N_STATE,
-                  "io_dtype": inp.io_dtype, "input_ring": 8, "state_in_place": True}
+                  "io_dtype": inp.io_dtype, "input_ring": len(dring), "state_in_place": True,
+                  "decode_path": args.decode_path}
         metric, unit = DECODE_METRIC, "rows/s"
         dom_kernel = "state_update"
+    flush_between = nsets == 0
+    if flush_between:
+        l2_note = "flushed before every timed step (256 MiB write, outside the step's events)"
+    else:
+        l2_note = (f"not flushed: the steps rotate through {max(nsets, 1)} buffer set(s) of "
+                   f"{set_bytes / 1e6:.1f} MB ({max(nsets, 1) * set_bytes / 1e6:.0f} MB >= 4x the "
+                   f"{l2_bytes / 2**20:.0f} MiB L2), so no step finds its data in L2, and the write-back "
+                   "of a step's dirty lines falls inside the following steps' timed regions")
 
     # ---- warm-up (also allocates the library's carry workspace before capture)
-    for _ in range(max(args.warmup, 3)):
-        flush.zero_()
-        step()
+    for k in range(max(args.warmup, 3)):
+        if flush_between:
+            flush.zero_()
+        step(k)
     torch.cuda.synchronize(dev)
     m.mssm_get_error()
 
@@ -363,9 +459,10 @@ def run_mssm(args):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for k in range(args.steps):
-            flush.zero_()
+            if flush_between:
+                flush.zero_()
             starts[k].record()
-            step()
+            step(k)
             ends[k].record()
     after = m.mssm_kernel_stats()
     launches = sum(after[k]["launches"] - before[k]["launches"] for k in after)
@@ -394,9 +491,10 @@ def run_mssm(args):
     # ---- per-kernel durations (same launches, events bracketing each kernel)
     m.mssm_set_option(m.MSSM_OPT_KERNEL_TIMING, 1)
     m.mssm_kernel_stats(reset=True)
-    for _ in range(args.steps):
-        flush.zero_()
-        step()
+    for k in range(args.steps):
+        if flush_between:
+            flush.zero_()
+        step(k)
     torch.cuda.synchronize(dev)
     ks = m.mssm_kernel_stats(reset=True)
     m.mssm_set_option(m.MSSM_OPT_KERNEL_TIMING, 0)
@@ -406,12 +504,16 @@ def run_mssm(args):
     dom = kern.get(dom_kernel)
     peak, peak_kind = measured_peaks()
     dom_ms = dom["ms_per_launch"] if dom else None
-    achieved = alg_bytes / (dom_ms / 1e3) / 1e9 if dom_ms else None
-    traffic, traffic_src = recorded_traffic(dom_kernel, args.workload)
-    roofline = {"bound": "hbm", "kernel": dom_kernel, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": (achieved / peak) if achieved else None, "peak_source": peak_kind,
-                "algorithmic_bytes_per_launch": alg_bytes,
-                "traffic": traffic, "traffic_source": traffic_src}
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    alu_peak = fp32_peak_tflops(sms, max_sm_mhz())
+    alg_flops = algorithmic_flops(units)
+    traffic, traffic_src = recorded_traffic(dom_kernel, args.workload, plan_string(config.get("plan")))
+    roofline = binding_roofline(alg_bytes, alg_flops, dom_ms, peak, alu_peak) if dom_ms else {"bound": None}
+    roofline.update({"kernel": dom_kernel, "ms_per_launch": dom_ms,
+                     "peak_source": f"HBM: {peak_kind} copy rate; FP32: {sms} SMs x 128 lanes x 2 x "
+                                    f"{max_sm_mhz():.0f} MHz",
+                     "algorithmic_bytes_per_launch": alg_bytes, "algorithmic_flops_per_launch": alg_flops,
+                     "traffic": traffic, "traffic_source": traffic_src})
 
     # ---- end to end: host buffers in pinned memory, copies inside the timed region
     e2e = None
@@ -423,7 +525,7 @@ def run_mssm(args):
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; no datasets or weights)",
-        "config": {**config, "l2": "flushed before every timed step (256 MiB write)",
+        "config": {**config, "l2": l2_note,
                    "parallelism": f"replicas x{world} (independent rows, no collective)",
                    "timing": "CUDA events per step inside one captured graph"},
         "hbm_gbs": step_gbs * world, "hbm_gbs_per_gpu": step_gbs,
@@ -521,6 +623,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--chunk-len", type=int, default=0, help="length split (0: automatic; multiple of 64)")
+    ap.add_argument("--decode-path", choices=["auto", "stream", "bulk_tile", "per_row"], default="auto",
+                    help="decode kernel (MSSM_OPT_DECODE_PATH)")
     ap.add_argument("--general-a", action="store_true",
                     help="disable the structured-A path (one exponential per state)")
     args = ap.parse_args(argv)

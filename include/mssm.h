@@ -200,14 +200,25 @@ mssm_status mssm_get_error(void *stream);
  *   MSSM_OPT_CHUNK_LEN (value 0, or a positive multiple of 64): length of the
  *     chunks a sequence is split into (a value >= L means no split); 0 restores
  *     the automatic choice.
+ *   MSSM_OPT_SCHEDULE (value 0..3): 0 automatic; otherwise force a schedule of
+ *     mssm_scan_plan (value = schedule + 1: 1 forward only, no split; 2 summaries
+ *     + forward; 3 chained).  A forced split schedule needs L > 64; otherwise the
+ *     plan falls back to forward only.
  *   MSSM_OPT_KERNEL_TIMING (value 0/1): when 1, every kernel launch is bracketed
  *     by two CUDA events recorded on the caller's stream (see mssm_kernel_stats).
+ *   MSSM_OPT_DECODE_PATH (value 0..3): the state-update kernel.  0 automatic
+ *     (2 when the state is one contiguous, 16-byte aligned [Bt, D, 16] range,
+ *     else 3); 1 persistent streaming kernel (a ring of bulk-copied tiles per
+ *     CTA); 2 one bulk-copied tile per CTA; 3 one thread per row, any layout.
+ *     1 and 2 need the contiguous layout and fall back to 3 without it.
  * Unknown options or invalid values return MSSM_ERR_INVALID_ARG.
  */
 typedef enum {
     MSSM_OPT_FORCE_GENERAL_A = 1,
     MSSM_OPT_CHUNK_LEN = 2,
-    MSSM_OPT_KERNEL_TIMING = 3
+    MSSM_OPT_KERNEL_TIMING = 3,
+    MSSM_OPT_SCHEDULE = 4,
+    MSSM_OPT_DECODE_PATH = 5
 } mssm_option;
 mssm_status mssm_set_option(int option, int64_t value);
 

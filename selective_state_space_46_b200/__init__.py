@@ -21,7 +21,8 @@ __all__ = [
     "mssm_state_update_ex",
     "mssm_get_error", "mssm_set_option", "mssm_shutdown", "mssm_version", "mssm_status_string",
     "mssm_last_error", "selective_scan_fwd", "state_update", "lib_path",
-    "MSSM_OPT_FORCE_GENERAL_A", "MSSM_OPT_CHUNK_LEN", "MSSM_OPT_KERNEL_TIMING", "mssm_kernel_stats", "mssm_scan_plan",
+    "MSSM_OPT_FORCE_GENERAL_A", "MSSM_OPT_CHUNK_LEN", "MSSM_OPT_KERNEL_TIMING", "MSSM_OPT_SCHEDULE", "SCHEDULES",
+    "MSSM_OPT_DECODE_PATH", "DECODE_PATHS", "mssm_kernel_stats", "mssm_scan_plan",
     "KERNEL_KINDS",
 ]
 
@@ -34,7 +35,10 @@ _lib = ctypes.CDLL(lib_path)
 
 MSSM_F32, MSSM_BF16 = 0, 1
 MSSM_OK, MSSM_ERR_INVALID_ARG, MSSM_ERR_UNSUPPORTED, MSSM_ERR_CUDA, MSSM_ERR_TIMEOUT = 0, 1, 2, 3, 4
-MSSM_OPT_FORCE_GENERAL_A, MSSM_OPT_CHUNK_LEN, MSSM_OPT_KERNEL_TIMING = 1, 2, 3
+MSSM_OPT_FORCE_GENERAL_A, MSSM_OPT_CHUNK_LEN, MSSM_OPT_KERNEL_TIMING, MSSM_OPT_SCHEDULE = 1, 2, 3, 4
+MSSM_OPT_DECODE_PATH = 5
+SCHEDULES = {"forward": 1, "summaries+forward": 2, "chained": 3}
+DECODE_PATHS = {"stream": 1, "bulk_tile": 2, "per_row": 3}
 KERNEL_KINDS = ("scan_chunk_state", "scan_out", "state_update")
 
 

@@ -1,6 +1,7 @@
 // C ABI of libmssm.so: argument validation, dtype/shape dispatch, the carry
 // workspace, status codes.  Every compute step runs in the kernels of scan.cu
 // and decode.cu; nothing here touches tensor contents on the host.
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -34,6 +35,8 @@ mssm_status cuda_fail(cudaError_t e, const char* what) {
 std::mutex g_mu;
 int g_force_general = 0;
 int64_t g_chunk_len = 0;
+int g_schedule = -1;
+int g_decode_path = 0;  // MSSM_OPT_DECODE_PATH  // -1 automatic, else the forced LaunchShape mode
 
 // ---- launch accounting and optional per-kernel event timing (diagnostics)
 int64_t g_launches[MSSM_KERNEL_KINDS] = {0, 0, 0};
@@ -158,7 +161,7 @@ int64_t round_seg(int64_t v) {
 // chained work item kItem, and the carry fold kFold per chunk.  Grid kernels
 // run their CTAs in waves of at most kMaxCta per SM (register limited) and
 // put ceil(warps / 4) warps on the busiest SMSP.
-LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forced_seg) {
+LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forced_seg, int forced_mode) {
   constexpr double kOut = 96.0, kSum = 55.0, kIpc1 = 0.6, kIpc2 = 0.7;
   constexpr double kStart = 4000.0, kLaunch = 6000.0, kItem = 4000.0, kFold = 200.0;
   auto ipc = [&](int64_t k) { return k <= 1 ? kIpc1 : kIpc2; };
@@ -172,7 +175,9 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
   };
   LaunchShape best{0, 32, L > 0 ? L : 1, 1, 0};
   double best_cost = -1.0;
+  if (forced_mode == 0) return LaunchShape{0, 32, L > 0 ? L : 1, 1, 0};
   auto consider = [&](const LaunchShape& sh, double cost) {
+    if (forced_mode > 0 && sh.mode != forced_mode) return;
     if (best_cost < 0.0 || cost < best_cost * 0.999) {
       best_cost = cost;
       best = sh;
@@ -191,6 +196,9 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
       if (nseg > 1) cost += grid_time(tiles * (nseg - 1), rows, double(seg), kSum) + kFold * double(nseg);
       consider(LaunchShape{nseg > 1 ? 1 : 0, rows, seg, nseg, 0}, cost);
       // chained: 32-row tiles, at most 8 one-warp CTAs per SM and never more CTAs than tiles
+      if (rows == 32 && nseg > 1 && forced_mode == 2 && tiles < 4 * int64_t(sms)) {
+        consider(LaunchShape{2, 32, seg, nseg, int(std::min<int64_t>(tiles, 8 * int64_t(sms)))}, 0.0);
+      }
       if (rows == 32 && nseg > 1) {
         const int64_t per_sm = tiles / sms < 8 ? tiles / sms : 8;
         if (per_sm >= 4) {
@@ -238,6 +246,14 @@ mssm_status mssm_set_option(int option, int64_t value) {
       if (value < 0 || value % mssm::kSegQuant != 0 || value > (int64_t(1) << 30))
         return fail(MSSM_ERR_INVALID_ARG, "CHUNK_LEN must be 0 or a positive multiple of %d", mssm::kSegQuant);
       g_chunk_len = value;
+      return MSSM_OK;
+    case MSSM_OPT_SCHEDULE:
+      if (value < 0 || value > 3) return fail(MSSM_ERR_INVALID_ARG, "SCHEDULE takes 0 (automatic) to 3");
+      g_schedule = int(value) - 1;
+      return MSSM_OK;
+    case MSSM_OPT_DECODE_PATH:
+      if (value < 0 || value > 3) return fail(MSSM_ERR_INVALID_ARG, "DECODE_PATH takes 0 (automatic) to 3");
+      g_decode_path = int(value);
       return MSSM_OK;
     case MSSM_OPT_KERNEL_TIMING:
       if (value != 0 && value != 1) return fail(MSSM_ERR_INVALID_ARG, "KERNEL_TIMING takes 0 or 1");
@@ -340,7 +356,7 @@ struct ScanPlan {
 ScanPlan scan_plan(ScanCall& call, int sm_count) {
   mssm::ScanArgs& a = call.a;
   a.force_general = g_force_general;
-  const LaunchShape shape = choose_shape(call.Bt, call.D, call.L, sm_count, g_chunk_len);
+  const LaunchShape shape = choose_shape(call.Bt, call.D, call.L, sm_count, g_chunk_len, g_schedule);
   ScanPlan plan;
   plan.mode = shape.mode;
   plan.rows_per_cta = shape.rows;
@@ -370,6 +386,7 @@ void scan_bind_workspace(mssm::ScanArgs& a, const ScanPlan& plan, void* ws) {
     a.ch_carry = reinterpret_cast<float*>(base + plan.count_bytes);
     return;
   }
+
   a.ws_count = reinterpret_cast<unsigned*>(base);
   a.ws_S = reinterpret_cast<float*>(base + plan.count_bytes);
   a.ws_H = reinterpret_cast<float*>(base + plan.count_bytes + plan.s_bytes);
@@ -584,7 +601,7 @@ static mssm_status state_update_impl(mssm_tensor* state, const mssm_tensor* x, c
   }
   if (same_ptr(out, state)) return fail(MSSM_ERR_INVALID_ARG, "out must not alias state");
   if (Bt == 0 || Dd == 0) return MSSM_OK;
-  if (Bt * Dd / 256 + 1 > int64_t(INT32_MAX)) return fail(MSSM_ERR_UNSUPPORTED, "too many rows for one launch");
+  if (Bt * Dd > int64_t(INT32_MAX)) return fail(MSSM_ERR_UNSUPPORTED, "Bt * D must fit in 31 bits");
 
   mssm::DecodeArgs a{};
   a.state = static_cast<float*>(state->data);
@@ -607,12 +624,16 @@ static mssm_status state_update_impl(mssm_tensor* state, const mssm_tensor* x, c
   a.vec_BC = aligned16(B->data) && aligned16(C->data) && B->stride[1] == 1 && C->stride[1] == 1 &&
              (B->stride[0] * es) % 16 == 0 && (C->stride[0] * es) % 16 == 0;
 
-  // one contiguous [rows][16] state range, 16-byte aligned: the bulk-copy kernel
-  const bool bulk = aligned16(state->data) && state->stride[1] == mssm::kN && state->stride[0] == Dd * mssm::kN;
+  // one contiguous [rows][16] state range, 16-byte aligned: the bulk-copy kernels
+  const bool contiguous = aligned16(state->data) && state->stride[1] == mssm::kN && state->stride[0] == Dd * mssm::kN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lk(g_mu);
+  mssm::DecodePath path = mssm::DecodePath::kPerRow;
+  if (contiguous)
+    path = g_decode_path == 1 ? mssm::DecodePath::kStream
+         : g_decode_path == 3 ? mssm::DecodePath::kPerRow : mssm::DecodePath::kBulkTile;
   cudaError_t e = tracked(MSSM_KERNEL_STATE_UPDATE, s,
-                          [&] { return mssm::launch_state_update(a, dt, z != nullptr, bulk, s); });
+                          [&] { return mssm::launch_state_update(a, dt, z != nullptr, path, s); });
   if (e != cudaSuccess) return cuda_fail(e, "state update launch");
   return MSSM_OK;
 }
@@ -646,7 +667,12 @@ mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int* 
     std::lock_guard<std::mutex> lk(g_mu);
     forced = g_chunk_len;
   }
-  const LaunchShape sh = choose_shape(Bt, D, L, sm_count, forced);
+  int forced_mode;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    forced_mode = g_schedule;
+  }
+  const LaunchShape sh = choose_shape(Bt, D, L, sm_count, forced, forced_mode);
   if (rows_per_cta) *rows_per_cta = sh.rows;
   if (chunk_len) *chunk_len = sh.seg;
   if (n_chunks) *n_chunks = sh.nseg;

@@ -21,22 +21,60 @@ cudaError_t device_error_word(unsigned int** out) {
   return cudaSuccess;
 }
 
+// SM count and the streaming kernels' shared-memory opt-in, once per device
+static cudaError_t stream_setup(int* sms) {
+  static int sm_cache[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!sm_cache[dev]) {
+    int v = 0;
+    e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int bytes = kStreamBufs * kStreamTileBytes;
+    if ((e = cudaFuncSetAttribute(state_update_stream_kernel<uint16_t, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(state_update_stream_kernel<uint16_t, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(state_update_stream_kernel<float, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(state_update_stream_kernel<float, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess)
+      return e;
+    sm_cache[dev] = v;
+  }
+  *sms = sm_cache[dev];
+  return cudaSuccess;
+}
+
 template <typename T, bool HAS_Z>
-static cudaError_t launch_decode_t(DecodeArgs a, bool bulk, cudaStream_t s) {
+static cudaError_t launch_decode_t(DecodeArgs a, DecodePath path, cudaStream_t s) {
   cudaError_t e = device_error_word(&a.err);
   if (e != cudaSuccess) return e;
   const int64_t rows = int64_t(a.Bt) * a.D;
   const int64_t blocks = (rows + kDecodeThreads - 1) / kDecodeThreads;
-  if (bulk)
+  if (path == DecodePath::kStream) {
+    int sms = 0;
+    if ((e = stream_setup(&sms)) != cudaSuccess) return e;
+    // as many CTAs as fit, with the tile count per CTA balanced: every CTA gets
+    // ceil(tiles / slots) tiles except the last, which gets what remains
+    const int64_t slots = int64_t(sms) * kStreamCtasPerSm;
+    const int64_t per = (blocks + slots - 1) / slots;
+    const int64_t grid = (blocks + per - 1) / per;
+    state_update_stream_kernel<T, HAS_Z>
+        <<<unsigned(grid), kDecodeThreads, kStreamBufs * kStreamTileBytes, s>>>(a);
+  } else if (path == DecodePath::kBulkTile) {
     state_update_bulk_kernel<T, HAS_Z><<<unsigned(blocks), kDecodeThreads, 0, s>>>(a);
-  else
+  } else {
     state_update_kernel<T, HAS_Z><<<unsigned(blocks), kDecodeThreads, 0, s>>>(a);
+  }
   return cudaGetLastError();
 }
 
-cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, bool bulk, cudaStream_t s) {
-  if (dtype == 1) return has_z ? launch_decode_t<uint16_t, true>(a, bulk, s) : launch_decode_t<uint16_t, false>(a, bulk, s);
-  return has_z ? launch_decode_t<float, true>(a, bulk, s) : launch_decode_t<float, false>(a, bulk, s);
+cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, DecodePath path, cudaStream_t s) {
+  if (dtype == 1) return has_z ? launch_decode_t<uint16_t, true>(a, path, s) : launch_decode_t<uint16_t, false>(a, path, s);
+  return has_z ? launch_decode_t<float, true>(a, path, s) : launch_decode_t<float, false>(a, path, s);
 }
 
 cudaError_t read_device_error(unsigned int* value, bool clear) {

@@ -83,11 +83,12 @@ struct DecodeRow {
   float x, dt, w, dl2;
 };
 
+// rows < 2^31 (checked on the host), so the row splits with 32-bit arithmetic
 template <typename T>
-__device__ __forceinline__ DecodeRow decode_row_scalars(const DecodeArgs& p, int64_t row) {
+__device__ __forceinline__ DecodeRow decode_row_scalars(const DecodeArgs& p, uint32_t row) {
   DecodeRow r;
-  r.b = int(row / p.D);
-  r.d = int(row - int64_t(r.b) * p.D);
+  r.b = int(row / uint32_t(p.D));
+  r.d = int(row - uint32_t(r.b) * uint32_t(p.D));
   r.x = ld_elem<T>(p.x, int64_t(r.b) * p.x_sb + int64_t(r.d) * p.x_sd);
   float dt = ld_elem<T>(p.dt, int64_t(r.b) * p.dt_sb + int64_t(r.d) * p.dt_sd);
   if (p.bias) dt += p.bias[int64_t(r.d) * p.bias_s];
@@ -152,7 +153,7 @@ __global__ void __launch_bounds__(kDecodeThreads) state_update_bulk_kernel(const
 
   const bool live = tid < nrows;
   DecodeRow r{};
-  if (live) r = decode_row_scalars<T>(p, r0 + tid);
+  if (live) r = decode_row_scalars<T>(p, uint32_t(r0) + uint32_t(tid));
 
   uint32_t done = 0;
   for (int it = 0; it < kDecodeSpinLimit && !done; ++it) {
@@ -193,15 +194,131 @@ __global__ void __launch_bounds__(kDecodeThreads) state_update_bulk_kernel(const
 }
 
 // ---------------------------------------------------------------------------
+// contiguous state, persistent streaming form: a grid of a few CTAs per SM,
+// each walking its tiles (blockIdx.x, blockIdx.x + gridDim.x, ...) through a
+// ring of kStreamBufs shared-memory tiles.  kStreamBufs - 1 bulk loads are kept
+// in flight ahead of the tile being updated, and the bulk store of a tile
+// overlaps the next tiles; so every SM keeps its share of the bytes moving for the whole
+// launch, with no per-CTA ramp-up or tail wave.
+// ---------------------------------------------------------------------------
+constexpr int kStreamBufs = 4;        // tiles resident per CTA
+constexpr int kStreamAhead = kStreamBufs - 1;
+constexpr int kStreamCtasPerSm = 3;   // 3 x 64 KB shared memory, 768 threads, <= 85 registers
+constexpr int kStreamTileBytes = kDecodeThreads * kN * 4;
+
+__device__ __forceinline__ uint32_t mbar_try_wait(uint32_t mb, uint32_t parity) {
+  uint32_t done;
+  asm volatile("{\n .reg .pred pr;\n mbarrier.try_wait.parity.shared::cta.b64 pr, [%1], %2;\n selp.u32 %0, 1, 0, pr;\n}"
+               : "=r"(done) : "r"(mb), "r"(parity) : "memory");
+  return done;
+}
+
+template <typename T, bool HAS_Z>
+__global__ void __launch_bounds__(kDecodeThreads, kStreamCtasPerSm) state_update_stream_kernel(const DecodeArgs p) {
+  extern __shared__ __align__(128) float ring_s[];  // kStreamBufs x [kDecodeThreads][16]
+  __shared__ __align__(8) unsigned long long mbar[kStreamBufs];
+  const int tid = threadIdx.x;
+  const uint32_t rows = uint32_t(p.Bt) * uint32_t(p.D);
+  const uint32_t ntiles = (rows + kDecodeThreads - 1) / kDecodeThreads;
+  if (blockIdx.x >= ntiles) return;
+  const uint32_t mine = (ntiles - 1 - blockIdx.x) / gridDim.x + 1;  // tiles of this CTA
+  const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(ring_s));
+  const uint32_t mb0 = static_cast<uint32_t>(__cvta_generic_to_shared(&mbar[0]));
+
+  // tile i of this CTA: global tile blockIdx.x + i * gridDim.x; the last tile may be partial
+  auto tile_rows = [&](uint32_t i) {
+    const uint32_t r0 = (blockIdx.x + i * gridDim.x) * uint32_t(kDecodeThreads);
+    return rows - r0 < uint32_t(kDecodeThreads) ? rows - r0 : uint32_t(kDecodeThreads);
+  };
+  auto tile_ptr = [&](uint32_t i) {
+    return p.state + size_t(blockIdx.x + i * gridDim.x) * kDecodeThreads * kN;
+  };
+  auto issue_load = [&](uint32_t i) {  // one thread
+    const uint32_t buf = i % kStreamBufs;
+    const uint32_t bytes = tile_rows(i) * kN * 4;
+    const uint32_t mb = mb0 + buf * 8;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(ring + buf * kStreamTileBytes), "l"(tile_ptr(i)), "r"(bytes), "r"(mb) : "memory");
+  };
+
+  if (tid == 0) {
+#pragma unroll
+    for (int k = 0; k < kStreamBufs; ++k)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mb0 + 8 * k) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (uint32_t j = 0; j < uint32_t(kStreamAhead) && j < mine; ++j) issue_load(j);
+  }
+
+  uint32_t i = 0;
+  bool ok = true;
+  for (; i < mine; ++i) {
+    const uint32_t buf = i % kStreamBufs;
+    const uint32_t nrows = tile_rows(i);
+    const bool live = uint32_t(tid) < nrows;
+    DecodeRow r{};
+    if (live) r = decode_row_scalars<T>(p, (blockIdx.x + i * gridDim.x) * uint32_t(kDecodeThreads) + tid);
+
+    uint32_t done = 0;
+    const uint32_t parity = (i / kStreamBufs) & 1u;
+    for (int it = 0; it < kDecodeSpinLimit && !done; ++it) done = mbar_try_wait(mb0 + buf * 8, parity);
+    if (!__syncthreads_and(done)) {
+      ok = false;
+      break;
+    }
+    if (live) {
+      float4* hs = reinterpret_cast<float4*>(ring_s + buf * (kDecodeThreads * kN) + tid * kN);
+      float y = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int q = (k + (tid >> 1)) & 3;  // lane-rotated quarter order: conflict-free
+        float4 h = hs[q];
+        y += decode_quarter<T>(p, r, q, h);
+        hs[q] = h;
+      }
+      decode_finish<T, HAS_Z>(p, r, y);
+    }
+    // generic-proxy writes of this tile -> visible to the bulk store
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (tid == 0) {
+      asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                   ::"l"(tile_ptr(i)), "r"(ring + buf * kStreamTileBytes), "r"(nrows * kN * 4) : "memory");
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      if (i + kStreamAhead < mine) {
+        // tile i + kStreamAhead reuses the buffer of tile i - 1, whose store is the older of
+        // the (at most) two stores in flight
+        asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        issue_load(i + kStreamAhead);
+      }
+    }
+  }
+  if (!ok && tid == 0) {
+    // record the error; give the loads still in flight (tiles i .. i + kStreamAhead - 1) a
+    // bounded time to land
+    atomicOr(p.err, 1u);
+    for (uint32_t j = i; j < i + kStreamAhead && j < mine; ++j) {
+      uint32_t done = 0;
+      for (int it = 0; it < kDecodeSpinLimit && !done; ++it)
+        done = mbar_try_wait(mb0 + (j % kStreamBufs) * 8, (j / kStreamBufs) & 1u);
+    }
+  }
+  if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // any layout: one thread per row
 // ---------------------------------------------------------------------------
 template <typename T, bool HAS_Z>
 __global__ void __launch_bounds__(kDecodeThreads) state_update_kernel(const DecodeArgs p) {
-  const int64_t row = int64_t(blockIdx.x) * kDecodeThreads + threadIdx.x;
-  const int64_t rows = int64_t(p.Bt) * p.D;
+  const uint32_t row = blockIdx.x * uint32_t(kDecodeThreads) + threadIdx.x;
+  const uint32_t rows = uint32_t(p.Bt) * uint32_t(p.D);
   if (row >= rows) return;
-  const int b = int(row / p.D);
-  const int d = int(row - int64_t(b) * p.D);
+  const int b = int(row / uint32_t(p.D));
+  const int d = int(row - uint32_t(b) * uint32_t(p.D));
   float* st = p.state + int64_t(b) * p.st_sb + int64_t(d) * p.st_sd;
   float4 h[4];
 #pragma unroll

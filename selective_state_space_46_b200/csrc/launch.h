@@ -17,7 +17,8 @@ cudaError_t launch_scan_chained(const ScanArgs& a, int grid, int dtype, bool has
 // Device address of this device's error word (cached per device).
 cudaError_t device_error_word(unsigned int** out);
 // bulk: the state is one contiguous [rows][16] range (bulk-copy kernel), else one thread per row.
-cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, bool bulk, cudaStream_t s);
+enum class DecodePath { kStream, kBulkTile, kPerRow };
+cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, DecodePath path, cudaStream_t s);
 // Reads (and optionally clears) the current device's error word.
 cudaError_t read_device_error(unsigned int* value, bool clear);
 

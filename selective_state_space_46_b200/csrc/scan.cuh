@@ -846,4 +846,5 @@ __global__ void __launch_bounds__(ROWS, 512 / ROWS) scan_chunk_state_kernel(cons
 }
 
 
+
 }  // namespace mssm

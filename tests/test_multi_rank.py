@@ -67,3 +67,31 @@ def test_algorithmic_bytes_match_the_stated_figures():
     assert abs(b1 / 1e6 - 50.9) < 0.1
     bd = bench.decode_algorithmic_bytes(256, 5120, 2)
     assert abs(bd / 1e6 - 178.6) < 0.3
+
+
+def test_binding_roofline_picks_the_slower_bound():
+    import bench
+    peak_fp32 = bench.fp32_peak_tflops(148, 1965.0)
+    assert abs(peak_fp32 - 74.45) < 0.01                 # 148 x 128 x 2 x 1.965 GHz
+    # prefill at 2 x 1536 x 2048: 96 flop against 8.09 B per element; the FP32 time
+    # (8.1 us) exceeds the copy-rate time (7.8 us), so the FP32 pipe is the bound
+    units = 2 * 1536 * 2048
+    r = bench.binding_roofline(bench.scan_algorithmic_bytes(2, 1536, 2048, 2), bench.algorithmic_flops(units),
+                               0.0405, 6539.5, peak_fp32)
+    assert r["bound"] == "alu" and r["unit"] == "TFLOP/s" and r["other"]["bound"] == "hbm"
+    assert abs(r["frac"] - r["achieved"] / peak_fp32) < 1e-12
+    # decode: 96 flop against 136 B per row -> HBM
+    rows = 256 * 5120
+    r = bench.binding_roofline(bench.decode_algorithmic_bytes(256, 5120, 2), bench.algorithmic_flops(rows),
+                               0.030, 6539.5, peak_fp32)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["achieved"] - 178.6e6 / 30e-6 / 1e9) < 15
+
+
+def test_ring_size_covers_four_l2():
+    import bench
+    l2 = 126 << 20
+    assert bench.ring_size(1347 << 20, l2) == 1                   # one set is already > 4x L2
+    r = bench.ring_size(50_900_000, l2)
+    assert r == 11 and r * 50_900_000 >= 4 * l2 and (r - 1) * 50_900_000 < 4 * l2
+    assert bench.ring_size(240_000, l2) == 0                      # tiny: flush instead

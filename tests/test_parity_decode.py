@@ -17,7 +17,20 @@ def dev_decode(inp):
                 dt_bias=to_dev(inp.dt_bias))
 
 
-def test_decode_workload_one_step(cuda_device):
+PATHS = ["auto", "stream", "bulk_tile", "per_row"]
+
+
+@pytest.fixture
+def decode_path(request):
+    """Force one state-update kernel for the test (MSSM_OPT_DECODE_PATH), restore automatic after."""
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_DECODE_PATH, m.DECODE_PATHS.get(request.param, 0))
+    yield request.param
+    m.mssm_set_option(m.MSSM_OPT_DECODE_PATH, 0)
+
+
+@pytest.mark.parametrize("decode_path", PATHS, indirect=True)
+def test_decode_workload_one_step(cuda_device, decode_path):
     import selective_state_space_46_b200 as m
     inp = synth.workload_inputs("decode_bf16_256x5120")
     dv = dev_decode(inp)
@@ -30,7 +43,25 @@ def test_decode_workload_one_step(cuda_device):
     check_close(to_f64(dv["state"]), st_ref, "f32", "state")
 
 
-def test_decode_64_distinct_steps(cuda_device):
+@pytest.mark.parametrize("decode_path", ["stream", "bulk_tile", "per_row"], indirect=True)
+@pytest.mark.parametrize("Bt,D", [(3, 4999), (37, 5003), (131, 5003), (1, 1), (1, 255), (2, 128)])
+def test_decode_ragged_tiles(cuda_device, decode_path, Bt, D):
+    """Row counts that leave a partial last tile, one or several tiles per CTA, and
+    (131 x 5003: 2561 tiles) CTAs that go round the shared-memory ring more than once."""
+    import selective_state_space_46_b200 as m
+    inp = synth.make_decode_inputs(Bt, D, io_dtype="bf16", seed=Bt * 7 + D)
+    dv = dev_decode(inp)
+    out = torch.empty_like(dv["x"])
+    m.mssm_state_update(dv["state"], dv["x"], dv["dt"], dv["A"], dv["B"], dv["C"], dv["D"], dv["z"], out)
+    torch.cuda.synchronize()
+    m.mssm_get_error()  # raises on a device-side timeout
+    st_ref, y_ref = oracle.state_update_inputs(inp)
+    check_close(to_f64(out), y_ref, "bf16", "y")
+    check_close(to_f64(dv["state"]), st_ref, "f32", "state")
+
+
+@pytest.mark.parametrize("decode_path", ["stream", "bulk_tile", "per_row"], indirect=True)
+def test_decode_64_distinct_steps(cuda_device, decode_path):
     import selective_state_space_46_b200 as m
     inp0 = synth.make_decode_inputs(16, 5120, seed=1, step_stream=0)
     state = to_dev(inp0.state)

@@ -19,6 +19,7 @@ def _reset_options():
     import selective_state_space_46_b200 as m
     m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 0)
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
+    m.mssm_set_option(m.MSSM_OPT_SCHEDULE, 0)
 
 
 @pytest.fixture(autouse=True)
@@ -33,6 +34,9 @@ def compare_full(inp, **kw):
     y_ref, h_ref = oracle.scan_inputs(inp)
     check_close(to_f64(out), y_ref, inp.io_dtype, "y")
     check_close(to_f64(last), h_ref, inp.io_dtype, "last_state")
+
+
+SPLIT_SCHEDULES = ["summaries+forward", "chained"]
 
 
 def random_A(dim, seed):
@@ -56,6 +60,14 @@ def test_workload_bf16_2x1536x2048_general_A_path():
     import selective_state_space_46_b200 as m
     m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 1)
     compare_full(synth.workload_inputs("scan_bf16_2x1536x2048"))
+
+
+@pytest.mark.parametrize("schedule", ["forward"] + SPLIT_SCHEDULES)
+def test_workload_bf16_2x1536x2048_each_schedule(schedule):
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_SCHEDULE, m.SCHEDULES[schedule])
+    compare_full(synth.workload_inputs("scan_bf16_2x1536x2048"))
+    m.mssm_get_error()
 
 
 def _sampled(name, rows_per_batch=6, seed=0):
@@ -132,9 +144,12 @@ def test_general_A_values(io):
 @pytest.mark.parametrize("chunk", [64, 128, 192, 320])
 @pytest.mark.parametrize("structured", [True, False])
 @pytest.mark.parametrize("io", ["bf16", "f32"])
-def test_chunked_carry(chunk, structured, io,):
+@pytest.mark.parametrize("schedule", SPLIT_SCHEDULES)
+def test_chunked_carry(chunk, structured, io, schedule):
     import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_SCHEDULE, m.SCHEDULES[schedule])
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, chunk)
+    assert m.mssm_scan_plan(2, 80, 1000)["schedule"] == schedule
     inp = synth.make_scan_inputs(2, 80, 1000, io_dtype=io, seed=chunk, delta_range=(1e-4, 1e-2))
     if not structured:
         inp.A = random_A(80, chunk)
