@@ -42,11 +42,13 @@ def _load():
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
         lib.oracle_scan_f64.argtypes = [I64, I64, I64, I64, P, P, P, P, P, P, P, P,
-                                        ctypes.c_int, P, P, P]
+                                        ctypes.c_int, ctypes.c_int, P, P, P]
         lib.oracle_scan_f64.restype = None
         lib.oracle_state_update_f64.argtypes = [I64, I64, I64, P, P, P, P, P, P, P, P, P,
-                                                ctypes.c_int, P]
+                                                ctypes.c_int, ctypes.c_int, P]
         lib.oracle_state_update_f64.restype = None
+        lib.oracle_causal_conv1d_f64.argtypes = [I64, I64, I64, I64, P, P, P, ctypes.c_int, P]
+        lib.oracle_causal_conv1d_f64.restype = None
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -65,11 +67,12 @@ def _ptr(a):
 
 
 def scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
-         h0=None) -> Tuple[np.ndarray, np.ndarray]:
+         h0=None, zoh=False) -> Tuple[np.ndarray, np.ndarray]:
     """Selective scan in fp64.
 
     Shapes: ``u, delta, z`` [Bt, D, L]; ``B, C`` [Bt, N, L]; ``A`` [D, N];
-    ``D, delta_bias`` [D]; ``h0`` [Bt, D, N] (zero when omitted).
+    ``D, delta_bias`` [D]; ``h0`` [Bt, D, N] (zero when omitted).  ``zoh``:
+    zero-order-hold input gain (exp(delta A) - 1) / A instead of delta.
     Returns ``(y [Bt, D, L], last_state [Bt, D, N])`` as float64.
     """
     u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
@@ -86,12 +89,12 @@ def scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
     last = np.empty((Bt, Dd, N), np.float64)
     _load().oracle_scan_f64(Bt, Dd, L, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
                             _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(softplus)),
-                            _ptr(h0), _ptr(out), _ptr(last))
+                            int(bool(zoh)), _ptr(h0), _ptr(out), _ptr(last))
     return out, last
 
 
 def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
-                 softplus=True) -> Tuple[np.ndarray, np.ndarray]:
+                 softplus=True, zoh=False) -> Tuple[np.ndarray, np.ndarray]:
     """One decode step in fp64 on a copy of ``state``.
 
     Shapes: ``state`` [Bt, D, N]; ``x, dt, z`` [Bt, D]; ``B, C`` [Bt, N]; ``A`` [D, N].
@@ -108,8 +111,48 @@ def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
     out = np.empty((Bt, Dd), np.float64)
     _load().oracle_state_update_f64(Bt, Dd, N, _ptr(st), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
                                     _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
-                                    int(bool(softplus)), _ptr(out))
+                                    int(bool(softplus)), int(bool(zoh)), _ptr(out))
     return st, out
+
+
+def causal_conv1d(x, w, bias=None, silu=True) -> np.ndarray:
+    """Causal depthwise conv1d along L (then SiLU) in fp64: ``x`` [Bt, D, L], ``w`` [D, K],
+    ``bias`` [D].  Returns [Bt, D, L]."""
+    x, w, bias = map(_f64, (x, w, bias))
+    Bt, Dd, L = x.shape
+    K = w.shape[1]
+    assert w.shape == (Dd, K) and (bias is None or bias.shape == (Dd,))
+    out = np.empty((Bt, Dd, L), np.float64)
+    _load().oracle_causal_conv1d_f64(Bt, Dd, L, K, _ptr(x), _ptr(w), _ptr(bias), int(bool(silu)), _ptr(out))
+    return out
+
+
+def scan_varlen(u, delta, A, B, C, cu_seqlens, D=None, z=None, delta_bias=None, softplus=True,
+                h0=None, zoh=False) -> Tuple[np.ndarray, np.ndarray]:
+    """Selective scan of several sequences packed along L (the varlen layout): ``u, delta,
+    z`` [1, D, T], ``B, C`` [1, N, T], ``cu_seqlens`` [S + 1] offsets (0 = c_0 <= ... <=
+    c_S = T).  Sequence s covers steps c_s .. c_(s+1) - 1 and starts from ``h0[s]`` (zero
+    when omitted): the state does not carry across a boundary.  Returns ``(y [1, D, T],
+    last_state [S, D, N])``.  Built only from ``scan`` on each slice."""
+    cu = np.asarray(cu_seqlens, np.int64)
+    Dd, N = np.shape(A)
+    T = np.shape(u)[-1]
+    assert cu[0] == 0 and cu[-1] == T and (np.diff(cu) >= 0).all()
+    S = len(cu) - 1
+    y = np.zeros((1, Dd, T), np.float64)
+    last = np.zeros((S, Dd, N), np.float64)
+    for s in range(S):
+        a, b = int(cu[s]), int(cu[s + 1])
+        h_init = None if h0 is None else np.asarray(h0, np.float64)[s:s + 1]
+        if b == a:
+            last[s] = 0.0 if h_init is None else h_init[0]
+            continue
+        sl = (lambda v: None if v is None else np.asarray(v)[..., a:b])
+        ys, hs = scan(sl(u), sl(delta), A, sl(B), sl(C), D, sl(z), delta_bias, softplus,
+                      h0=h_init, zoh=zoh)
+        y[..., a:b] = ys
+        last[s] = hs[0]
+    return y, last
 
 
 # --------------------------------------------------------------------------
@@ -117,10 +160,10 @@ def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
 # --------------------------------------------------------------------------
 
 
-def scan_inputs(inp, h0=None):
+def scan_inputs(inp, h0=None, zoh=False):
     """Oracle scan of a whole ``synth.ScanInputs`` problem."""
     return scan(inp.f64("u"), inp.f64("delta"), inp.f64("A"), inp.f64("B"), inp.f64("C"),
-                inp.f64("D"), inp.f64("z"), inp.f64("delta_bias"), inp.softplus, h0=h0)
+                inp.f64("D"), inp.f64("z"), inp.f64("delta_bias"), inp.softplus, h0=h0, zoh=zoh)
 
 
 def scan_rows(inp, rows: Sequence[Tuple[int, int]]):
@@ -160,9 +203,9 @@ def _widen_batch(inp, name, b):
     return to_f64(a[b:b + 1], inp.io_dtype)
 
 
-def state_update_inputs(inp, state=None):
+def state_update_inputs(inp, state=None, zoh=False):
     """Oracle decode step of a ``synth.DecodeInputs`` batch (``state`` overrides ``inp.state``)."""
     st = inp.state if state is None else state
     return state_update(st, inp.f64("x"), inp.f64("dt"), inp.f64("A"), inp.f64("B"),
                         inp.f64("C"), inp.f64("D"), inp.f64("z"), inp.f64("dt_bias"),
-                        inp.softplus)
+                        inp.softplus, zoh=zoh)

@@ -12,7 +12,10 @@
  *     for t = 0 .. L-1:
  *       delta = delta_raw[b,d,t] + bias[d]               (bias optional)
  *       delta = softplus(delta) = log(1 + exp(delta))    (if softplus_flag)
- *       for n:  h[n] = exp(delta * A[d,n]) * h[n] + delta * B[b,n,t] * u[b,d,t]
+ *       for n:  h[n] = exp(delta * A[d,n]) * h[n] + Bbar[n] * u[b,d,t]
+ *               Bbar[n] = delta * B[b,n,t]                         (Euler, the default)
+ *               Bbar[n] = (exp(delta * A[d,n]) - 1) / A[d,n] * B[b,n,t]   (zero-order hold;
+ *                         delta * B[b,n,t] where A[d,n] = 0, the limit)
  *       y = sum_n C[b,n,t] * h[n] + D[d] * u[b,d,t]      (D optional)
  *       y = y * z / (1 + exp(-z))   with z = z[b,d,t]    (gate optional)
  *       out[b,d,t] = y
@@ -32,9 +35,14 @@
  *  - same page, section Discretization, Recurrent View: one recurrence step is
  *    exactly the decode update (oracle_state_update_f64 below).
  *
+ *  - "Linear Attention vs Softmax Attention ...", section Core Concepts, and
+ *    "Mamba selective state space", the discretisation equations: the
+ *    zero-order-hold input matrix (delta A)^-1 (exp(delta A) - I) delta B, which
+ *    for a diagonal A is (exp(delta A_n) - 1) / A_n * B_n per state (zoh_flag).
+ *
  * Readings where the pages leave a choice open:
- *  - B_bar = delta*B (the page's code), not the zero-order-hold form printed in
- *    the pages' equations.
+ *  - B_bar = delta*B (the page's code) by default; the zero-order-hold form
+ *    printed in the pages' equations is the zoh_flag option.
  *  - softplus is the exact log(1 + exp(x)) with no threshold (the listing calls
  *    F.softplus with defaults; the threshold-20 shortcut differs by < 2.1e-9).
  *  - bias absent means 0; D absent means no skip; z absent means no gate.
@@ -61,6 +69,15 @@ static double sp_exact(double x)
     return log1p(exp(x));
 }
 
+/* Zero-order-hold input gain (exp(dt * a) - 1) / a, with expm1 so that small
+ * dt * a loses nothing to cancellation; its limit dt where a = 0. */
+static double zoh_gain(double dt, double a)
+{
+    if (a == 0.0)
+        return dt;
+    return expm1(dt * a) / a;
+}
+
 /* silu(z) = z * sigmoid(z) = z / (1 + exp(-z)). */
 static double silu(double z)
 {
@@ -83,13 +100,14 @@ int oracle_num_threads(void)
  *   A                : [D, N]
  *   Dskip, bias      : [D]
  *   h0, last_state   : [Bt, D, N]
- * Nullable: Dskip, z, bias, h0, last_state.
+ * Nullable: Dskip, z, bias, h0, last_state.  zoh_flag selects the zero-order-hold
+ * input gain instead of delta.
  */
 void oracle_scan_f64(int64_t Bt, int64_t D, int64_t L, int64_t N,
                      const double *u, const double *delta, const double *A,
                      const double *B, const double *C, const double *Dskip,
                      const double *z, const double *bias, int softplus_flag,
-                     const double *h0, double *out, double *last_state)
+                     int zoh_flag, const double *h0, double *out, double *last_state)
 {
     int64_t rows = Bt * D;
 #pragma omp parallel for schedule(dynamic, 4)
@@ -114,6 +132,8 @@ void oracle_scan_f64(int64_t Bt, int64_t D, int64_t L, int64_t N,
             for (int64_t n = 0; n < N; ++n) {
                 double a_bar = exp(dt * Ad[n]);
                 double b_bar = dt * Bb[n * L + t];
+                if (zoh_flag)
+                    b_bar = zoh_gain(dt, Ad[n]) * Bb[n * L + t];
                 h[n] = a_bar * h[n] + b_bar * x;
                 y += Cb[n * L + t] * h[n];
             }
@@ -139,7 +159,7 @@ void oracle_state_update_f64(int64_t Bt, int64_t D, int64_t N, double *state,
                              const double *x, const double *dt_in, const double *A,
                              const double *B, const double *C, const double *Dskip,
                              const double *z, const double *bias, int softplus_flag,
-                             double *out)
+                             int zoh_flag, double *out)
 {
     int64_t rows = Bt * D;
 #pragma omp parallel for schedule(static)
@@ -152,7 +172,8 @@ void oracle_state_update_f64(int64_t Bt, int64_t D, int64_t N, double *state,
         double *h = state + r * N;
         double y = 0.0;
         for (int64_t n = 0; n < N; ++n) {
-            h[n] = exp(dt * A[d * N + n]) * h[n] + dt * B[b * N + n] * xv;
+            double gain = zoh_flag ? zoh_gain(dt, A[d * N + n]) : dt;
+            h[n] = exp(dt * A[d * N + n]) * h[n] + gain * B[b * N + n] * xv;
             y += C[b * N + n] * h[n];
         }
         if (Dskip)
@@ -162,3 +183,35 @@ void oracle_state_update_f64(int64_t Bt, int64_t D, int64_t N, double *state,
         out[r] = y;
     }
 }
+
+/*
+ * Causal depthwise 1-D convolution along L, optionally followed by SiLU: the step
+ * that feeds the scan its input u in the listed layer ("Linear Attention vs Softmax
+ * Attention ...", section Implementation: a grouped Conv1d with one group per
+ * channel, kernel size K, padding K - 1, truncated to the first L outputs, then
+ * SiLU).  With x = 0 before the start of the sequence:
+ *   out[b,d,t] = act(bias[d] + sum_{j=0}^{K-1} w[d,j] * x[b,d,t + j - (K-1)])
+ *   x, out : [Bt, D, L]     w : [D, K]     bias : [D] (nullable)
+ */
+void oracle_causal_conv1d_f64(int64_t Bt, int64_t D, int64_t L, int64_t K,
+                              const double *x, const double *w, const double *bias,
+                              int silu_flag, double *out)
+{
+    int64_t rows = Bt * D;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t d = r % D;
+        const double *xr = x + r * L;
+        const double *wd = w + d * K;
+        for (int64_t t = 0; t < L; ++t) {
+            double acc = bias ? bias[d] : 0.0;
+            for (int64_t j = 0; j < K; ++j) {
+                int64_t src = t + j - (K - 1);
+                if (src >= 0)
+                    acc += wd[j] * xr[src];
+            }
+            out[r * L + t] = silu_flag ? silu(acc) : acc;
+        }
+    }
+}
+

@@ -300,6 +300,143 @@ def test_softplus_and_silu_spot_values():
 
 
 # ---------------------------------------------------------------------------
+# 7b. zero-order hold ("Linear Attention vs Softmax Attention ...", Core Concepts;
+#     "Mamba selective state space", discretisation equations)
+# ---------------------------------------------------------------------------
+
+def test_zoh_constant_input_is_exact():
+    """With the step, A, B and u held constant, the zero-order-hold recurrence is exact:
+    after t steps of size dt the state equals the continuous solution of h' = A h + B u
+    from h(0) = 0 at time t dt, (exp(A t dt) - 1) / A * B u, whatever dt is."""
+    rng = np.random.default_rng(21)
+    D, L = 3, 40
+    A = -np.exp(rng.uniform(-2.0, 1.0, size=(D, N)))
+    for dt in (0.01, 0.37):
+        u = np.full((1, D, L), 0.8)
+        delta = np.full((1, D, L), dt)
+        Bv = rng.standard_normal(N)
+        B = np.repeat(Bv[None, :, None], L, axis=2)
+        C = np.ones((1, N, L))
+        y, last = oracle.scan(u, delta, A, B, C, None, None, None, softplus=False, zoh=True)
+        tt = dt * np.arange(1, L + 1)
+        h = np.expm1(A[:, :, None] * tt[None, None, :]) / A[:, :, None] * Bv[None, :, None] * 0.8
+        np.testing.assert_allclose(y[0], h.sum(axis=1), rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(last[0], h[:, :, -1], rtol=1e-12, atol=1e-13)
+
+
+def test_zoh_small_A_is_euler():
+    """As A -> 0, (exp(dt A) - 1) / A -> dt: the two discretisations agree to O(dt^2 A)."""
+    rng = np.random.default_rng(22)
+    p = rand_problem(rng, 1, 4, 30)
+    p["A"] = np.full_like(p["A"], -1e-9)
+    y_e, h_e = oracle.scan(**p, softplus=True)
+    y_z, h_z = oracle.scan(**p, softplus=True, zoh=True)
+    np.testing.assert_allclose(y_z, y_e, rtol=1e-7, atol=1e-9)
+    np.testing.assert_allclose(h_z, h_e, rtol=1e-7, atol=1e-9)
+
+
+def test_zoh_decode_steps_reproduce_scan():
+    rng = np.random.default_rng(23)
+    p = rand_problem(rng, 2, 5, 16)
+    y, last = oracle.scan(**p, softplus=True, zoh=True)
+    state = np.zeros((2, 5, N))
+    for t in range(16):
+        state, yt = oracle.state_update(state, p["u"][..., t], p["delta"][..., t], p["A"],
+                                        p["B"][..., t], p["C"][..., t], p["D"], p["z"][..., t],
+                                        p["delta_bias"], True, zoh=True)
+        np.testing.assert_allclose(yt, y[..., t], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(state, last, rtol=1e-13, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# 7c. causal depthwise conv1d + SiLU feeding the scan ("Linear Attention vs Softmax
+#     Attention ...", section Implementation: grouped Conv1d, padding K - 1, truncated)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("silu", [False, True])
+def test_conv1d_matches_numpy_convolve(silu):
+    rng = np.random.default_rng(31)
+    Bt, D, L, K = 2, 5, 23, 4
+    x = rng.standard_normal((Bt, D, L))
+    w = rng.standard_normal((D, K))
+    b = rng.standard_normal(D)
+    out = oracle.causal_conv1d(x, w, b, silu=silu)
+    # cross-correlation with left zero padding == the first L outputs of a full convolution
+    # with the reversed filter
+    ref = np.stack([np.stack([np.convolve(x[i, d], w[d][::-1])[:L] + b[d] for d in range(D)])
+                    for i in range(Bt)])
+    if silu:
+        ref = ref * sigmoid_ref(ref)
+    np.testing.assert_allclose(out, ref, rtol=1e-13, atol=1e-14)
+
+
+def test_conv1d_matches_torch_conv1d():
+    import torch
+    rng = np.random.default_rng(32)
+    Bt, D, L, K = 3, 4, 17, 4
+    x = rng.standard_normal((Bt, D, L))
+    w = rng.standard_normal((D, K))
+    b = rng.standard_normal(D)
+    ref = torch.nn.functional.conv1d(torch.from_numpy(x), torch.from_numpy(w)[:, None, :],
+                                     torch.from_numpy(b), padding=K - 1, groups=D)[..., :L]
+    ref = torch.nn.functional.silu(ref).numpy()
+    np.testing.assert_allclose(oracle.causal_conv1d(x, w, b, silu=True), ref, rtol=1e-13, atol=1e-14)
+
+
+def test_conv1d_impulse_response():
+    # a unit impulse at t0 comes out as the filter read backwards: out[t0 + m] = w[K - 1 - m]
+    K, L, t0 = 4, 12, 3
+    w = np.array([[0.5, -1.0, 2.0, 3.0]])
+    x = np.zeros((1, 1, L))
+    x[0, 0, t0] = 1.0
+    out = oracle.causal_conv1d(x, w, None, silu=False)[0, 0]
+    expect = np.zeros(L)
+    for m in range(K):
+        expect[t0 + m] = w[0, K - 1 - m]
+    np.testing.assert_array_equal(out, expect)
+
+
+# ---------------------------------------------------------------------------
+# 7d. packed variable-length sequences: the state restarts at every boundary
+# ---------------------------------------------------------------------------
+
+def test_varlen_single_sequence_is_the_scan():
+    rng = np.random.default_rng(41)
+    p = rand_problem(rng, 1, 3, 25)
+    y, last = oracle.scan(**p, softplus=True)
+    yv, lv = oracle.scan_varlen(p["u"], p["delta"], p["A"], p["B"], p["C"], [0, 25], p["D"], p["z"],
+                                p["delta_bias"], True)
+    np.testing.assert_array_equal(yv, y)
+    np.testing.assert_array_equal(lv, last)
+
+
+def test_varlen_sequences_are_isolated():
+    rng = np.random.default_rng(42)
+    p = rand_problem(rng, 1, 3, 40)
+    cu = [0, 9, 9, 30, 40]  # includes an empty sequence
+    h0 = rng.standard_normal((4, 3, N))
+    y, last = oracle.scan_varlen(p["u"], p["delta"], p["A"], p["B"], p["C"], cu, p["D"], p["z"],
+                                 p["delta_bias"], True, h0=h0)
+    # perturbing sequence 0 changes nothing in sequences 2 and 3
+    q = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in p.items()}
+    q["u"][..., :9] += 1.0
+    q["B"][..., :9] -= 0.5
+    y2, last2 = oracle.scan_varlen(q["u"], q["delta"], q["A"], q["B"], q["C"], cu, q["D"], q["z"],
+                                   q["delta_bias"], True, h0=h0)
+    np.testing.assert_array_equal(y2[..., 9:], y[..., 9:])
+    np.testing.assert_array_equal(last2[1:], last[1:])
+    assert np.abs(y2[..., :9] - y[..., :9]).max() > 1e-3
+    # the empty sequence hands back its initial state
+    np.testing.assert_array_equal(last[1], h0[1])
+    # with zero initial states, the scan of sequence 3 alone is the same
+    y0, _ = oracle.scan_varlen(p["u"], p["delta"], p["A"], p["B"], p["C"], cu, p["D"], p["z"],
+                               p["delta_bias"], True)
+    sl = {k: (v[..., 30:] if k in ("u", "delta", "B", "C", "z") else v) for k, v in p.items()}
+    ys, _ = oracle.scan(**sl, softplus=True)
+    np.testing.assert_array_equal(y0[..., 30:], ys)
+
+
+# ---------------------------------------------------------------------------
 # 8. hand-derived worked example (tests/golden/halving_decay.txt)
 # ---------------------------------------------------------------------------
 
@@ -343,7 +480,16 @@ MUTANTS = {
     "softplus_is_exp": ("dt = sp_exact(dt);\n            double x = ur[t];",
                         "dt = exp(dt);\n            double x = ur[t];"),
     "A_channel_ignored": ("const double *Ad = A + d * N;", "const double *Ad = A;"),
-    "decode_dropped_dt_on_input": ("+ dt * B[b * N + n] * xv;", "+ B[b * N + n] * xv;"),
+    "decode_dropped_dt_on_input": ("zoh_gain(dt, A[d * N + n]) : dt;", "zoh_gain(dt, A[d * N + n]) : 1.0;"),
+    "zoh_gain_sign_flipped": ("return expm1(dt * a) / a;", "return expm1(-dt * a) / a;"),
+    "zoh_gain_not_divided": ("return expm1(dt * a) / a;", "return expm1(dt * a);"),
+    "zoh_gain_is_exp": ("return expm1(dt * a) / a;", "return exp(dt * a) / a;"),
+    "scan_zoh_ignored": ("b_bar = zoh_gain(dt, Ad[n]) * Bb[n * L + t];", "b_bar = dt * Bb[n * L + t];"),
+    "decode_zoh_ignored": ("double gain = zoh_flag ? zoh_gain(dt, A[d * N + n]) : dt;", "double gain = dt;"),
+    "conv_filter_reversed": ("acc += wd[j] * xr[src];", "acc += wd[K - 1 - j] * xr[src];"),
+    "conv_window_off_by_one": ("int64_t src = t + j - (K - 1);", "int64_t src = t + j - K;"),
+    "conv_bias_dropped": ("double acc = bias ? bias[d] : 0.0;", "double acc = 0.0;"),
+    "conv_silu_dropped": ("silu_flag ? silu(acc) : acc;", "acc;"),
     "decode_bias_dropped": ("double dt = dt_in[r] + (bias ? bias[d] : 0.0);", "double dt = dt_in[r];"),
     "decode_gate_dropped": ("            y *= silu(z[r]);\n        out[r] = y;", "        out[r] = y;"),
 }
@@ -362,6 +508,12 @@ PIN_CALLS = [
     test_linear_in_u,
     test_softplus_and_silu_spot_values,
     test_golden_halving_decay,
+    test_zoh_constant_input_is_exact,
+    test_zoh_small_A_is_euler,
+    test_zoh_decode_steps_reproduce_scan,
+    lambda: test_conv1d_matches_numpy_convolve(True),
+    test_conv1d_matches_torch_conv1d,
+    test_conv1d_impulse_response,
 ]
 
 
@@ -379,8 +531,11 @@ def _count_failures(lib_path):
     import ctypes
     lib = ctypes.CDLL(lib_path)
     P, I64 = ctypes.c_void_p, ctypes.c_int64
-    lib.oracle_scan_f64.argtypes = [I64, I64, I64, I64, P, P, P, P, P, P, P, P, ctypes.c_int, P, P, P]
-    lib.oracle_state_update_f64.argtypes = [I64, I64, I64, P, P, P, P, P, P, P, P, P, ctypes.c_int, P]
+    lib.oracle_scan_f64.argtypes = [I64, I64, I64, I64, P, P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                    P, P, P]
+    lib.oracle_state_update_f64.argtypes = [I64, I64, I64, P, P, P, P, P, P, P, P, P, ctypes.c_int,
+                                            ctypes.c_int, P]
+    lib.oracle_causal_conv1d_f64.argtypes = [I64, I64, I64, I64, P, P, P, ctypes.c_int, P]
     lib.oracle_num_threads.restype = ctypes.c_int
     saved = oracle._lib
     oracle._lib = lib
