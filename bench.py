@@ -160,7 +160,8 @@ def max_sm_mhz(default: float = 1965.0) -> float:
 KERNEL_SOURCES = {
     "scan_out": ("device_common.cuh", "scan.cuh", "scan.cu"),
     "scan_chunk_state": ("device_common.cuh", "scan.cuh", "scan.cu"),
-    "state_update": ("device_common.cuh", "decode.cuh", "decode.cu"),
+    # the automatic choice among the decode kernels is made in api.cu
+    "state_update": ("device_common.cuh", "decode.cuh", "decode.cu", "api.cu"),
 }
 
 
@@ -507,7 +508,8 @@ def run_mssm(args):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     alu_peak = fp32_peak_tflops(sms, max_sm_mhz())
     alg_flops = algorithmic_flops(units)
-    traffic, traffic_src = recorded_traffic(dom_kernel, args.workload, plan_string(config.get("plan")))
+    plan_key = plan_string(config.get("plan")) if kind == "scan" else f"decode_path={args.decode_path}"
+    traffic, traffic_src = recorded_traffic(dom_kernel, args.workload, plan_key)
     roofline = binding_roofline(alg_bytes, alg_flops, dom_ms, peak, alu_peak) if dom_ms else {"bound": None}
     roofline.update({"kernel": dom_kernel, "ms_per_launch": dom_ms,
                      "peak_source": f"HBM: {peak_kind} copy rate; FP32: {sms} SMs x 128 lanes x 2 x "

@@ -206,11 +206,15 @@ mssm_status mssm_get_error(void *stream);
  *     plan falls back to forward only.
  *   MSSM_OPT_KERNEL_TIMING (value 0/1): when 1, every kernel launch is bracketed
  *     by two CUDA events recorded on the caller's stream (see mssm_kernel_stats).
- *   MSSM_OPT_DECODE_PATH (value 0..3): the state-update kernel.  0 automatic
- *     (2 when the state is one contiguous, 16-byte aligned [Bt, D, 16] range,
- *     else 3); 1 persistent streaming kernel (a ring of bulk-copied tiles per
- *     CTA); 2 one bulk-copied tile per CTA; 3 one thread per row, any layout.
- *     1 and 2 need the contiguous layout and fall back to 3 without it.
+ *   MSSM_OPT_DECODE_PATH (value 0..3): the state-update kernel.  0 automatic:
+ *     the first of 1, 2, 3 whose layout conditions hold.  1 persistent streaming
+ *     kernel (per CTA a block of 128 channels and a ring of bulk-copied tiles);
+ *     needs the state as one contiguous, 16-byte aligned [Bt, D, 16] range, x,
+ *     dt and z with unit channel stride and 16-byte aligned batch rows, D a
+ *     multiple of 8 (bf16) or 4 (f32), and B, C with unit n stride and 16-byte
+ *     aligned batch rows.  2 one bulk-copied tile of 256 rows per CTA; needs the
+ *     contiguous state.  3 one thread per row, any layout.  A forced path whose
+ *     conditions fail falls back to the next one that holds.
  * Unknown options or invalid values return MSSM_ERR_INVALID_ARG.
  */
 typedef enum {

@@ -628,10 +628,16 @@ static mssm_status state_update_impl(mssm_tensor* state, const mssm_tensor* x, c
   const bool contiguous = aligned16(state->data) && state->stride[1] == mssm::kN && state->stride[0] == Dd * mssm::kN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lk(g_mu);
+  // every per-row input a contiguous, 16-byte aligned run per batch: the streaming kernel
+  auto runs = [&](const mssm_tensor* t) {
+    return !t || (aligned16(t->data) && t->stride[1] == 1 && (t->stride[0] * es) % 16 == 0);
+  };
+  const bool streamable = contiguous && runs(x) && runs(dt_t) && runs(z) && a.vec_BC &&
+                          (Dd * es) % 16 == 0;
   mssm::DecodePath path = mssm::DecodePath::kPerRow;
-  if (contiguous)
-    path = g_decode_path == 1 ? mssm::DecodePath::kStream
-         : g_decode_path == 3 ? mssm::DecodePath::kPerRow : mssm::DecodePath::kBulkTile;
+  if (g_decode_path != 3 && contiguous) {
+    path = (g_decode_path == 2 || !streamable) ? mssm::DecodePath::kBulkTile : mssm::DecodePath::kStream;
+  }
   cudaError_t e = tracked(MSSM_KERNEL_STATE_UPDATE, s,
                           [&] { return mssm::launch_state_update(a, dt, z != nullptr, path, s); });
   if (e != cudaSuccess) return cuda_fail(e, "state update launch");

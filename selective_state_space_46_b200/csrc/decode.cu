@@ -32,20 +32,33 @@ static cudaError_t stream_setup(int* sms) {
     int v = 0;
     e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const int bytes = kStreamBufs * kStreamTileBytes;
+    const int b16 = kStreamBufs * int(StreamSlot<uint16_t>::kBytes);
+    const int b32 = kStreamBufs * int(StreamSlot<float>::kBytes);
     if ((e = cudaFuncSetAttribute(state_update_stream_kernel<uint16_t, true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess ||
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, b16)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(state_update_stream_kernel<uint16_t, false>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess ||
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, b16)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(state_update_stream_kernel<float, true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess ||
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, b32)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(state_update_stream_kernel<float, false>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess)
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, b32)) != cudaSuccess)
       return e;
     sm_cache[dev] = v;
   }
   *sms = sm_cache[dev];
   return cudaSuccess;
+}
+
+// Batch groups of the streaming kernel: as many CTAs per channel block as fill the
+// resident slots, but no more groups than batches.
+int stream_groups(int Bt, int D, int sms) {
+  const int nblk = (D + kStreamRows - 1) / kStreamRows;
+  int groups = (sms * kStreamCtasPerSm) / nblk;
+  if (groups < 1) groups = 1;
+  if (groups > Bt) groups = Bt;
+  // same number of batches per CTA with as few groups as that needs
+  const int per = (Bt + groups - 1) / groups;
+  return (Bt + per - 1) / per;
 }
 
 template <typename T, bool HAS_Z>
@@ -57,13 +70,10 @@ static cudaError_t launch_decode_t(DecodeArgs a, DecodePath path, cudaStream_t s
   if (path == DecodePath::kStream) {
     int sms = 0;
     if ((e = stream_setup(&sms)) != cudaSuccess) return e;
-    // as many CTAs as fit, with the tile count per CTA balanced: every CTA gets
-    // ceil(tiles / slots) tiles except the last, which gets what remains
-    const int64_t slots = int64_t(sms) * kStreamCtasPerSm;
-    const int64_t per = (blocks + slots - 1) / slots;
-    const int64_t grid = (blocks + per - 1) / per;
+    a.groups = stream_groups(a.Bt, a.D, sms);
+    const int64_t nblk = (a.D + kStreamRows - 1) / kStreamRows;
     state_update_stream_kernel<T, HAS_Z>
-        <<<unsigned(grid), kDecodeThreads, kStreamBufs * kStreamTileBytes, s>>>(a);
+        <<<unsigned(nblk * a.groups), kStreamRows, kStreamBufs * StreamSlot<T>::kBytes, s>>>(a);
   } else if (path == DecodePath::kBulkTile) {
     state_update_bulk_kernel<T, HAS_Z><<<unsigned(blocks), kDecodeThreads, 0, s>>>(a);
   } else {

@@ -53,6 +53,7 @@ struct DecodeArgs {
   int vec_state;  // every row's state starts 16-byte aligned
   int vec_A;      // A rows 16-byte aligned with unit n stride
   int vec_BC;     // B and C rows 16-byte aligned with unit n stride
+  int groups;     // streaming kernel: batch groups (CTAs per channel block)
   unsigned int* err;  // device error word: bit 0 = a bulk copy did not complete in time
 };
 
@@ -194,17 +195,38 @@ __global__ void __launch_bounds__(kDecodeThreads) state_update_bulk_kernel(const
 }
 
 // ---------------------------------------------------------------------------
-// contiguous state, persistent streaming form: a grid of a few CTAs per SM,
-// each walking its tiles (blockIdx.x, blockIdx.x + gridDim.x, ...) through a
-// ring of kStreamBufs shared-memory tiles.  kStreamBufs - 1 bulk loads are kept
-// in flight ahead of the tile being updated, and the bulk store of a tile
-// overlaps the next tiles; so every SM keeps its share of the bytes moving for the whole
-// launch, with no per-CTA ramp-up or tail wave.
+// persistent streaming form.  A CTA owns one block of kStreamRows channels and
+// walks the batches b = g, g + G, g + 2G, ... of that block (g, G: its batch
+// group and the group count).  Per (batch, channel block) tile, one thread
+// issues bulk copies of everything the tile reads -- the contiguous 8 KB of
+// state, the x / dt / z runs of the block and the batch's B and C rows -- into
+// one slot of a shared-memory ring, all counted on the slot's mbarrier;
+// kStreamBufs - 1 tiles are in flight ahead of the one being updated, and the
+// updated state leaves by a bulk store that overlaps the following tiles.  The
+// block's A rows, skip weights and biases are loaded once per CTA into
+// registers.  So no thread waits on a global load inside the loop: the only
+// waits are the (bounded) mbarrier waits the ring hides.
+//
+// Needs: contiguous 16-byte-aligned state; x, dt (and z) with unit channel
+// stride, 16-byte-aligned batch rows and D a multiple of 16 / sizeof(T); B and
+// C with unit n stride and 16-byte-aligned batch rows (the host checks all).
 // ---------------------------------------------------------------------------
-constexpr int kStreamBufs = 4;        // tiles resident per CTA
+constexpr int kStreamRows = 128;      // channels per CTA, one thread each
+constexpr int kStreamBufs = 4;        // ring slots per CTA
 constexpr int kStreamAhead = kStreamBufs - 1;
-constexpr int kStreamCtasPerSm = 3;   // 3 x 64 KB shared memory, 768 threads, <= 85 registers
-constexpr int kStreamTileBytes = kDecodeThreads * kN * 4;
+constexpr int kStreamCtasPerSm = 5;   // 5 x (4 x <= 9.9 KB) shared memory, 640 threads
+
+template <typename T>
+struct StreamSlot {
+  static constexpr uint32_t kState = 0;
+  static constexpr uint32_t kX = kStreamRows * kN * 4;
+  static constexpr uint32_t kDt = kX + kStreamRows * sizeof(T);
+  static constexpr uint32_t kZ = kDt + kStreamRows * sizeof(T);
+  static constexpr uint32_t kB = kZ + kStreamRows * sizeof(T);
+  static constexpr uint32_t kC = kB + kN * sizeof(T);
+  static constexpr uint32_t kBytes = kC + kN * sizeof(T);
+  static_assert(kBytes % 16 == 0 && kX % 16 == 0 && kB % 16 == 0, "slot layout must keep 16-byte alignment");
+};
 
 __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t mb, uint32_t parity) {
   uint32_t done;
@@ -213,33 +235,49 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t mb, uint32_t parity) 
   return done;
 }
 
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t mb) {
+  asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(mb) : "memory");
+}
+
+// value j of a run of T stored in shared memory
+template <typename T>
+__device__ __forceinline__ float smem_elem(const unsigned char* base, int j) {
+  return Elem<T>::load(reinterpret_cast<const T*>(base) + j);
+}
+
 template <typename T, bool HAS_Z>
-__global__ void __launch_bounds__(kDecodeThreads, kStreamCtasPerSm) state_update_stream_kernel(const DecodeArgs p) {
-  extern __shared__ __align__(128) float ring_s[];  // kStreamBufs x [kDecodeThreads][16]
+__global__ void __launch_bounds__(kStreamRows, kStreamCtasPerSm) state_update_stream_kernel(const DecodeArgs p) {
+  using L = StreamSlot<T>;
+  extern __shared__ __align__(128) unsigned char ring_s[];  // kStreamBufs slots of L::kBytes
   __shared__ __align__(8) unsigned long long mbar[kStreamBufs];
   const int tid = threadIdx.x;
-  const uint32_t rows = uint32_t(p.Bt) * uint32_t(p.D);
-  const uint32_t ntiles = (rows + kDecodeThreads - 1) / kDecodeThreads;
-  if (blockIdx.x >= ntiles) return;
-  const uint32_t mine = (ntiles - 1 - blockIdx.x) / gridDim.x + 1;  // tiles of this CTA
+  const int nblk = (p.D + kStreamRows - 1) / kStreamRows;
+  const int cb = int(blockIdx.x % uint32_t(nblk));
+  const int g = int(blockIdx.x / uint32_t(nblk));
+  if (g >= p.Bt || g >= p.groups) return;
+  const int c0 = cb * kStreamRows;
+  const int nrows = p.D - c0 < kStreamRows ? p.D - c0 : kStreamRows;
+  const uint32_t mine = uint32_t(p.Bt - 1 - g) / uint32_t(p.groups) + 1;  // batches of this CTA
+  const bool live = tid < nrows;
+  const int d = c0 + (live ? tid : nrows - 1);
   const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(ring_s));
   const uint32_t mb0 = static_cast<uint32_t>(__cvta_generic_to_shared(&mbar[0]));
+  constexpr uint32_t ES = sizeof(T);
+  const uint32_t run_bytes = uint32_t(nrows) * ES;  // a multiple of 16 (D % (16 / ES) == 0)
+  const uint32_t tile_bytes = uint32_t(nrows) * kN * 4 + (HAS_Z ? 3u : 2u) * run_bytes + 2u * kN * ES;
 
-  // tile i of this CTA: global tile blockIdx.x + i * gridDim.x; the last tile may be partial
-  auto tile_rows = [&](uint32_t i) {
-    const uint32_t r0 = (blockIdx.x + i * gridDim.x) * uint32_t(kDecodeThreads);
-    return rows - r0 < uint32_t(kDecodeThreads) ? rows - r0 : uint32_t(kDecodeThreads);
-  };
-  auto tile_ptr = [&](uint32_t i) {
-    return p.state + size_t(blockIdx.x + i * gridDim.x) * kDecodeThreads * kN;
-  };
-  auto issue_load = [&](uint32_t i) {  // one thread
-    const uint32_t buf = i % kStreamBufs;
-    const uint32_t bytes = tile_rows(i) * kN * 4;
-    const uint32_t mb = mb0 + buf * 8;
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(bytes) : "memory");
-    asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(ring + buf * kStreamTileBytes), "l"(tile_ptr(i)), "r"(bytes), "r"(mb) : "memory");
+  auto issue = [&](uint32_t i) {  // one thread
+    const int64_t b = int64_t(g) + int64_t(i) * p.groups;
+    const uint32_t slot = ring + (i % kStreamBufs) * L::kBytes;
+    const uint32_t mb = mb0 + (i % kStreamBufs) * 8;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(tile_bytes) : "memory");
+    bulk_load(slot + L::kState, p.state + (b * p.D + c0) * kN, uint32_t(nrows) * kN * 4, mb);
+    bulk_load(slot + L::kX, static_cast<const T*>(p.x) + b * p.x_sb + c0, run_bytes, mb);
+    bulk_load(slot + L::kDt, static_cast<const T*>(p.dt) + b * p.dt_sb + c0, run_bytes, mb);
+    if constexpr (HAS_Z) bulk_load(slot + L::kZ, static_cast<const T*>(p.z) + b * p.z_sb + c0, run_bytes, mb);
+    bulk_load(slot + L::kB, static_cast<const T*>(p.B) + b * p.B_sb, kN * ES, mb);
+    bulk_load(slot + L::kC, static_cast<const T*>(p.C) + b * p.C_sb, kN * ES, mb);
   };
 
   if (tid == 0) {
@@ -249,56 +287,85 @@ __global__ void __launch_bounds__(kDecodeThreads, kStreamCtasPerSm) state_update
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  if (tid == 0) {
-    for (uint32_t j = 0; j < uint32_t(kStreamAhead) && j < mine; ++j) issue_load(j);
+  if (tid == 0)
+    for (uint32_t j = 0; j < uint32_t(kStreamAhead) && j < mine; ++j) issue(j);
+
+  // per-channel constants, once per CTA.  The state row is visited in the lane-rotated
+  // quarter order q = (kq + rot) & 3 (bank-conflict free), so A is stored pre-rotated:
+  // a2r[4 kq + e] = A[d, 4 q + e] * log2(e), and the loop indexes it with constants.
+  const int rot = (tid >> 1) & 3;
+  float a2r[kN];
+  {
+    const float* Ar = p.A + int64_t(d) * p.A_sd;
+#pragma unroll
+    for (int kq = 0; kq < 4; ++kq)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a2r[4 * kq + e] = Ar[int64_t(4 * ((kq + rot) & 3) + e) * p.A_sn] * kLog2e;
   }
+  const float bias = p.bias ? p.bias[int64_t(d) * p.bias_s] : 0.0f;
+  const float Dd = p.Dskip ? p.Dskip[int64_t(d) * p.D_s] : 0.0f;
 
   uint32_t i = 0;
   bool ok = true;
   for (; i < mine; ++i) {
-    const uint32_t buf = i % kStreamBufs;
-    const uint32_t nrows = tile_rows(i);
-    const bool live = uint32_t(tid) < nrows;
-    DecodeRow r{};
-    if (live) r = decode_row_scalars<T>(p, (blockIdx.x + i * gridDim.x) * uint32_t(kDecodeThreads) + tid);
-
+    const uint32_t k = i % kStreamBufs;
+    const unsigned char* slot = ring_s + k * L::kBytes;
     uint32_t done = 0;
-    const uint32_t parity = (i / kStreamBufs) & 1u;
-    for (int it = 0; it < kDecodeSpinLimit && !done; ++it) done = mbar_try_wait(mb0 + buf * 8, parity);
+    for (int it = 0; it < kDecodeSpinLimit && !done; ++it) done = mbar_try_wait(mb0 + k * 8, (i / kStreamBufs) & 1u);
     if (!__syncthreads_and(done)) {
       ok = false;
       break;
     }
     if (live) {
-      float4* hs = reinterpret_cast<float4*>(ring_s + buf * (kDecodeThreads * kN) + tid * kN);
+      const int64_t b = int64_t(g) + int64_t(i) * p.groups;
+      const float x = smem_elem<T>(slot + L::kX, tid);
+      float dt = smem_elem<T>(slot + L::kDt, tid) + bias;
+      if (p.softplus) dt = softplus_f(dt);
+      const float w = dt * x;
+      float4* hs = reinterpret_cast<float4*>(const_cast<unsigned char*>(slot) + L::kState + tid * (kN * 4));
       float y = 0.0f;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int q = (k + (tid >> 1)) & 3;  // lane-rotated quarter order: conflict-free
+      for (int kq = 0; kq < 4; ++kq) {
+        const int q = (kq + rot) & 3;
         float4 h = hs[q];
-        y += decode_quarter<T>(p, r, q, h);
-        hs[q] = h;
+        float hv[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int n = 4 * q + e;
+          hv[e] = fmaf(ex2f(dt * a2r[4 * kq + e]), hv[e], w * smem_elem<T>(slot + L::kB, n));
+          y = fmaf(smem_elem<T>(slot + L::kC, n), hv[e], y);
+        }
+        hs[q] = make_float4(hv[0], hv[1], hv[2], hv[3]);
       }
-      decode_finish<T, HAS_Z>(p, r, y);
+      y = fmaf(Dd, x, y);
+      if constexpr (HAS_Z) y *= gate_f<T>(smem_elem<T>(slot + L::kZ, tid));
+      T* o = static_cast<T*>(p.out) + b * p.o_sb + int64_t(d) * p.o_sd;
+      if constexpr (sizeof(T) == 2) {
+        *o = f_to_bf16(y);
+      } else {
+        *o = y;
+      }
     }
-    // generic-proxy writes of this tile -> visible to the bulk store
+    // generic-proxy accesses of this slot -> ordered before the bulk store and the next bulk load
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
     if (tid == 0) {
+      const int64_t b = int64_t(g) + int64_t(i) * p.groups;
       asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
-                   ::"l"(tile_ptr(i)), "r"(ring + buf * kStreamTileBytes), "r"(nrows * kN * 4) : "memory");
+                   ::"l"(p.state + (b * p.D + c0) * kN), "r"(ring + k * L::kBytes + L::kState),
+                   "r"(uint32_t(nrows) * kN * 4) : "memory");
       asm volatile("cp.async.bulk.commit_group;" ::: "memory");
       if (i + kStreamAhead < mine) {
-        // tile i + kStreamAhead reuses the buffer of tile i - 1, whose store is the older of
+        // tile i + kStreamAhead takes the slot of tile i - 1, whose store is the older of
         // the (at most) two stores in flight
         asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-        issue_load(i + kStreamAhead);
+        issue(i + kStreamAhead);
       }
     }
   }
   if (!ok && tid == 0) {
     // record the error; give the loads still in flight (tiles i .. i + kStreamAhead - 1) a
-    // bounded time to land
+    // bounded time to land before the CTA's shared memory is released
     atomicOr(p.err, 1u);
     for (uint32_t j = i; j < i + kStreamAhead && j < mine; ++j) {
       uint32_t done = 0;

@@ -44,19 +44,23 @@ def test_decode_workload_one_step(cuda_device, decode_path):
 
 
 @pytest.mark.parametrize("decode_path", ["stream", "bulk_tile", "per_row"], indirect=True)
-@pytest.mark.parametrize("Bt,D", [(3, 4999), (37, 5003), (131, 5003), (1, 1), (1, 255), (2, 128)])
-def test_decode_ragged_tiles(cuda_device, decode_path, Bt, D):
-    """Row counts that leave a partial last tile, one or several tiles per CTA, and
-    (131 x 5003: 2561 tiles) CTAs that go round the shared-memory ring more than once."""
+@pytest.mark.parametrize("Bt,D,io", [(3, 4999, "bf16"), (37, 5003, "bf16"), (131, 5003, "bf16"), (1, 1, "bf16"),
+                                     (1, 255, "bf16"), (2, 128, "bf16"), (3, 5000, "bf16"), (131, 4104, "bf16"),
+                                     (300, 8, "bf16"), (5, 1028, "f32"), (7, 130, "f32")])
+def test_decode_ragged_tiles(cuda_device, decode_path, Bt, D, io):
+    """Row counts that leave a partial last tile or channel block, one or several tiles per
+    CTA, CTAs that go round the shared-memory ring more than once (131 x 4104: 22 batch
+    groups of up to 6 batches; 131 x 5003: 2561 tiles of 256 rows), and shapes the streaming
+    kernel cannot take (D not a multiple of 16 bytes), where the path falls back."""
     import selective_state_space_46_b200 as m
-    inp = synth.make_decode_inputs(Bt, D, io_dtype="bf16", seed=Bt * 7 + D)
+    inp = synth.make_decode_inputs(Bt, D, io_dtype=io, seed=Bt * 7 + D)
     dv = dev_decode(inp)
     out = torch.empty_like(dv["x"])
     m.mssm_state_update(dv["state"], dv["x"], dv["dt"], dv["A"], dv["B"], dv["C"], dv["D"], dv["z"], out)
     torch.cuda.synchronize()
     m.mssm_get_error()  # raises on a device-side timeout
     st_ref, y_ref = oracle.state_update_inputs(inp)
-    check_close(to_f64(out), y_ref, "bf16", "y")
+    check_close(to_f64(out), y_ref, io, "y")
     check_close(to_f64(dv["state"]), st_ref, "f32", "state")
 
 
@@ -79,9 +83,11 @@ def test_decode_64_distinct_steps(cuda_device, decode_path):
 
 @pytest.mark.parametrize("io", ["bf16", "f32"])
 @pytest.mark.parametrize("with_z,with_D", [(True, True), (False, False)])
-def test_decode_variants(cuda_device, io, with_z, with_D):
+@pytest.mark.parametrize("dim", [77, 128])
+def test_decode_variants(cuda_device, io, with_z, with_D, dim):
+    """Optional gate, skip and bias on the automatic path (D = 128: streaming kernel; 77: not)."""
     import selective_state_space_46_b200 as m
-    inp = synth.make_decode_inputs(3, 77, io_dtype=io, seed=4, with_z=with_z, with_D=with_D, dt_bias=True)
+    inp = synth.make_decode_inputs(3, dim, io_dtype=io, seed=4, with_z=with_z, with_D=with_D, dt_bias=True)
     dv = dev_decode(inp)
     out = m.state_update(dv["state"], dv["x"], dv["dt"], dv["A"], dv["B"], dv["C"], dv["D"], dv["z"],
                          dt_bias=dv["dt_bias"], softplus=True)
