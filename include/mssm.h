@@ -7,6 +7,7 @@
  *   delta_t   = softplus(delta_raw_t + bias_d)          (softplus and bias optional)
  *   A_bar_tn  = exp(delta_t * A_dn)
  *   h_tn      = A_bar_tn * h_(t-1)n + delta_t * B_tn * u_t          (h_(-1) = 0)
+ *               (optionally the zero-order-hold input term and a given h_(-1))
  *   y_t       = sum_n C_tn * h_tn + D_d * u_t                       (D optional)
  *   out_t     = y_t * silu(z_t)                                     (z optional)
  *
@@ -113,6 +114,47 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor *u, const mssm_tensor *del
                                     int softplus_flag, mssm_tensor *out,
                                     mssm_tensor *last_state, void *stream);
 
+/* Discretisation of the input term (mssm_selective_scan_fwd_ex, mssm_state_update_ex). */
+typedef enum {
+    MSSM_DISC_EULER = 0, /* B_bar = delta * B: the listed layer's loop ("Linear Attention vs
+                            Softmax Attention ...", section Implementation); the default */
+    MSSM_DISC_ZOH = 1    /* B_bar = (exp(delta A) - 1) / A * B per state: the zero-order hold
+                            of the same page's Core Concepts, item 3, and of "State Space Models
+                            in Large Language Models ...", section Discretization, for diagonal
+                            A; delta * B where A = 0 (the limit) */
+} mssm_discretization;
+
+/*
+ * Optional inputs of mssm_selective_scan_fwd_ex.  Set struct_size to
+ * sizeof(mssm_scan_ext); fields may be appended in later versions.
+ *   discretization  mssm_discretization
+ *   h0              [Bt, D, N] f32, n stride 1: the state before step 0 (NULL: zero),
+ *                   e.g. the last_state of the previous piece of a sequence processed
+ *                   in parts (prefill in pieces, resume).  Must not alias out or
+ *                   last_state.
+ */
+typedef struct {
+    int32_t struct_size;
+    int32_t discretization;
+    const mssm_tensor *h0;
+} mssm_scan_ext;
+
+/*
+ * mssm_selective_scan_fwd_ex: mssm_selective_scan_fwd with the options of `ext`
+ * (NULL: none, i.e. the plain call).  Same arguments, results, workspace and
+ * errors otherwise; an invalid ext (struct_size too small, unknown
+ * discretization, h0 of the wrong shape, dtype or n stride, h0 aliasing an
+ * output) is MSSM_ERR_INVALID_ARG.  With h0 given, the scan equals running the
+ * recurrence from h0: splitting a sequence at any step and passing the first
+ * part's last_state as the second part's h0 reproduces the whole-sequence call.
+ */
+mssm_status mssm_selective_scan_fwd_ex(const mssm_tensor *u, const mssm_tensor *delta,
+                                       const mssm_tensor *A, const mssm_tensor *B,
+                                       const mssm_tensor *C, const mssm_tensor *D,
+                                       const mssm_tensor *z, const mssm_tensor *delta_bias,
+                                       int softplus_flag, const mssm_scan_ext *ext,
+                                       mssm_tensor *out, mssm_tensor *last_state, void *stream);
+
 /*
  * mssm_selective_scan_fwd_noalloc: the same scan, same arguments and results,
  * for callers that cannot allocate device memory during the call.  Examples: a
@@ -156,8 +198,11 @@ mssm_status mssm_selective_scan_fwd_noalloc(const mssm_tensor *u, const mssm_ten
  * This entry point applies delta = softplus(dt) (no bias).  The same step as
  * one iteration of mssm_selective_scan_fwd's recurrence ("State Space Models
  * in Large Language Models ...", section Discretization, recurrent view).
- * When `state` is one contiguous 16-byte-aligned [Bt*D][16] range, each CTA
- * moves its 16 KB tile with a bulk copy in and out of shared memory.
+ * When `state` is one contiguous 16-byte-aligned [Bt*D][16] range (and the
+ * per-row inputs are aligned runs), a persistent kernel streams each (batch,
+ * 128-channel block) tile and its inputs through shared memory with bulk
+ * copies (see MSSM_OPT_DECODE_PATH); its bounded waits report
+ * MSSM_ERR_TIMEOUT through mssm_get_error if they ever give up.
  */
 mssm_status mssm_state_update(mssm_tensor *state, const mssm_tensor *x, const mssm_tensor *dt,
                               const mssm_tensor *A, const mssm_tensor *B, const mssm_tensor *C,
@@ -165,16 +210,17 @@ mssm_status mssm_state_update(mssm_tensor *state, const mssm_tensor *x, const ms
                               void *stream);
 
 /*
- * As mssm_state_update, with an optional per-channel dt_bias [D] f32 (NULL: none)
- * and an explicit softplus flag, so that a sequence of decode steps reproduces
- * mssm_selective_scan_fwd called with the same bias and flag.
+ * As mssm_state_update, with an optional per-channel dt_bias [D] f32 (NULL: none),
+ * an explicit softplus flag and the discretisation (mssm_discretization), so
+ * that a sequence of decode steps reproduces mssm_selective_scan_fwd_ex called
+ * with the same bias, flag and discretisation.
  */
 mssm_status mssm_state_update_ex(mssm_tensor *state, const mssm_tensor *x,
                                  const mssm_tensor *dt, const mssm_tensor *A,
                                  const mssm_tensor *B, const mssm_tensor *C,
                                  const mssm_tensor *D, const mssm_tensor *z,
                                  const mssm_tensor *dt_bias, int softplus_flag,
-                                 mssm_tensor *out, void *stream);
+                                 int discretization, mssm_tensor *out, void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *mssm_status_string(mssm_status status);

@@ -35,10 +35,11 @@
  *  - same page, section Discretization, Recurrent View: one recurrence step is
  *    exactly the decode update (oracle_state_update_f64 below).
  *
- *  - "Linear Attention vs Softmax Attention ...", section Core Concepts, and
- *    "Mamba selective state space", the discretisation equations: the
- *    zero-order-hold input matrix (delta A)^-1 (exp(delta A) - I) delta B, which
- *    for a diagonal A is (exp(delta A_n) - 1) / A_n * B_n per state (zoh_flag).
+ *  - "Linear Attention vs Softmax Attention ...", section Core Concepts, item 3,
+ *    and "State Space Models in Large Language Models ...", section
+ *    Discretization: the zero-order-hold input matrix
+ *    (delta A)^-1 (exp(delta A) - I) delta B, which for a diagonal A is
+ *    (exp(delta A_n) - 1) / A_n * B_n per state (zoh_flag).
  *
  * Readings where the pages leave a choice open:
  *  - B_bar = delta*B (the page's code) by default; the zero-order-hold form

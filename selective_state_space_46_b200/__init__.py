@@ -23,6 +23,7 @@ __all__ = [
     "mssm_last_error", "selective_scan_fwd", "state_update", "lib_path",
     "MSSM_OPT_FORCE_GENERAL_A", "MSSM_OPT_CHUNK_LEN", "MSSM_OPT_KERNEL_TIMING", "MSSM_OPT_SCHEDULE", "SCHEDULES",
     "MSSM_OPT_DECODE_PATH", "DECODE_PATHS", "mssm_kernel_stats", "mssm_scan_plan",
+    "mssm_selective_scan_fwd_ex", "MSSM_DISC_EULER", "MSSM_DISC_ZOH",
     "KERNEL_KINDS",
 ]
 
@@ -37,6 +38,7 @@ MSSM_F32, MSSM_BF16 = 0, 1
 MSSM_OK, MSSM_ERR_INVALID_ARG, MSSM_ERR_UNSUPPORTED, MSSM_ERR_CUDA, MSSM_ERR_TIMEOUT = 0, 1, 2, 3, 4
 MSSM_OPT_FORCE_GENERAL_A, MSSM_OPT_CHUNK_LEN, MSSM_OPT_KERNEL_TIMING, MSSM_OPT_SCHEDULE = 1, 2, 3, 4
 MSSM_OPT_DECODE_PATH = 5
+MSSM_DISC_EULER, MSSM_DISC_ZOH = 0, 1
 SCHEDULES = {"forward": 1, "summaries+forward": 2, "chained": 3}
 DECODE_PATHS = {"stream": 1, "bulk_tile": 2, "per_row": 3}
 KERNEL_KINDS = ("scan_chunk_state", "scan_out", "state_update")
@@ -47,15 +49,23 @@ class mssm_tensor(ctypes.Structure):
                 ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
 
 
+class mssm_scan_ext(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_int32), ("discretization", ctypes.c_int32),
+                ("h0", ctypes.POINTER(mssm_tensor))]
+
+
 _P = ctypes.POINTER(mssm_tensor)
 _V = ctypes.c_void_p
 _lib.mssm_selective_scan_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, _V]
 _lib.mssm_selective_scan_fwd.restype = ctypes.c_int
+_lib.mssm_selective_scan_fwd_ex.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int,
+                                            ctypes.POINTER(mssm_scan_ext), _P, _P, _V]
+_lib.mssm_selective_scan_fwd_ex.restype = ctypes.c_int
 _lib.mssm_selective_scan_fwd_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, _V]
 _lib.mssm_selective_scan_fwd_noalloc.restype = ctypes.c_int
 _lib.mssm_state_update.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _V]
 _lib.mssm_state_update.restype = ctypes.c_int
-_lib.mssm_state_update_ex.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _V]
+_lib.mssm_state_update_ex.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _V]
 _lib.mssm_state_update_ex.restype = ctypes.c_int
 _lib.mssm_status_string.argtypes = [ctypes.c_int]
 _lib.mssm_status_string.restype = ctypes.c_char_p
@@ -169,6 +179,18 @@ def mssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, 
                                         _ref(ds[8]), _ref(ds[9]), _stream(stream, u)))
 
 
+def mssm_selective_scan_fwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state,
+                               h0=None, discretization=MSSM_DISC_EULER, stream=None) -> None:
+    """Marshal torch tensors into ``mssm_selective_scan_fwd_ex``: the scan from an initial
+    state ``h0`` [Bt, D, N] (None: zero) with the given discretisation (see include/mssm.h)."""
+    ds = [_desc(t) for t in (u, delta, A, B, C, D, z, delta_bias, out, last_state)]
+    dh = _desc(h0)
+    ext = mssm_scan_ext(ctypes.sizeof(mssm_scan_ext), int(discretization),
+                        None if dh is None else ctypes.pointer(dh[1]))
+    _check(_lib.mssm_selective_scan_fwd_ex(*[_ref(x) for x in ds[:8]], int(softplus_flag), ctypes.byref(ext),
+                                           _ref(ds[8]), _ref(ds[9]), _stream(stream, u)))
+
+
 def mssm_selective_scan_fwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state,
                                     stream=None) -> None:
     """Marshal torch tensors into ``mssm_selective_scan_fwd_noalloc``: the same scan for
@@ -185,11 +207,11 @@ def mssm_state_update(state, x, dt, A, B, C, D, z, out, stream=None) -> None:
 
 
 def mssm_state_update_ex(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, out,
-                         stream=None) -> None:
+                         discretization=MSSM_DISC_EULER, stream=None) -> None:
     """Marshal torch tensors into ``mssm_state_update_ex`` (state updated in place)."""
     ds = [_desc(t) for t in (state, x, dt, A, B, C, D, z, dt_bias)]
     do = _desc(out)
-    _check(_lib.mssm_state_update_ex(*[_ref(v) for v in ds], int(softplus_flag), _ref(do),
+    _check(_lib.mssm_state_update_ex(*[_ref(v) for v in ds], int(softplus_flag), int(discretization), _ref(do),
                                      _stream(stream, x)))
 
 
@@ -198,25 +220,31 @@ def mssm_state_update_ex(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, ou
 # --------------------------------------------------------------------------
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
-                       out=None, last_state=None, return_last_state=True,
+                       out=None, last_state=None, return_last_state=True, h0=None, zoh=False,
                        stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Allocate ``out`` (and ``last_state``) with torch and run the scan on the GPU."""
+    """Allocate ``out`` (and ``last_state``) with torch and run the scan on the GPU
+    (from ``h0`` when given; zero-order-hold input term when ``zoh``)."""
     if not u.is_cuda:
         raise ValueError("selective_scan_fwd runs on CUDA tensors only")
     if out is None:
         out = torch.empty_like(u, memory_format=torch.contiguous_format)
     if last_state is None and return_last_state:
         last_state = torch.empty(u.shape[0], u.shape[1], A.shape[1], device=u.device, dtype=torch.float32)
-    mssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, out, last_state, stream)
+    if h0 is None and not zoh:
+        mssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, out, last_state, stream)
+    else:
+        mssm_selective_scan_fwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus, out, last_state, h0=h0,
+                                   discretization=MSSM_DISC_ZOH if zoh else MSSM_DISC_EULER, stream=stream)
     return out, last_state
 
 
 def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, softplus=True, out=None,
-                 stream=None) -> torch.Tensor:
+                 zoh=False, stream=None) -> torch.Tensor:
     """Run one decode step on the GPU (``state`` updated in place); returns ``out``."""
     if not x.is_cuda:
         raise ValueError("state_update runs on CUDA tensors only")
     if out is None:
         out = torch.empty_like(x, memory_format=torch.contiguous_format)
-    mssm_state_update_ex(state, x, dt, A, B, C, D, z, dt_bias, softplus, out, stream)
+    mssm_state_update_ex(state, x, dt, A, B, C, D, z, dt_bias, softplus, out,
+                         discretization=MSSM_DISC_ZOH if zoh else MSSM_DISC_EULER, stream=stream)
     return out

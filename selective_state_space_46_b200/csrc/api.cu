@@ -341,6 +341,32 @@ mssm_status scan_prepare(const mssm_tensor* u, const mssm_tensor* delta, const m
   return MSSM_OK;
 }
 
+// The optional inputs of mssm_selective_scan_fwd_ex: initial state and discretisation.
+mssm_status scan_prepare_ext(const mssm_scan_ext* ext, const mssm_tensor* out, const mssm_tensor* last_state,
+                             ScanCall& call) {
+  if (!ext) return MSSM_OK;
+  if (ext->struct_size < int32_t(sizeof(mssm_scan_ext)))
+    return fail(MSSM_ERR_INVALID_ARG, "ext->struct_size = %d; expected at least %d", int(ext->struct_size),
+                int(sizeof(mssm_scan_ext)));
+  if (ext->discretization != MSSM_DISC_EULER && ext->discretization != MSSM_DISC_ZOH)
+    return fail(MSSM_ERR_INVALID_ARG, "ext->discretization must be MSSM_DISC_EULER or MSSM_DISC_ZOH");
+  call.a.zoh = ext->discretization == MSSM_DISC_ZOH;
+  const mssm_tensor* h0 = ext->h0;
+  if (h0) {
+    const int64_t s_bdn[3] = {call.Bt, call.D, mssm::kN};
+    mssm_status st = check(h0, "h0", 3, s_bdn, MSSM_F32, true);
+    if (st != MSSM_OK) return st;
+    if (same_ptr(h0, out) || same_ptr(h0, last_state))
+      return fail(MSSM_ERR_INVALID_ARG, "h0 must not alias out or last_state");
+    if (call.noop) return MSSM_OK;
+    call.a.h0 = static_cast<const float*>(h0->data);
+    call.a.h0_sb = h0->stride[0];
+    call.a.h0_sd = h0->stride[1];
+    call.a.vec_h0 = aligned16(h0->data) && (h0->stride[0] * 4) % 16 == 0 && (h0->stride[1] * 4) % 16 == 0;
+  }
+  return MSSM_OK;
+}
+
 // Plans the launch (caller holds g_mu) and returns the carry workspace layout.
 struct ScanPlan {
   int mode = 0;
@@ -420,20 +446,8 @@ mssm_status scan_launch(ScanCall& call, const ScanPlan& plan, void* ws, cudaStre
   return MSSM_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* delta,
-                                    const mssm_tensor* A, const mssm_tensor* B,
-                                    const mssm_tensor* C, const mssm_tensor* D,
-                                    const mssm_tensor* z, const mssm_tensor* delta_bias,
-                                    int softplus_flag, mssm_tensor* out, mssm_tensor* last_state,
-                                    void* stream) {
-  ScanCall call;
-  mssm_status st = scan_prepare(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state, call);
-  if (st != MSSM_OK || call.noop) return st;
-
+// The allocating scan of a prepared call: plan, grow the workspace if needed, launch.
+mssm_status scan_fwd_impl(ScanCall& call, void* stream) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -500,6 +514,35 @@ mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* del
     scan_bind_workspace(call.a, layout, ds->ws);
   }
   return scan_launch(call, plan, ds->ws, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+mssm_status mssm_selective_scan_fwd(const mssm_tensor* u, const mssm_tensor* delta,
+                                    const mssm_tensor* A, const mssm_tensor* B,
+                                    const mssm_tensor* C, const mssm_tensor* D,
+                                    const mssm_tensor* z, const mssm_tensor* delta_bias,
+                                    int softplus_flag, mssm_tensor* out, mssm_tensor* last_state,
+                                    void* stream) {
+  ScanCall call;
+  mssm_status st = scan_prepare(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state, call);
+  if (st != MSSM_OK || call.noop) return st;
+  return scan_fwd_impl(call, stream);
+}
+
+mssm_status mssm_selective_scan_fwd_ex(const mssm_tensor* u, const mssm_tensor* delta,
+                                       const mssm_tensor* A, const mssm_tensor* B,
+                                       const mssm_tensor* C, const mssm_tensor* D,
+                                       const mssm_tensor* z, const mssm_tensor* delta_bias,
+                                       int softplus_flag, const mssm_scan_ext* ext, mssm_tensor* out,
+                                       mssm_tensor* last_state, void* stream) {
+  ScanCall call;
+  mssm_status st = scan_prepare(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state, call);
+  if (st != MSSM_OK) return st;
+  if ((st = scan_prepare_ext(ext, out, last_state, call)) != MSSM_OK || call.noop) return st;
+  return scan_fwd_impl(call, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -572,7 +615,9 @@ mssm_status mssm_selective_scan_fwd_noalloc(const mssm_tensor* u, const mssm_ten
 static mssm_status state_update_impl(mssm_tensor* state, const mssm_tensor* x, const mssm_tensor* dt_t,
                                      const mssm_tensor* A, const mssm_tensor* B, const mssm_tensor* C,
                                      const mssm_tensor* D, const mssm_tensor* z, const mssm_tensor* bias,
-                                     int softplus_flag, mssm_tensor* out, void* stream) {
+                                     int softplus_flag, int discretization, mssm_tensor* out, void* stream) {
+  if (discretization != MSSM_DISC_EULER && discretization != MSSM_DISC_ZOH)
+    return fail(MSSM_ERR_INVALID_ARG, "discretization must be MSSM_DISC_EULER or MSSM_DISC_ZOH");
   if (!x) return fail(MSSM_ERR_INVALID_ARG, "x: null tensor descriptor");
   if (x->ndim != 2) return fail(MSSM_ERR_INVALID_ARG, "x: expected 2 dims [Bt, D]");
   const int dt = x->dtype;
@@ -618,6 +663,7 @@ static mssm_status state_update_impl(mssm_tensor* state, const mssm_tensor* x, c
   a.bias = bias ? static_cast<const float*>(bias->data) : nullptr; a.bias_s = bias ? bias->stride[0] : 0;
   a.Bt = int(Bt); a.D = int(Dd);
   a.softplus = softplus_flag != 0;
+  a.zoh = discretization == MSSM_DISC_ZOH;
   a.vec_state = aligned16(state->data) && (state->stride[0] * 4) % 16 == 0 && (state->stride[1] * 4) % 16 == 0;
   a.vec_A = aligned16(A->data) && A->stride[1] == 1 && (A->stride[0] * 4) % 16 == 0;
   const int64_t es = int64_t(esize(dt));
@@ -648,14 +694,14 @@ mssm_status mssm_state_update(mssm_tensor* state, const mssm_tensor* x, const ms
                               const mssm_tensor* A, const mssm_tensor* B, const mssm_tensor* C,
                               const mssm_tensor* D, const mssm_tensor* z, mssm_tensor* out,
                               void* stream) {
-  return state_update_impl(state, x, dt, A, B, C, D, z, nullptr, 1, out, stream);
+  return state_update_impl(state, x, dt, A, B, C, D, z, nullptr, 1, MSSM_DISC_EULER, out, stream);
 }
 
 mssm_status mssm_state_update_ex(mssm_tensor* state, const mssm_tensor* x, const mssm_tensor* dt,
                                  const mssm_tensor* A, const mssm_tensor* B, const mssm_tensor* C,
                                  const mssm_tensor* D, const mssm_tensor* z, const mssm_tensor* dt_bias,
-                                 int softplus_flag, mssm_tensor* out, void* stream) {
-  return state_update_impl(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, out, stream);
+                                 int softplus_flag, int discretization, mssm_tensor* out, void* stream) {
+  return state_update_impl(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, discretization, out, stream);
 }
 
 mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int* rows_per_cta,

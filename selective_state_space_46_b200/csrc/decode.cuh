@@ -54,6 +54,7 @@ struct DecodeArgs {
   int vec_A;      // A rows 16-byte aligned with unit n stride
   int vec_BC;     // B and C rows 16-byte aligned with unit n stride
   int groups;     // streaming kernel: batch groups (CTAs per channel block)
+  int zoh;        // zero-order-hold input gain (exp(dt A) - 1) / A instead of dt
   unsigned int* err;  // device error word: bit 0 = a bulk copy did not complete in time
 };
 
@@ -100,16 +101,25 @@ __device__ __forceinline__ DecodeRow decode_row_scalars(const DecodeArgs& p, uin
   return r;
 }
 
+// One state: h <- exp(dt a) h + g x b, g = dt (Euler) or (exp(dt a) - 1) / a (zero-order hold).
+__device__ __forceinline__ float decode_state(bool zoh, float h, float a, float b, float dt, float dl2, float x,
+                                              float w) {
+  const float e = ex2f(dl2 * a);
+  if (zoh) return fmaf(e, h, zoh_gain_f(e, dt, a, a != 0.0f ? rcpf(a) : 0.0f) * x * b);
+  return fmaf(e, h, w * b);
+}
+
 // Update one 16-byte quarter q (states 4q..4q+3); returns the partial readout.
 template <typename T>
 __device__ __forceinline__ float decode_quarter(const DecodeArgs& p, const DecodeRow& r, int q, float4& h) {
   const float4 a = load4<float>(p.A, int64_t(r.d) * p.A_sd + int64_t(4 * q) * p.A_sn, p.A_sn, p.vec_A != 0);
   const float4 bv = load4<T>(p.B, int64_t(r.b) * p.B_sb + int64_t(4 * q) * p.B_sn, p.B_sn, p.vec_BC != 0);
   const float4 cv = load4<T>(p.C, int64_t(r.b) * p.C_sb + int64_t(4 * q) * p.C_sn, p.C_sn, p.vec_BC != 0);
-  h.x = fmaf(ex2f(r.dl2 * a.x), h.x, r.w * bv.x);
-  h.y = fmaf(ex2f(r.dl2 * a.y), h.y, r.w * bv.y);
-  h.z = fmaf(ex2f(r.dl2 * a.z), h.z, r.w * bv.z);
-  h.w = fmaf(ex2f(r.dl2 * a.w), h.w, r.w * bv.w);
+  const bool zoh = p.zoh != 0;
+  h.x = decode_state(zoh, h.x, a.x, bv.x, r.dt, r.dl2, r.x, r.w);
+  h.y = decode_state(zoh, h.y, a.y, bv.y, r.dt, r.dl2, r.x, r.w);
+  h.z = decode_state(zoh, h.z, a.z, bv.z, r.dt, r.dl2, r.x, r.w);
+  h.w = decode_state(zoh, h.w, a.w, bv.w, r.dt, r.dl2, r.x, r.w);
   return fmaf(cv.x, h.x, fmaf(cv.y, h.y, fmaf(cv.z, h.z, cv.w * h.w)));
 }
 
@@ -332,7 +342,13 @@ __global__ void __launch_bounds__(kStreamRows, kStreamCtasPerSm) state_update_st
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int n = 4 * q + e;
-          hv[e] = fmaf(ex2f(dt * a2r[4 * kq + e]), hv[e], w * smem_elem<T>(slot + L::kB, n));
+          const float ed = ex2f(dt * a2r[4 * kq + e]);
+          float g = w;
+          if (p.zoh) {
+            const float an = a2r[4 * kq + e] * kLn2;
+            g = zoh_gain_f(ed, dt, an, an != 0.0f ? rcpf(an) : 0.0f) * x;
+          }
+          hv[e] = fmaf(ed, hv[e], g * smem_elem<T>(slot + L::kB, n));
           y = fmaf(smem_elem<T>(slot + L::kC, n), hv[e], y);
         }
         hs[q] = make_float4(hv[0], hv[1], hv[2], hv[3]);

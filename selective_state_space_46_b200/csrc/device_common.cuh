@@ -47,6 +47,23 @@ __device__ __forceinline__ float softplus_f(float v) {
   return (v > 20.0f) ? v : r;
 }
 
+// Zero-order hold ("Linear Attention vs Softmax Attention ...", Core Concepts, item 3;
+// "State Space Models in Large Language Models ...", Discretization): the input gain of state n is
+// (exp(delta A_n) - 1) / A_n = delta * phi(delta A_n), phi(x) = expm1(x) / x.
+// For |x| < 1/16, phi is its Taylor polynomial through x^4/120 (truncation below
+// x^5/720 < 1.4e-9 relative), which avoids the cancellation of exp(x) - 1; for
+// larger |x|, |exp(x) - 1| >= 0.06, so (e - 1) from the SFU exponential keeps a
+// relative error below 4e-6.
+__device__ __forceinline__ float expm1_over_x_small(float x) {
+  return fmaf(x, fmaf(x, fmaf(x, fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f), 1.0f / 6.0f), 0.5f), 1.0f);
+}
+// gain = (e - 1) / a with e = exp(dt a) already computed; inv_a = 1 / a (unused when |dt a| < 1/16,
+// which covers a = 0, where the gain is dt)
+__device__ __forceinline__ float zoh_gain_f(float e, float dt, float a, float inv_a) {
+  const float x = dt * a;
+  return (fabsf(x) < 0.0625f) ? dt * expm1_over_x_small(x) : (e - 1.0f) * inv_a;
+}
+
 // silu(z) = z / (1 + e^-z); e^-z overflowing to +inf gives 0, as it should.
 __device__ __forceinline__ float silu_f(float z) {
   return z * rcpf(1.0f + ex2f(-z * kLog2e));

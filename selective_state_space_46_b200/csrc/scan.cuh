@@ -64,6 +64,10 @@ struct ScanArgs {
   int64_t bias_s;
   float* last_state;
   int64_t ls_sb, ls_sd;  // n stride 1
+  const float* h0;       // [Bt, D, 16] initial state (n stride 1), or null for zero
+  int64_t h0_sb, h0_sd;
+  int vec_h0;            // h0 rows are 16-byte aligned
+  int zoh;               // zero-order-hold input gain (exp(delta A) - 1) / A instead of delta
   int Bt, D, L;
   int force_general;
   int nseg, seg_len;
@@ -174,11 +178,13 @@ template <typename T, int ROWS> struct BCStage {
     }
   }
 
-  __device__ __forceinline__ void store(float* s) const {  // s: [kTC][32]
+  // B rows are scaled for the discretisation: ln 2 (Euler, base-2 step s), 1 / (n + 1)
+  // (zero-order hold on the structured-A path), or 1 (zero-order hold, general A)
+  __device__ __forceinline__ void store(float* s, int bmode = 0) const {  // s: [kTC][32]
     const int tid = threadIdx.x;
     const int r = tid / kThreadsPerRow;
     const int t = (tid % kThreadsPerRow) * kVals;
-    const float scale = (r < 16) ? kLn2 : 1.0f;
+    const float scale = (r >= 16) ? 1.0f : bmode == 0 ? kLn2 : bmode == 1 ? 1.0f / float(r + 1) : 1.0f;
 #pragma unroll
     for (int j = 0; j < kVals; ++j) {
       float v;
@@ -264,6 +270,7 @@ struct RowParams {
   float bias2;   // bias * log2(e)
   float Dd;      // skip weight
   float A0;      // A[d, 0]
+  float invA0;   // 1 / A[d, 0] (0 when A[d, 0] = 0)
   f2_t Ap[8];    // A[d, n] pairs (general path)
 };
 
@@ -293,9 +300,17 @@ __device__ __forceinline__ void decay(float s, const RowParams& rp, f2_t (&dA)[8
 // Per-step scalars of one block: x = decay base 2^(s A_0) (structured A) or s
 // (general A), w = s * u.  PARTIAL: steps at or past `valid` become identity
 // steps (s = 0: A_bar = 1 and no input).
-template <typename T, bool SOFTPLUS, bool STRUCT, bool PARTIAL>
+//
+// Zero-order hold (ZOH): the input term of state n is G_n B_n u with G_n =
+// (exp(delta A_n) - 1) / A_n.  Structured A: exp(delta A_n) - 1 = E (1 + a + ... + a^n)
+// with a = exp(delta A_0) and E = a - 1, and A_n = (n+1) A_0, so G_n B_n u =
+// (E / A_0) u * P_n * B_n / (n+1) with P_n = sum_{i<=n} a^i: w = (E / A_0) u here
+// (E / A_0 = delta phi(delta A_0), see zoh_gain_f), B is staged divided by n + 1, and
+// the recurrence forms w P_n by a running FMA over the powers it already has.
+// General A: w = u and the recurrence takes G_n per state.  sv[j] = s (for the sum S).
+template <typename T, bool SOFTPLUS, bool STRUCT, bool PARTIAL, bool ZOH = false>
 __device__ __forceinline__ void block_scalars(const uint4& ru, const uint4& rd, int valid, const RowParams& rp,
-                                              float* x, float* w) {
+                                              float* x, float* w, float* sv = nullptr) {
   constexpr int S = 16 / int(sizeof(T));
 #pragma unroll
   for (int j = 0; j < S; ++j) {
@@ -307,27 +322,60 @@ __device__ __forceinline__ void block_scalars(const uint4& ru, const uint4& rd, 
       uu = (j < valid) ? uu : 0.0f;
     }
     x[j] = STRUCT ? ex2f(s * rp.A0) : s;
-    w[j] = s * uu;
+    if constexpr (!ZOH) {
+      w[j] = s * uu;
+    } else if constexpr (STRUCT) {
+      const float dt = s * kLn2;
+      w[j] = zoh_gain_f(x[j], dt, rp.A0, rp.invA0) * uu;
+    } else {
+      w[j] = uu;
+    }
+    if (sv) sv[j] = s;
   }
 }
 
 // Recurrence and readout of one block; yout[j] = C_t . h_t (before skip and gate).
-template <typename T, bool STRUCT>
+// READOUT = false: the recurrence only (chunk summaries by a forward sweep).
+// invA: 1 / A[d, n] pairs, used by the zero-order hold on the general path only.
+template <typename T, bool STRUCT, bool ZOH = false, bool READOUT = true>
 __device__ __forceinline__ void block_recurrence(const float* bcrow, const float* x, const float* w,
-                                                 const RowParams& rp, f2_t (&h2)[8], float* yout) {
+                                                 const RowParams& rp, f2_t (&h2)[8], float* yout,
+                                                 const f2_t* invA = nullptr) {
   constexpr int S = 16 / int(sizeof(T));
 #pragma unroll
   for (int j = 0; j < S; ++j) {
     f2_t dA[8];
+    f2_t gw[8];  // ZOH: per-state multiplier of the staged B
     if constexpr (STRUCT) {
       powers16(x[j], dA);
+      if constexpr (ZOH) {
+        // w P_n, n = 0..15, as a running FMA over a^1 .. a^15
+        float run = w[j];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float alo, ahi;
+          f2split(dA[k], alo, ahi);  // a^(2k+1), a^(2k+2)
+          const float p_lo = run;
+          const float p_hi = fmaf(w[j], alo, p_lo);
+          run = fmaf(w[j], ahi, p_hi);
+          gw[k] = f2(p_lo, p_hi);
+        }
+      }
     } else {
       const f2_t s2 = f2(x[j], x[j]);
+      const float dt = x[j] * kLn2;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         float lo, hi;
         f2split(mul2(s2, rp.Ap[k]), lo, hi);
-        dA[k] = f2(ex2f(lo), ex2f(hi));
+        const float elo = ex2f(lo), ehi = ex2f(hi);
+        dA[k] = f2(elo, ehi);
+        if constexpr (ZOH) {
+          float alo, ahi, ilo, ihi;
+          f2split(rp.Ap[k], alo, ahi);
+          f2split(invA[k], ilo, ihi);
+          gw[k] = f2(zoh_gain_f(elo, dt, alo, ilo) * w[j], zoh_gain_f(ehi, dt, ahi, ihi) * w[j]);
+        }
       }
     }
     const f2_t w2 = f2(w[j], w[j]);
@@ -335,25 +383,45 @@ __device__ __forceinline__ void block_recurrence(const float* bcrow, const float
     f2_t ya = 0ull;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const ulonglong2 bb = q[k];      // ln2 * B, pairs (4k, 4k+1), (4k+2, 4k+3)
+      const ulonglong2 bb = q[k];      // scaled B, pairs (4k, 4k+1), (4k+2, 4k+3)
       const ulonglong2 cc = q[4 + k];  // C pairs
-      h2[2 * k] = fma2(dA[2 * k], h2[2 * k], mul2(w2, bb.x));
-      h2[2 * k + 1] = fma2(dA[2 * k + 1], h2[2 * k + 1], mul2(w2, bb.y));
-      ya = (k == 0) ? mul2(cc.x, h2[0]) : fma2(cc.x, h2[2 * k], ya);
-      ya = fma2(cc.y, h2[2 * k + 1], ya);
+      const f2_t m0 = ZOH ? gw[2 * k] : w2;
+      const f2_t m1 = ZOH ? gw[2 * k + 1] : w2;
+      h2[2 * k] = fma2(dA[2 * k], h2[2 * k], mul2(m0, bb.x));
+      h2[2 * k + 1] = fma2(dA[2 * k + 1], h2[2 * k + 1], mul2(m1, bb.y));
+      if constexpr (READOUT) {
+        ya = (k == 0) ? mul2(cc.x, h2[0]) : fma2(cc.x, h2[2 * k], ya);
+        ya = fma2(cc.y, h2[2 * k + 1], ya);
+      }
     }
-    float a0, a1;
-    f2split(ya, a0, a1);
-    yout[j] = a0 + a1;
+    if constexpr (READOUT) {
+      float a0, a1;
+      f2split(ya, a0, a1);
+      yout[j] = a0 + a1;
+    }
   }
 }
 
-template <typename T, int ROWS, bool HAS_Z, bool SOFTPLUS, bool STRUCT>
+// READOUT = false: no output, no z; ssum returns the sum of s over the steps (the
+// chunk-summary sweep of the zero-order-hold discretisation).
+template <typename T, int ROWS, bool HAS_Z, bool SOFTPLUS, bool STRUCT, bool ZOH = false, bool READOUT = true>
 __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[kTC * 32], uint4* slots,
                                               int b, int t0, int t1, const T* urow, const T* dlrow,
                                               const T* zrow, T* orow, bool row_ok, const RowParams& rp,
-                                              f2_t (&h2)[8]) {
+                                              f2_t (&h2)[8], float* ssum = nullptr) {
   constexpr int S = 16 / int(sizeof(T));
+  constexpr bool LOAD_Z = HAS_Z && READOUT;
+  const int bmode = !ZOH ? 0 : STRUCT ? 1 : 2;
+  f2_t invA[8];
+  if constexpr (ZOH && !STRUCT) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float lo, hi;
+      f2split(rp.Ap[k], lo, hi);
+      invA[k] = f2(lo != 0.0f ? rcpf(lo) : 0.0f, hi != 0.0f ? rcpf(hi) : 0.0f);
+    }
+  }
+  float sacc = 0.0f;
   constexpr int kBlkPerChunk = kTC / S;
   const int tid = threadIdx.x;
   const bool vec = p.vec_rows != 0;
@@ -367,14 +435,19 @@ __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[k
     const int st = k % kStages;
     fetch_block<T>(slot(st, 0), urow, t, t1, vec);
     fetch_block<T>(slot(st, 1), dlrow, t, t1, vec);
-    if constexpr (HAS_Z) fetch_block<T>(slot(st, 2), zrow, t, t1, vec);
+    if constexpr (LOAD_Z) fetch_block<T>(slot(st, 2), zrow, t, t1, vec);
   };
   auto scalars = [&](int k, const uint4& ru, const uint4& rd, float* x, float* w) {
     const int valid = t1 - (t0 + k * S);
+    float sv[S];
     if (valid >= S)
-      block_scalars<T, SOFTPLUS, STRUCT, false>(ru, rd, S, rp, x, w);
+      block_scalars<T, SOFTPLUS, STRUCT, false, ZOH>(ru, rd, S, rp, x, w, READOUT ? nullptr : sv);
     else
-      block_scalars<T, SOFTPLUS, STRUCT, true>(ru, rd, valid, rp, x, w);
+      block_scalars<T, SOFTPLUS, STRUCT, true, ZOH>(ru, rd, valid, rp, x, w, READOUT ? nullptr : sv);
+    if constexpr (!READOUT) {
+#pragma unroll
+      for (int j = 0; j < S; ++j) sacc += sv[j];
+    }
   };
 #pragma unroll
   for (int k = 0; k < kStages - 1; ++k) {
@@ -384,12 +457,12 @@ __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[k
 
   BCStage<T, ROWS> stage;
   stage.load(p, b, t0, t1);
-  stage.store(bc_s[0]);
+  stage.store(bc_s[0], bmode);
 
   // block 0's scalars
   cp_wait<kStages - 2>();
   uint4 ru = *slot(0, 0);
-  uint4 rz = HAS_Z ? *slot(0, 2) : make_uint4(0u, 0u, 0u, 0u);
+  uint4 rz = LOAD_Z ? *slot(0, 2) : make_uint4(0u, 0u, 0u, 0u);
   float xc[S], wc[S];
   scalars(0, ru, *slot(0, 1), xc, wc);
   __syncthreads();
@@ -410,19 +483,21 @@ __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[k
         cp_wait<kStages - 2>();
         const int st = (k + 1) % kStages;
         run = *slot(st, 0);
-        if constexpr (HAS_Z) rzn = *slot(st, 2);
+        if constexpr (LOAD_Z) rzn = *slot(st, 2);
         scalars(k + 1, run, *slot(st, 1), xn, wn);
       }
       // this block: recurrence, readout, skip, gate, store
       float y[S];
-      block_recurrence<T, STRUCT>(bcb + kb * S * 32, xc, wc, rp, h2, y);
+      block_recurrence<T, STRUCT, ZOH, READOUT>(bcb + kb * S * 32, xc, wc, rp, h2, y, invA);
+      if constexpr (READOUT) {
 #pragma unroll
-      for (int j = 0; j < S; ++j) {
-        float v = fmaf(rp.Dd, blk_at<T>(ru, j), y[j]);
-        if constexpr (HAS_Z) v *= gate_f<T>(blk_at<T>(rz, j));
-        y[j] = v;
+        for (int j = 0; j < S; ++j) {
+          float v = fmaf(rp.Dd, blk_at<T>(ru, j), y[j]);
+          if constexpr (HAS_Z) v *= gate_f<T>(blk_at<T>(rz, j));
+          y[j] = v;
+        }
+        if (row_ok) store_block<T>(orow, t0 + k * S, t1, vec, y);
       }
-      if (row_ok) store_block<T>(orow, t0 + k * S, t1, vec, y);
 #pragma unroll
       for (int j = 0; j < S; ++j) {
         xc[j] = xn[j];
@@ -431,10 +506,11 @@ __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[k
       ru = run;
       rz = rzn;
     }
-    if (c + 1 < nchunks) stage.store(bc_s[(c + 1) & 1]);
+    if (c + 1 < nchunks) stage.store(bc_s[(c + 1) & 1], bmode);
     __syncthreads();
   }
   cp_wait<0>();
+  if (ssum) *ssum = sacc;
 }
 
 template <int ROWS>
@@ -444,6 +520,7 @@ __device__ __forceinline__ bool load_row_params(const ScanArgs& p, int dc, RowPa
   rp.Dd = p.Dskip ? p.Dskip[int64_t(dc) * p.D_s] : 0.0f;
   const float* Ar = p.A + int64_t(dc) * p.A_sd;
   rp.A0 = Ar[0];
+  rp.invA0 = rp.A0 != 0.0f ? 1.0f / rp.A0 : 0.0f;
   bool st = true;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -454,9 +531,43 @@ __device__ __forceinline__ bool load_row_params(const ScanArgs& p, int dc, RowPa
   return st;
 }
 
+// The initial state of row (b, d): h0[b, d, :] when given, else zero.
+__device__ __forceinline__ void load_h0(const ScanArgs& p, int b, int d, f2_t (&h2)[8]) {
+  if (!p.h0) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) h2[k] = 0ull;
+    return;
+  }
+  const float* src = p.h0 + int64_t(b) * p.h0_sb + int64_t(d) * p.h0_sd;
+  if (p.vec_h0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(src) + i);
+      h2[2 * i] = f2(v.x, v.y);
+      h2[2 * i + 1] = f2(v.z, v.w);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) h2[k] = f2(__ldg(src + 2 * k), __ldg(src + 2 * k + 1));
+  }
+}
+
+// The forward sweep with the A path chosen at run time (uniform per CTA).
+template <typename T, int ROWS, bool HAS_Z, bool SOFTPLUS, bool ZOH>
+__device__ __forceinline__ void forward_any(const ScanArgs& p, float (*bc_s)[kTC * 32], uint4* slots, int b,
+                                            int t0, int t1, const T* urow, const T* dlrow, const T* zrow, T* orow,
+                                            bool row_ok, const RowParams& rp, bool structured, f2_t (&h2)[8]) {
+  if (structured)
+    forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, true, ZOH>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
+                                                       row_ok, rp, h2);
+  else
+    forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, false, ZOH>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
+                                                        row_ok, rp, h2);
+}
+
 // 64-row CTAs are used when the grid must fill 16 warps per SM (128 registers);
 // 32-row CTAs when the rows alone limit occupancy, so they may use up to 224.
-template <typename T, int ROWS, bool HAS_Z, bool SOFTPLUS>
+template <typename T, int ROWS, bool HAS_Z, bool SOFTPLUS, bool ZOH>
 __global__ void __launch_bounds__(ROWS, ROWS == 32 ? 9 : 8) scan_out_kernel(const ScanArgs p) {
   __shared__ __align__(16) float bc_s[2][kTC * 32];
   __shared__ __align__(16) uint4 slots[kStages * 3 * ROWS];
@@ -491,16 +602,11 @@ __global__ void __launch_bounds__(ROWS, ROWS == 32 ? 9 : 8) scan_out_kernel(cons
       h2[2 * i + 1] = f2(v.z, v.w);
     }
   } else {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) h2[k] = 0ull;
+    load_h0(p, b, dc, h2);
   }
 
-  if (structured)
-    forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, true>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
-                                                  row_ok, rp, h2);
-  else
-    forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, false>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
-                                                   row_ok, rp, h2);
+  forward_any<T, ROWS, HAS_Z, SOFTPLUS, ZOH>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow, row_ok, rp,
+                                             structured, h2);
 
   if (seg == p.nseg - 1 && row_ok && p.last_state) {
     float* dst = p.last_state + int64_t(b) * p.ls_sb + int64_t(d) * p.ls_sd;
@@ -545,7 +651,7 @@ __device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-template <typename T, bool HAS_Z, bool SOFTPLUS>
+template <typename T, bool HAS_Z, bool SOFTPLUS, bool ZOH>
 __global__ void __launch_bounds__(32, 8) scan_out_chained_kernel(const ScanArgs p) {
   constexpr int ROWS = 32;
   __shared__ __align__(16) float bc_s[2][kTC * 32];
@@ -576,8 +682,12 @@ __global__ void __launch_bounds__(32, 8) scan_out_chained_kernel(const ScanArgs 
     const bool st = load_row_params<ROWS>(p, dc, rp);
 
     f2_t h2[8];
+    if (c == 0) {
+      load_h0(p, b, dc, h2);
+    } else {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) h2[k] = 0ull;
+      for (int k = 0; k < 8; ++k) h2[k] = 0ull;
+    }
     if (c > 0) {
       if (tid == 0) {
         unsigned v = ld_acquire_u32(p.ch_flags + tile);
@@ -600,12 +710,8 @@ __global__ void __launch_bounds__(32, 8) scan_out_chained_kernel(const ScanArgs 
       }
     }
     const bool structured = __syncthreads_and(st) && !p.force_general;
-    if (structured)
-      forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, true>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
-                                                    row_ok, rp, h2);
-    else
-      forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, false>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
-                                                     row_ok, rp, h2);
+    forward_any<T, ROWS, HAS_Z, SOFTPLUS, ZOH>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow, row_ok, rp,
+                                               structured, h2);
     float v[16];
 #pragma unroll
     for (int k = 0; k < 8; ++k) f2split(h2[k], v[2 * k], v[2 * k + 1]);
@@ -751,7 +857,7 @@ __device__ __forceinline__ void backward_chunk(const ScanArgs& p, float (*bc_s)[
   Ssum = Tacc;
 }
 
-template <typename T, int ROWS, bool SOFTPLUS>
+template <typename T, int ROWS, bool SOFTPLUS, bool ZOH>
 __global__ void __launch_bounds__(ROWS, 512 / ROWS) scan_chunk_state_kernel(const ScanArgs p) {
   __shared__ __align__(16) float bc_s[2][kTC * 32];
   __shared__ __align__(16) uint4 slots[kStages * 3 * ROWS];
@@ -775,10 +881,20 @@ __global__ void __launch_bounds__(ROWS, 512 / ROWS) scan_chunk_state_kernel(cons
 #pragma unroll
   for (int k = 0; k < 8; ++k) H2[k] = 0ull;
   float Ssum = 0.0f;
-  if (structured)
+  if constexpr (ZOH) {
+    // zero-order hold: the summary is the chunk's end state from zero by a forward sweep
+    // (the backward form would need every step's own powers as well as the suffix decay)
+    if (structured)
+      forward_chunk<T, ROWS, false, SOFTPLUS, true, true, false>(p, bc_s, slots, b, t0, t1, urow, dlrow, nullptr,
+                                                                 nullptr, false, rp, H2, &Ssum);
+    else
+      forward_chunk<T, ROWS, false, SOFTPLUS, false, true, false>(p, bc_s, slots, b, t0, t1, urow, dlrow,
+                                                                  nullptr, nullptr, false, rp, H2, &Ssum);
+  } else if (structured) {
     backward_chunk<T, ROWS, SOFTPLUS, true>(p, bc_s, slots, b, t0, t1, urow, dlrow, rp, H2, Ssum);
-  else
+  } else {
     backward_chunk<T, ROWS, SOFTPLUS, false>(p, bc_s, slots, b, t0, t1, urow, dlrow, rp, H2, Ssum);
+  }
 
   const int64_t rows_total = int64_t(p.Bt) * p.tiles_per_batch * ROWS;
   const int64_t rowg = int64_t(tile) * ROWS + tid;
@@ -804,8 +920,7 @@ __global__ void __launch_bounds__(ROWS, 512 / ROWS) scan_chunk_state_kernel(cons
   if (!s_last) return;
   __threadfence();
   f2_t h[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) h[k] = 0ull;
+  load_h0(p, b, dc, h);
   const int nrec = p.nseg - 1;
   // records are prefetched one ahead so the serial walk waits on arithmetic, not on L2
   float4 nv[4];

@@ -138,6 +138,51 @@ def test_scan_validation(lib, case, expect):
     assert last_error(lib)
 
 
+class Ext(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_int32), ("discretization", ctypes.c_int32),
+                ("h0", ctypes.POINTER(T))]
+
+
+@pytest.mark.parametrize("case", ["short_struct", "bad_disc", "h0_shape", "h0_dtype", "h0_inner_stride",
+                                  "h0_aliases_last_state"])
+def test_scan_ext_validation(lib, case):
+    a = scan_args()
+    h0 = mk([2, 8, 16], 0)
+    ext = Ext(ctypes.sizeof(Ext), 0, ctypes.pointer(h0))
+    expect = INVALID
+    if case == "short_struct":
+        ext.struct_size = 4
+    elif case == "bad_disc":
+        ext.discretization = 2
+    elif case == "h0_shape":
+        ext.h0 = ctypes.pointer(mk([2, 8, 8], 0))
+        expect = INVALID
+    elif case == "h0_dtype":
+        ext.h0 = ctypes.pointer(mk([2, 8, 16], 1))
+    elif case == "h0_inner_stride":
+        ext.h0 = ctypes.pointer(mk([2, 8, 16], 0, stride=[256, 32, 2]))
+        expect = UNSUPPORTED
+    elif case == "h0_aliases_last_state":
+        h0.data = a["last_state"].data
+    P = lambda t: None if t is None else ctypes.byref(t)  # noqa: E731
+    f = lib.mssm_selective_scan_fwd_ex
+    f.restype = ctypes.c_int
+    st = f(P(a["u"]), P(a["delta"]), P(a["A"]), P(a["B"]), P(a["C"]), P(a["D"]), P(a["z"]), P(a["delta_bias"]),
+           1, ctypes.byref(ext), P(a["out"]), P(a["last_state"]), None)
+    assert st == expect, last_error(lib)
+    assert last_error(lib)
+
+
+def test_decode_ex_rejects_unknown_discretization(lib):
+    P = ctypes.byref
+    f = lib.mssm_state_update_ex
+    f.restype = ctypes.c_int
+    st, x, dt = mk([4, 8, 16], 0), mk([4, 8], 1), mk([4, 8], 1)
+    A, B, C, D, z, out = mk([8, 16], 0), mk([4, 16], 1), mk([4, 16], 1), mk([8], 0), mk([4, 8], 1), mk([4, 8], 1)
+    assert f(P(st), P(x), P(dt), P(A), P(B), P(C), P(D), P(z), None, 1, 5, P(out), None) == INVALID
+    assert "discretization" in last_error(lib)
+
+
 def test_empty_problem_is_noop(lib):
     # Bt == 0 returns OK without touching the device
     a = scan_args(Bt=0)

@@ -300,8 +300,8 @@ def test_softplus_and_silu_spot_values():
 
 
 # ---------------------------------------------------------------------------
-# 7b. zero-order hold ("Linear Attention vs Softmax Attention ...", Core Concepts;
-#     "Mamba selective state space", discretisation equations)
+# 7b. zero-order hold ("Linear Attention vs Softmax Attention ...", Core Concepts, item 3;
+#     "State Space Models in Large Language Models ...", Discretization)
 # ---------------------------------------------------------------------------
 
 def test_zoh_constant_input_is_exact():
