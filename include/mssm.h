@@ -261,6 +261,11 @@ mssm_status mssm_get_error(void *stream);
  *     aligned batch rows.  2 one bulk-copied tile of 256 rows per CTA; needs the
  *     contiguous state.  3 one thread per row, any layout.  A forced path whose
  *     conditions fail falls back to the next one that holds.
+ *   MSSM_OPT_TEST_HOOKS (value 0/1, for testing failure detection only): when 1,
+ *     the chained scan schedule publishes no carried states, so every chunk after
+ *     the first gives up its bounded wait (about 0.5 s), runs from a zero state
+ *     and sets the device error word; mssm_get_error then reports
+ *     MSSM_ERR_TIMEOUT.  No fault, trap or unbounded wait is involved.
  * Unknown options or invalid values return MSSM_ERR_INVALID_ARG.
  */
 typedef enum {
@@ -268,7 +273,8 @@ typedef enum {
     MSSM_OPT_CHUNK_LEN = 2,
     MSSM_OPT_KERNEL_TIMING = 3,
     MSSM_OPT_SCHEDULE = 4,
-    MSSM_OPT_DECODE_PATH = 5
+    MSSM_OPT_DECODE_PATH = 5,
+    MSSM_OPT_TEST_HOOKS = 6
 } mssm_option;
 mssm_status mssm_set_option(int option, int64_t value);
 

@@ -36,7 +36,8 @@ std::mutex g_mu;
 int g_force_general = 0;
 int64_t g_chunk_len = 0;
 int g_schedule = -1;
-int g_decode_path = 0;  // MSSM_OPT_DECODE_PATH  // -1 automatic, else the forced LaunchShape mode
+int g_decode_path = 0;  // MSSM_OPT_DECODE_PATH
+int g_test_hooks = 0;   // MSSM_OPT_TEST_HOOKS  // -1 automatic, else the forced LaunchShape mode
 
 // ---- launch accounting and optional per-kernel event timing (diagnostics)
 int64_t g_launches[MSSM_KERNEL_KINDS] = {0, 0, 0};
@@ -251,6 +252,10 @@ mssm_status mssm_set_option(int option, int64_t value) {
       if (value < 0 || value > 3) return fail(MSSM_ERR_INVALID_ARG, "SCHEDULE takes 0 (automatic) to 3");
       g_schedule = int(value) - 1;
       return MSSM_OK;
+    case MSSM_OPT_TEST_HOOKS:
+      if (value < 0 || value > 1) return fail(MSSM_ERR_INVALID_ARG, "TEST_HOOKS takes 0 or 1");
+      g_test_hooks = int(value);
+      return MSSM_OK;
     case MSSM_OPT_DECODE_PATH:
       if (value < 0 || value > 3) return fail(MSSM_ERR_INVALID_ARG, "DECODE_PATH takes 0 (automatic) to 3");
       g_decode_path = int(value);
@@ -382,6 +387,7 @@ struct ScanPlan {
 ScanPlan scan_plan(ScanCall& call, int sm_count) {
   mssm::ScanArgs& a = call.a;
   a.force_general = g_force_general;
+  a.test_no_publish = g_test_hooks & 1;
   const LaunchShape shape = choose_shape(call.Bt, call.D, call.L, sm_count, g_chunk_len, g_schedule);
   ScanPlan plan;
   plan.mode = shape.mode;

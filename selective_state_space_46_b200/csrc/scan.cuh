@@ -84,6 +84,7 @@ struct ScanArgs {
   unsigned* ch_flags;    // [tiles]: chunks of the tile whose carried state is published
   float* ch_carry;       // [tiles * 32][16]: carried state between consecutive chunks
   unsigned* err;         // device error word: bit 1 = a chained wait gave up
+  int test_no_publish;   // test hook: the chained kernel publishes no carried states
 };
 
 // ---------------------------------------------------------------------------
@@ -733,7 +734,7 @@ __global__ void __launch_bounds__(32, 8) scan_out_chained_kernel(const ScanArgs 
       for (int i = 0; i < 4; ++i) __stcg(dst + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
       __threadfence();
       __syncthreads();
-      if (tid == 0) st_release_u32(p.ch_flags + tile, unsigned(c + 1));
+      if (tid == 0 && !p.test_no_publish) st_release_u32(p.ch_flags + tile, unsigned(c + 1));
     }
     __syncthreads();
   }

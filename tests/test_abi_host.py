@@ -214,6 +214,8 @@ def test_options_and_strings(lib):
     assert lib.mssm_set_option(5, 4) == INVALID and lib.mssm_set_option(5, -1) == INVALID
     for v in (1, 2, 3, 0):
         assert lib.mssm_set_option(5, v) == 0
+    assert lib.mssm_set_option(6, 2) == INVALID
+    assert lib.mssm_set_option(6, 1) == 0 and lib.mssm_set_option(6, 0) == 0
     assert lib.mssm_set_option(2, 128) == 0
     assert lib.mssm_set_option(2, 0) == 0
     lib.mssm_status_string.restype = ctypes.c_char_p
