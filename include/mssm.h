@@ -56,7 +56,8 @@ extern "C" {
 
 typedef enum {
     MSSM_F32 = 0,
-    MSSM_BF16 = 1
+    MSSM_BF16 = 1,
+    MSSM_I32 = 2  /* index tensors only (cu_seqlens) */
 } mssm_dtype;
 
 typedef enum {
@@ -128,15 +129,29 @@ typedef enum {
  * Optional inputs of mssm_selective_scan_fwd_ex.  Set struct_size to
  * sizeof(mssm_scan_ext); fields may be appended in later versions.
  *   discretization  mssm_discretization
- *   h0              [Bt, D, N] f32, n stride 1: the state before step 0 (NULL: zero),
- *                   e.g. the last_state of the previous piece of a sequence processed
- *                   in parts (prefill in pieces, resume).  Must not alias out or
- *                   last_state.
+ *   h0              [S, D, N] f32, n stride 1: the state before the first step of each
+ *                   sequence (NULL: zero), e.g. the last_state of the previous piece of
+ *                   a sequence processed in parts (prefill in pieces, resume).  S = Bt,
+ *                   or the number of packed sequences.  Must not alias out or last_state.
+ *   cu_seqlens      [S + 1] int32 DEVICE tensor, or NULL: packed variable-length
+ *                   sequences.  u, delta, z, out are then [1, D, T] and B, C [1, N, T];
+ *                   sequence s covers steps cu_seqlens[s] .. cu_seqlens[s+1] - 1, starts
+ *                   from h0[s] (or zero), and its final state goes to last_state[s]
+ *                   ([S, D, N]).  Offsets must be non-decreasing within [0, T].
+ *   max_seqlen      host value >= every sequence length (used to plan the launch; only
+ *                   read with cu_seqlens).  Offsets outside [0, T], decreasing offsets
+ *                   or a longer sequence are clamped on the device and reported as
+ *                   MSSM_ERR_INVALID_ARG by mssm_get_error; the outputs are then undefined.
+ * The packed layout is the one the listed layer's batch would take with its padding
+ * removed; a sequence boundary resets the state, as if each sequence were its own batch
+ * row (the pages' scan has no state across batch rows).
  */
 typedef struct {
     int32_t struct_size;
     int32_t discretization;
     const mssm_tensor *h0;
+    const mssm_tensor *cu_seqlens;
+    int64_t max_seqlen;
 } mssm_scan_ext;
 
 /*
@@ -230,11 +245,13 @@ const char *mssm_last_error(void);
 
 /*
  * Synchronises `stream` and reports an asynchronous failure of the work queued
- * on it: MSSM_ERR_CUDA (with the CUDA error text in mssm_last_error()), or
+ * on it: MSSM_ERR_CUDA (with the CUDA error text in mssm_last_error());
  * MSSM_ERR_TIMEOUT when a bounded device-side wait gave up since the last call
- * (the decode kernel waits, with an iteration limit, for its own bulk copy; on
- * giving up it leaves that tile's state rows unchanged).  Clears the device
- * error word.  No kernel waits on another CTA or on the host.
+ * (the decode kernels wait, with an iteration limit, for their own bulk copies
+ * and on giving up leave that tile's state rows unchanged; the chained scan
+ * schedule waits for the previous chunk's carried state and on giving up runs
+ * the chunk from zero); MSSM_ERR_INVALID_ARG when a scan met inconsistent
+ * cu_seqlens.  Clears the device error word.  No kernel waits on the host.
  */
 mssm_status mssm_get_error(void *stream);
 

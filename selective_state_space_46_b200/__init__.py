@@ -52,7 +52,8 @@ class mssm_tensor(ctypes.Structure):
 
 class mssm_scan_ext(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_int32), ("discretization", ctypes.c_int32),
-                ("h0", ctypes.POINTER(mssm_tensor))]
+                ("h0", ctypes.POINTER(mssm_tensor)), ("cu_seqlens", ctypes.POINTER(mssm_tensor)),
+                ("max_seqlen", ctypes.c_int64)]
 
 
 _P = ctypes.POINTER(mssm_tensor)
@@ -92,7 +93,8 @@ class MssmError(RuntimeError):
         self.status = status
 
 
-_DT = {torch.float32: MSSM_F32, torch.bfloat16: MSSM_BF16}
+MSSM_I32 = 2
+_DT = {torch.float32: MSSM_F32, torch.bfloat16: MSSM_BF16, torch.int32: MSSM_I32}
 
 
 def _desc(t: Optional[torch.Tensor]):
@@ -181,13 +183,17 @@ def mssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, 
 
 
 def mssm_selective_scan_fwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state,
-                               h0=None, discretization=MSSM_DISC_EULER, stream=None) -> None:
+                               h0=None, discretization=MSSM_DISC_EULER, cu_seqlens=None, max_seqlen=0,
+                               stream=None) -> None:
     """Marshal torch tensors into ``mssm_selective_scan_fwd_ex``: the scan from an initial
-    state ``h0`` [Bt, D, N] (None: zero) with the given discretisation (see include/mssm.h)."""
+    state ``h0`` (None: zero) with the given discretisation, over packed sequences when
+    ``cu_seqlens`` (int32 device offsets) and ``max_seqlen`` are given (see include/mssm.h)."""
     ds = [_desc(t) for t in (u, delta, A, B, C, D, z, delta_bias, out, last_state)]
     dh = _desc(h0)
+    dc = _desc(cu_seqlens)
     ext = mssm_scan_ext(ctypes.sizeof(mssm_scan_ext), int(discretization),
-                        None if dh is None else ctypes.pointer(dh[1]))
+                        None if dh is None else ctypes.pointer(dh[1]),
+                        None if dc is None else ctypes.pointer(dc[1]), int(max_seqlen))
     _check(_lib.mssm_selective_scan_fwd_ex(*[_ref(x) for x in ds[:8]], int(softplus_flag), ctypes.byref(ext),
                                            _ref(ds[8]), _ref(ds[9]), _stream(stream, u)))
 
@@ -222,20 +228,26 @@ def mssm_state_update_ex(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, ou
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                        out=None, last_state=None, return_last_state=True, h0=None, zoh=False,
+                       cu_seqlens=None, max_seqlen=None,
                        stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Allocate ``out`` (and ``last_state``) with torch and run the scan on the GPU
-    (from ``h0`` when given; zero-order-hold input term when ``zoh``)."""
+    (from ``h0`` when given; zero-order-hold input term when ``zoh``; packed sequences
+    when ``cu_seqlens`` is given, with ``max_seqlen`` read back from it if omitted)."""
     if not u.is_cuda:
         raise ValueError("selective_scan_fwd runs on CUDA tensors only")
     if out is None:
         out = torch.empty_like(u, memory_format=torch.contiguous_format)
+    nstate = u.shape[0] if cu_seqlens is None else cu_seqlens.shape[0] - 1
     if last_state is None and return_last_state:
-        last_state = torch.empty(u.shape[0], u.shape[1], A.shape[1], device=u.device, dtype=torch.float32)
-    if h0 is None and not zoh:
+        last_state = torch.empty(nstate, u.shape[1], A.shape[1], device=u.device, dtype=torch.float32)
+    if cu_seqlens is not None and max_seqlen is None:
+        max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if nstate > 0 else 0
+    if h0 is None and not zoh and cu_seqlens is None:
         mssm_selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, out, last_state, stream)
     else:
         mssm_selective_scan_fwd_ex(u, delta, A, B, C, D, z, delta_bias, softplus, out, last_state, h0=h0,
-                                   discretization=MSSM_DISC_ZOH if zoh else MSSM_DISC_EULER, stream=stream)
+                                   discretization=MSSM_DISC_ZOH if zoh else MSSM_DISC_EULER,
+                                   cu_seqlens=cu_seqlens, max_seqlen=max_seqlen or 0, stream=stream)
     return out, last_state
 
 

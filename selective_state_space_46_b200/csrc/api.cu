@@ -101,9 +101,11 @@ DeviceState* device_state(int dev) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-size_t esize(int dtype) { return dtype == MSSM_BF16 ? 2 : 4; }
+size_t esize(int dtype) { return dtype == MSSM_BF16 ? 2 : 4; }  // f32, i32: 4
 
-const char* dname(int dtype) { return dtype == MSSM_BF16 ? "bf16" : dtype == MSSM_F32 ? "f32" : "?"; }
+const char* dname(int dtype) {
+  return dtype == MSSM_BF16 ? "bf16" : dtype == MSSM_F32 ? "f32" : dtype == MSSM_I32 ? "i32" : "?";
+}
 
 // Shape/dtype check of one tensor.  shape entries < 0 are not checked.
 mssm_status check(const mssm_tensor* t, const char* name, int ndim, const int64_t* shape,
@@ -279,13 +281,16 @@ struct ScanCall {
   bool has_z = false;
   bool softplus = false;
   bool noop = false;       // Bt * D == 0: nothing to launch
-  int64_t Bt = 0, D = 0, L = 0;
+  int64_t Bt = 0, D = 0, L = 0;  // as planned: packed sequences plan S x D x max_seqlen
 };
 
+// state_batches: the leading size of last_state (and h0) when it is not Bt (packed
+// sequences: their count), else -1.
 mssm_status scan_prepare(const mssm_tensor* u, const mssm_tensor* delta, const mssm_tensor* A,
                          const mssm_tensor* B, const mssm_tensor* C, const mssm_tensor* D,
                          const mssm_tensor* z, const mssm_tensor* delta_bias, int softplus_flag,
-                         mssm_tensor* out, mssm_tensor* last_state, ScanCall& call) {
+                         mssm_tensor* out, mssm_tensor* last_state, ScanCall& call,
+                         int64_t state_batches = -1) {
   if (!u) return fail(MSSM_ERR_INVALID_ARG, "u: null tensor descriptor");
   if (u->ndim != 3) return fail(MSSM_ERR_INVALID_ARG, "u: expected 3 dims [Bt, D, L]");
   const int dt = u->dtype;
@@ -295,7 +300,7 @@ mssm_status scan_prepare(const mssm_tensor* u, const mssm_tensor* delta, const m
   if (N != mssm::kN)
     return fail(MSSM_ERR_UNSUPPORTED, "state size N = %lld; this build supports N = %d", (long long)N, mssm::kN);
   const int64_t s_bdl[3] = {Bt, Dd, L}, s_bnl[3] = {Bt, N, L}, s_dn[2] = {Dd, N}, s_d[1] = {Dd},
-                s_bdn[3] = {Bt, Dd, N};
+                s_bdn[3] = {state_batches >= 0 ? state_batches : Bt, Dd, N};
   mssm_status st;
   if ((st = check(u, "u", 3, s_bdl, dt, true)) != MSSM_OK) return st;
   if ((st = check(delta, "delta", 3, s_bdl, dt, true)) != MSSM_OK) return st;
@@ -346,16 +351,50 @@ mssm_status scan_prepare(const mssm_tensor* u, const mssm_tensor* delta, const m
   return MSSM_OK;
 }
 
-// The optional inputs of mssm_selective_scan_fwd_ex: initial state and discretisation.
-mssm_status scan_prepare_ext(const mssm_scan_ext* ext, const mssm_tensor* out, const mssm_tensor* last_state,
-                             ScanCall& call) {
+// First checks of an mssm_scan_ext; returns the packed-sequence count through nseq
+// (-1 without cu_seqlens).
+mssm_status scan_ext_header(const mssm_scan_ext* ext, int64_t* nseq) {
+  *nseq = -1;
   if (!ext) return MSSM_OK;
   if (ext->struct_size < int32_t(sizeof(mssm_scan_ext)))
     return fail(MSSM_ERR_INVALID_ARG, "ext->struct_size = %d; expected at least %d", int(ext->struct_size),
                 int(sizeof(mssm_scan_ext)));
   if (ext->discretization != MSSM_DISC_EULER && ext->discretization != MSSM_DISC_ZOH)
     return fail(MSSM_ERR_INVALID_ARG, "ext->discretization must be MSSM_DISC_EULER or MSSM_DISC_ZOH");
+  const mssm_tensor* cu = ext->cu_seqlens;
+  if (cu) {
+    const int64_t any[1] = {-1};
+    mssm_status st = check(cu, "cu_seqlens", 1, any, MSSM_I32, true);
+    if (st != MSSM_OK) return st;
+    if (cu->shape[0] < 1) return fail(MSSM_ERR_INVALID_ARG, "cu_seqlens: expected S + 1 >= 1 offsets");
+    if (cu->shape[0] - 1 > INT32_MAX) return fail(MSSM_ERR_UNSUPPORTED, "too many sequences");
+    *nseq = cu->shape[0] - 1;
+  }
+  return MSSM_OK;
+}
+
+// The optional inputs of mssm_selective_scan_fwd_ex: initial state, discretisation and
+// packed sequences (after scan_prepare has checked the main tensors).
+mssm_status scan_prepare_ext(const mssm_scan_ext* ext, const mssm_tensor* out, const mssm_tensor* last_state,
+                             ScanCall& call) {
+  if (!ext) return MSSM_OK;
   call.a.zoh = ext->discretization == MSSM_DISC_ZOH;
+  const mssm_tensor* cu = ext->cu_seqlens;
+  if (cu) {
+    if (call.Bt != 1)
+      return fail(MSSM_ERR_INVALID_ARG, "with cu_seqlens, u/delta/z/out must be [1, D, T] (got Bt = %lld)",
+                  (long long)call.Bt);
+    const int64_t S = cu->shape[0] - 1;
+    if (ext->max_seqlen < 0 || ext->max_seqlen > call.L)
+      return fail(MSSM_ERR_INVALID_ARG, "max_seqlen = %lld must lie in [0, T = %lld]",
+                  (long long)ext->max_seqlen, (long long)call.L);
+    // plan as S independent rows of max_seqlen steps; the kernels read each sequence's range
+    call.Bt = S;
+    call.L = ext->max_seqlen;
+    call.noop = (S == 0 || call.D == 0);
+    call.a.Bt = int(S);
+    call.a.cu_seqlens = static_cast<const int*>(cu->data);
+  }
   const mssm_tensor* h0 = ext->h0;
   if (h0) {
     const int64_t s_bdn[3] = {call.Bt, call.D, mssm::kN};
@@ -427,10 +466,9 @@ void scan_bind_workspace(mssm::ScanArgs& a, const ScanPlan& plan, void* ws) {
 // The kernel launches of a planned call (caller holds g_mu).  `ws` is the
 // workspace base the plan was bound to (mode 2 zeroes its ticket and flags).
 mssm_status scan_launch(ScanCall& call, const ScanPlan& plan, void* ws, cudaStream_t s) {
-  cudaError_t e;
+  cudaError_t e = mssm::device_error_word(&call.a.err);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
   if (plan.mode == 2) {
-    e = mssm::device_error_word(&call.a.err);
-    if (e != cudaSuccess) return cuda_fail(e, "device error word");
     e = cudaMemsetAsync(ws, 0, plan.count_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(chained schedule flags)");
     e = tracked(MSSM_KERNEL_SCAN_OUT, s, [&] {
@@ -544,8 +582,11 @@ mssm_status mssm_selective_scan_fwd_ex(const mssm_tensor* u, const mssm_tensor* 
                                        const mssm_tensor* z, const mssm_tensor* delta_bias,
                                        int softplus_flag, const mssm_scan_ext* ext, mssm_tensor* out,
                                        mssm_tensor* last_state, void* stream) {
+  int64_t nseq = -1;
+  mssm_status st = scan_ext_header(ext, &nseq);
+  if (st != MSSM_OK) return st;
   ScanCall call;
-  mssm_status st = scan_prepare(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state, call);
+  st = scan_prepare(u, delta, A, B, C, D, z, delta_bias, softplus_flag, out, last_state, call, nseq);
   if (st != MSSM_OK) return st;
   if ((st = scan_prepare_ext(ext, out, last_state, call)) != MSSM_OK || call.noop) return st;
   return scan_fwd_impl(call, stream);
@@ -780,6 +821,12 @@ mssm_status mssm_get_error(void* stream) {
   if (word & 1u)
     return fail(MSSM_ERR_TIMEOUT, "a decode bulk copy did not complete within its bounded wait; "
                 "the state rows of that tile were left unchanged");
+  if (word & 2u)
+    return fail(MSSM_ERR_TIMEOUT, "a chained scan chunk gave up waiting for the previous chunk's "
+                "carried state and ran from a zero state");
+  if (word & 4u)
+    return fail(MSSM_ERR_INVALID_ARG, "cu_seqlens held an offset outside [0, T], a decreasing offset "
+                "or a sequence longer than max_seqlen; the scan outputs are undefined");
   return MSSM_OK;
 }
 

@@ -85,7 +85,38 @@ struct ScanArgs {
   float* ch_carry;       // [tiles * 32][16]: carried state between consecutive chunks
   unsigned* err;         // device error word: bit 1 = a chained wait gave up
   int test_no_publish;   // test hook: the chained kernel publishes no carried states
+  // packed variable-length sequences: Bt is the sequence count, the data has one batch row,
+  // sequence v covers steps cu_seqlens[v] .. cu_seqlens[v+1] - 1 of it (null: plain batches)
+  const int* cu_seqlens;
 };
+
+// The steps of virtual batch v: data batch row b, first step tb, length len, and the
+// index of its last chunk.  Offsets outside [0, L], decreasing offsets, or a sequence
+// longer than the planned nseg * seg_len are clamped and flagged (error word bit 2).
+struct SeqRange {
+  int b, tb, len, last_seg;
+};
+__device__ __forceinline__ SeqRange seq_range(const ScanArgs& p, int v) {
+  SeqRange r;
+  if (!p.cu_seqlens) {
+    r.b = v;
+    r.tb = 0;
+    r.len = p.L;
+  } else {
+    int a = __ldg(p.cu_seqlens + v), e = __ldg(p.cu_seqlens + v + 1);
+    const int cap = p.nseg * p.seg_len;
+    bool bad = a < 0 || a > p.L || e < a || e > p.L || e - a > cap;
+    a = min(max(a, 0), p.L);
+    e = min(max(e, a), p.L);
+    if (e - a > cap) e = a + cap;
+    if (bad && threadIdx.x == 0 && p.err) atomicOr(p.err, 4u);
+    r.b = 0;
+    r.tb = a;
+    r.len = e - a;
+  }
+  r.last_seg = r.len > 0 ? (r.len - 1) / p.seg_len : 0;
+  return r;
+}
 
 // ---------------------------------------------------------------------------
 // small device helpers
@@ -223,30 +254,32 @@ __device__ __forceinline__ void fetch_block(uint4* slot, const T* row, int t, in
   }
 }
 
-// Store a block of y (S steps of fp32 values) at step t, clipped at t_end.
+// Store a block of y (S steps of fp32 values) at step t, clipped to [t_lo, t_end).
 template <typename T>
-__device__ __forceinline__ void store_block(T* row, int t, int t_end, bool vec, const float* y) {
+__device__ __forceinline__ void store_block(T* row, int t, int t_lo, int t_end, bool vec, const float* y) {
   constexpr int S = 16 / int(sizeof(T));
+  const bool whole = vec && t >= t_lo && t + S <= t_end;
   if constexpr (sizeof(T) == 2) {
     const uint32_t w0 = pack_bf16x2(y[0], y[1]), w1 = pack_bf16x2(y[2], y[3]);
     const uint32_t w2 = pack_bf16x2(y[4], y[5]), w3 = pack_bf16x2(y[6], y[7]);
-    if (vec && t + S <= t_end) {
+    if (whole) {
       *reinterpret_cast<uint4*>(row + t) = make_uint4(w0, w1, w2, w3);
     } else {
       const uint32_t w[4] = {w0, w1, w2, w3};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        if (t + 2 * i < t_end) row[t + 2 * i] = uint16_t(w[i] & 0xffffu);
-        if (t + 2 * i + 1 < t_end) row[t + 2 * i + 1] = uint16_t(w[i] >> 16);
+        const int ta = t + 2 * i, tb = t + 2 * i + 1;
+        if (ta >= t_lo && ta < t_end) row[ta] = uint16_t(w[i] & 0xffffu);
+        if (tb >= t_lo && tb < t_end) row[tb] = uint16_t(w[i] >> 16);
       }
     }
   } else {
-    if (vec && t + S <= t_end) {
+    if (whole) {
       *reinterpret_cast<float4*>(row + t) = make_float4(y[0], y[1], y[2], y[3]);
     } else {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        if (t + i < t_end) row[t + i] = y[i];
+        if (t + i >= t_lo && t + i < t_end) row[t + i] = y[i];
     }
   }
 }
@@ -299,8 +332,8 @@ __device__ __forceinline__ void decay(float s, const RowParams& rp, f2_t (&dA)[8
 // ---------------------------------------------------------------------------
 
 // Per-step scalars of one block: x = decay base 2^(s A_0) (structured A) or s
-// (general A), w = s * u.  PARTIAL: steps at or past `valid` become identity
-// steps (s = 0: A_bar = 1 and no input).
+// (general A), w = s * u.  PARTIAL: steps before `lo` or at or past `valid` become
+// identity steps (s = 0: A_bar = 1 and no input).
 //
 // Zero-order hold (ZOH): the input term of state n is G_n B_n u with G_n =
 // (exp(delta A_n) - 1) / A_n.  Structured A: exp(delta A_n) - 1 = E (1 + a + ... + a^n)
@@ -310,8 +343,8 @@ __device__ __forceinline__ void decay(float s, const RowParams& rp, f2_t (&dA)[8
 // the recurrence forms w P_n by a running FMA over the powers it already has.
 // General A: w = u and the recurrence takes G_n per state.  sv[j] = s (for the sum S).
 template <typename T, bool SOFTPLUS, bool STRUCT, bool PARTIAL, bool ZOH = false>
-__device__ __forceinline__ void block_scalars(const uint4& ru, const uint4& rd, int valid, const RowParams& rp,
-                                              float* x, float* w, float* sv = nullptr) {
+__device__ __forceinline__ void block_scalars(const uint4& ru, const uint4& rd, int lo, int valid,
+                                              const RowParams& rp, float* x, float* w, float* sv = nullptr) {
   constexpr int S = 16 / int(sizeof(T));
 #pragma unroll
   for (int j = 0; j < S; ++j) {
@@ -319,8 +352,9 @@ __device__ __forceinline__ void block_scalars(const uint4& ru, const uint4& rd, 
     float s = SOFTPLUS ? softplus2(v2) : v2;
     float uu = blk_at<T>(ru, j);
     if constexpr (PARTIAL) {
-      s = (j < valid) ? s : 0.0f;
-      uu = (j < valid) ? uu : 0.0f;
+      const bool in = j >= lo && j < valid;
+      s = in ? s : 0.0f;
+      uu = in ? uu : 0.0f;
     }
     x[j] = STRUCT ? ex2f(s * rp.A0) : s;
     if constexpr (!ZOH) {
@@ -426,25 +460,30 @@ __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[k
   constexpr int kBlkPerChunk = kTC / S;
   const int tid = threadIdx.x;
   const bool vec = p.vec_rows != 0;
-  const int nblk = (t1 - t0 + S - 1) / S;
-  const int nchunks = (t1 - t0 + kTC - 1) / kTC;
-  if (nchunks <= 0) return;
+  if (t1 <= t0) return;
+  // blocks are aligned to S-step boundaries of the row; a chunk that starts inside a block
+  // (packed sequences) runs its first `head` steps as identity steps and stores nothing there
+  const int ta = t0 - t0 % S;
+  const int head = t0 - ta;
+  const int nblk = (t1 - ta + S - 1) / S;
+  const int nchunks = (t1 - ta + kTC - 1) / kTC;
 
   auto slot = [&](int stage, int tensor) { return slots + (stage * 3 + tensor) * ROWS + tid; };
   auto issue = [&](int k) {
-    const int t = t0 + k * S;
+    const int t = ta + k * S;
     const int st = k % kStages;
     fetch_block<T>(slot(st, 0), urow, t, t1, vec);
     fetch_block<T>(slot(st, 1), dlrow, t, t1, vec);
     if constexpr (LOAD_Z) fetch_block<T>(slot(st, 2), zrow, t, t1, vec);
   };
   auto scalars = [&](int k, const uint4& ru, const uint4& rd, float* x, float* w) {
-    const int valid = t1 - (t0 + k * S);
+    const int valid = t1 - (ta + k * S);
+    const int lo = k == 0 ? head : 0;
     float sv[S];
-    if (valid >= S)
-      block_scalars<T, SOFTPLUS, STRUCT, false, ZOH>(ru, rd, S, rp, x, w, READOUT ? nullptr : sv);
+    if (valid >= S && lo == 0)
+      block_scalars<T, SOFTPLUS, STRUCT, false, ZOH>(ru, rd, 0, S, rp, x, w, READOUT ? nullptr : sv);
     else
-      block_scalars<T, SOFTPLUS, STRUCT, true, ZOH>(ru, rd, valid, rp, x, w, READOUT ? nullptr : sv);
+      block_scalars<T, SOFTPLUS, STRUCT, true, ZOH>(ru, rd, lo, valid, rp, x, w, READOUT ? nullptr : sv);
     if constexpr (!READOUT) {
 #pragma unroll
       for (int j = 0; j < S; ++j) sacc += sv[j];
@@ -457,7 +496,7 @@ __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[k
   }
 
   BCStage<T, ROWS> stage;
-  stage.load(p, b, t0, t1);
+  stage.load(p, b, ta, t1);
   stage.store(bc_s[0], bmode);
 
   // block 0's scalars
@@ -470,7 +509,7 @@ __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[k
 
   int k = 0;
   for (int c = 0; c < nchunks; ++c) {
-    const int cs = t0 + c * kTC;
+    const int cs = ta + c * kTC;
     if (c + 1 < nchunks) stage.load(p, b, cs + kTC, t1);
     const float* bcb = bc_s[c & 1];
 #pragma unroll 1
@@ -497,7 +536,7 @@ __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[k
           if constexpr (HAS_Z) v *= gate_f<T>(blk_at<T>(rz, j));
           y[j] = v;
         }
-        if (row_ok) store_block<T>(orow, t0 + k * S, t1, vec, y);
+        if (row_ok) store_block<T>(orow, ta + k * S, t0, t1, vec, y);
       }
 #pragma unroll
       for (int j = 0; j < S; ++j) {
@@ -575,12 +614,15 @@ __global__ void __launch_bounds__(ROWS, ROWS == 32 ? 9 : 8) scan_out_kernel(cons
   const int tid = threadIdx.x;
   const int tile = blockIdx.x;
   const int seg = blockIdx.y;
-  const int b = tile / p.tiles_per_batch;
-  const int d = (tile - b * p.tiles_per_batch) * ROWS + tid;
+  const int vb = tile / p.tiles_per_batch;  // batch, or sequence of a packed batch
+  const SeqRange sr = seq_range(p, vb);
+  if (seg > sr.last_seg) return;  // past the end of a shorter packed sequence
+  const int b = sr.b;
+  const int d = (tile - vb * p.tiles_per_batch) * ROWS + tid;
   const bool row_ok = d < p.D;
   const int dc = row_ok ? d : p.D - 1;
-  const int t0 = seg * p.seg_len;
-  const int t1 = min(p.L, t0 + p.seg_len);
+  const int t0 = sr.tb + seg * p.seg_len;
+  const int t1 = sr.tb + min(sr.len, (seg + 1) * p.seg_len);
 
   const T* urow = static_cast<const T*>(p.u) + int64_t(b) * p.u_sb + int64_t(dc) * p.u_sd;
   const T* dlrow = static_cast<const T*>(p.delta) + int64_t(b) * p.dl_sb + int64_t(dc) * p.dl_sd;
@@ -603,14 +645,14 @@ __global__ void __launch_bounds__(ROWS, ROWS == 32 ? 9 : 8) scan_out_kernel(cons
       h2[2 * i + 1] = f2(v.z, v.w);
     }
   } else {
-    load_h0(p, b, dc, h2);
+    load_h0(p, vb, dc, h2);
   }
 
   forward_any<T, ROWS, HAS_Z, SOFTPLUS, ZOH>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow, row_ok, rp,
                                              structured, h2);
 
-  if (seg == p.nseg - 1 && row_ok && p.last_state) {
-    float* dst = p.last_state + int64_t(b) * p.ls_sb + int64_t(d) * p.ls_sd;
+  if (seg == sr.last_seg && row_ok && p.last_state) {
+    float* dst = p.last_state + int64_t(vb) * p.ls_sb + int64_t(d) * p.ls_sd;
     float v[16];
 #pragma unroll
     for (int k = 0; k < 8; ++k) f2split(h2[k], v[2 * k], v[2 * k + 1]);
@@ -669,12 +711,16 @@ __global__ void __launch_bounds__(32, 8) scan_out_chained_kernel(const ScanArgs 
     if (item >= nitems) break;
     const int c = item / ntiles;
     const int tile = item - c * ntiles;
-    const int b = tile / p.tiles_per_batch;
-    const int d = (tile - b * p.tiles_per_batch) * ROWS + tid;
+    const int vb = tile / p.tiles_per_batch;  // batch, or sequence of a packed batch
+    const SeqRange sr = seq_range(p, vb);
+    __syncthreads();                         // every thread has read s_item
+    if (c > sr.last_seg) continue;           // past the end of a shorter packed sequence
+    const int b = sr.b;
+    const int d = (tile - vb * p.tiles_per_batch) * ROWS + tid;
     const bool row_ok = d < p.D;
     const int dc = row_ok ? d : p.D - 1;
-    const int t0 = c * p.seg_len;
-    const int t1 = min(p.L, t0 + p.seg_len);
+    const int t0 = sr.tb + c * p.seg_len;
+    const int t1 = sr.tb + min(sr.len, (c + 1) * p.seg_len);
     const T* urow = static_cast<const T*>(p.u) + int64_t(b) * p.u_sb + int64_t(dc) * p.u_sd;
     const T* dlrow = static_cast<const T*>(p.delta) + int64_t(b) * p.dl_sb + int64_t(dc) * p.dl_sd;
     const T* zrow = HAS_Z ? static_cast<const T*>(p.z) + int64_t(b) * p.z_sb + int64_t(dc) * p.z_sd : nullptr;
@@ -684,7 +730,7 @@ __global__ void __launch_bounds__(32, 8) scan_out_chained_kernel(const ScanArgs 
 
     f2_t h2[8];
     if (c == 0) {
-      load_h0(p, b, dc, h2);
+      load_h0(p, vb, dc, h2);
     } else {
 #pragma unroll
       for (int k = 0; k < 8; ++k) h2[k] = 0ull;
@@ -716,9 +762,9 @@ __global__ void __launch_bounds__(32, 8) scan_out_chained_kernel(const ScanArgs 
     float v[16];
 #pragma unroll
     for (int k = 0; k < 8; ++k) f2split(h2[k], v[2 * k], v[2 * k + 1]);
-    if (c == p.nseg - 1) {
+    if (c == sr.last_seg) {
       if (row_ok && p.last_state) {
-        float* dst = p.last_state + int64_t(b) * p.ls_sb + int64_t(d) * p.ls_sd;
+        float* dst = p.last_state + int64_t(vb) * p.ls_sb + int64_t(d) * p.ls_sd;
         if (p.vec_ls) {
 #pragma unroll
           for (int i = 0; i < 4; ++i)
@@ -858,7 +904,9 @@ __device__ __forceinline__ void backward_chunk(const ScanArgs& p, float (*bc_s)[
   Ssum = Tacc;
 }
 
-template <typename T, int ROWS, bool SOFTPLUS, bool ZOH>
+// FWD: summaries by the forward sweep (zero-order hold, packed sequences whose chunks start
+// inside a 16-byte block); otherwise by the cheaper backward sweep.
+template <typename T, int ROWS, bool SOFTPLUS, bool ZOH, bool FWD>
 __global__ void __launch_bounds__(ROWS, 512 / ROWS) scan_chunk_state_kernel(const ScanArgs p) {
   __shared__ __align__(16) float bc_s[2][kTC * 32];
   __shared__ __align__(16) uint4 slots[kStages * 3 * ROWS];
@@ -866,11 +914,14 @@ __global__ void __launch_bounds__(ROWS, 512 / ROWS) scan_chunk_state_kernel(cons
   const int tid = threadIdx.x;
   const int tile = blockIdx.x;
   const int seg = blockIdx.y;  // 0 .. nseg-2
-  const int b = tile / p.tiles_per_batch;
-  const int d = (tile - b * p.tiles_per_batch) * ROWS + tid;
+  const int vb = tile / p.tiles_per_batch;  // batch, or sequence of a packed batch
+  const SeqRange sr = seq_range(p, vb);
+  if (seg >= sr.last_seg) return;  // the last chunk of a sequence needs no summary
+  const int b = sr.b;
+  const int d = (tile - vb * p.tiles_per_batch) * ROWS + tid;
   const int dc = d < p.D ? d : p.D - 1;
-  const int t0 = seg * p.seg_len;
-  const int t1 = t0 + p.seg_len;
+  const int t0 = sr.tb + seg * p.seg_len;
+  const int t1 = t0 + p.seg_len;  // not the last chunk: always full
 
   const T* urow = static_cast<const T*>(p.u) + int64_t(b) * p.u_sb + int64_t(dc) * p.u_sd;
   const T* dlrow = static_cast<const T*>(p.delta) + int64_t(b) * p.dl_sb + int64_t(dc) * p.dl_sd;
@@ -882,15 +933,15 @@ __global__ void __launch_bounds__(ROWS, 512 / ROWS) scan_chunk_state_kernel(cons
 #pragma unroll
   for (int k = 0; k < 8; ++k) H2[k] = 0ull;
   float Ssum = 0.0f;
-  if constexpr (ZOH) {
-    // zero-order hold: the summary is the chunk's end state from zero by a forward sweep
-    // (the backward form would need every step's own powers as well as the suffix decay)
+  if constexpr (ZOH || FWD) {
+    // the summary is the chunk's end state from zero by a forward sweep (for the zero-order
+    // hold the backward form would need every step's own powers as well as the suffix decay)
     if (structured)
-      forward_chunk<T, ROWS, false, SOFTPLUS, true, true, false>(p, bc_s, slots, b, t0, t1, urow, dlrow, nullptr,
-                                                                 nullptr, false, rp, H2, &Ssum);
+      forward_chunk<T, ROWS, false, SOFTPLUS, true, ZOH, false>(p, bc_s, slots, b, t0, t1, urow, dlrow, nullptr,
+                                                                nullptr, false, rp, H2, &Ssum);
     else
-      forward_chunk<T, ROWS, false, SOFTPLUS, false, true, false>(p, bc_s, slots, b, t0, t1, urow, dlrow,
-                                                                  nullptr, nullptr, false, rp, H2, &Ssum);
+      forward_chunk<T, ROWS, false, SOFTPLUS, false, ZOH, false>(p, bc_s, slots, b, t0, t1, urow, dlrow,
+                                                                 nullptr, nullptr, false, rp, H2, &Ssum);
   } else if (structured) {
     backward_chunk<T, ROWS, SOFTPLUS, true>(p, bc_s, slots, b, t0, t1, urow, dlrow, rp, H2, Ssum);
   } else {
@@ -916,13 +967,13 @@ __global__ void __launch_bounds__(ROWS, 512 / ROWS) scan_chunk_state_kernel(cons
   // over H_k.  Nobody waits: the fold runs in whichever CTA arrives last.
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&p.ws_count[tile], 1u) == unsigned(p.nseg - 2));
+  if (tid == 0) s_last = (atomicAdd(&p.ws_count[tile], 1u) == unsigned(sr.last_seg - 1));
   __syncthreads();
   if (!s_last) return;
   __threadfence();
   f2_t h[8];
-  load_h0(p, b, dc, h);
-  const int nrec = p.nseg - 1;
+  load_h0(p, vb, dc, h);
+  const int nrec = sr.last_seg;
   // records are prefetched one ahead so the serial walk waits on arithmetic, not on L2
   float4 nv[4];
   float nS = 0.0f;

@@ -13,7 +13,15 @@ struct ScanDispatch {
   template <typename T, int ROWS, bool SP>
   static cudaError_t chunk_state_t(const ScanArgs& a, cudaStream_t s) {
     dim3 g(a.Bt * a.tiles_per_batch, a.nseg - 1);
-    scan_chunk_state_kernel<T, ROWS, SP, ZOH><<<g, ROWS, 0, s>>>(a);
+    // packed sequences take the forward-sweep summaries (their chunks may start inside a block)
+    if constexpr (ZOH) {
+      scan_chunk_state_kernel<T, ROWS, SP, true, true><<<g, ROWS, 0, s>>>(a);
+    } else {
+      if (a.cu_seqlens)
+        scan_chunk_state_kernel<T, ROWS, SP, false, true><<<g, ROWS, 0, s>>>(a);
+      else
+        scan_chunk_state_kernel<T, ROWS, SP, false, false><<<g, ROWS, 0, s>>>(a);
+    }
     return cudaGetLastError();
   }
   template <typename T, int ROWS, bool HAS_Z, bool SP>

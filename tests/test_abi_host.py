@@ -140,7 +140,7 @@ def test_scan_validation(lib, case, expect):
 
 class Ext(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_int32), ("discretization", ctypes.c_int32),
-                ("h0", ctypes.POINTER(T))]
+                ("h0", ctypes.POINTER(T)), ("cu_seqlens", ctypes.POINTER(T)), ("max_seqlen", ctypes.c_int64)]
 
 
 @pytest.mark.parametrize("case", ["short_struct", "bad_disc", "h0_shape", "h0_dtype", "h0_inner_stride",
@@ -170,6 +170,36 @@ def test_scan_ext_validation(lib, case):
     st = f(P(a["u"]), P(a["delta"]), P(a["A"]), P(a["B"]), P(a["C"]), P(a["D"]), P(a["z"]), P(a["delta_bias"]),
            1, ctypes.byref(ext), P(a["out"]), P(a["last_state"]), None)
     assert st == expect, last_error(lib)
+    assert last_error(lib)
+
+
+@pytest.mark.parametrize("case", ["cu_dtype", "cu_2d", "batch_not_1", "last_state_batches", "max_seqlen_big",
+                                  "h0_batches"])
+def test_scan_varlen_validation(lib, case):
+    S, D, Tn = 3, 8, 40
+    a = scan_args(Bt=1, D=D, L=Tn)
+    a["last_state"] = mk([S, D, 16], 0)
+    cu = mk([S + 1], 2)
+    ext = Ext(ctypes.sizeof(Ext), 0, None, ctypes.pointer(cu), 20)
+    if case == "cu_dtype":
+        ext.cu_seqlens = ctypes.pointer(mk([S + 1], 0))
+    elif case == "cu_2d":
+        ext.cu_seqlens = ctypes.pointer(mk([1, S + 1], 2))
+    elif case == "batch_not_1":
+        a = scan_args(Bt=2, D=D, L=Tn)
+        a["last_state"] = mk([S, D, 16], 0)
+    elif case == "last_state_batches":
+        a["last_state"] = mk([1, D, 16], 0)
+    elif case == "max_seqlen_big":
+        ext.max_seqlen = Tn + 1
+    elif case == "h0_batches":
+        ext.h0 = ctypes.pointer(mk([1, D, 16], 0))
+    P = lambda t: None if t is None else ctypes.byref(t)  # noqa: E731
+    f = lib.mssm_selective_scan_fwd_ex
+    f.restype = ctypes.c_int
+    st = f(P(a["u"]), P(a["delta"]), P(a["A"]), P(a["B"]), P(a["C"]), P(a["D"]), P(a["z"]), P(a["delta_bias"]),
+           1, ctypes.byref(ext), P(a["out"]), P(a["last_state"]), None)
+    assert st == INVALID, (st, last_error(lib))
     assert last_error(lib)
 
 
