@@ -266,8 +266,9 @@ class ClockSampler:
 # reference arm: the fp64 CPU oracle on the host cores
 # --------------------------------------------------------------------------
 
-def oracle_sample(workload: str, rows: int):
-    """A bounded sample of the workload for the CPU oracle: the first ``rows`` channels of batch 0."""
+def oracle_sample(workload: str, rows: int, zoh: bool = False):
+    """A bounded sample of the workload for the CPU oracle: the first ``rows`` channels of batch 0
+    (of every packed sequence, for a packed workload)."""
     import oracle
     inp = synth.workload_inputs(workload)
     if isinstance(inp, synth.ScanInputs):
@@ -276,9 +277,14 @@ def oracle_sample(workload: str, rows: int):
                     B=inp.f64("B")[:1], C=inp.f64("C")[:1], D=None if inp.D is None else inp.f64("D")[:d],
                     z=None if inp.z is None else inp.f64("z")[:1, :d],
                     delta_bias=None if inp.delta_bias is None else inp.f64("delta_bias")[:d],
-                    softplus=inp.softplus)
+                    softplus=inp.softplus, zoh=zoh)
         units = d * inp.length
-        desc = f"batch 0, channels 0..{d - 1}, all {inp.length} steps ({units} elements)"
+        disc = ", zero-order hold" if zoh else ""
+        if inp.cu_seqlens is not None:
+            cu = inp.cu_seqlens
+            desc = (f"channels 0..{d - 1} of all {len(cu) - 1} packed sequences ({units} elements{disc})")
+            return (lambda: oracle.scan_varlen(cu_seqlens=cu, **args)), units, desc
+        desc = f"batch 0, channels 0..{d - 1}, all {inp.length} steps ({units} elements{disc})"
         return (lambda: oracle.scan(**args)), units, desc
     b = max(1, min(inp.batch, rows // inp.dim if rows >= inp.dim else 1))
     args = dict(state=inp.state[:b], x=inp.f64("x")[:b], dt=inp.f64("dt")[:b], A=inp.f64("A"),
@@ -288,11 +294,11 @@ def oracle_sample(workload: str, rows: int):
     return (lambda: oracle.state_update(**args)), units, f"batches 0..{b - 1} ({units} rows)"
 
 
-def cpu_baseline(workload: str, budget_s: float = 10.0):
+def cpu_baseline(workload: str, budget_s: float = 10.0, zoh: bool = False):
     import oracle
     is_scan = WORKLOADS_KIND[workload] == "scan"
     rows = 512 if is_scan else 256 * 5120
-    fn, units, desc = oracle_sample(workload, rows)
+    fn, units, desc = oracle_sample(workload, rows, zoh)
     fn()  # build + warm
     t0 = time.perf_counter()
     n = 0
@@ -315,7 +321,7 @@ def run_reference(args):
         return 0
     import oracle
     is_scan = WORKLOADS_KIND[args.workload] == "scan"
-    fn, units, desc = oracle_sample(args.workload, 256 if is_scan else 256 * 5120)
+    fn, units, desc = oracle_sample(args.workload, 256 if is_scan else 256 * 5120, args.zoh)
     for _ in range(max(args.warmup, 0)):
         fn()
     times = []
@@ -389,26 +395,41 @@ def run_mssm(args):
         inp = synth.workload_inputs(args.workload, seed=seed)
         host = {k: getattr(inp, k) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
         units = inp.batch * inp.dim * inp.length
+        varlen = inp.cu_seqlens is not None
+        nstate = len(inp.cu_seqlens) - 1 if varlen else inp.batch
+        max_seqlen = int(np.diff(inp.cu_seqlens).max()) if varlen else inp.length
         alg_bytes = scan_algorithmic_bytes(inp.batch, inp.dim, inp.length, io_bytes, inp.z is not None,
-                                           inp.D is not None, inp.delta_bias is not None)
+                                           inp.D is not None, inp.delta_bias is not None, last_state=False)
+        alg_bytes += nstate * inp.dim * N_STATE * 4 + (4 * (nstate + 1) if varlen else 0)
         nsets = ring_size(alg_bytes, l2_bytes)
         d = {k: to_dev(v) for k, v in host.items()}
+        cu_d = torch.from_numpy(inp.cu_seqlens).to(dev) if varlen else None
         sets = []
         for k in range(max(nsets, 1)):
             dk = d if k == 0 else {**d, **{n: d[n].clone() for n in ("u", "delta", "B", "C", "z") if d[n] is not None}}
-            sets.append((dk, torch.empty_like(d["u"]), torch.empty(inp.batch, inp.dim, N_STATE, device=dev)))
+            sets.append((dk, torch.empty_like(d["u"]), torch.empty(nstate, inp.dim, N_STATE, device=dev)))
+        disc = m.MSSM_DISC_ZOH if args.zoh else m.MSSM_DISC_EULER
 
         def step(k=0):
             dk, out_k, last_k = sets[k % len(sets)]
-            m.mssm_selective_scan_fwd(dk["u"], dk["delta"], dk["A"], dk["B"], dk["C"], dk["D"], dk["z"],
-                                      dk["delta_bias"], inp.softplus, out_k, last_k)
+            if varlen or args.zoh:
+                m.mssm_selective_scan_fwd_ex(dk["u"], dk["delta"], dk["A"], dk["B"], dk["C"], dk["D"], dk["z"],
+                                             dk["delta_bias"], inp.softplus, out_k, last_k, discretization=disc,
+                                             cu_seqlens=cu_d, max_seqlen=max_seqlen if varlen else 0)
+            else:
+                m.mssm_selective_scan_fwd(dk["u"], dk["delta"], dk["A"], dk["B"], dk["C"], dk["D"], dk["z"],
+                                          dk["delta_bias"], inp.softplus, out_k, last_k)
         config = {"workload": args.workload, "batch": inp.batch, "channels": inp.dim, "length": inp.length,
                   "state": N_STATE, "io_dtype": inp.io_dtype, "gate": inp.z is not None,
                   "softplus_bias": inp.delta_bias is not None, "D_skip": inp.D is not None,
                   "exp_path": "general (one exponential per state)" if args.general_a
                   else "structured A (powers of one exponential)",
+                  "discretization": "zero-order hold" if args.zoh else "euler",
                   "chunk_len": args.chunk_len or "auto",
-                  "plan": m.mssm_scan_plan(inp.batch, inp.dim, inp.length)}
+                  "plan": m.mssm_scan_plan(nstate, inp.dim, max_seqlen,
+                                           total_len=inp.length if varlen else -1)}
+        if varlen:
+            config.update({"sequences": nstate, "max_seqlen": max_seqlen, "packed_length": inp.length})
         metric, unit = METRIC, "elems/s"
         dom_kernel = "scan_out"
         set_bytes = alg_bytes
@@ -536,7 +557,7 @@ def run_mssm(args):
         "source_hash": kernel_source_hash(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds, args.zoh)
     if world > 1:
         dist.barrier()
         del g
@@ -563,20 +584,27 @@ def run_e2e(args, kind, inp, d, dev, m, units, world):
     if kind == "scan":
         names = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
         h = {k: pin(getattr(inp, k)) for k in names}
+        varlen = inp.cu_seqlens is not None
+        if varlen:
+            h["cu_seqlens"] = torch.from_numpy(inp.cu_seqlens).pin_memory()
         dd = {k: (None if v is None else torch.empty(v.shape, dtype=v.dtype, device=dev)) for k, v in h.items()}
         out = torch.empty_like(dd["u"])
-        last = torch.empty(inp.batch, inp.dim, N_STATE, device=dev)
+        nstate = len(inp.cu_seqlens) - 1 if varlen else inp.batch
+        max_seqlen = int(np.diff(inp.cu_seqlens).max()) if varlen else 0
+        last = torch.empty(nstate, inp.dim, N_STATE, device=dev)
         y_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         s_host = torch.empty(last.shape, dtype=last.dtype).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in h.values() if v is not None)
         d2h = y_host.numel() * y_host.element_size() + s_host.numel() * s_host.element_size()
+        disc = m.MSSM_DISC_ZOH if args.zoh else m.MSSM_DISC_EULER
 
         def one():
-            for k in names:
+            for k in h:
                 if h[k] is not None:
                     dd[k].copy_(h[k], non_blocking=True)
-            m.mssm_selective_scan_fwd(dd["u"], dd["delta"], dd["A"], dd["B"], dd["C"], dd["D"], dd["z"],
-                                      dd["delta_bias"], inp.softplus, out, last)
+            m.mssm_selective_scan_fwd_ex(dd["u"], dd["delta"], dd["A"], dd["B"], dd["C"], dd["D"], dd["z"],
+                                         dd["delta_bias"], inp.softplus, out, last, discretization=disc,
+                                         cu_seqlens=dd.get("cu_seqlens"), max_seqlen=max_seqlen)
             y_host.copy_(out, non_blocking=True)
             s_host.copy_(last, non_blocking=True)
     else:
@@ -627,6 +655,7 @@ def main(argv=None):
     ap.add_argument("--chunk-len", type=int, default=0, help="length split (0: automatic; multiple of 64)")
     ap.add_argument("--decode-path", choices=["auto", "stream", "bulk_tile", "per_row"], default="auto",
                     help="decode kernel (MSSM_OPT_DECODE_PATH)")
+    ap.add_argument("--zoh", action="store_true", help="zero-order-hold discretisation (scan workloads)")
     ap.add_argument("--general-a", action="store_true",
                     help="disable the structured-A path (one exponential per state)")
     args = ap.parse_args(argv)

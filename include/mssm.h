@@ -308,6 +308,13 @@ mssm_status mssm_set_option(int option, int64_t value);
 mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int *rows_per_cta,
                            int64_t *chunk_len, int64_t *n_chunks, int *schedule);
 
+/*
+ * The same query for S packed sequences of at most max_seqlen steps summing to
+ * total_len (the T of mssm_scan_ext.cu_seqlens; total_len < 0: S full sequences).
+ */
+mssm_status mssm_scan_plan_packed(int64_t S, int64_t D, int64_t max_seqlen, int64_t total_len, int sm_count,
+                                  int *rows_per_cta, int64_t *chunk_len, int64_t *n_chunks, int *schedule);
+
 /* Kernel kinds counted by mssm_kernel_stats. */
 typedef enum {
     MSSM_KERNEL_SCAN_CHUNK_STATE = 0, /* chunk summaries + carry fold (split scans only) */

@@ -85,6 +85,10 @@ _lib.mssm_scan_plan.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, 
                                 ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int64),
                                 ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int)]
 _lib.mssm_scan_plan.restype = ctypes.c_int
+_lib.mssm_scan_plan_packed.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                       ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int64),
+                                       ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int)]
+_lib.mssm_scan_plan_packed.restype = ctypes.c_int
 
 
 class MssmError(RuntimeError):
@@ -159,11 +163,12 @@ def mssm_kernel_stats(reset: bool = False) -> dict:
     return {k: {"launches": launches[i], "timed": timed[i], "ms": ms[i]} for i, k in enumerate(KERNEL_KINDS)}
 
 
-def mssm_scan_plan(Bt: int, D: int, L: int, sm_count: int = 0) -> dict:
-    """Launch plan of the scan for a [Bt, D, L] problem (host only, launches nothing)."""
+def mssm_scan_plan(Bt: int, D: int, L: int, sm_count: int = 0, total_len: int = -1) -> dict:
+    """Launch plan of the scan for a [Bt, D, L] problem, or for Bt packed sequences of at most
+    L steps summing to ``total_len`` (host only, launches nothing)."""
     rows, seg, nseg, sched = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int()
-    _check(_lib.mssm_scan_plan(Bt, D, L, sm_count, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg),
-                               ctypes.byref(sched)))
+    _check(_lib.mssm_scan_plan_packed(Bt, D, L, total_len, sm_count, ctypes.byref(rows), ctypes.byref(seg),
+                                      ctypes.byref(nseg), ctypes.byref(sched)))
     return {"rows_per_cta": rows.value, "chunk_len": seg.value, "n_chunks": nseg.value,
             "schedule": ("forward", "summaries+forward", "chained")[sched.value]}
 

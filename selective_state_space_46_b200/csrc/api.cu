@@ -164,8 +164,15 @@ int64_t round_seg(int64_t v) {
 // chained work item kItem, and the carry fold kFold per chunk.  Grid kernels
 // run their CTAs in waves of at most kMaxCta per SM (register limited) and
 // put ceil(warps / 4) warps on the busiest SMSP.
-LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forced_seg, int forced_mode) {
-  constexpr double kOut = 96.0, kSum = 55.0, kIpc1 = 0.6, kIpc2 = 0.7;
+//
+// Packed sequences (total_len >= 0: the sum of the Bt sequence lengths, each at most L)
+// count only the chunks that hold steps, about total_len / seg + Bt per row tile column,
+// and pay the forward-sweep summary (kSumFwd).  A chained tile runs its chunks one after
+// another, so the chained schedule costs at least nseg items, which is what rules it out
+// for a few long sequences among short ones.
+LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forced_seg, int forced_mode,
+                         int64_t total_len = -1) {
+  constexpr double kOut = 96.0, kSum = 55.0, kSumFwd = 70.0, kIpc1 = 0.6, kIpc2 = 0.7;
   constexpr double kStart = 4000.0, kLaunch = 6000.0, kItem = 4000.0, kFold = 200.0;
   auto ipc = [&](int64_t k) { return k <= 1 ? kIpc1 : kIpc2; };
   auto grid_time = [&](int64_t ctas, int rows, double steps, double instr) {
@@ -186,8 +193,10 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
       best = sh;
     }
   };
+  const bool packed = total_len >= 0;
   for (int rows : {32, 64}) {
-    const int64_t tiles = Bt * ((D + rows - 1) / rows);
+    const int64_t tpb = (D + rows - 1) / rows;
+    const int64_t tiles = Bt * tpb;
     for (int64_t want = 1; want <= 64; ++want) {
       int64_t seg = forced_seg > 0 ? forced_seg : round_seg((L + want - 1) / want);
       int64_t nseg = L > 0 ? (L + seg - 1) / seg : 1;
@@ -195,8 +204,15 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
         seg *= 2;
         nseg = (L + seg - 1) / seg;
       }
-      double cost = grid_time(tiles * nseg, rows, double(seg), kOut);
-      if (nseg > 1) cost += grid_time(tiles * (nseg - 1), rows, double(seg), kSum) + kFold * double(nseg);
+      // CTAs (items) that hold steps; the rest of a packed grid exits at once
+      int64_t out_items = tiles * nseg, sum_items = tiles * (nseg - 1);
+      if (packed) {
+        out_items = std::min<int64_t>(out_items, tpb * ((total_len + seg - 1) / seg + Bt));
+        sum_items = std::min<int64_t>(sum_items, tpb * (total_len / seg));
+      }
+      double cost = grid_time(out_items, rows, double(seg), kOut);
+      if (nseg > 1)
+        cost += grid_time(sum_items, rows, double(seg), packed ? kSumFwd : kSum) + kFold * double(nseg);
       consider(LaunchShape{nseg > 1 ? 1 : 0, rows, seg, nseg, 0}, cost);
       // chained: 32-row tiles, at most 8 one-warp CTAs per SM and never more CTAs than tiles
       if (rows == 32 && nseg > 1 && forced_mode == 2 && tiles < 4 * int64_t(sms)) {
@@ -208,7 +224,7 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
           // each CTA takes whole items; k warps share an SMSP's issue
           const int64_t grid = per_sm * sms;
           const int64_t k = (per_sm + 3) / 4;
-          const int64_t rounds = (tiles * nseg + grid - 1) / grid;
+          const int64_t rounds = std::max<int64_t>((out_items + grid - 1) / grid, nseg);
           const double item = double(seg) * kOut * double(k) / ipc(k) + kItem;
           consider(LaunchShape{2, 32, seg, nseg, int(grid)}, double(rounds) * item + kLaunch);
         }
@@ -282,6 +298,7 @@ struct ScanCall {
   bool softplus = false;
   bool noop = false;       // Bt * D == 0: nothing to launch
   int64_t Bt = 0, D = 0, L = 0;  // as planned: packed sequences plan S x D x max_seqlen
+  int64_t total_len = -1;        // packed sequences: their summed length (the packed row's T)
 };
 
 // state_batches: the leading size of last_state (and h0) when it is not Bt (packed
@@ -389,6 +406,7 @@ mssm_status scan_prepare_ext(const mssm_scan_ext* ext, const mssm_tensor* out, c
       return fail(MSSM_ERR_INVALID_ARG, "max_seqlen = %lld must lie in [0, T = %lld]",
                   (long long)ext->max_seqlen, (long long)call.L);
     // plan as S independent rows of max_seqlen steps; the kernels read each sequence's range
+    call.total_len = call.L;
     call.Bt = S;
     call.L = ext->max_seqlen;
     call.noop = (S == 0 || call.D == 0);
@@ -427,7 +445,8 @@ ScanPlan scan_plan(ScanCall& call, int sm_count) {
   mssm::ScanArgs& a = call.a;
   a.force_general = g_force_general;
   a.test_no_publish = g_test_hooks & 1;
-  const LaunchShape shape = choose_shape(call.Bt, call.D, call.L, sm_count, g_chunk_len, g_schedule);
+  const LaunchShape shape =
+      choose_shape(call.Bt, call.D, call.L, sm_count, g_chunk_len, g_schedule, call.total_len);
   ScanPlan plan;
   plan.mode = shape.mode;
   plan.rows_per_cta = shape.rows;
@@ -753,6 +772,12 @@ mssm_status mssm_state_update_ex(mssm_tensor* state, const mssm_tensor* x, const
 
 mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int* rows_per_cta,
                            int64_t* chunk_len, int64_t* n_chunks, int* schedule) {
+  return mssm_scan_plan_packed(Bt, D, L, -1, sm_count, rows_per_cta, chunk_len, n_chunks, schedule);
+}
+
+mssm_status mssm_scan_plan_packed(int64_t S, int64_t D, int64_t max_seqlen, int64_t total_len, int sm_count,
+                                  int* rows_per_cta, int64_t* chunk_len, int64_t* n_chunks, int* schedule) {
+  const int64_t Bt = S, L = max_seqlen;
   if (Bt < 0 || D < 0 || L < 0) return fail(MSSM_ERR_INVALID_ARG, "negative size");
   if (sm_count <= 0) {
     int dev = 0, v = 0;
@@ -771,7 +796,7 @@ mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int* 
     std::lock_guard<std::mutex> lk(g_mu);
     forced_mode = g_schedule;
   }
-  const LaunchShape sh = choose_shape(Bt, D, L, sm_count, forced, forced_mode);
+  const LaunchShape sh = choose_shape(Bt, D, L, sm_count, forced, forced_mode, total_len);
   if (rows_per_cta) *rows_per_cta = sh.rows;
   if (chunk_len) *chunk_len = sh.seg;
   if (n_chunks) *n_chunks = sh.nseg;

@@ -107,6 +107,7 @@ class ScanInputs:
     z: Optional[np.ndarray]  # [batch, dim, length]
     delta_bias: Optional[np.ndarray]  # [dim] f32
     softplus: bool
+    cu_seqlens: Optional[np.ndarray] = None  # [S + 1] int32 offsets when the batch row packs S sequences
 
     def f64(self, name: str) -> Optional[np.ndarray]:
         a = getattr(self, name)
@@ -204,9 +205,19 @@ WORKLOADS = {
     # long context, slow decay spanning many chunks
     "scan_bf16_1x2048x131072": dict(kind="scan", batch=1, dim=2048, length=131072,
                                     io_dtype="bf16", delta_range=(1e-4, 1e-2), with_z=True),
+    # packed variable-length prefill: 32 sequences of 64..4096 steps (log-uniform) over
+    # Mamba-130M's 1536 channels, concatenated along L without padding
+    "scan_varlen_bf16_1536x32seq": dict(kind="scan", batch=1, dim=1536, nseq=32, len_range=(64, 4096),
+                                        io_dtype="bf16", delta_range=(1e-3, 1e-1), with_z=True),
     # one-token decode state update, timed over successive steps
     "decode_bf16_256x5120": dict(kind="decode", batch=256, dim=5120, io_dtype="bf16"),
 }
+
+
+def varlen_lengths(nseq: int, lo: int, hi: int, seed: int = 0) -> np.ndarray:
+    """Sequence lengths, log-uniform in [lo, hi], from their own stream."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 99])))
+    return np.exp(rng.uniform(np.log(lo), np.log(hi), size=nseq)).astype(np.int64)
 
 
 def workload_inputs(name: str, seed: int = 0, batch: Optional[int] = None,
@@ -216,6 +227,12 @@ def workload_inputs(name: str, seed: int = 0, batch: Optional[int] = None,
     kind = w.pop("kind")
     if batch is not None:
         w["batch"] = batch
+    if kind == "scan" and "nseq" in w:
+        lengths = varlen_lengths(w["nseq"], *w["len_range"], seed=seed)
+        inp = make_scan_inputs(1, w["dim"], int(lengths.sum()), io_dtype=w["io_dtype"], seed=seed,
+                               delta_range=w["delta_range"], with_z=w["with_z"])
+        inp.cu_seqlens = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+        return inp
     if kind == "scan":
         return make_scan_inputs(w["batch"], w["dim"], w["length"], io_dtype=w["io_dtype"],
                                 seed=seed, delta_range=w["delta_range"], with_z=w["with_z"])
