@@ -160,8 +160,7 @@ def max_sm_mhz(default: float = 1965.0) -> float:
 KERNEL_SOURCES = {
     "scan_out": ("device_common.cuh", "scan.cuh", "scan.cu", "scan_zoh.cu", "scan_dispatch.cuh"),
     "scan_chunk_state": ("device_common.cuh", "scan.cuh", "scan.cu", "scan_zoh.cu", "scan_dispatch.cuh"),
-    # the automatic choice among the decode kernels is made in api.cu
-    "state_update": ("device_common.cuh", "decode.cuh", "decode.cu", "api.cu"),
+    "state_update": ("device_common.cuh", "decode.cuh", "decode.cu"),
 }
 
 
