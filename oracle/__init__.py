@@ -127,6 +127,31 @@ def causal_conv1d(x, w, bias=None, silu=True) -> np.ndarray:
     return out
 
 
+def causal_conv1d_varlen(x, w, cu_seqlens, bias=None, silu=True) -> np.ndarray:
+    """Causal conv1d (then SiLU) of packed sequences: ``x`` [1, D, T] with ``cu_seqlens``
+    offsets; every sequence sees zeros before its own first step.  Built only from
+    ``causal_conv1d`` on each slice."""
+    cu = np.asarray(cu_seqlens, np.int64)
+    x = np.asarray(x, np.float64)
+    out = np.zeros(x.shape, np.float64)
+    for s in range(len(cu) - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        if b > a:
+            out[..., a:b] = causal_conv1d(x[..., a:b], w, bias, silu)
+    return out
+
+
+def causal_conv1d_update(conv_state, x, w, bias=None, silu=True):
+    """One decode step of the causal conv1d: ``conv_state`` [Bt, D, K-1] holds the previous
+    K-1 inputs (oldest first), ``x`` [Bt, D] the new one.  Returns ``(new_state, out [Bt, D])``:
+    the conv (then SiLU) at the newest position of the window [state, x], and the window
+    without its oldest input.  Built only from ``causal_conv1d`` on the window."""
+    st = np.asarray(conv_state, np.float64)
+    win = np.concatenate([st, np.asarray(x, np.float64)[..., None]], axis=-1)  # [Bt, D, K]
+    out = causal_conv1d(win, w, bias, silu)[..., -1]
+    return win[..., 1:].copy(), out
+
+
 def scan_varlen(u, delta, A, B, C, cu_seqlens, D=None, z=None, delta_bias=None, softplus=True,
                 h0=None, zoh=False) -> Tuple[np.ndarray, np.ndarray]:
     """Selective scan of several sequences packed along L (the varlen layout): ``u, delta,

@@ -396,6 +396,33 @@ def test_conv1d_impulse_response():
     np.testing.assert_array_equal(out, expect)
 
 
+def test_conv1d_update_chain_is_the_conv():
+    """T decode steps of the conv from a zero window give the prefill conv, step by step."""
+    rng = np.random.default_rng(33)
+    Bt, D, L, K = 2, 3, 11, 4
+    x = rng.standard_normal((Bt, D, L))
+    w = rng.standard_normal((D, K))
+    b = rng.standard_normal(D)
+    full = oracle.causal_conv1d(x, w, b, silu=True)
+    st = np.zeros((Bt, D, K - 1))
+    for t in range(L):
+        st, o = oracle.causal_conv1d_update(st, x[..., t], w, b, silu=True)
+        np.testing.assert_allclose(o, full[..., t], rtol=1e-14, atol=1e-15)
+    np.testing.assert_array_equal(st, x[..., L - K + 1:])
+
+
+def test_conv1d_varlen_restarts_at_boundaries():
+    rng = np.random.default_rng(34)
+    D, K = 3, 4
+    cu = [0, 2, 2, 9, 15]
+    x = rng.standard_normal((1, D, 15))
+    w = rng.standard_normal((D, K))
+    out = oracle.causal_conv1d_varlen(x, w, cu, None, silu=False)
+    # the third sequence alone, from zeros: its first outputs see only its own inputs
+    np.testing.assert_allclose(out[..., 9:], oracle.causal_conv1d(x[..., 9:], w, None, silu=False), rtol=1e-15)
+    np.testing.assert_allclose(out[0, :, 9], w[:, K - 1] * x[0, :, 9], rtol=1e-15)
+
+
 # ---------------------------------------------------------------------------
 # 7d. packed variable-length sequences: the state restarts at every boundary
 # ---------------------------------------------------------------------------
