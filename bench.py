@@ -45,6 +45,7 @@ import synth  # noqa: E402
 
 METRIC = "selective-scan B·D·L elems/s and achieved HBM GB/s vs ~8 TB/s B200 peak"
 DECODE_METRIC = "selective state update rows/s and achieved HBM GB/s vs ~8 TB/s B200 peak"
+CONV_METRIC = "causal conv1d + SiLU B·D·L elems/s and achieved HBM GB/s vs ~8 TB/s B200 peak"
 DEFAULT_WORKLOAD = "scan_bf16_2x1536x2048"
 L2_FLUSH_BYTES = 256 << 20
 NOMINAL_HBM_GBS = 8000.0
@@ -161,6 +162,7 @@ KERNEL_SOURCES = {
     "scan_out": ("device_common.cuh", "scan.cuh", "scan.cu", "scan_zoh.cu", "scan_dispatch.cuh"),
     "scan_chunk_state": ("device_common.cuh", "scan.cuh", "scan.cu", "scan_zoh.cu", "scan_dispatch.cuh"),
     "state_update": ("device_common.cuh", "decode.cuh", "decode.cu"),
+    "conv": ("device_common.cuh", "conv.cuh", "conv.cu"),
 }
 
 
@@ -285,6 +287,13 @@ def oracle_sample(workload: str, rows: int, zoh: bool = False):
             return (lambda: oracle.scan_varlen(cu_seqlens=cu, **args)), units, desc
         desc = f"batch 0, channels 0..{d - 1}, all {inp.length} steps ({units} elements{disc})"
         return (lambda: oracle.scan(**args)), units, desc
+    if isinstance(inp, synth.ConvInputs):
+        d = min(rows, inp.dim)
+        x = synth.to_f64(inp.x[:1, :d], inp.io_dtype)
+        w, bias = inp.weight[:d].astype(np.float64), inp.bias[:d].astype(np.float64)
+        units = d * inp.length
+        return ((lambda: oracle.causal_conv1d(x, w, bias, True)), units,
+                f"batch 0, channels 0..{d - 1}, all {inp.length} steps ({units} elements)")
     b = max(1, min(inp.batch, rows // inp.dim if rows >= inp.dim else 1))
     args = dict(state=inp.state[:b], x=inp.f64("x")[:b], dt=inp.f64("dt")[:b], A=inp.f64("A"),
                 B=inp.f64("B")[:b], C=inp.f64("C")[:b], D=inp.f64("D"), z=inp.f64("z")[:b],
@@ -295,7 +304,7 @@ def oracle_sample(workload: str, rows: int, zoh: bool = False):
 
 def cpu_baseline(workload: str, budget_s: float = 10.0, zoh: bool = False):
     import oracle
-    is_scan = WORKLOADS_KIND[workload] == "scan"
+    is_scan = WORKLOADS_KIND[workload] in ("scan", "conv")
     rows = 512 if is_scan else 256 * 5120
     fn, units, desc = oracle_sample(workload, rows, zoh)
     fn()  # build + warm
@@ -319,7 +328,8 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
-    is_scan = WORKLOADS_KIND[args.workload] == "scan"
+    kind = WORKLOADS_KIND[args.workload]
+    is_scan = kind in ("scan", "conv")
     fn, units, desc = oracle_sample(args.workload, 256 if is_scan else 256 * 5120, args.zoh)
     for _ in range(max(args.warmup, 0)):
         fn()
@@ -332,7 +342,8 @@ def run_reference(args):
     value = units / (ms / 1e3)
     unit = "elems/s" if is_scan else "rows/s"
     line = {
-        "impl": "reference", "metric": METRIC if is_scan else DECODE_METRIC, "value": value, "unit": unit,
+        "impl": "reference", "metric": {"scan": METRIC, "conv": CONV_METRIC}.get(kind, DECODE_METRIC),
+        "value": value, "unit": unit,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)", "config": {"workload": args.workload, "sample": desc},
@@ -432,6 +443,26 @@ def run_mssm(args):
         metric, unit = METRIC, "elems/s"
         dom_kernel = "scan_out"
         set_bytes = alg_bytes
+    elif kind == "conv":
+        inp = synth.workload_inputs(args.workload, seed=seed)
+        units = inp.batch * inp.dim * inp.length
+        K = inp.weight.shape[1]
+        alg_bytes = 2 * units * io_bytes + inp.dim * (K + 1) * 4
+        set_bytes = alg_bytes
+        nsets = ring_size(alg_bytes, l2_bytes)
+        x0 = to_dev(inp.x)
+        xs = [x0] + [x0.clone() for _ in range(max(nsets, 1) - 1)]
+        outs_c = [torch.empty_like(x0) for _ in xs]
+        w_d, b_d = to_dev(inp.weight), to_dev(inp.bias)
+        d = {"x": x0}
+
+        def step(k=0):
+            j = k % len(xs)
+            m.mssm_causal_conv1d_fwd(xs[j], w_d, b_d, outs_c[j], None, 0, True)
+        config = {"workload": args.workload, "batch": inp.batch, "channels": inp.dim, "length": inp.length,
+                  "kernel_size": K, "io_dtype": inp.io_dtype, "activation": "silu"}
+        metric, unit = CONV_METRIC, "elems/s"
+        dom_kernel = "conv"
     else:
         ring = [synth.workload_inputs(args.workload, seed=seed, step_stream=k) for k in range(8)]
         inp = ring[0]
@@ -527,8 +558,10 @@ def run_mssm(args):
     dom_ms = dom["ms_per_launch"] if dom else None
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     alu_peak = fp32_peak_tflops(sms, max_sm_mhz())
-    alg_flops = algorithmic_flops(units)
-    plan_key = plan_string(config.get("plan")) if kind == "scan" else f"decode_path={args.decode_path}"
+    # the conv: K FMAs per element (its SiLU runs on the SFU)
+    alg_flops = algorithmic_flops(units) if kind != "conv" else units * 2 * inp.weight.shape[1]
+    plan_key = (plan_string(config.get("plan")) if kind == "scan" else
+                f"decode_path={args.decode_path}" if kind == "decode" else None)
     traffic, traffic_src = recorded_traffic(dom_kernel, args.workload, plan_key)
     roofline = binding_roofline(alg_bytes, alg_flops, dom_ms, peak, alu_peak) if dom_ms else {"bound": None}
     roofline.update({"kernel": dom_kernel, "ms_per_launch": dom_ms,
@@ -540,7 +573,7 @@ def run_mssm(args):
     # ---- end to end: host buffers in pinned memory, copies inside the timed region
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, kind, inp, d if kind == "scan" else None, dev, m, units, world)
+        e2e = run_e2e(args, kind, inp, d if kind in ("scan", "conv") else None, dev, m, units, world)
 
     step_gbs = alg_bytes / (ms_per_step / 1e3) / 1e9
     line = {
@@ -580,7 +613,20 @@ def run_e2e(args, kind, inp, d, dev, m, units, world):
             t = torch.from_numpy(np.ascontiguousarray(a, np.float32))
         return t.pin_memory()
 
-    if kind == "scan":
+    if kind == "conv":
+        hx = pin(inp.x)
+        xd = torch.empty(hx.shape, dtype=hx.dtype, device=dev)
+        w_d, b_d = pin(inp.weight).to(dev), pin(inp.bias).to(dev)
+        out = torch.empty_like(xd)
+        y_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = hx.numel() * hx.element_size()
+        d2h = y_host.numel() * y_host.element_size()
+
+        def one():
+            xd.copy_(hx, non_blocking=True)
+            m.mssm_causal_conv1d_fwd(xd, w_d, b_d, out, None, 0, True)
+            y_host.copy_(out, non_blocking=True)
+    elif kind == "scan":
         names = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
         h = {k: pin(getattr(inp, k)) for k in names}
         varlen = inp.cu_seqlens is not None
@@ -635,7 +681,7 @@ def run_e2e(args, kind, inp, d, dev, m, units, world):
     t1.record()
     torch.cuda.synchronize(dev)
     ms = reduce_max(t0.elapsed_time(t1), dist if world > 1 else None) / steps
-    return {"value": units * world / (ms / 1e3), "unit": "elems/s" if kind == "scan" else "rows/s",
+    return {"value": units * world / (ms / 1e3), "unit": "elems/s" if kind in ("scan", "conv") else "rows/s",
             "ms_per_step": ms, "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "path": "pinned host buffers -> H2D copies -> C-ABI call -> D2H of y and final state"}
 

@@ -237,6 +237,41 @@ mssm_status mssm_state_update_ex(mssm_tensor *state, const mssm_tensor *x,
                                  const mssm_tensor *dt_bias, int softplus_flag,
                                  int discretization, mssm_tensor *out, void *stream);
 
+/*
+ * Causal depthwise conv1d + SiLU: the step that produces the scan's input u from
+ * the in-projection's x branch ("Linear Attention vs Softmax Attention ...",
+ * section Implementation: the listed layer's grouped Conv1d with one group per
+ * channel, kernel size K, padding K - 1, the output truncated to the first L
+ * steps, then SiLU):
+ *
+ *   out[b,d,t] = act(bias[d] + sum_{k<K} weight[d,k] * x[b,d,t-(K-1)+k]),  x = 0 before t = 0
+ *
+ *   x, out      [Bt, D, L]  bf16|f32 (same dtype), L stride 1; out must not alias x
+ *   weight      [D, K] f32, 1 <= K <= 4;   bias [D] f32 or NULL
+ *   cu_seqlens  NULL, or [S + 1] int32 DEVICE offsets of packed sequences in a
+ *               [1, D, T] x (as in mssm_scan_ext): every sequence sees zeros before
+ *               its own first step; out outside every sequence is left unwritten
+ *   max_seqlen  host bound on the sequence lengths (read only with cu_seqlens)
+ *   silu_flag   1: act = SiLU, 0: identity
+ * Inconsistent offsets are clamped and reported by mssm_get_error
+ * (MSSM_ERR_INVALID_ARG).  The output is written in the scan's u layout.
+ */
+mssm_status mssm_causal_conv1d_fwd(const mssm_tensor *x, const mssm_tensor *weight, const mssm_tensor *bias,
+                                   const mssm_tensor *cu_seqlens, int64_t max_seqlen, int silu_flag,
+                                   mssm_tensor *out, void *stream);
+
+/*
+ * One decode step of the same conv, conv_state updated IN PLACE:
+ *   conv_state [Bt, D, K-1]  dtype of x: the previous K-1 inputs, oldest first
+ *   x, out     [Bt, D]       bf16|f32
+ *   weight [D, K] f32 with 2 <= K <= 4;  bias [D] f32 or NULL
+ * out = act(bias + sum_k weight[d,k] * window[k]) over window = [conv_state, x];
+ * conv_state then drops its oldest input and appends x.  Steps from a zero state
+ * reproduce mssm_causal_conv1d_fwd step by step.
+ */
+mssm_status mssm_causal_conv1d_update(mssm_tensor *conv_state, const mssm_tensor *x, const mssm_tensor *weight,
+                                      const mssm_tensor *bias, int silu_flag, mssm_tensor *out, void *stream);
+
 /* Static, human-readable name of a status code. */
 const char *mssm_status_string(mssm_status status);
 
@@ -320,7 +355,8 @@ typedef enum {
     MSSM_KERNEL_SCAN_CHUNK_STATE = 0, /* chunk summaries + carry fold (split scans only) */
     MSSM_KERNEL_SCAN_OUT = 1,         /* forward sweep with fused epilogue */
     MSSM_KERNEL_STATE_UPDATE = 2,     /* decode step */
-    MSSM_KERNEL_KINDS = 3
+    MSSM_KERNEL_CONV = 3,             /* causal conv1d (prefill and decode step) */
+    MSSM_KERNEL_KINDS = 4
 } mssm_kernel_kind;
 
 /*

@@ -24,6 +24,7 @@ __all__ = [
     "MSSM_OPT_FORCE_GENERAL_A", "MSSM_OPT_CHUNK_LEN", "MSSM_OPT_KERNEL_TIMING", "MSSM_OPT_SCHEDULE", "SCHEDULES",
     "MSSM_OPT_DECODE_PATH", "DECODE_PATHS", "MSSM_OPT_TEST_HOOKS", "MSSM_ERR_TIMEOUT", "mssm_kernel_stats", "mssm_scan_plan",
     "mssm_selective_scan_fwd_ex", "MSSM_DISC_EULER", "MSSM_DISC_ZOH",
+    "mssm_causal_conv1d_fwd", "mssm_causal_conv1d_update", "causal_conv1d", "causal_conv1d_update",
     "KERNEL_KINDS",
 ]
 
@@ -42,7 +43,7 @@ MSSM_OPT_TEST_HOOKS = 6
 MSSM_DISC_EULER, MSSM_DISC_ZOH = 0, 1
 SCHEDULES = {"forward": 1, "summaries+forward": 2, "chained": 3}
 DECODE_PATHS = {"stream": 1, "bulk_tile": 2, "per_row": 3}
-KERNEL_KINDS = ("scan_chunk_state", "scan_out", "state_update")
+KERNEL_KINDS = ("scan_chunk_state", "scan_out", "state_update", "conv")
 
 
 class mssm_tensor(ctypes.Structure):
@@ -69,6 +70,10 @@ _lib.mssm_state_update.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _V]
 _lib.mssm_state_update.restype = ctypes.c_int
 _lib.mssm_state_update_ex.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _V]
 _lib.mssm_state_update_ex.restype = ctypes.c_int
+_lib.mssm_causal_conv1d_fwd.argtypes = [_P, _P, _P, _P, ctypes.c_int64, ctypes.c_int, _P, _V]
+_lib.mssm_causal_conv1d_fwd.restype = ctypes.c_int
+_lib.mssm_causal_conv1d_update.argtypes = [_P, _P, _P, _P, ctypes.c_int, _P, _V]
+_lib.mssm_causal_conv1d_update.restype = ctypes.c_int
 _lib.mssm_status_string.argtypes = [ctypes.c_int]
 _lib.mssm_status_string.restype = ctypes.c_char_p
 _lib.mssm_last_error.restype = ctypes.c_char_p
@@ -227,9 +232,44 @@ def mssm_state_update_ex(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, ou
                                      _stream(stream, x)))
 
 
+def mssm_causal_conv1d_fwd(x, weight, bias, out, cu_seqlens=None, max_seqlen=0, silu_flag=True,
+                           stream=None) -> None:
+    """Marshal torch tensors into ``mssm_causal_conv1d_fwd`` (see include/mssm.h)."""
+    ds = [_desc(t) for t in (x, weight, bias, cu_seqlens)]
+    _check(_lib.mssm_causal_conv1d_fwd(*[_ref(v) for v in ds], int(max_seqlen), int(silu_flag), _ref(_desc(out)),
+                                       _stream(stream, x)))
+
+
+def mssm_causal_conv1d_update(conv_state, x, weight, bias, out, silu_flag=True, stream=None) -> None:
+    """Marshal torch tensors into ``mssm_causal_conv1d_update`` (conv_state updated in place)."""
+    ds = [_desc(t) for t in (conv_state, x, weight, bias)]
+    _check(_lib.mssm_causal_conv1d_update(*[_ref(v) for v in ds], int(silu_flag), _ref(_desc(out)),
+                                          _stream(stream, x)))
+
+
 # --------------------------------------------------------------------------
 # allocation conveniences (torch allocates; the library computes)
 # --------------------------------------------------------------------------
+
+def causal_conv1d(x, weight, bias=None, silu=True, cu_seqlens=None, max_seqlen=None, out=None,
+                  stream=None) -> torch.Tensor:
+    """Causal depthwise conv1d (+ SiLU) of ``x`` [Bt, D, L] on the GPU; returns ``out``."""
+    if not x.is_cuda:
+        raise ValueError("causal_conv1d runs on CUDA tensors only")
+    if out is None:
+        out = torch.empty_like(x, memory_format=torch.contiguous_format)
+    if cu_seqlens is not None and max_seqlen is None:
+        max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if cu_seqlens.numel() > 1 else 0
+    mssm_causal_conv1d_fwd(x, weight, bias, out, cu_seqlens, max_seqlen or 0, silu, stream)
+    return out
+
+
+def causal_conv1d_update(conv_state, x, weight, bias=None, silu=True, out=None, stream=None) -> torch.Tensor:
+    """One decode step of the conv on the GPU (``conv_state`` updated in place); returns ``out``."""
+    if out is None:
+        out = torch.empty_like(x, memory_format=torch.contiguous_format)
+    mssm_causal_conv1d_update(conv_state, x, weight, bias, out, silu, stream)
+    return out
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True,
                        out=None, last_state=None, return_last_state=True, h0=None, zoh=False,

@@ -40,7 +40,7 @@ int g_decode_path = 0;  // MSSM_OPT_DECODE_PATH
 int g_test_hooks = 0;   // MSSM_OPT_TEST_HOOKS  // -1 automatic, else the forced LaunchShape mode
 
 // ---- launch accounting and optional per-kernel event timing (diagnostics)
-int64_t g_launches[MSSM_KERNEL_KINDS] = {0, 0, 0};
+int64_t g_launches[MSSM_KERNEL_KINDS] = {};
 int g_timing = 0;
 struct TimedLaunch {
   int kind;
@@ -48,8 +48,8 @@ struct TimedLaunch {
 };
 std::vector<TimedLaunch> g_pending;
 std::vector<cudaEvent_t> g_event_pool;
-double g_time_ms[MSSM_KERNEL_KINDS] = {0, 0, 0};
-int64_t g_timed[MSSM_KERNEL_KINDS] = {0, 0, 0};
+double g_time_ms[MSSM_KERNEL_KINDS] = {};
+int64_t g_timed[MSSM_KERNEL_KINDS] = {};
 
 cudaEvent_t take_event() {
   if (!g_event_pool.empty()) {
@@ -768,6 +768,100 @@ mssm_status mssm_state_update_ex(mssm_tensor* state, const mssm_tensor* x, const
                                  const mssm_tensor* D, const mssm_tensor* z, const mssm_tensor* dt_bias,
                                  int softplus_flag, int discretization, mssm_tensor* out, void* stream) {
   return state_update_impl(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, discretization, out, stream);
+}
+
+mssm_status mssm_causal_conv1d_fwd(const mssm_tensor* x, const mssm_tensor* weight, const mssm_tensor* bias,
+                                   const mssm_tensor* cu_seqlens, int64_t max_seqlen, int silu_flag,
+                                   mssm_tensor* out, void* stream) {
+  if (!x) return fail(MSSM_ERR_INVALID_ARG, "x: null tensor descriptor");
+  if (x->ndim != 3) return fail(MSSM_ERR_INVALID_ARG, "x: expected 3 dims [Bt, D, L]");
+  const int dt = x->dtype;
+  if (dt != MSSM_F32 && dt != MSSM_BF16) return fail(MSSM_ERR_INVALID_ARG, "x: dtype must be f32 or bf16");
+  if (!weight || weight->ndim != 2) return fail(MSSM_ERR_INVALID_ARG, "weight: expected 2 dims [D, K]");
+  const int64_t Bt = x->shape[0], Dd = x->shape[1], L = x->shape[2], K = weight->shape[1];
+  if (K < 1 || K > mssm::kConvMaxK)
+    return fail(MSSM_ERR_UNSUPPORTED, "kernel size K = %lld; this build supports 1..%d", (long long)K,
+                mssm::kConvMaxK);
+  const int64_t s_bdl[3] = {Bt, Dd, L}, s_dk[2] = {Dd, K}, s_d[1] = {Dd}, any[1] = {-1};
+  mssm_status st;
+  if ((st = check(x, "x", 3, s_bdl, dt, true)) != MSSM_OK) return st;
+  if ((st = check(out, "out", 3, s_bdl, dt, true)) != MSSM_OK) return st;
+  if ((st = check(weight, "weight", 2, s_dk, MSSM_F32, false)) != MSSM_OK) return st;
+  if (bias && (st = check(bias, "bias", 1, s_d, MSSM_F32, false)) != MSSM_OK) return st;
+  if (same_ptr(out, x)) return fail(MSSM_ERR_INVALID_ARG, "out must not alias x");
+  if (Bt > INT32_MAX || Dd > INT32_MAX || L > INT32_MAX / 2 || Bt * Dd > int64_t(INT32_MAX))
+    return fail(MSSM_ERR_UNSUPPORTED, "size too large");
+  int64_t S = Bt, Lmax = L;
+  if (cu_seqlens) {
+    if ((st = check(cu_seqlens, "cu_seqlens", 1, any, MSSM_I32, true)) != MSSM_OK) return st;
+    if (cu_seqlens->shape[0] < 1) return fail(MSSM_ERR_INVALID_ARG, "cu_seqlens: expected S + 1 >= 1 offsets");
+    if (Bt != 1) return fail(MSSM_ERR_INVALID_ARG, "with cu_seqlens, x must be [1, D, T]");
+    if (max_seqlen < 0 || max_seqlen > L) return fail(MSSM_ERR_INVALID_ARG, "max_seqlen must lie in [0, T]");
+    S = cu_seqlens->shape[0] - 1;
+    Lmax = max_seqlen;
+    if (S * Dd > int64_t(INT32_MAX)) return fail(MSSM_ERR_UNSUPPORTED, "S * D must fit in 31 bits");
+  }
+  if (S == 0 || Dd == 0 || Lmax == 0) return MSSM_OK;
+
+  mssm::ConvArgs a{};
+  a.x = x->data; a.out = out->data;
+  a.x_sb = x->stride[0]; a.x_sd = x->stride[1]; a.o_sb = out->stride[0]; a.o_sd = out->stride[1];
+  a.w = static_cast<const float*>(weight->data); a.w_sd = weight->stride[0]; a.w_sk = weight->stride[1];
+  a.bias = bias ? static_cast<const float*>(bias->data) : nullptr; a.bias_s = bias ? bias->stride[0] : 0;
+  a.Bt = int(S); a.D = int(Dd); a.L = int(L); a.K = int(K);
+  a.vec = rows_vec(x) && rows_vec(out);
+  a.cu_seqlens = cu_seqlens ? static_cast<const int*>(cu_seqlens->data) : nullptr;
+  cudaError_t e = mssm::device_error_word(&a.err);
+  if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  // warp items of kConvPieces pieces of 32 16-byte blocks
+  const int64_t item = int64_t(mssm::kConvPieces) * 32 * (16 / int64_t(esize(dt)));
+  const int64_t items64 = (Lmax + item - 1) / item;
+  if (items64 > 65535) return fail(MSSM_ERR_UNSUPPORTED, "sequence too long for the conv grid (%lld pieces)",
+                                   (long long)items64);
+  const int items = int(items64);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lk(g_mu);
+  e = tracked(MSSM_KERNEL_CONV, s, [&] { return mssm::launch_causal_conv1d(a, items, dt, silu_flag != 0, s); });
+  if (e != cudaSuccess) return cuda_fail(e, "conv1d kernel launch");
+  return MSSM_OK;
+}
+
+mssm_status mssm_causal_conv1d_update(mssm_tensor* conv_state, const mssm_tensor* x, const mssm_tensor* weight,
+                                      const mssm_tensor* bias, int silu_flag, mssm_tensor* out, void* stream) {
+  if (!x) return fail(MSSM_ERR_INVALID_ARG, "x: null tensor descriptor");
+  if (x->ndim != 2) return fail(MSSM_ERR_INVALID_ARG, "x: expected 2 dims [Bt, D]");
+  const int dt = x->dtype;
+  if (dt != MSSM_F32 && dt != MSSM_BF16) return fail(MSSM_ERR_INVALID_ARG, "x: dtype must be f32 or bf16");
+  if (!weight || weight->ndim != 2) return fail(MSSM_ERR_INVALID_ARG, "weight: expected 2 dims [D, K]");
+  const int64_t Bt = x->shape[0], Dd = x->shape[1], K = weight->shape[1];
+  if (K < 2 || K > mssm::kConvMaxK)
+    return fail(MSSM_ERR_UNSUPPORTED, "kernel size K = %lld; the update supports 2..%d", (long long)K,
+                mssm::kConvMaxK);
+  const int64_t s_bd[2] = {Bt, Dd}, s_dk[2] = {Dd, K}, s_d[1] = {Dd}, s_st[3] = {Bt, Dd, K - 1};
+  mssm_status st;
+  if ((st = check(x, "x", 2, s_bd, dt, false)) != MSSM_OK) return st;
+  if ((st = check(out, "out", 2, s_bd, dt, false)) != MSSM_OK) return st;
+  if ((st = check(conv_state, "conv_state", 3, s_st, dt, false)) != MSSM_OK) return st;
+  if ((st = check(weight, "weight", 2, s_dk, MSSM_F32, false)) != MSSM_OK) return st;
+  if (bias && (st = check(bias, "bias", 1, s_d, MSSM_F32, false)) != MSSM_OK) return st;
+  if (same_ptr(out, x) || same_ptr(out, conv_state) || same_ptr(conv_state, x))
+    return fail(MSSM_ERR_INVALID_ARG, "out, x and conv_state must not alias");
+  if (Bt * Dd > int64_t(INT32_MAX)) return fail(MSSM_ERR_UNSUPPORTED, "Bt * D must fit in 31 bits");
+  if (Bt == 0 || Dd == 0) return MSSM_OK;
+  mssm::ConvUpdateArgs a{};
+  a.state = conv_state->data;
+  a.st_sb = conv_state->stride[0]; a.st_sd = conv_state->stride[1]; a.st_sk = conv_state->stride[2];
+  a.x = x->data; a.out = out->data;
+  a.x_sb = x->stride[0]; a.x_sd = x->stride[1]; a.o_sb = out->stride[0]; a.o_sd = out->stride[1];
+  a.w = static_cast<const float*>(weight->data); a.w_sd = weight->stride[0]; a.w_sk = weight->stride[1];
+  a.bias = bias ? static_cast<const float*>(bias->data) : nullptr; a.bias_s = bias ? bias->stride[0] : 0;
+  a.Bt = int(Bt); a.D = int(Dd); a.K = int(K);
+  a.silu = silu_flag != 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lk(g_mu);
+  cudaError_t e = tracked(MSSM_KERNEL_CONV, s, [&] { return mssm::launch_causal_conv1d_update(a, dt, s); });
+  if (e != cudaSuccess) return cuda_fail(e, "conv1d update kernel launch");
+  return MSSM_OK;
 }
 
 mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int* rows_per_cta,

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 
+#include "conv.cuh"
 #include "decode.cuh"
 #include "scan.cuh"
 
@@ -19,6 +20,9 @@ cudaError_t device_error_word(unsigned int** out);
 // bulk: the state is one contiguous [rows][16] range (bulk-copy kernel), else one thread per row.
 enum class DecodePath { kStream, kBulkTile, kPerRow };
 cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, DecodePath path, cudaStream_t s);
+// Causal conv1d + SiLU: grid (ceil(rows / kConvWarps), items); one decode step of it.
+cudaError_t launch_causal_conv1d(const ConvArgs& a, int items, int dtype, bool silu, cudaStream_t s);
+cudaError_t launch_causal_conv1d_update(const ConvUpdateArgs& a, int dtype, cudaStream_t s);
 // Reads (and optionally clears) the current device's error word.
 cudaError_t read_device_error(unsigned int* value, bool clear);
 

@@ -205,6 +205,8 @@ WORKLOADS = {
     # long context, slow decay spanning many chunks
     "scan_bf16_1x2048x131072": dict(kind="scan", batch=1, dim=2048, length=131072,
                                     io_dtype="bf16", delta_range=(1e-4, 1e-2), with_z=True),
+    # the causal conv1d (K = 4) + SiLU that produces u, at the Mamba-130M prefill shape
+    "conv_bf16_2x1536x2048": dict(kind="conv", batch=2, dim=1536, length=2048, io_dtype="bf16", K=4),
     # packed variable-length prefill: 32 sequences of 64..4096 steps (log-uniform) over
     # Mamba-130M's 1536 channels, concatenated along L without padding
     "scan_varlen_bf16_1536x32seq": dict(kind="scan", batch=1, dim=1536, nseq=32, len_range=(64, 4096),
@@ -212,6 +214,28 @@ WORKLOADS = {
     # one-token decode state update, timed over successive steps
     "decode_bf16_256x5120": dict(kind="decode", batch=256, dim=5120, io_dtype="bf16"),
 }
+
+
+@dataclasses.dataclass
+class ConvInputs:
+    """One causal conv1d problem: ``x`` [batch, dim, length] in ``io_dtype`` storage,
+    ``weight`` [dim, K] and ``bias`` [dim] float32."""
+    batch: int
+    dim: int
+    length: int
+    io_dtype: str
+    x: np.ndarray
+    weight: np.ndarray
+    bias: np.ndarray
+
+
+def make_conv_inputs(batch: int, dim: int, length: int, K: int = 4, *, io_dtype: str = "bf16",
+                     seed: int = 0) -> ConvInputs:
+    """x ~ N(0, 1); weight ~ N(0, 1/K) (unit-variance output before SiLU); bias ~ N(0, 0.25)."""
+    x = _store(_normal(seed, 20, (batch, dim, length)), io_dtype)
+    w = _normal(seed, 21, (dim, K), std=1.0 / np.sqrt(K)).astype(np.float32)
+    b = _normal(seed, 22, (dim,), std=0.5).astype(np.float32)
+    return ConvInputs(batch, dim, length, io_dtype, x, w, b)
 
 
 def varlen_lengths(nseq: int, lo: int, hi: int, seed: int = 0) -> np.ndarray:
@@ -236,5 +260,7 @@ def workload_inputs(name: str, seed: int = 0, batch: Optional[int] = None,
     if kind == "scan":
         return make_scan_inputs(w["batch"], w["dim"], w["length"], io_dtype=w["io_dtype"],
                                 seed=seed, delta_range=w["delta_range"], with_z=w["with_z"])
+    if kind == "conv":
+        return make_conv_inputs(w["batch"], w["dim"], w["length"], w["K"], io_dtype=w["io_dtype"], seed=seed)
     return make_decode_inputs(w["batch"], w["dim"], io_dtype=w["io_dtype"], seed=seed,
                               step_stream=step_stream)

@@ -203,6 +203,26 @@ def test_scan_varlen_validation(lib, case):
     assert last_error(lib)
 
 
+def test_conv_validation(lib):
+    P = lambda t: None if t is None else ctypes.byref(t)  # noqa: E731
+    f = lib.mssm_causal_conv1d_fwd
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    x, out = mk([2, 8, 32], 1), mk([2, 8, 32], 1)
+    assert f(P(x), P(mk([8, 5], 0)), None, None, 0, 1, P(out), None) == UNSUPPORTED  # K = 5
+    assert f(P(x), P(mk([8, 4], 1)), None, None, 0, 1, P(out), None) == INVALID      # bf16 weight
+    out.data = x.data
+    assert f(P(x), P(mk([8, 4], 0)), None, None, 0, 1, P(out), None) == INVALID      # alias
+    out = mk([2, 8, 32], 1)
+    assert f(P(x), P(mk([8, 4], 0)), None, P(mk([3], 2)), 10, 1, P(out), None) == INVALID  # Bt != 1
+    g = lib.mssm_causal_conv1d_update
+    g.restype = ctypes.c_int
+    g.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    xs, os_ = mk([2, 8], 1), mk([2, 8], 1)
+    assert g(P(mk([2, 8, 0], 1)), P(xs), P(mk([8, 1], 0)), None, 1, P(os_), None) == UNSUPPORTED  # K = 1
+    assert g(P(mk([2, 8, 2], 1)), P(xs), P(mk([8, 4], 0)), None, 1, P(os_), None) == INVALID      # state K-1
+
+
 def test_decode_ex_rejects_unknown_discretization(lib):
     P = ctypes.byref
     f = lib.mssm_state_update_ex
