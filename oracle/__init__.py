@@ -48,6 +48,9 @@ def _load():
                                                 ctypes.c_int, ctypes.c_int, P]
         lib.oracle_state_update_f64.restype = None
         lib.oracle_causal_conv1d_f64.argtypes = [I64, I64, I64, I64, P, P, P, ctypes.c_int, P]
+        lib.oracle_scan_bwd_f64.argtypes = [I64, I64, I64, I64, P, P, P, P, P, P, P, P, ctypes.c_int,
+                                            P, P, P, P, P, P, P, P, P]
+        lib.oracle_scan_bwd_f64.restype = None
         lib.oracle_causal_conv1d_f64.restype = None
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -113,6 +116,28 @@ def state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
                                     _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
                                     int(bool(softplus)), int(bool(zoh)), _ptr(out))
     return st, out
+
+
+def scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, dout=None) -> dict:
+    """Gradients of ``scan`` (Euler, zero initial state) with respect to every input, for
+    dLoss/dout = ``dout`` [Bt, D, L].  Returns a dict with du, ddelta, dA, dB, dC and, when
+    the inputs are given, dD, dz, ddelta_bias (float64)."""
+    u, delta, A, B, C, dout = map(_f64, (u, delta, A, B, C, dout))
+    D, z, delta_bias = map(_f64, (D, z, delta_bias))
+    Bt, Dd, L = u.shape
+    N = A.shape[1]
+    if N > 64:
+        raise ValueError("oracle supports N <= 64")
+    assert dout.shape == u.shape
+    out = dict(du=np.empty_like(u), ddelta=np.empty_like(u), dA=np.empty_like(A), dB=np.empty_like(B),
+               dC=np.empty_like(C), dD=None if D is None else np.empty_like(D),
+               dz=None if z is None else np.empty_like(z),
+               ddelta_bias=None if delta_bias is None else np.empty_like(delta_bias))
+    _load().oracle_scan_bwd_f64(Bt, Dd, L, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                _ptr(z), _ptr(delta_bias), int(bool(softplus)), _ptr(dout),
+                                _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dA"]), _ptr(out["dB"]),
+                                _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dz"]), _ptr(out["ddelta_bias"]))
+    return out
 
 
 def causal_conv1d(x, w, bias=None, silu=True) -> np.ndarray:

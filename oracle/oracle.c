@@ -57,6 +57,7 @@
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #ifdef _OPENMP
 #include <omp.h>
@@ -216,3 +217,100 @@ void oracle_causal_conv1d_f64(int64_t Bt, int64_t D, int64_t L, int64_t K,
     }
 }
 
+
+/* sigmoid(x) = 1 / (1 + exp(-x)). */
+static double sigm(double x)
+{
+    return 1.0 / (1.0 + exp(-x));
+}
+
+/*
+ * Gradients of the selective scan (Euler discretisation, zero initial state) with
+ * respect to every input, given dout = dLoss/dout.  The forward is the loop of
+ * oracle_scan_f64; this is its reverse-mode chain rule written out step by step,
+ * from the last step to the first, keeping every state of the forward (the pages'
+ * kernel recomputes them: "Mamba selective state space", the hardware-aware scan;
+ * here they are simply stored).  Per row, with g[n] = dLoss/dh_t[n]:
+ *   gy     = dout_t * silu(z_t)                 dz_t = dout_t * y_t * silu'(z_t)
+ *   dD    += gy * u_t                           du_t = gy * D
+ *   g[n]  += gy * C_tn                          dC_tn += gy * h_tn
+ *   with a = exp(dt A_n):  ddt += g[n] (A_n a h_(t-1)n + B_tn u_t)
+ *                          dA_n += g[n] dt a h_(t-1)n,  dB_tn += g[n] dt u_t,
+ *                          du_t += g[n] dt B_tn,        g[n] *= a
+ *   ddelta_t = ddt * sigmoid(delta_t + bias) (softplus) or ddt;  dbias += ddelta_t
+ * dB and dC sum over the channels of a batch; dA, dD and dbias over batches and steps.
+ * Outputs are overwritten; nullable: Dskip/dD, z/dz, bias/dbias.  Serial.
+ */
+void oracle_scan_bwd_f64(int64_t Bt, int64_t D, int64_t L, int64_t N,
+                         const double *u, const double *delta, const double *A,
+                         const double *B, const double *C, const double *Dskip,
+                         const double *z, const double *bias, int softplus_flag,
+                         const double *dout, double *du, double *ddelta, double *dA,
+                         double *dB, double *dC, double *dD, double *dz, double *dbias)
+{
+    for (int64_t i = 0; i < D * N; ++i) dA[i] = 0.0;
+    for (int64_t i = 0; i < Bt * N * L; ++i) { dB[i] = 0.0; dC[i] = 0.0; }
+    if (dD) for (int64_t i = 0; i < D; ++i) dD[i] = 0.0;
+    if (dbias) for (int64_t i = 0; i < D; ++i) dbias[i] = 0.0;
+    double *hs = (double *)malloc(sizeof(double) * (size_t)((L + 1) * N));
+    double *dts = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    double *ys = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    double g[64];
+    for (int64_t r = 0; r < Bt * D; ++r) {
+        int64_t b = r / D, d = r % D;
+        const double *ur = u + r * L, *dr = delta + r * L;
+        const double *zr = z ? z + r * L : NULL;
+        const double *Bb = B + b * N * L, *Cb = C + b * N * L, *Ad = A + d * N;
+        /* forward, keeping h_t (hs row t+1; row 0 = h_(-1) = 0), dt_t and y_t */
+        for (int64_t n = 0; n < N; ++n) hs[n] = 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            double step = dr[t] + (bias ? bias[d] : 0.0);
+            if (softplus_flag) step = sp_exact(step);
+            dts[t] = step;
+            double y = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                double h = exp(step * Ad[n]) * hs[t * N + n] + step * Bb[n * L + t] * ur[t];
+                hs[(t + 1) * N + n] = h;
+                y += Cb[n * L + t] * h;
+            }
+            if (Dskip) y += Dskip[d] * ur[t];
+            ys[t] = y;
+        }
+        /* reverse */
+        for (int64_t n = 0; n < N; ++n) g[n] = 0.0;
+        for (int64_t t = L - 1; t >= 0; --t) {
+            double gy = dout[r * L + t];
+            if (zr) {
+                double s = sigm(zr[t]);
+                dz[r * L + t] = dout[r * L + t] * ys[t] * s * (1.0 + zr[t] * (1.0 - s));
+                gy *= zr[t] * s;
+            }
+            double dut = 0.0;
+            if (Dskip) {
+                dD[d] += gy * ur[t];
+                dut = gy * Dskip[d];
+            }
+            double dt = dts[t], ddt = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                g[n] += gy * Cb[n * L + t];
+                dC[b * N * L + n * L + t] += gy * hs[(t + 1) * N + n];
+            }
+            for (int64_t n = 0; n < N; ++n) {
+                double a = exp(dt * Ad[n]);
+                double hp = hs[t * N + n];
+                ddt += g[n] * (Ad[n] * a * hp + Bb[n * L + t] * ur[t]);
+                dA[d * N + n] += g[n] * dt * a * hp;
+                dB[b * N * L + n * L + t] += g[n] * dt * ur[t];
+                dut += g[n] * dt * Bb[n * L + t];
+                g[n] *= a;
+            }
+            du[r * L + t] = dut;
+            double draw = softplus_flag ? ddt * sigm(dr[t] + (bias ? bias[d] : 0.0)) : ddt;
+            ddelta[r * L + t] = draw;
+            if (dbias) dbias[d] += draw;
+        }
+    }
+    free(hs);
+    free(dts);
+    free(ys);
+}

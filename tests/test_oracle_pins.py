@@ -464,6 +464,49 @@ def test_varlen_sequences_are_isolated():
 
 
 # ---------------------------------------------------------------------------
+# 7e. backward: every gradient against central finite differences of the forward
+# ---------------------------------------------------------------------------
+
+def _fd_check_bwd(softplus, with_z, with_D, seed, n_probe=24):
+    rng = np.random.default_rng(seed)
+    p = rand_problem(rng, 2, 3, 7, with_z=with_z, with_D=with_D)
+    if not softplus:  # keep the raw step positive, as softplus would
+        p["delta"] = 0.2 * np.abs(p["delta"])
+        p["delta_bias"] = rng.uniform(0.01, 0.1, size=p["delta_bias"].shape)
+    dout = rng.standard_normal(p["u"].shape)
+    g = oracle.scan_bwd(**p, softplus=softplus, dout=dout)
+
+    def loss(q):
+        return float((oracle.scan(**q, softplus=softplus)[0] * dout).sum())
+
+    eps = 1e-6
+    for name in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias"):
+        if p[name] is None:
+            assert g.get("d" + name) is None
+            continue
+        grad = g["d" + name]
+        idxs = list(np.ndindex(p[name].shape))
+        pick = rng.choice(len(idxs), size=min(n_probe, len(idxs)), replace=False)
+        for i in pick:
+            idx = idxs[i]
+            q = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in p.items()}
+            q[name][idx] += eps
+            lp = loss(q)
+            q[name][idx] -= 2 * eps
+            lm = loss(q)
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-6 * (1 + abs(fd)), (name, idx, fd, grad[idx])
+
+
+def test_backward_matches_finite_differences():
+    _fd_check_bwd(True, True, True, seed=51)
+
+
+def test_backward_without_softplus_gate_or_skip():
+    _fd_check_bwd(False, False, False, seed=52)
+
+
+# ---------------------------------------------------------------------------
 # 8. hand-derived worked example (tests/golden/halving_decay.txt)
 # ---------------------------------------------------------------------------
 
@@ -513,6 +556,15 @@ MUTANTS = {
     "zoh_gain_is_exp": ("return expm1(dt * a) / a;", "return exp(dt * a) / a;"),
     "scan_zoh_ignored": ("b_bar = zoh_gain(dt, Ad[n]) * Bb[n * L + t];", "b_bar = dt * Bb[n * L + t];"),
     "decode_zoh_ignored": ("double gain = zoh_flag ? zoh_gain(dt, A[d * N + n]) : dt;", "double gain = dt;"),
+    "bwd_no_decay_propagation": ("                g[n] *= a;\n", "\n"),
+    "bwd_dA_without_dt": ("dA[d * N + n] += g[n] * dt * a * hp;", "dA[d * N + n] += g[n] * a * hp;"),
+    "bwd_dB_uses_C": ("dB[b * N * L + n * L + t] += g[n] * dt * ur[t];",
+                      "dB[b * N * L + n * L + t] += g[n] * dt * Cb[n * L + t];"),
+    "bwd_dC_uses_previous_state": ("dC[b * N * L + n * L + t] += gy * hs[(t + 1) * N + n];",
+                                   "dC[b * N * L + n * L + t] += gy * hs[t * N + n];"),
+    "bwd_softplus_derivative_dropped": ("double draw = softplus_flag ? ddt * sigm(dr[t] + (bias ? bias[d] : 0.0)) : ddt;",
+                                        "double draw = ddt;"),
+    "bwd_gate_derivative_sign": ("s * (1.0 + zr[t] * (1.0 - s));", "s * (1.0 - zr[t] * (1.0 - s));"),
     "conv_filter_reversed": ("acc += wd[j] * xr[src];", "acc += wd[K - 1 - j] * xr[src];"),
     "conv_window_off_by_one": ("int64_t src = t + j - (K - 1);", "int64_t src = t + j - K;"),
     "conv_bias_dropped": ("double acc = bias ? bias[d] : 0.0;", "double acc = 0.0;"),
@@ -539,6 +591,8 @@ PIN_CALLS = [
     test_zoh_small_A_is_euler,
     test_zoh_decode_steps_reproduce_scan,
     lambda: test_conv1d_matches_numpy_convolve(True),
+    test_backward_matches_finite_differences,
+    test_backward_without_softplus_gate_or_skip,
     test_conv1d_matches_torch_conv1d,
     test_conv1d_impulse_response,
 ]
@@ -563,6 +617,8 @@ def _count_failures(lib_path):
     lib.oracle_state_update_f64.argtypes = [I64, I64, I64, P, P, P, P, P, P, P, P, P, ctypes.c_int,
                                             ctypes.c_int, P]
     lib.oracle_causal_conv1d_f64.argtypes = [I64, I64, I64, I64, P, P, P, ctypes.c_int, P]
+    lib.oracle_scan_bwd_f64.argtypes = [I64, I64, I64, I64, P, P, P, P, P, P, P, P, ctypes.c_int,
+                                        P, P, P, P, P, P, P, P, P]
     lib.oracle_num_threads.restype = ctypes.c_int
     saved = oracle._lib
     oracle._lib = lib
