@@ -46,6 +46,8 @@ import synth  # noqa: E402
 METRIC = "selective-scan B·D·L elems/s and achieved HBM GB/s vs ~8 TB/s B200 peak"
 DECODE_METRIC = "selective state update rows/s and achieved HBM GB/s vs ~8 TB/s B200 peak"
 CONV_METRIC = "causal conv1d + SiLU B·D·L elems/s and achieved HBM GB/s vs ~8 TB/s B200 peak"
+BWD_METRIC = "selective-scan backward B·D·L elems/s and achieved HBM GB/s vs ~8 TB/s B200 peak"
+BWD_FLOP_PER_STATE = 22  # the forward recomputed (6) and the reverse step (16) per (element, state)
 DEFAULT_WORKLOAD = "scan_bf16_2x1536x2048"
 L2_FLUSH_BYTES = 256 << 20
 NOMINAL_HBM_GBS = 8000.0
@@ -267,7 +269,7 @@ class ClockSampler:
 # reference arm: the fp64 CPU oracle on the host cores
 # --------------------------------------------------------------------------
 
-def oracle_sample(workload: str, rows: int, zoh: bool = False):
+def oracle_sample(workload: str, rows: int, zoh: bool = False, backward: bool = False):
     """A bounded sample of the workload for the CPU oracle: the first ``rows`` channels of batch 0
     (of every packed sequence, for a packed workload)."""
     import oracle
@@ -281,6 +283,11 @@ def oracle_sample(workload: str, rows: int, zoh: bool = False):
                     softplus=inp.softplus, zoh=zoh)
         units = d * inp.length
         disc = ", zero-order hold" if zoh else ""
+        if backward:
+            dout = np.random.default_rng(7).standard_normal(args["u"].shape)
+            bargs = {k: v for k, v in args.items() if k != "zoh"}
+            desc = f"backward, batch 0, channels 0..{d - 1}, all {inp.length} steps ({units} elements, serial)"
+            return (lambda: oracle.scan_bwd(dout=dout, **bargs)), units, desc
         if inp.cu_seqlens is not None:
             cu = inp.cu_seqlens
             desc = (f"channels 0..{d - 1} of all {len(cu) - 1} packed sequences ({units} elements{disc})")
@@ -302,11 +309,11 @@ def oracle_sample(workload: str, rows: int, zoh: bool = False):
     return (lambda: oracle.state_update(**args)), units, f"batches 0..{b - 1} ({units} rows)"
 
 
-def cpu_baseline(workload: str, budget_s: float = 10.0, zoh: bool = False):
+def cpu_baseline(workload: str, budget_s: float = 10.0, zoh: bool = False, backward: bool = False):
     import oracle
     is_scan = WORKLOADS_KIND[workload] in ("scan", "conv")
-    rows = 512 if is_scan else 256 * 5120
-    fn, units, desc = oracle_sample(workload, rows, zoh)
+    rows = (64 if backward else 512) if is_scan else 256 * 5120
+    fn, units, desc = oracle_sample(workload, rows, zoh, backward)
     fn()  # build + warm
     t0 = time.perf_counter()
     n = 0
@@ -316,7 +323,8 @@ def cpu_baseline(workload: str, budget_s: float = 10.0, zoh: bool = False):
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 10000:
             break
-    return {"value": units * n / el, "unit": "elems/s" if is_scan else "rows/s", "cores": oracle.num_threads(),
+    return {"value": units * n / el, "unit": "elems/s" if is_scan else "rows/s",
+            "cores": 1 if backward else oracle.num_threads(),
             "kind": "oracle", "sample": f"{desc}, repeated {n}x over {el:.1f} s (fp64, OpenMP over rows)"}
 
 
@@ -330,7 +338,8 @@ def run_reference(args):
     import oracle
     kind = WORKLOADS_KIND[args.workload]
     is_scan = kind in ("scan", "conv")
-    fn, units, desc = oracle_sample(args.workload, 256 if is_scan else 256 * 5120, args.zoh)
+    fn, units, desc = oracle_sample(args.workload, (32 if args.backward else 256) if is_scan else 256 * 5120,
+                                    args.zoh, args.backward)
     for _ in range(max(args.warmup, 0)):
         fn()
     times = []
@@ -342,7 +351,8 @@ def run_reference(args):
     value = units / (ms / 1e3)
     unit = "elems/s" if is_scan else "rows/s"
     line = {
-        "impl": "reference", "metric": {"scan": METRIC, "conv": CONV_METRIC}.get(kind, DECODE_METRIC),
+        "impl": "reference",
+        "metric": BWD_METRIC if args.backward else {"scan": METRIC, "conv": CONV_METRIC}.get(kind, DECODE_METRIC),
         "value": value, "unit": unit,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -443,6 +453,30 @@ def run_mssm(args):
         metric, unit = METRIC, "elems/s"
         dom_kernel = "scan_out"
         set_bytes = alg_bytes
+        if args.backward:
+            if varlen or args.zoh:
+                raise SystemExit("--backward covers the Euler scan of plain batches")
+            # reads u, delta, z, dout, B, C; writes du, ddelta, dz (io dtype) and dB, dC (fp32)
+            n_io = 7 if inp.z is not None else 5
+            alg_bytes = (units * io_bytes * n_io + 2 * inp.batch * N_STATE * inp.length * (io_bytes + 4)
+                         + inp.dim * N_STATE * 8 + inp.dim * 16)
+            rng = np.random.default_rng(seed + 7)
+            dout_h = rng.standard_normal(inp.u.shape).astype(np.float32)
+            if inp.io_dtype == "bf16":
+                dout_h = synth.f32_to_bf16_bits(dout_h)
+            dout_d = to_dev(dout_h)
+            grads = [m.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["z"],
+                                          d["delta_bias"], inp.softplus, dout_d) for _ in range(2)]
+
+            def step(k=0):
+                dk = sets[k % len(sets)][0]
+                gk = grads[k % 2]
+                m.mssm_selective_scan_bwd(dk["u"], dk["delta"], dk["A"], dk["B"], dk["C"], dk["D"], dk["z"],
+                                          dk["delta_bias"], inp.softplus, dout_d, gk["du"], gk["ddelta"],
+                                          gk["dA"], gk["dB"], gk["dC"], gk["dD"], gk["dz"], gk["ddelta_bias"])
+            metric = BWD_METRIC
+            dom_kernel = "scan_bwd"
+            config["pass"] = "backward (passes A, B, C)"
     elif kind == "conv":
         inp = synth.workload_inputs(args.workload, seed=seed)
         units = inp.batch * inp.dim * inp.length
@@ -558,8 +592,13 @@ def run_mssm(args):
     dom_ms = dom["ms_per_launch"] if dom else None
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     alu_peak = fp32_peak_tflops(sms, max_sm_mhz())
-    # the conv: K FMAs per element (its SiLU runs on the SFU)
-    alg_flops = algorithmic_flops(units) if kind != "conv" else units * 2 * inp.weight.shape[1]
+    # the conv: K FMAs per element (its SiLU runs on the SFU); the backward: BWD_FLOP_PER_STATE
+    if kind == "conv":
+        alg_flops = units * 2 * inp.weight.shape[1]
+    elif kind == "scan" and args.backward:
+        alg_flops = units * N_STATE * BWD_FLOP_PER_STATE
+    else:
+        alg_flops = algorithmic_flops(units)
     plan_key = (plan_string(config.get("plan")) if kind == "scan" else
                 f"decode_path={args.decode_path}" if kind == "decode" else None)
     traffic, traffic_src = recorded_traffic(dom_kernel, args.workload, plan_key)
@@ -589,7 +628,7 @@ def run_mssm(args):
         "source_hash": kernel_source_hash(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds, args.zoh)
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds, args.zoh, args.backward)
     if world > 1:
         dist.barrier()
         del g
@@ -626,6 +665,32 @@ def run_e2e(args, kind, inp, d, dev, m, units, world):
             xd.copy_(hx, non_blocking=True)
             m.mssm_causal_conv1d_fwd(xd, w_d, b_d, out, None, 0, True)
             y_host.copy_(out, non_blocking=True)
+    elif kind == "scan" and args.backward:
+        names = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
+        h = {k: pin(getattr(inp, k)) for k in names}
+        rng = np.random.default_rng(7)
+        dout_h = rng.standard_normal(inp.u.shape).astype(np.float32)
+        h["dout"] = pin(synth.f32_to_bf16_bits(dout_h) if inp.io_dtype == "bf16" else dout_h)
+        dd = {k: (None if v is None else torch.empty(v.shape, dtype=v.dtype, device=dev)) for k, v in h.items()}
+        for k in h:
+            if h[k] is not None:
+                dd[k].copy_(h[k])
+        g = m.selective_scan_bwd(dd["u"], dd["delta"], dd["A"], dd["B"], dd["C"], dd["D"], dd["z"],
+                                 dd["delta_bias"], inp.softplus, dd["dout"])
+        g_host = {k: (None if v is None else torch.empty(v.shape, dtype=v.dtype).pin_memory()) for k, v in g.items()}
+        h2d = sum(v.numel() * v.element_size() for v in h.values() if v is not None)
+        d2h = sum(v.numel() * v.element_size() for v in g_host.values() if v is not None)
+
+        def one():
+            for k in h:
+                if h[k] is not None:
+                    dd[k].copy_(h[k], non_blocking=True)
+            m.mssm_selective_scan_bwd(dd["u"], dd["delta"], dd["A"], dd["B"], dd["C"], dd["D"], dd["z"],
+                                      dd["delta_bias"], inp.softplus, dd["dout"], g["du"], g["ddelta"], g["dA"],
+                                      g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"])
+            for k, v in g.items():
+                if v is not None:
+                    g_host[k].copy_(v, non_blocking=True)
     elif kind == "scan":
         names = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
         h = {k: pin(getattr(inp, k)) for k in names}
@@ -701,6 +766,7 @@ def main(argv=None):
     ap.add_argument("--decode-path", choices=["auto", "stream", "bulk_tile", "per_row"], default="auto",
                     help="decode kernel (MSSM_OPT_DECODE_PATH)")
     ap.add_argument("--zoh", action="store_true", help="zero-order-hold discretisation (scan workloads)")
+    ap.add_argument("--backward", action="store_true", help="time the backward scan instead (scan workloads)")
     ap.add_argument("--general-a", action="store_true",
                     help="disable the structured-A path (one exponential per state)")
     args = ap.parse_args(argv)

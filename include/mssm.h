@@ -238,6 +238,32 @@ mssm_status mssm_state_update_ex(mssm_tensor *state, const mssm_tensor *x,
                                  int discretization, mssm_tensor *out, void *stream);
 
 /*
+ * Backward of mssm_selective_scan_fwd (Euler discretisation, zero initial state,
+ * no packed sequences): the gradients of Loss with respect to every input, given
+ * dout = dLoss/dout.  The states are recomputed, never stored: the forward's
+ * chunk summaries give every 64-step chunk's start state, a reverse pass of chunk
+ * summaries gives every chunk's incoming dLoss/dh, and every chunk then sweeps its
+ * recomputed states backwards ("Mamba selective state space", the hardware-aware
+ * scan: intermediates are recomputed in the backward pass).
+ *   inputs     as for mssm_selective_scan_fwd, plus dout [Bt, D, L] dtype of u
+ *   du, ddelta [Bt, D, L] dtype of u, written (ddelta: with respect to delta before
+ *              the bias and softplus)
+ *   dz         [Bt, D, L] dtype of u, written; given exactly when z is
+ *   dA         [D, N] f32; dB, dC [Bt, N, L] f32 (summed over channels);
+ *   dD, ddelta_bias [D] f32, given exactly when D / delta_bias are
+ * The f32 gradients must be dense; they are zeroed and accumulated with atomic
+ * adds, so their rounding order is not fixed.  Uses a per-device workspace of
+ * about (2 x 68 x L / 64) bytes per row, grown with cudaMalloc on demand (which
+ * synchronises the device) and freed by mssm_shutdown().
+ */
+mssm_status mssm_selective_scan_bwd(const mssm_tensor *u, const mssm_tensor *delta, const mssm_tensor *A,
+                                    const mssm_tensor *B, const mssm_tensor *C, const mssm_tensor *D,
+                                    const mssm_tensor *z, const mssm_tensor *delta_bias, int softplus_flag,
+                                    const mssm_tensor *dout, mssm_tensor *du, mssm_tensor *ddelta,
+                                    mssm_tensor *dA, mssm_tensor *dB, mssm_tensor *dC, mssm_tensor *dD,
+                                    mssm_tensor *dz, mssm_tensor *ddelta_bias, void *stream);
+
+/*
  * Causal depthwise conv1d + SiLU: the step that produces the scan's input u from
  * the in-projection's x branch ("Linear Attention vs Softmax Attention ...",
  * section Implementation: the listed layer's grouped Conv1d with one group per
@@ -356,7 +382,8 @@ typedef enum {
     MSSM_KERNEL_SCAN_OUT = 1,         /* forward sweep with fused epilogue */
     MSSM_KERNEL_STATE_UPDATE = 2,     /* decode step */
     MSSM_KERNEL_CONV = 3,             /* causal conv1d (prefill and decode step) */
-    MSSM_KERNEL_KINDS = 4
+    MSSM_KERNEL_SCAN_BWD = 4,         /* backward scan (passes B and C; pass A counts as CHUNK_STATE) */
+    MSSM_KERNEL_KINDS = 5
 } mssm_kernel_kind;
 
 /*

@@ -25,6 +25,7 @@ __all__ = [
     "MSSM_OPT_DECODE_PATH", "DECODE_PATHS", "MSSM_OPT_TEST_HOOKS", "MSSM_ERR_TIMEOUT", "mssm_kernel_stats", "mssm_scan_plan",
     "mssm_selective_scan_fwd_ex", "MSSM_DISC_EULER", "MSSM_DISC_ZOH",
     "mssm_causal_conv1d_fwd", "mssm_causal_conv1d_update", "causal_conv1d", "causal_conv1d_update",
+    "mssm_selective_scan_bwd", "selective_scan_bwd",
     "KERNEL_KINDS",
 ]
 
@@ -43,7 +44,7 @@ MSSM_OPT_TEST_HOOKS = 6
 MSSM_DISC_EULER, MSSM_DISC_ZOH = 0, 1
 SCHEDULES = {"forward": 1, "summaries+forward": 2, "chained": 3}
 DECODE_PATHS = {"stream": 1, "bulk_tile": 2, "per_row": 3}
-KERNEL_KINDS = ("scan_chunk_state", "scan_out", "state_update", "conv")
+KERNEL_KINDS = ("scan_chunk_state", "scan_out", "state_update", "conv", "scan_bwd")
 
 
 class mssm_tensor(ctypes.Structure):
@@ -70,6 +71,8 @@ _lib.mssm_state_update.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _V]
 _lib.mssm_state_update.restype = ctypes.c_int
 _lib.mssm_state_update_ex.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _V]
 _lib.mssm_state_update_ex.restype = ctypes.c_int
+_lib.mssm_selective_scan_bwd.argtypes = [_P] * 8 + [ctypes.c_int] + [_P] * 9 + [_V]
+_lib.mssm_selective_scan_bwd.restype = ctypes.c_int
 _lib.mssm_causal_conv1d_fwd.argtypes = [_P, _P, _P, _P, ctypes.c_int64, ctypes.c_int, _P, _V]
 _lib.mssm_causal_conv1d_fwd.restype = ctypes.c_int
 _lib.mssm_causal_conv1d_update.argtypes = [_P, _P, _P, _P, ctypes.c_int, _P, _V]
@@ -230,6 +233,29 @@ def mssm_state_update_ex(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, ou
     do = _desc(out)
     _check(_lib.mssm_state_update_ex(*[_ref(v) for v in ds], int(softplus_flag), int(discretization), _ref(do),
                                      _stream(stream, x)))
+
+
+def mssm_selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, dout, du, ddelta, dA, dB, dC,
+                            dD, dz, ddelta_bias, stream=None) -> None:
+    """Marshal torch tensors into ``mssm_selective_scan_bwd`` (see include/mssm.h)."""
+    ds = [_desc(t) for t in (u, delta, A, B, C, D, z, delta_bias)]
+    gs = [_desc(t) for t in (dout, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias)]
+    _check(_lib.mssm_selective_scan_bwd(*[_ref(x) for x in ds], int(softplus_flag), *[_ref(x) for x in gs],
+                                        _stream(stream, u)))
+
+
+def selective_scan_bwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=True, dout=None,
+                       stream=None) -> dict:
+    """Allocate the gradients with torch and run the backward scan on the GPU."""
+    f32 = dict(device=u.device, dtype=torch.float32)
+    g = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u), dA=torch.empty(A.shape, **f32),
+             dB=torch.empty(B.shape, **f32), dC=torch.empty(C.shape, **f32),
+             dD=None if D is None else torch.empty(D.shape, **f32),
+             dz=None if z is None else torch.empty_like(z),
+             ddelta_bias=None if delta_bias is None else torch.empty(delta_bias.shape, **f32))
+    mssm_selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus, dout, g["du"], g["ddelta"], g["dA"],
+                            g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"], stream)
+    return g
 
 
 def mssm_causal_conv1d_fwd(x, weight, bias, out, cu_seqlens=None, max_seqlen=0, silu_flag=True,

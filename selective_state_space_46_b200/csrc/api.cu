@@ -84,6 +84,8 @@ struct DeviceState {
   size_t ws_bytes = 0;
   int64_t count_cap = 0;  // arrival counters at the start of ws (a region only counters ever use)
   int sm_count = 0;
+  void* bwd_ws = nullptr;  // the backward scan's checkpoints and chunk gradients
+  size_t bwd_bytes = 0;
 };
 std::vector<DeviceState> g_dev;
 
@@ -770,6 +772,151 @@ mssm_status mssm_state_update_ex(mssm_tensor* state, const mssm_tensor* x, const
   return state_update_impl(state, x, dt, A, B, C, D, z, dt_bias, softplus_flag, discretization, out, stream);
 }
 
+mssm_status mssm_selective_scan_bwd(const mssm_tensor* u, const mssm_tensor* delta, const mssm_tensor* A,
+                                    const mssm_tensor* B, const mssm_tensor* C, const mssm_tensor* D,
+                                    const mssm_tensor* z, const mssm_tensor* delta_bias, int softplus_flag,
+                                    const mssm_tensor* dout, mssm_tensor* du, mssm_tensor* ddelta,
+                                    mssm_tensor* dA, mssm_tensor* dB, mssm_tensor* dC, mssm_tensor* dD,
+                                    mssm_tensor* dz, mssm_tensor* ddelta_bias, void* stream) {
+  // the forward's checks, with dout in the place of out (its shape, dtype and layout)
+  ScanCall call;
+  mssm_status st = scan_prepare(u, delta, A, B, C, D, z, delta_bias, softplus_flag,
+                                const_cast<mssm_tensor*>(dout), nullptr, call);
+  if (st != MSSM_OK) return st;
+  const int dt = u->dtype;
+  const int64_t Bt = u->shape[0], Dd = u->shape[1], L = u->shape[2], N = mssm::kN;
+  const int64_t s_bdl[3] = {Bt, Dd, L}, s_bnl[3] = {Bt, N, L}, s_dn[2] = {Dd, N}, s_d[1] = {Dd};
+  if ((st = check(du, "du", 3, s_bdl, dt, true)) != MSSM_OK) return st;
+  if ((st = check(ddelta, "ddelta", 3, s_bdl, dt, true)) != MSSM_OK) return st;
+  if ((st = check(dA, "dA", 2, s_dn, MSSM_F32, true)) != MSSM_OK) return st;
+  if ((st = check(dB, "dB", 3, s_bnl, MSSM_F32, true)) != MSSM_OK) return st;
+  if ((st = check(dC, "dC", 3, s_bnl, MSSM_F32, true)) != MSSM_OK) return st;
+  if (!D != !dD) return fail(MSSM_ERR_INVALID_ARG, "dD must be given exactly when D is");
+  if (!z != !dz) return fail(MSSM_ERR_INVALID_ARG, "dz must be given exactly when z is");
+  if (!delta_bias != !ddelta_bias)
+    return fail(MSSM_ERR_INVALID_ARG, "ddelta_bias must be given exactly when delta_bias is");
+  if (dD && (st = check(dD, "dD", 1, s_d, MSSM_F32, true)) != MSSM_OK) return st;
+  if (dz && (st = check(dz, "dz", 3, s_bdl, dt, true)) != MSSM_OK) return st;
+  if (ddelta_bias && (st = check(ddelta_bias, "ddelta_bias", 1, s_d, MSSM_F32, true)) != MSSM_OK) return st;
+  // the accumulated gradients are zeroed and atomically added: they must be dense
+  auto dense = [](const mssm_tensor* t) {
+    int64_t want = 1;
+    for (int i = t->ndim - 1; i >= 0; --i) {
+      if (t->shape[i] > 1 && t->stride[i] != want) return false;
+      want *= t->shape[i];
+    }
+    return true;
+  };
+  for (const mssm_tensor* t : {static_cast<const mssm_tensor*>(dA), static_cast<const mssm_tensor*>(dB),
+                               static_cast<const mssm_tensor*>(dC), static_cast<const mssm_tensor*>(dD),
+                               static_cast<const mssm_tensor*>(ddelta_bias)})
+    if (t && !dense(t)) return fail(MSSM_ERR_UNSUPPORTED, "dA, dB, dC, dD and ddelta_bias must be dense");
+  const mssm_tensor* ins[] = {u, delta, A, B, C, D, z, delta_bias, dout};
+  const mssm_tensor* outs[] = {du, ddelta, dA, dB, dC, dD, dz, ddelta_bias};
+  for (const mssm_tensor* o : outs) {
+    if (!o) continue;
+    for (const mssm_tensor* i : ins)
+      if (same_ptr(o, i)) return fail(MSSM_ERR_INVALID_ARG, "gradients must not alias the inputs");
+    for (const mssm_tensor* o2 : outs)
+      if (o2 != o && same_ptr(o, o2)) return fail(MSSM_ERR_INVALID_ARG, "gradients must not alias each other");
+  }
+  if (call.noop) return MSSM_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lk(g_mu);
+  // zero the accumulated gradients
+  cudaError_t e = cudaSuccess;
+  auto zero = [&](const mssm_tensor* t, size_t elems) {
+    if (t && e == cudaSuccess && elems) e = cudaMemsetAsync(t->data, 0, elems * 4, s);
+  };
+  zero(dA, size_t(Dd * N));
+  zero(dB, size_t(Bt * N * L));
+  zero(dC, size_t(Bt * N * L));
+  zero(dD, size_t(Dd));
+  zero(ddelta_bias, size_t(Dd));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(gradients)");
+  if (L == 0) return MSSM_OK;
+
+  // workspace: pass A's chunk states (H, S, counters) and pass B's (G, S, Q, counters)
+  const int64_t tpb = (Dd + mssm::kBwdRows - 1) / mssm::kBwdRows;
+  const int64_t tiles = Bt * tpb, rows_total = tiles * mssm::kBwdRows;
+  const int64_t nseg = (L + mssm::kBwdChunk - 1) / mssm::kBwdChunk;
+  if (nseg > 65535 || tiles > INT32_MAX) return fail(MSSM_ERR_UNSUPPORTED, "problem too large for the backward grid");
+  auto al = [](size_t v) { return (v + 255) / 256 * 256; };
+  const size_t cnt_b = al(size_t(tiles) * 4);
+  const size_t hA_b = al(size_t(nseg - 1) * rows_total * mssm::kN * 4), sA_b = al(size_t(nseg - 1) * rows_total * 4);
+  const size_t g_b = al(size_t(nseg) * rows_total * mssm::kN * 4), sB_b = al(size_t(nseg) * rows_total * 4);
+  const size_t need = 2 * cnt_b + hA_b + sA_b + 2 * g_b + sB_b;
+  int dev = -1;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  DeviceState* ds = device_state(dev);
+  if (ds->bwd_bytes < need) {
+    if (ds->bwd_ws) {
+      e = cudaFree(ds->bwd_ws);  // synchronises the device
+      ds->bwd_ws = nullptr;
+      ds->bwd_bytes = 0;
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFree(backward workspace)");
+    }
+    if ((e = cudaMalloc(&ds->bwd_ws, need)) != cudaSuccess) {
+      ds->bwd_ws = nullptr;
+      return cuda_fail(e, "cudaMalloc(backward workspace)");
+    }
+    ds->bwd_bytes = need;
+  }
+  char* base = static_cast<char*>(ds->bwd_ws);
+  unsigned* cntA = reinterpret_cast<unsigned*>(base);
+  unsigned* cntB = reinterpret_cast<unsigned*>(base + cnt_b);
+  float* hA = reinterpret_cast<float*>(base + 2 * cnt_b);
+  float* sA = reinterpret_cast<float*>(base + 2 * cnt_b + hA_b);
+  float* gB = reinterpret_cast<float*>(base + 2 * cnt_b + hA_b + sA_b);
+  float* qB = reinterpret_cast<float*>(base + 2 * cnt_b + hA_b + sA_b + g_b);
+  float* sB = reinterpret_cast<float*>(base + 2 * cnt_b + hA_b + sA_b + 2 * g_b);
+  if ((e = cudaMemsetAsync(base, 0, 2 * cnt_b, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(counters)");
+
+  // pass A: the forward chunk summaries and their fold give every chunk's start state
+  if (nseg > 1) {
+    mssm::ScanArgs a = call.a;
+    a.force_general = g_force_general;
+    a.tiles_per_batch = int(tpb);
+    a.seg_len = mssm::kBwdChunk;
+    a.nseg = int(nseg);
+    a.ws_H = hA;
+    a.ws_S = sA;
+    a.ws_count = cntA;
+    a.h0 = nullptr;
+    a.zoh = 0;
+    a.cu_seqlens = nullptr;
+    if ((e = mssm::device_error_word(&a.err)) != cudaSuccess) return cuda_fail(e, "device error word");
+    e = tracked(MSSM_KERNEL_SCAN_CHUNK_STATE, s,
+                [&] { return mssm::launch_scan_chunk_state(a, mssm::kBwdRows, dt, softplus_flag != 0, s); });
+    if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel launch (backward pass A)");
+  }
+  // passes B and C
+  mssm::BwdArgs b{};
+  b.u = u->data; b.delta = delta->data; b.z = z ? z->data : nullptr; b.dout = dout->data;
+  b.u_sb = u->stride[0]; b.u_sd = u->stride[1]; b.dl_sb = delta->stride[0]; b.dl_sd = delta->stride[1];
+  b.z_sb = z ? z->stride[0] : 0; b.z_sd = z ? z->stride[1] : 0;
+  b.g_sb = dout->stride[0]; b.g_sd = dout->stride[1];
+  b.B = B->data; b.C = C->data;
+  b.B_sb = B->stride[0]; b.B_sn = B->stride[1]; b.C_sb = C->stride[0]; b.C_sn = C->stride[1];
+  b.A = static_cast<const float*>(A->data); b.A_sd = A->stride[0]; b.A_sn = A->stride[1];
+  b.Dskip = D ? static_cast<const float*>(D->data) : nullptr; b.D_s = D ? D->stride[0] : 0;
+  b.bias = delta_bias ? static_cast<const float*>(delta_bias->data) : nullptr;
+  b.bias_s = delta_bias ? delta_bias->stride[0] : 0;
+  b.du = du->data; b.ddelta = ddelta->data; b.dz = dz ? dz->data : nullptr;
+  b.du_sb = du->stride[0]; b.du_sd = du->stride[1]; b.dd_sb = ddelta->stride[0]; b.dd_sd = ddelta->stride[1];
+  b.dz_sb = dz ? dz->stride[0] : 0; b.dz_sd = dz ? dz->stride[1] : 0;
+  b.dA = static_cast<float*>(dA->data); b.dB = static_cast<float*>(dB->data); b.dC = static_cast<float*>(dC->data);
+  b.dD = dD ? static_cast<float*>(dD->data) : nullptr;
+  b.dbias = ddelta_bias ? static_cast<float*>(ddelta_bias->data) : nullptr;
+  b.Bt = int(Bt); b.D = int(Dd); b.L = int(L);
+  b.softplus = softplus_flag != 0;
+  b.nseg = int(nseg); b.tiles_per_batch = int(tpb);
+  b.hstart = hA; b.ws_G = gB; b.ws_S = sB; b.ws_Q = qB; b.ws_count = cntB;
+  e = tracked(MSSM_KERNEL_SCAN_BWD, s, [&] { return mssm::launch_scan_bwd(b, dt, z != nullptr, s); });
+  if (e != cudaSuccess) return cuda_fail(e, "backward scan kernel launch");
+  return MSSM_OK;
+}
+
 mssm_status mssm_causal_conv1d_fwd(const mssm_tensor* x, const mssm_tensor* weight, const mssm_tensor* bias,
                                    const mssm_tensor* cu_seqlens, int64_t max_seqlen, int silu_flag,
                                    mssm_tensor* out, void* stream) {
@@ -955,12 +1102,21 @@ mssm_status mssm_shutdown(void) {
   int prev = -1;
   if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
   for (size_t i = 0; i < g_dev.size(); ++i) {
-    if (!g_dev[i].ws) continue;
+    if (!g_dev[i].ws && !g_dev[i].bwd_ws) continue;
     cudaSetDevice(int(i));
-    cudaError_t e = cudaFree(g_dev[i].ws);
-    if (e != cudaSuccess) st = cuda_fail(e, "cudaFree(workspace)");
+    if (g_dev[i].ws) {
+      cudaError_t e = cudaFree(g_dev[i].ws);
+      if (e != cudaSuccess) st = cuda_fail(e, "cudaFree(workspace)");
+    }
+    if (g_dev[i].bwd_ws) {
+      cudaError_t e = cudaFree(g_dev[i].bwd_ws);
+      if (e != cudaSuccess) st = cuda_fail(e, "cudaFree(backward workspace)");
+    }
     g_dev[i].ws = nullptr;
     g_dev[i].ws_bytes = 0;
+    g_dev[i].count_cap = 0;
+    g_dev[i].bwd_ws = nullptr;
+    g_dev[i].bwd_bytes = 0;
   }
   if (prev >= 0) cudaSetDevice(prev);
   return st;

@@ -1,0 +1,24 @@
+// Instantiation and launch of the backward scan kernels (passes B and C; pass A is the
+// forward chunk-summary kernel of scan.cu).
+#include "launch.h"
+
+namespace mssm {
+
+template <typename T, bool HAS_Z>
+static cudaError_t bwd_t(const BwdArgs& a, cudaStream_t s) {
+  const unsigned tiles = unsigned(a.Bt * a.tiles_per_batch);
+  if (a.nseg > 1) {
+    scan_bwd_summary_kernel<T, HAS_Z><<<dim3(tiles, a.nseg - 1), kBwdRows, 0, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  scan_bwd_kernel<T, HAS_Z><<<dim3(tiles, a.nseg), kBwdRows, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scan_bwd(const BwdArgs& a, int dtype, bool has_z, cudaStream_t s) {
+  if (dtype == 1) return has_z ? bwd_t<uint16_t, true>(a, s) : bwd_t<uint16_t, false>(a, s);
+  return has_z ? bwd_t<float, true>(a, s) : bwd_t<float, false>(a, s);
+}
+
+}  // namespace mssm

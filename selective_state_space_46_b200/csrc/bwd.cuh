@@ -1,0 +1,370 @@
+// Backward of the selective scan (Euler discretisation, zero initial state), sm_100a.
+//
+// The forward per row (b, d) and state n is h_t = a_t h_(t-1) + dt_t B_t u_t with
+// a_t = exp(dt_t A_n), y_t = C_t . h_t + D u_t, out_t = y_t silu(z_t).  Its reverse-mode
+// chain rule runs from the last step to the first with g = dLoss/dh_t:
+//   gy = dout silu(z);  g += gy C_t;  dC_t += gy h_t;  ddt += g (A a h_(t-1) + B_t u_t);
+//   dA += g dt a h_(t-1);  dB_t += g dt u;  du += g dt B_t (+ gy D);  g *= a.
+// The fused forward never stores the states, so the backward recomputes them
+// ("Mamba selective state space", the hardware-aware scan: intermediates are
+// recomputed in the backward pass instead of being written).
+//
+// Three chunk-parallel passes over chunks of kBwdChunk steps, one thread per row:
+//  A. the forward chunk summaries and their fold (scan_chunk_state_kernel) give
+//     every chunk's start state;
+//  B. scan_bwd_summary_kernel: every chunk but the first runs the g recurrence
+//     from a zero incoming gradient, giving G_c (what it sends to the chunk
+//     before) and S_c (its summed step); the last CTA of a row tile folds them
+//     backwards, Q_(c-1) = exp(A S_c) Q_c + G_c, into each chunk's incoming Q_c;
+//  C. scan_bwd_kernel: every chunk recomputes its states forward from its start
+//     state, in sub-chunks of kBwdSub steps kept in shared memory, and sweeps them
+//     backwards from Q_c, writing du, ddelta, dz and accumulating dA, dD, dbias
+//     (per row, then one atomic add per CTA) and dB, dC (a warp transpose-reduction
+//     over the 32 rows, then one atomic add per lane and step).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "device_common.cuh"
+
+namespace mssm {
+
+constexpr int kBwdChunk = 64;  // steps per chunk (the forward summaries' quantum)
+constexpr int kBwdSub = 16;    // steps per recomputed sub-chunk kept in shared memory
+constexpr int kBwdRows = 32;   // rows per CTA (one warp)
+
+struct BwdArgs {
+  const void* u;
+  const void* delta;
+  const void* z;
+  const void* dout;
+  int64_t u_sb, u_sd, dl_sb, dl_sd, z_sb, z_sd, g_sb, g_sd;  // L stride 1
+  const void* B;
+  const void* C;
+  int64_t B_sb, B_sn, C_sb, C_sn;  // L stride 1
+  const float* A;
+  int64_t A_sd, A_sn;
+  const float* Dskip;
+  int64_t D_s;
+  const float* bias;
+  int64_t bias_s;
+  void* du;
+  void* ddelta;
+  void* dz;
+  int64_t du_sb, du_sd, dd_sb, dd_sd, dz_sb, dz_sd;
+  float* dA;  // [D, N] contiguous, accumulated
+  float* dB;  // [Bt, N, L] contiguous, accumulated
+  float* dC;
+  float* dD;     // [D], accumulated, or null
+  float* dbias;  // [D], accumulated, or null
+  int Bt, D, L;
+  int softplus;
+  int nseg, tiles_per_batch;
+  const float* hstart;  // [nseg-1][rows][16]: start state of chunk k+1 at k (pass A)
+  float* ws_G;          // [nseg][rows][16]: pass B outgoing gradient of chunk c
+  float* ws_S;          // [nseg][rows]: pass B summed step of chunk c
+  float* ws_Q;          // [nseg][rows][16]: incoming gradient of chunk c (pass B fold)
+  unsigned* ws_count;   // [tiles]: pass B arrivals, reset by the folding CTA
+};
+
+template <typename T>
+__device__ __forceinline__ float bwd_ld(const void* base, int64_t off) {
+  return Elem<T>::load(static_cast<const T*>(base) + off);
+}
+template <typename T>
+__device__ __forceinline__ void bwd_st(void* base, int64_t off, float v) {
+  if constexpr (sizeof(T) == 2) {
+    static_cast<uint16_t*>(base)[off] = f_to_bf16(v);
+  } else {
+    static_cast<float*>(base)[off] = v;
+  }
+}
+
+// dt of one step: softplus(delta + bias) or delta + bias; also sigmoid(delta + bias), the
+// derivative of softplus (1 without softplus)
+__device__ __forceinline__ float bwd_dt(float raw, float bias, bool softplus, float& dsp) {
+  const float v = raw + bias;
+  if (!softplus) {
+    dsp = 1.0f;
+    return v;
+  }
+  const float e = ex2f(-v * kLog2e);
+  dsp = rcpf(1.0f + e);  // sigmoid(v)
+  return softplus_f(v);
+}
+
+// silu(z) and its derivative sigma(z) (1 + z (1 - sigma(z)))
+__device__ __forceinline__ void bwd_silu(float z, float& s, float& ds) {
+  const float sg = rcpf(1.0f + ex2f(-z * kLog2e));
+  s = z * sg;
+  ds = sg * fmaf(z, 1.0f - sg, 1.0f);
+}
+
+// Row constants: A (natural units, and times log2 e), skip, bias.
+struct BwdRow {
+  float A[kN], A2[kN];
+  float Dd, bias;
+};
+__device__ __forceinline__ void bwd_row(const BwdArgs& p, int d, BwdRow& r) {
+#pragma unroll
+  for (int n = 0; n < kN; ++n) {
+    r.A[n] = p.A[int64_t(d) * p.A_sd + int64_t(n) * p.A_sn];
+    r.A2[n] = r.A[n] * kLog2e;
+  }
+  r.Dd = p.Dskip ? p.Dskip[int64_t(d) * p.D_s] : 0.0f;
+  r.bias = p.bias ? p.bias[int64_t(d) * p.bias_s] : 0.0f;
+}
+
+// B and C of steps [t0, t0 + kBwdChunk) of batch b into shared memory, fp32 [t][32]
+// (B in 0..15, C in 16..31); zero past L.  Each of the 32 threads loads one row of B or C.
+template <typename T>
+__device__ __forceinline__ void bwd_stage_bc(const BwdArgs& p, int b, int t0, float (*bc)[32]) {
+  const int r = threadIdx.x;
+  const T* base = r < 16 ? static_cast<const T*>(p.B) + int64_t(b) * p.B_sb + int64_t(r) * p.B_sn
+                         : static_cast<const T*>(p.C) + int64_t(b) * p.C_sb + int64_t(r - 16) * p.C_sn;
+  for (int j = 0; j < kBwdChunk; ++j) {
+    const int t = t0 + j;
+    bc[j][r] = t < p.L ? Elem<T>::load(base + t) : 0.0f;
+  }
+}
+
+// Reduce 32 per-lane quantities v[0..31] over the warp: lane i returns the sum of v[i]
+// over all lanes (31 shuffles, the recursive-halving transpose).
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool upper = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      // keep the half this lane is responsible for, send the other half to lane ^ w
+      const float keep = upper ? v[i + w] : v[i];
+      const float send = upper ? v[i] : v[i + w];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  return v[0];
+}
+
+// ---------------------------------------------------------------------------
+// pass B: the g recurrence of chunk c >= 1 from a zero incoming gradient; fold
+// ---------------------------------------------------------------------------
+template <typename T, bool HAS_Z>
+__global__ void __launch_bounds__(kBwdRows) scan_bwd_summary_kernel(const BwdArgs p) {
+  __shared__ __align__(16) float bc_s[kBwdChunk][32];
+  __shared__ int s_last;
+  const int tid = threadIdx.x;
+  const int tile = blockIdx.x;
+  const int c = blockIdx.y + 1;
+  const int b = tile / p.tiles_per_batch;
+  const int d = (tile - b * p.tiles_per_batch) * kBwdRows + tid;
+  const int dc = d < p.D ? d : p.D - 1;
+  const int t0 = c * kBwdChunk;
+  const int t1 = min(p.L, t0 + kBwdChunk);
+  BwdRow r;
+  bwd_row(p, dc, r);
+  bwd_stage_bc<T>(p, b, t0, bc_s);
+  __syncthreads();
+
+  float g[kN];
+#pragma unroll
+  for (int n = 0; n < kN; ++n) g[n] = 0.0f;
+  float ssum = 0.0f;
+  const int64_t ro = int64_t(b) * p.dl_sb + int64_t(dc) * p.dl_sd;
+  const int64_t go = int64_t(b) * p.g_sb + int64_t(dc) * p.g_sd;
+  const int64_t zo = int64_t(b) * p.z_sb + int64_t(dc) * p.z_sd;
+  for (int t = t1 - 1; t >= t0; --t) {
+    float dsp;
+    const float dt = bwd_dt(bwd_ld<T>(p.delta, ro + t), r.bias, p.softplus, dsp);
+    float gy = bwd_ld<T>(p.dout, go + t);
+    if constexpr (HAS_Z) {
+      float s, ds;
+      bwd_silu(bwd_ld<T>(p.z, zo + t), s, ds);
+      gy *= s;
+    }
+    const float* cr = bc_s[t - t0] + 16;
+#pragma unroll
+    for (int n = 0; n < kN; ++n) g[n] = ex2f(dt * r.A2[n]) * fmaf(gy, cr[n], g[n]);
+    ssum += dt;
+  }
+  const int64_t rows_total = int64_t(p.Bt) * p.tiles_per_batch * kBwdRows;
+  const int64_t rowg = int64_t(tile) * kBwdRows + tid;
+  {
+    float4* dst = reinterpret_cast<float4*>(p.ws_G + (int64_t(c) * rows_total + rowg) * kN);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) __stcg(dst + i, make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]));
+    __stcg(p.ws_S + int64_t(c) * rows_total + rowg, ssum);
+  }
+  // the last CTA of the row tile folds backwards: Q_(nseg-1) = 0, Q_(c-1) = exp(A S_c) Q_c + G_c
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&p.ws_count[tile], 1u) == unsigned(p.nseg - 2));
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  float q[kN];
+#pragma unroll
+  for (int n = 0; n < kN; ++n) q[n] = 0.0f;
+  for (int k = p.nseg - 1; k >= 0; --k) {
+    float4* qd = reinterpret_cast<float4*>(p.ws_Q + (int64_t(k) * rows_total + rowg) * kN);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) __stcg(qd + i, make_float4(q[4 * i], q[4 * i + 1], q[4 * i + 2], q[4 * i + 3]));
+    if (k == 0) break;
+    const float sk = __ldcg(p.ws_S + int64_t(k) * rows_total + rowg);
+    const float4* gs = reinterpret_cast<const float4*>(p.ws_G + (int64_t(k) * rows_total + rowg) * kN);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 gv = __ldcg(gs + i);
+      q[4 * i] = fmaf(ex2f(sk * r.A2[4 * i]), q[4 * i], gv.x);
+      q[4 * i + 1] = fmaf(ex2f(sk * r.A2[4 * i + 1]), q[4 * i + 1], gv.y);
+      q[4 * i + 2] = fmaf(ex2f(sk * r.A2[4 * i + 2]), q[4 * i + 2], gv.z);
+      q[4 * i + 3] = fmaf(ex2f(sk * r.A2[4 * i + 3]), q[4 * i + 3], gv.w);
+    }
+  }
+  if (tid == 0) p.ws_count[tile] = 0u;
+}
+
+// ---------------------------------------------------------------------------
+// pass C: recompute the chunk's states and sweep them backwards
+// ---------------------------------------------------------------------------
+template <typename T, bool HAS_Z>
+__global__ void __launch_bounds__(kBwdRows) scan_bwd_kernel(const BwdArgs p) {
+  __shared__ __align__(16) float bc_s[kBwdChunk][32];
+  __shared__ __align__(16) float hsub[kBwdChunk / kBwdSub][kN][kBwdRows];  // sub-chunk start states
+  __shared__ __align__(16) float hbuf[kBwdSub][kN][kBwdRows];              // states of one sub-chunk
+  const int tid = threadIdx.x;
+  const int tile = blockIdx.x;
+  const int c = blockIdx.y;
+  const int b = tile / p.tiles_per_batch;
+  const int d = (tile - b * p.tiles_per_batch) * kBwdRows + tid;
+  const bool row_ok = d < p.D;
+  const int dc = row_ok ? d : p.D - 1;
+  const int t0 = c * kBwdChunk;
+  const int t1 = min(p.L, t0 + kBwdChunk);
+  const int64_t rows_total = int64_t(p.Bt) * p.tiles_per_batch * kBwdRows;
+  const int64_t rowg = int64_t(tile) * kBwdRows + tid;
+  BwdRow r;
+  bwd_row(p, dc, r);
+  bwd_stage_bc<T>(p, b, t0, bc_s);
+  __syncthreads();
+
+  const int64_t uo = int64_t(b) * p.u_sb + int64_t(dc) * p.u_sd;
+  const int64_t ro = int64_t(b) * p.dl_sb + int64_t(dc) * p.dl_sd;
+  const int64_t go = int64_t(b) * p.g_sb + int64_t(dc) * p.g_sd;
+  const int64_t zo = int64_t(b) * p.z_sb + int64_t(dc) * p.z_sd;
+
+  // forward from the chunk's start state, keeping the start state of every sub-chunk
+  float h[kN];
+  if (c == 0) {
+#pragma unroll
+    for (int n = 0; n < kN; ++n) h[n] = 0.0f;
+  } else {
+    const float4* src = reinterpret_cast<const float4*>(p.hstart + (int64_t(c - 1) * rows_total + rowg) * kN);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = __ldcg(src + i);
+      h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
+    }
+  }
+  auto step_fwd = [&](int t) {
+    float dsp;
+    const float dt = bwd_dt(bwd_ld<T>(p.delta, ro + t), r.bias, p.softplus, dsp);
+    const float w = dt * bwd_ld<T>(p.u, uo + t);
+    const float* br = bc_s[t - t0];
+#pragma unroll
+    for (int n = 0; n < kN; ++n) h[n] = fmaf(ex2f(dt * r.A2[n]), h[n], w * br[n]);
+  };
+  const int nsub = (t1 - t0 + kBwdSub - 1) / kBwdSub;
+  for (int k = 0; k < nsub; ++k) {
+#pragma unroll
+    for (int n = 0; n < kN; ++n) hsub[k][n][tid] = h[n];
+    if (k + 1 < nsub)
+      for (int t = t0 + k * kBwdSub; t < t0 + (k + 1) * kBwdSub; ++t) step_fwd(t);
+  }
+
+  // backward from the incoming gradient
+  float g[kN], dA[kN];
+  {
+    const float4* src = reinterpret_cast<const float4*>(p.ws_Q + (int64_t(c) * rows_total + rowg) * kN);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = c + 1 < p.nseg ? __ldcg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      g[4 * i] = v.x; g[4 * i + 1] = v.y; g[4 * i + 2] = v.z; g[4 * i + 3] = v.w;
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < kN; ++n) dA[n] = 0.0f;
+  float dDacc = 0.0f, dbacc = 0.0f;
+  for (int k = nsub - 1; k >= 0; --k) {
+    const int ts = t0 + k * kBwdSub;
+    const int te = min(t1, ts + kBwdSub);
+    // recompute this sub-chunk's states into hbuf
+#pragma unroll
+    for (int n = 0; n < kN; ++n) h[n] = hsub[k][n][tid];
+    for (int t = ts; t < te; ++t) {
+      step_fwd(t);
+#pragma unroll
+      for (int n = 0; n < kN; ++n) hbuf[t - ts][n][tid] = h[n];
+    }
+    // sweep it backwards
+    for (int t = te - 1; t >= ts; --t) {
+      float dsp;
+      const float raw = bwd_ld<T>(p.delta, ro + t);
+      const float dt = bwd_dt(raw, r.bias, p.softplus, dsp);
+      const float uu = bwd_ld<T>(p.u, uo + t);
+      const float gout = bwd_ld<T>(p.dout, go + t);
+      float gy = gout;
+      float yv = 0.0f;
+      const float* br = bc_s[t - t0];
+      const float* cr = br + 16;
+      float red[32];  // dB (0..15) and dC (16..31) partials of this row
+#pragma unroll
+      for (int n = 0; n < kN; ++n) yv = fmaf(cr[n], hbuf[t - ts][n][tid], yv);
+      yv = fmaf(r.Dd, uu, yv);
+      if constexpr (HAS_Z) {
+        float s, ds;
+        const float zz = bwd_ld<T>(p.z, zo + t);
+        bwd_silu(zz, s, ds);
+        if (row_ok) bwd_st<T>(p.dz, int64_t(b) * p.dz_sb + int64_t(d) * p.dz_sd + t, gout * yv * ds);
+        gy = gout * s;
+      }
+      float du = gy * r.Dd;
+      dDacc = fmaf(gy, uu, dDacc);
+      float ddt = 0.0f;
+#pragma unroll
+      for (int n = 0; n < kN; ++n) {
+        const float ht = hbuf[t - ts][n][tid];
+        const float hp = t > ts ? hbuf[t - ts - 1][n][tid] : hsub[k][n][tid];
+        g[n] = fmaf(gy, cr[n], g[n]);
+        red[16 + n] = row_ok ? gy * ht : 0.0f;
+        const float a = ex2f(dt * r.A2[n]);
+        const float gah = g[n] * a * hp;
+        ddt = fmaf(g[n], br[n] * uu, fmaf(r.A[n], gah, ddt));
+        dA[n] = fmaf(gah, dt, dA[n]);
+        red[n] = row_ok ? g[n] * dt * uu : 0.0f;
+        du = fmaf(g[n] * dt, br[n], du);
+        g[n] *= a;
+      }
+      const float draw = ddt * dsp;
+      dbacc += draw;
+      if (row_ok) {
+        bwd_st<T>(p.du, int64_t(b) * p.du_sb + int64_t(d) * p.du_sd + t, du);
+        bwd_st<T>(p.ddelta, int64_t(b) * p.dd_sb + int64_t(d) * p.dd_sd + t, draw);
+      }
+      const float tot = warp_transpose_sum(red);
+      // lane i holds dB (i < 16) or dC (i >= 16) of state i % 16 summed over the 32 rows
+      float* dst = tid < 16 ? p.dB + (int64_t(b) * kN + tid) * p.L + t
+                            : p.dC + (int64_t(b) * kN + (tid - 16)) * p.L + t;
+      atomicAdd(dst, tot);
+    }
+  }
+  if (row_ok) {
+#pragma unroll
+    for (int n = 0; n < kN; ++n) atomicAdd(p.dA + int64_t(d) * kN + n, dA[n]);
+    if (p.dD) atomicAdd(p.dD + d, dDacc);
+    if (p.dbias) atomicAdd(p.dbias + d, dbacc);
+  }
+}
+
+}  // namespace mssm

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 
+#include "bwd.cuh"
 #include "conv.cuh"
 #include "decode.cuh"
 #include "scan.cuh"
@@ -23,6 +24,9 @@ cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, Deco
 // Causal conv1d + SiLU: grid (ceil(rows / kConvWarps), items); one decode step of it.
 cudaError_t launch_causal_conv1d(const ConvArgs& a, int items, int dtype, bool silu, cudaStream_t s);
 cudaError_t launch_causal_conv1d_update(const ConvUpdateArgs& a, int dtype, cudaStream_t s);
+// Backward scan, passes B and C (pass A: launch_scan_chunk_state with 32-row tiles and
+// chunks of kBwdChunk steps, into the same workspace rows).
+cudaError_t launch_scan_bwd(const BwdArgs& a, int dtype, bool has_z, cudaStream_t s);
 // Reads (and optionally clears) the current device's error word.
 cudaError_t read_device_error(unsigned int* value, bool clear);
 
