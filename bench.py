@@ -406,6 +406,7 @@ def run_mssm(args):
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, args.chunk_len)
     m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 1 if args.general_a else 0)
     m.mssm_set_option(m.MSSM_OPT_DECODE_PATH, m.DECODE_PATHS.get(args.decode_path, 0))
+    m.mssm_set_option(m.MSSM_OPT_SCHEDULE, m.SCHEDULES.get(args.schedule, 0))
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -766,6 +767,8 @@ def main(argv=None):
     ap.add_argument("--decode-path", choices=["auto", "stream", "bulk_tile", "per_row"], default="auto",
                     help="decode kernel (MSSM_OPT_DECODE_PATH)")
     ap.add_argument("--zoh", action="store_true", help="zero-order-hold discretisation (scan workloads)")
+    ap.add_argument("--schedule", choices=["auto", "forward", "summaries+forward", "chained", "fused"],
+                    default="auto", help="force a scan schedule (MSSM_OPT_SCHEDULE)")
     ap.add_argument("--backward", action="store_true", help="time the backward scan instead (scan workloads)")
     ap.add_argument("--general-a", action="store_true",
                     help="disable the structured-A path (one exponential per state)")

@@ -324,10 +324,11 @@ mssm_status mssm_get_error(void *stream);
  *   MSSM_OPT_CHUNK_LEN (value 0, or a positive multiple of 64): length of the
  *     chunks a sequence is split into (a value >= L means no split); 0 restores
  *     the automatic choice.
- *   MSSM_OPT_SCHEDULE (value 0..3): 0 automatic; otherwise force a schedule of
+ *   MSSM_OPT_SCHEDULE (value 0..4): 0 automatic; otherwise force a schedule of
  *     mssm_scan_plan (value = schedule + 1: 1 forward only, no split; 2 summaries
- *     + forward; 3 chained).  A forced split schedule needs L > 64; otherwise the
- *     plan falls back to forward only.
+ *     + forward; 3 chained; 4 fused single pass).  A forced split schedule needs
+ *     L > 64; otherwise the plan falls back to forward only.  The fused schedule
+ *     takes plain batches only (packed sequences fall back to the automatic plan).
  *   MSSM_OPT_KERNEL_TIMING (value 0/1): when 1, every kernel launch is bracketed
  *     by two CUDA events recorded on the caller's stream (see mssm_kernel_stats).
  *   MSSM_OPT_DECODE_PATH (value 0..3): the state-update kernel.  0 automatic:
@@ -363,7 +364,9 @@ mssm_status mssm_set_option(int option, int64_t value);
  * number of chunks (1 = no split) and schedule: 0 = one forward kernel,
  * 1 = chunk-summary kernel + forward kernel, 2 = persistent chained forward
  * kernel (chunks of a tile run in order, each starting from the state the
- * previous one published).  Honours MSSM_OPT_CHUNK_LEN.  Launches nothing; any
+ * previous one published), 3 = fused single pass (one persistent kernel: every
+ * chunk summarises itself, looks back over the published summaries of the
+ * chunks before it for its start state, then runs forward).  Honours MSSM_OPT_CHUNK_LEN.  Launches nothing; any
  * output pointer may be NULL.
  */
 mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int *rows_per_cta,

@@ -42,7 +42,7 @@ MSSM_OPT_FORCE_GENERAL_A, MSSM_OPT_CHUNK_LEN, MSSM_OPT_KERNEL_TIMING, MSSM_OPT_S
 MSSM_OPT_DECODE_PATH = 5
 MSSM_OPT_TEST_HOOKS = 6
 MSSM_DISC_EULER, MSSM_DISC_ZOH = 0, 1
-SCHEDULES = {"forward": 1, "summaries+forward": 2, "chained": 3}
+SCHEDULES = {"forward": 1, "summaries+forward": 2, "chained": 3, "fused": 4}
 DECODE_PATHS = {"stream": 1, "bulk_tile": 2, "per_row": 3}
 KERNEL_KINDS = ("scan_chunk_state", "scan_out", "state_update", "conv", "scan_bwd")
 
@@ -178,7 +178,7 @@ def mssm_scan_plan(Bt: int, D: int, L: int, sm_count: int = 0, total_len: int = 
     _check(_lib.mssm_scan_plan_packed(Bt, D, L, total_len, sm_count, ctypes.byref(rows), ctypes.byref(seg),
                                       ctypes.byref(nseg), ctypes.byref(sched)))
     return {"rows_per_cta": rows.value, "chunk_len": seg.value, "n_chunks": nseg.value,
-            "schedule": ("forward", "summaries+forward", "chained")[sched.value]}
+            "schedule": ("forward", "summaries+forward", "chained", "fused")[sched.value]}
 
 
 def mssm_get_error(stream=None) -> None:

@@ -216,6 +216,10 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
       if (nseg > 1)
         cost += grid_time(sum_items, rows, double(seg), packed ? kSumFwd : kSum) + kFold * double(nseg);
       consider(LaunchShape{nseg > 1 ? 1 : 0, rows, seg, nseg, 0}, cost);
+      // fused single pass (forced only, until measured): 32-row tiles, persistent one-warp CTAs
+      if (rows == 32 && nseg > 1 && forced_mode == 3 && !packed) {
+        consider(LaunchShape{3, 32, seg, nseg, int(std::min<int64_t>(tiles * nseg, 8 * int64_t(sms)))}, 0.0);
+      }
       // chained: 32-row tiles, at most 8 one-warp CTAs per SM and never more CTAs than tiles
       if (rows == 32 && nseg > 1 && forced_mode == 2 && tiles < 4 * int64_t(sms)) {
         consider(LaunchShape{2, 32, seg, nseg, int(std::min<int64_t>(tiles, 8 * int64_t(sms)))}, 0.0);
@@ -269,7 +273,7 @@ mssm_status mssm_set_option(int option, int64_t value) {
       g_chunk_len = value;
       return MSSM_OK;
     case MSSM_OPT_SCHEDULE:
-      if (value < 0 || value > 3) return fail(MSSM_ERR_INVALID_ARG, "SCHEDULE takes 0 (automatic) to 3");
+      if (value < 0 || value > 4) return fail(MSSM_ERR_INVALID_ARG, "SCHEDULE takes 0 (automatic) to 4");
       g_schedule = int(value) - 1;
       return MSSM_OK;
     case MSSM_OPT_TEST_HOOKS:
@@ -466,6 +470,11 @@ ScanPlan scan_plan(ScanCall& call, int sm_count) {
   } else if (shape.mode == 2) {
     plan.count_bytes = ((size_t(tiles + 1) * 4 + 255) / 256) * 256;
     plan.h_bytes = size_t(tiles) * 32 * mssm::kN * 4;
+  } else if (shape.mode == 3) {
+    const size_t recs = size_t(tiles) * size_t(shape.nseg);
+    plan.count_bytes = ((size_t(recs + 1) * 4 + 255) / 256) * 256;
+    plan.s_bytes = ((recs * 32 * 4 + 255) / 256) * 256;
+    plan.h_bytes = 2 * recs * 32 * mssm::kN * 4;  // summaries and end states
   }
   return plan;
 }
@@ -476,6 +485,14 @@ void scan_bind_workspace(mssm::ScanArgs& a, const ScanPlan& plan, void* ws) {
     a.ch_ticket = reinterpret_cast<unsigned*>(base);
     a.ch_flags = reinterpret_cast<unsigned*>(base) + 1;
     a.ch_carry = reinterpret_cast<float*>(base + plan.count_bytes);
+    return;
+  }
+  if (plan.mode == 3) {
+    a.ch_ticket = reinterpret_cast<unsigned*>(base);
+    a.lb_flags = reinterpret_cast<unsigned*>(base) + 1;
+    a.lb_S = reinterpret_cast<float*>(base + plan.count_bytes);
+    a.lb_H = reinterpret_cast<float*>(base + plan.count_bytes + plan.s_bytes);
+    a.lb_I = a.lb_H + plan.h_bytes / 8;
     return;
   }
 
@@ -489,6 +506,15 @@ void scan_bind_workspace(mssm::ScanArgs& a, const ScanPlan& plan, void* ws) {
 mssm_status scan_launch(ScanCall& call, const ScanPlan& plan, void* ws, cudaStream_t s) {
   cudaError_t e = mssm::device_error_word(&call.a.err);
   if (e != cudaSuccess) return cuda_fail(e, "device error word");
+  if (plan.mode == 3) {
+    e = cudaMemsetAsync(ws, 0, plan.count_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(fused schedule flags)");
+    e = tracked(MSSM_KERNEL_SCAN_OUT, s, [&] {
+      return mssm::launch_scan_fused(call.a, plan.grid, call.dtype, call.has_z, call.softplus, s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "fused scan kernel launch");
+    return MSSM_OK;
+  }
   if (plan.mode == 2) {
     e = cudaMemsetAsync(ws, 0, plan.count_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(chained schedule flags)");
@@ -521,7 +547,7 @@ mssm_status scan_fwd_impl(ScanCall& call, void* stream) {
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceState* ds = device_state(dev);
   const ScanPlan plan = scan_plan(call, ds->sm_count);
-  if (plan.mode == 2) {
+  if (plan.mode == 2 || plan.mode == 3) {
     // ticket, flags and carried states: zeroed by scan_launch where they must be
     const size_t need = plan.need() + size_t(ds->count_cap) * 4;
     if (ds->ws_bytes < need) {

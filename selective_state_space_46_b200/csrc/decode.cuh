@@ -222,9 +222,9 @@ __global__ void __launch_bounds__(kDecodeThreads) state_update_bulk_kernel(const
 // C with unit n stride and 16-byte-aligned batch rows (the host checks all).
 // ---------------------------------------------------------------------------
 constexpr int kStreamRows = 128;      // channels per CTA, one thread each
-constexpr int kStreamBufs = 4;        // ring slots per CTA
+constexpr int kStreamBufs = 8;        // ring slots per CTA (swept: 3..8 slots x 3..6 CTAs; 8 x 3 best)
 constexpr int kStreamAhead = kStreamBufs - 1;
-constexpr int kStreamCtasPerSm = 5;   // 5 x (4 x <= 9.9 KB) shared memory, 640 threads
+constexpr int kStreamCtasPerSm = 3;   // 3 x (8 x <= 9.9 KB) shared memory, 384 threads
 
 template <typename T>
 struct StreamSlot {

@@ -16,6 +16,8 @@ cudaError_t launch_scan_chunk_state(const ScanArgs& a, int rows, int dtype, bool
 cudaError_t launch_scan_out(const ScanArgs& a, int rows, int dtype, bool has_z, bool softplus, cudaStream_t s);
 // Persistent chained forward kernel (32-row tiles), `grid` one-warp CTAs.
 cudaError_t launch_scan_chained(const ScanArgs& a, int grid, int dtype, bool has_z, bool softplus, cudaStream_t s);
+// Fused single-pass (look-back) kernel, `grid` persistent one-warp CTAs.
+cudaError_t launch_scan_fused(const ScanArgs& a, int grid, int dtype, bool has_z, bool softplus, cudaStream_t s);
 // Device address of this device's error word (cached per device).
 cudaError_t device_error_word(unsigned int** out);
 // bulk: the state is one contiguous [rows][16] range (bulk-copy kernel), else one thread per row.

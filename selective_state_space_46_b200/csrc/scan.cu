@@ -9,6 +9,11 @@ cudaError_t launch_scan_chained(const ScanArgs& a, int grid, int dtype, bool has
   return ScanDispatch<false>::chained(a, grid, dtype, has_z, sp, s);
 }
 
+cudaError_t launch_scan_fused(const ScanArgs& a, int grid, int dtype, bool has_z, bool sp, cudaStream_t s) {
+  if (a.zoh) return launch_scan_fused_zoh(a, grid, dtype, has_z, sp, s);
+  return ScanDispatch<false>::fused(a, grid, dtype, has_z, sp, s);
+}
+
 cudaError_t launch_scan_chunk_state(const ScanArgs& a, int rows, int dtype, bool sp, cudaStream_t s) {
   if (a.zoh) return launch_scan_chunk_state_zoh(a, rows, dtype, sp, s);
   return ScanDispatch<false>::chunk_state(a, rows, dtype, sp, s);

@@ -83,6 +83,12 @@ struct ScanArgs {
   unsigned* ch_ticket;   // work-item counter
   unsigned* ch_flags;    // [tiles]: chunks of the tile whose carried state is published
   float* ch_carry;       // [tiles * 32][16]: carried state between consecutive chunks
+  // fused schedule (scan_fused_kernel): per (tile, chunk) flags (zeroed before each launch),
+  // summaries and end states; the ticket is ch_ticket
+  unsigned* lb_flags;    // [tiles][nseg]: 1 = summary published, 2 = end state published
+  float* lb_S;           // [tiles][nseg][32]
+  float* lb_H;           // [tiles][nseg][32][16]
+  float* lb_I;           // [tiles][nseg][32][16]
   unsigned* err;         // device error word: bit 1 = a chained wait gave up
   int test_no_publish;   // test hook: the chained kernel publishes no carried states
   // packed variable-length sequences: Bt is the sequence count, the data has one batch row,
@@ -1013,5 +1019,199 @@ __global__ void __launch_bounds__(ROWS, 512 / ROWS) scan_chunk_state_kernel(cons
 }
 
 
+
+}  // namespace mssm
+
+namespace mssm {
+
+// ---------------------------------------------------------------------------
+// Fused single-pass schedule: chunk summaries, carries and the forward sweep in
+// one persistent kernel (a decoupled look-back over the chunks of a row tile).
+//
+// Work items (tile, chunk) are taken in chunk-major order from an atomic ticket.
+// An item of chunk c first summarises its chunk (S_c, H_c) -- unless it is the
+// last chunk, whose summary nobody reads -- and publishes it (flag 1), then looks
+// back over chunks c-1, c-2, ... composing their published summaries until it
+// meets a published end state (flag 2), which gives its start state; it then
+// publishes its own end state (flag 2) and runs the forward sweep.  Chunk 0's
+// end state follows from its summary and h0 without looking back.  Every wait is
+// on an item taken earlier, whose own waits are on items earlier still, so the
+// waits always end; each is bounded anyway (kChainSpinLimit polls): if one gives
+// up, the item records bit 1 of the device error word and treats the missing
+// prefix as a zero state.  Records: flags [tiles][nseg], S [tiles][nseg][32],
+// H and end states [tiles][nseg][32][16].
+// ---------------------------------------------------------------------------
+template <bool STRUCT>
+__device__ __forceinline__ void lb_decay(float S, const RowParams& rp, f2_t (&e)[8]) {
+  // 2^(S A_n): the chunk's decay over summed base-2 step S
+  const f2_t S2 = f2(S, S);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float lo, hi;
+    f2split(mul2(S2, rp.Ap[k]), lo, hi);
+    e[k] = f2(ex2f(lo), ex2f(hi));
+  }
+}
+
+template <typename T, bool HAS_Z, bool SOFTPLUS, bool ZOH>
+__global__ void __launch_bounds__(32, 8) scan_fused_kernel(const ScanArgs p) {
+  constexpr int ROWS = 32;
+  __shared__ __align__(16) float bc_s[2][kTC * 32];
+  __shared__ __align__(16) uint4 slots[kStages * 3 * ROWS];
+  __shared__ int s_item;
+  __shared__ unsigned s_flag;
+  const int tid = threadIdx.x;
+  const int ntiles = p.Bt * p.tiles_per_batch;
+  const int nitems = ntiles * p.nseg;
+  for (;;) {
+    if (tid == 0) s_item = int(atomicAdd(p.ch_ticket, 1u));
+    __syncthreads();
+    const int item = s_item;
+    if (item >= nitems) break;
+    const int c = item / ntiles;
+    const int tile = item - c * ntiles;
+    const int b = tile / p.tiles_per_batch;
+    const int d = (tile - b * p.tiles_per_batch) * ROWS + tid;
+    const bool row_ok = d < p.D;
+    const int dc = row_ok ? d : p.D - 1;
+    const int t0 = c * p.seg_len;
+    const int t1 = min(p.L, t0 + p.seg_len);
+    const T* urow = static_cast<const T*>(p.u) + int64_t(b) * p.u_sb + int64_t(dc) * p.u_sd;
+    const T* dlrow = static_cast<const T*>(p.delta) + int64_t(b) * p.dl_sb + int64_t(dc) * p.dl_sd;
+    const T* zrow = HAS_Z ? static_cast<const T*>(p.z) + int64_t(b) * p.z_sb + int64_t(dc) * p.z_sd : nullptr;
+    T* orow = static_cast<T*>(p.out) + int64_t(b) * p.o_sb + int64_t(dc) * p.o_sd;
+    RowParams rp;
+    const bool st = load_row_params<ROWS>(p, dc, rp);
+    const bool structured = __syncthreads_and(st) && !p.force_general;
+    const int64_t recbase = int64_t(tile) * p.nseg;  // record of chunk k: (recbase + k) * ROWS + tid
+    const bool publish = !p.test_no_publish;
+
+    auto store16 = [&](float* dst, const f2_t (&v)[8]) {
+      float4* q = reinterpret_cast<float4*>(dst);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float a0, a1, a2, a3;
+        f2split(v[2 * i], a0, a1);
+        f2split(v[2 * i + 1], a2, a3);
+        __stcg(q + i, make_float4(a0, a1, a2, a3));
+      }
+    };
+    auto load16 = [&](const float* src, f2_t (&v)[8]) {
+      const float4* q = reinterpret_cast<const float4*>(src);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 x = __ldcg(q + i);
+        v[2 * i] = f2(x.x, x.y);
+        v[2 * i + 1] = f2(x.z, x.w);
+      }
+    };
+    auto release = [&](int k, unsigned flag) {  // records of chunk k written by every thread
+      __threadfence();
+      __syncthreads();
+      if (tid == 0 && publish) st_release_u32(p.lb_flags + recbase + k, flag);
+    };
+
+    // 1. this chunk's summary (not for the last chunk: nobody reads it)
+    f2_t H[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) H[k] = 0ull;
+    float S = 0.0f;
+    const bool last = c == p.nseg - 1;
+    if (!last) {
+      if constexpr (ZOH) {
+        if (structured)
+          forward_chunk<T, ROWS, false, SOFTPLUS, true, true, false>(p, bc_s, slots, b, t0, t1, urow, dlrow,
+                                                                     nullptr, nullptr, false, rp, H, &S);
+        else
+          forward_chunk<T, ROWS, false, SOFTPLUS, false, true, false>(p, bc_s, slots, b, t0, t1, urow, dlrow,
+                                                                      nullptr, nullptr, false, rp, H, &S);
+      } else {
+        if (structured)
+          backward_chunk<T, ROWS, SOFTPLUS, true>(p, bc_s, slots, b, t0, t1, urow, dlrow, rp, H, S);
+        else
+          backward_chunk<T, ROWS, SOFTPLUS, false>(p, bc_s, slots, b, t0, t1, urow, dlrow, rp, H, S);
+      }
+    }
+    const int64_t myrec = (recbase + c) * ROWS + tid;
+    f2_t carry[8];
+    if (c == 0) {
+      load_h0(p, b, dc, carry);
+    } else {
+      if (!last) {
+        store16(p.lb_H + myrec * kN, H);
+        __stcg(p.lb_S + myrec, S);
+        release(c, 1u);
+      }
+      // 2. look back: compose the published summaries of chunks c-1, c-2, ... (later ones
+      // first) until a published end state; (Sacc, Hacc) is the map of the chunks in between
+      f2_t Hacc[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) Hacc[k] = 0ull;
+      float Sacc = 0.0f;
+      bool found = false;
+      for (int k = c - 1; k >= 0; --k) {
+        if (tid == 0) {
+          unsigned v = ld_acquire_u32(p.lb_flags + recbase + k);
+          for (int it = 0; v == 0u && it < kChainSpinLimit; ++it) {
+            __nanosleep(64);
+            v = ld_acquire_u32(p.lb_flags + recbase + k);
+          }
+          if (v == 0u) atomicOr(p.err, 2u);
+          s_flag = v;
+        }
+        __syncthreads();
+        const unsigned f = s_flag;
+        __syncthreads();
+        if (f == 0u) break;  // gave up: the prefix before chunk k is taken as zero
+        const int64_t rk = (recbase + k) * ROWS + tid;
+        f2_t e[8];
+        lb_decay<true>(Sacc, rp, e);
+        f2_t v[8];
+        if (f >= 2u) {
+          load16(p.lb_I + rk * kN, v);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) Hacc[q] = fma2(e[q], v[q], Hacc[q]);
+          found = true;
+          break;
+        }
+        load16(p.lb_H + rk * kN, v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) Hacc[q] = fma2(e[q], v[q], Hacc[q]);
+        Sacc += __ldcg(p.lb_S + rk);
+      }
+      (void)found;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) carry[q] = Hacc[q];
+    }
+    // this chunk's end state for the chunks after it: 2^(A S) carry + H
+    if (!last) {
+      f2_t e[8], I[8];
+      lb_decay<true>(S, rp, e);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) I[q] = fma2(e[q], carry[q], H[q]);
+      store16(p.lb_I + myrec * kN, I);
+      release(c, 2u);
+    }
+
+    // 3. the forward sweep from the carried state
+    forward_any<T, ROWS, HAS_Z, SOFTPLUS, ZOH>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow, row_ok, rp,
+                                               structured, carry);
+    if (last && row_ok && p.last_state) {
+      float* dst = p.last_state + int64_t(b) * p.ls_sb + int64_t(d) * p.ls_sd;
+      float v[16];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) f2split(carry[k], v[2 * k], v[2 * k + 1]);
+      if (p.vec_ls) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      } else {
+#pragma unroll
+        for (int n = 0; n < 16; ++n) dst[n] = v[n];
+      }
+    }
+    __syncthreads();
+  }
+}
 
 }  // namespace mssm

@@ -35,6 +35,19 @@ struct ScanDispatch {
     scan_out_chained_kernel<T, HAS_Z, SP, ZOH><<<grid, 32, 0, s>>>(a);
     return cudaGetLastError();
   }
+  template <typename T, bool HAS_Z, bool SP>
+  static cudaError_t fused_t(const ScanArgs& a, int grid, cudaStream_t s) {
+    scan_fused_kernel<T, HAS_Z, SP, ZOH><<<grid, 32, 0, s>>>(a);
+    return cudaGetLastError();
+  }
+  template <typename T>
+  static cudaError_t fused_d(const ScanArgs& a, int grid, bool has_z, bool sp, cudaStream_t s) {
+    if (has_z) return sp ? fused_t<T, true, true>(a, grid, s) : fused_t<T, true, false>(a, grid, s);
+    return sp ? fused_t<T, false, true>(a, grid, s) : fused_t<T, false, false>(a, grid, s);
+  }
+  static cudaError_t fused(const ScanArgs& a, int grid, int dtype, bool has_z, bool sp, cudaStream_t s) {
+    return dtype == 1 ? fused_d<uint16_t>(a, grid, has_z, sp, s) : fused_d<float>(a, grid, has_z, sp, s);
+  }
   template <typename T>
   static cudaError_t chained_d(const ScanArgs& a, int grid, bool has_z, bool sp, cudaStream_t s) {
     if (has_z) return sp ? chained_t<T, true, true>(a, grid, s) : chained_t<T, true, false>(a, grid, s);
@@ -66,5 +79,6 @@ struct ScanDispatch {
 cudaError_t launch_scan_chunk_state_zoh(const ScanArgs& a, int rows, int dtype, bool sp, cudaStream_t s);
 cudaError_t launch_scan_out_zoh(const ScanArgs& a, int rows, int dtype, bool has_z, bool sp, cudaStream_t s);
 cudaError_t launch_scan_chained_zoh(const ScanArgs& a, int grid, int dtype, bool has_z, bool sp, cudaStream_t s);
+cudaError_t launch_scan_fused_zoh(const ScanArgs& a, int grid, int dtype, bool has_z, bool sp, cudaStream_t s);
 
 }  // namespace mssm

@@ -7,6 +7,10 @@ cudaError_t launch_scan_chained_zoh(const ScanArgs& a, int grid, int dtype, bool
   return ScanDispatch<true>::chained(a, grid, dtype, has_z, sp, s);
 }
 
+cudaError_t launch_scan_fused_zoh(const ScanArgs& a, int grid, int dtype, bool has_z, bool sp, cudaStream_t s) {
+  return ScanDispatch<true>::fused(a, grid, dtype, has_z, sp, s);
+}
+
 cudaError_t launch_scan_chunk_state_zoh(const ScanArgs& a, int rows, int dtype, bool sp, cudaStream_t s) {
   return ScanDispatch<true>::chunk_state(a, rows, dtype, sp, s);
 }

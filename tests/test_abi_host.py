@@ -259,8 +259,8 @@ def test_options_and_strings(lib):
     assert lib.mssm_set_option(1, 2) == INVALID
     assert lib.mssm_set_option(2, 100) == INVALID      # not a multiple of 64
     assert lib.mssm_set_option(99, 0) == INVALID
-    assert lib.mssm_set_option(4, 4) == INVALID
-    assert lib.mssm_set_option(4, 3) == 0 and lib.mssm_set_option(4, 0) == 0
+    assert lib.mssm_set_option(4, 5) == INVALID
+    assert lib.mssm_set_option(4, 4) == 0 and lib.mssm_set_option(4, 3) == 0 and lib.mssm_set_option(4, 0) == 0
     assert lib.mssm_set_option(5, 4) == INVALID and lib.mssm_set_option(5, -1) == INVALID
     for v in (1, 2, 3, 0):
         assert lib.mssm_set_option(5, v) == 0
@@ -304,7 +304,7 @@ def test_scan_plan_host_only(lib):
     assert lib.mssm_set_option(2, 0) == 0
     assert f(-1, 64, 1000, 148, None, None, None, None) == INVALID
     # every schedule can be forced (forward-only never splits)
-    for value, mode in ((1, 0), (2, 1), (3, 2)):
+    for value, mode in ((1, 0), (2, 1), (3, 2), (4, 3)):
         assert lib.mssm_set_option(4, value) == 0
         assert f(2, 1536, 2048, 148, ctypes.byref(rows), ctypes.byref(seg), ctypes.byref(nseg), ctypes.byref(sched)) == 0
         assert sched.value == mode and (nseg.value == 1) == (mode == 0)

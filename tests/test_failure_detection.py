@@ -16,14 +16,15 @@ from gpu_util import check_close, dev_scan_inputs, to_f64
 pytestmark = pytest.mark.gpu
 
 
-def test_chained_wait_timeout_is_reported_and_recoverable(cuda_device):
+@pytest.mark.parametrize("schedule", ["chained", "fused"])
+def test_chained_wait_timeout_is_reported_and_recoverable(cuda_device, schedule):
     import selective_state_space_46_b200 as m
     inp = synth.make_scan_inputs(1, 32, 128, io_dtype="f32", seed=3)
     dev = dev_scan_inputs(inp)
-    m.mssm_set_option(m.MSSM_OPT_SCHEDULE, m.SCHEDULES["chained"])
+    m.mssm_set_option(m.MSSM_OPT_SCHEDULE, m.SCHEDULES[schedule])
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 64)  # two chunks: one bounded wait
     try:
-        assert m.mssm_scan_plan(1, 32, 128)["schedule"] == "chained"
+        assert m.mssm_scan_plan(1, 32, 128)["schedule"] == schedule
         m.mssm_get_error()  # start from a clear error word
         m.mssm_set_option(m.MSSM_OPT_TEST_HOOKS, 1)
         m.selective_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dev["D"], dev["z"],

@@ -15,7 +15,7 @@ from gpu_util import check_close, dev_scan_inputs, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
-SCHEDULES = ["forward", "summaries+forward", "chained"]
+SCHEDULES = ["forward", "summaries+forward", "chained", "fused"]
 
 
 def _reset():

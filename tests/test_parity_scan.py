@@ -36,7 +36,7 @@ def compare_full(inp, **kw):
     check_close(to_f64(last), h_ref, inp.io_dtype, "last_state")
 
 
-SPLIT_SCHEDULES = ["summaries+forward", "chained"]
+SPLIT_SCHEDULES = ["summaries+forward", "chained", "fused"]
 
 
 def random_A(dim, seed):
