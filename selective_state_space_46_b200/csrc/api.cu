@@ -938,6 +938,9 @@ mssm_status mssm_selective_scan_bwd(const mssm_tensor* u, const mssm_tensor* del
   b.softplus = softplus_flag != 0;
   b.nseg = int(nseg); b.tiles_per_batch = int(tpb);
   b.hstart = hA; b.ws_G = gB; b.ws_S = sB; b.ws_Q = qB; b.ws_count = cntB;
+  b.vec_rows = rows_vec(u) && rows_vec(delta) && rows_vec(dout) && rows_vec(du) && rows_vec(ddelta) &&
+               (!z || (rows_vec(z) && rows_vec(dz)));
+  b.force_general = g_force_general;
   e = tracked(MSSM_KERNEL_SCAN_BWD, s, [&] { return mssm::launch_scan_bwd(b, dt, z != nullptr, s); });
   if (e != cudaSuccess) return cuda_fail(e, "backward scan kernel launch");
   return MSSM_OK;

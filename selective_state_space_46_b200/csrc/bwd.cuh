@@ -17,10 +17,11 @@
 //     before) and S_c (its summed step); the last CTA of a row tile folds them
 //     backwards, Q_(c-1) = exp(A S_c) Q_c + G_c, into each chunk's incoming Q_c;
 //  C. scan_bwd_kernel: every chunk recomputes its states forward from its start
-//     state, in sub-chunks of kBwdSub steps kept in shared memory, and sweeps them
-//     backwards from Q_c, writing du, ddelta, dz and accumulating dA, dD, dbias
-//     (per row, then one atomic add per CTA) and dB, dC (a warp transpose-reduction
-//     over the 32 rows, then one atomic add per lane and step).
+//     state, window by window (kBwdWin steps held in registers, the windows' start
+//     states in shared memory), and sweeps them backwards from Q_c, writing du,
+//     ddelta, dz and accumulating dA, dD, dbias (per row, then one atomic add per
+//     CTA) and dB, dC (a warp transpose-reduction over the 32 rows, then one atomic
+//     add per lane and step).
 #pragma once
 
 #include <cstdint>
@@ -31,7 +32,6 @@
 namespace mssm {
 
 constexpr int kBwdChunk = 64;  // steps per chunk (the forward summaries' quantum)
-constexpr int kBwdSub = 16;    // steps per recomputed sub-chunk kept in shared memory
 constexpr int kBwdRows = 32;   // rows per CTA (one warp)
 
 struct BwdArgs {
@@ -61,6 +61,8 @@ struct BwdArgs {
   int Bt, D, L;
   int softplus;
   int nseg, tiles_per_batch;
+  int vec_rows;       // u, delta, dout, z, du, ddelta, dz rows start 16-byte aligned
+  int force_general;  // never take the structured-A powers
   const float* hstart;  // [nseg-1][rows][16]: start state of chunk k+1 at k (pass A)
   float* ws_G;          // [nseg][rows][16]: pass B outgoing gradient of chunk c
   float* ws_S;          // [nseg][rows]: pass B summed step of chunk c
@@ -226,13 +228,200 @@ __global__ void __launch_bounds__(kBwdRows) scan_bwd_summary_kernel(const BwdArg
 }
 
 // ---------------------------------------------------------------------------
-// pass C: recompute the chunk's states and sweep them backwards
+// pass C: recompute the chunk's states and sweep them backwards.  The chunk is
+// walked in windows of kBwdWin steps: a first forward sweep leaves each window's
+// start state in shared memory (2 KB per window for the warp); then, window by
+// window from the last, the window's kBwdWin states are recomputed into
+// registers and swept backwards.  The window's inputs are read once, as 16-byte
+// blocks where the rows allow.
 // ---------------------------------------------------------------------------
+constexpr int kBwdWin = 8;
+
+// steps [t, t + kBwdWin) of a row (zero past t_end)
+template <typename T>
+__device__ __forceinline__ void bwd_load_win(const void* base, int64_t off, int t, int t_end, bool vec,
+                                             float (&v)[kBwdWin]) {
+  const T* row = static_cast<const T*>(base) + off;
+  if (vec && t + kBwdWin <= t_end) {
+    if constexpr (sizeof(T) == 2) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(row + t));
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = bf16lo(ws[i]);
+        v[2 * i + 1] = bf16hi(ws[i]);
+      }
+    } else {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(row + t));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(row + t) + 1);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kBwdWin; ++j) v[j] = t + j < t_end ? Elem<T>::load(row + t + j) : 0.0f;
+  }
+}
+
+// steps [t, t + kBwdWin) of an output row, clipped at t_end
+template <typename T>
+__device__ __forceinline__ void bwd_store_win(void* base, int64_t off, int t, int t_end, bool vec,
+                                              const float (&v)[kBwdWin]) {
+  T* row = static_cast<T*>(base) + off;
+  if (vec && t + kBwdWin <= t_end) {
+    if constexpr (sizeof(T) == 2) {
+      *reinterpret_cast<uint4*>(row + t) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                                      pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    } else {
+      reinterpret_cast<float4*>(row + t)[0] = make_float4(v[0], v[1], v[2], v[3]);
+      reinterpret_cast<float4*>(row + t)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kBwdWin; ++j) {
+      if (t + j < t_end) {
+        if constexpr (sizeof(T) == 2) {
+          row[t + j] = f_to_bf16(v[j]);
+        } else {
+          row[t + j] = v[j];
+        }
+      }
+    }
+  }
+}
+
+// a_n = exp(dt A_n) for the 16 states: powers of exp(dt A_0) on the structured path
+template <bool STRUCT>
+__device__ __forceinline__ void bwd_decay(float dt, const BwdRow& r, float (&a)[kN]) {
+  if constexpr (STRUCT) {
+    const float a1 = ex2f(dt * r.A2[0]);
+    a[0] = a1;
+#pragma unroll
+    for (int n = 1; n < kN; ++n) a[n] = a[n - 1] * a1;
+  } else {
+#pragma unroll
+    for (int n = 0; n < kN; ++n) a[n] = ex2f(dt * r.A2[n]);
+  }
+}
+
+template <typename T, bool HAS_Z, bool STRUCT>
+__device__ __forceinline__ void bwd_chunk(const BwdArgs& p, const BwdRow& r, float (*bc)[32],
+                                          float (*hwin)[kN][kBwdRows], int b, int d, bool row_ok, int dc,
+                                          int t0, int t1, float (&h)[kN], float (&g)[kN], float (&dA)[kN],
+                                          float& dDacc, float& dbacc) {
+  const int tid = threadIdx.x;
+  const int64_t uo = int64_t(b) * p.u_sb + int64_t(dc) * p.u_sd;
+  const int64_t ro = int64_t(b) * p.dl_sb + int64_t(dc) * p.dl_sd;
+  const int64_t go = int64_t(b) * p.g_sb + int64_t(dc) * p.g_sd;
+  const int64_t zo = int64_t(b) * p.z_sb + int64_t(dc) * p.z_sd;
+  const int64_t duo = int64_t(b) * p.du_sb + int64_t(dc) * p.du_sd;
+  const int64_t ddo = int64_t(b) * p.dd_sb + int64_t(dc) * p.dd_sd;
+  const int64_t dzo = int64_t(b) * p.dz_sb + int64_t(dc) * p.dz_sd;
+  const bool vin = p.vec_rows != 0;
+  const int nwin = (t1 - t0 + kBwdWin - 1) / kBwdWin;
+  // forward: every window's start state
+  for (int w = 0; w < nwin; ++w) {
+#pragma unroll
+    for (int n = 0; n < kN; ++n) hwin[w][n][tid] = h[n];
+    if (w + 1 == nwin) break;
+    const int tw = t0 + w * kBwdWin;
+    float uu[kBwdWin], dl[kBwdWin];
+    bwd_load_win<T>(p.u, uo, tw, t1, vin, uu);
+    bwd_load_win<T>(p.delta, ro, tw, t1, vin, dl);
+#pragma unroll
+    for (int j = 0; j < kBwdWin; ++j) {
+      float dsp, a[kN];
+      const float dt = bwd_dt(dl[j], r.bias, p.softplus, dsp);
+      bwd_decay<STRUCT>(dt, r, a);
+      const float wv = dt * uu[j];
+      const float* br = bc[tw - t0 + j];
+#pragma unroll
+      for (int n = 0; n < kN; ++n) h[n] = fmaf(a[n], h[n], wv * br[n]);
+    }
+  }
+  // backward, window by window
+  for (int w = nwin - 1; w >= 0; --w) {
+    const int tw = t0 + w * kBwdWin;
+    float uu[kBwdWin], dl[kBwdWin], go_[kBwdWin], zz[kBwdWin];
+    bwd_load_win<T>(p.u, uo, tw, t1, vin, uu);
+    bwd_load_win<T>(p.delta, ro, tw, t1, vin, dl);
+    bwd_load_win<T>(p.dout, go, tw, t1, vin, go_);
+    if constexpr (HAS_Z) bwd_load_win<T>(p.z, zo, tw, t1, vin, zz);
+    // recompute the window's states into registers
+    float hs[kBwdWin + 1][kN];  // hs[0]: the window's start state, hs[j + 1]: after step j
+#pragma unroll
+    for (int n = 0; n < kN; ++n) hs[0][n] = hwin[w][n][tid];
+#pragma unroll
+    for (int j = 0; j < kBwdWin; ++j) {
+      float dsp, a[kN];
+      const float dt = bwd_dt(dl[j], r.bias, p.softplus, dsp);
+      bwd_decay<STRUCT>(dt, r, a);
+      const float wv = dt * uu[j];
+      const float* br = bc[tw - t0 + j];
+#pragma unroll
+      for (int n = 0; n < kN; ++n) hs[j + 1][n] = fmaf(a[n], hs[j][n], wv * br[n]);
+    }
+    float du_w[kBwdWin], dd_w[kBwdWin], dz_w[kBwdWin];
+#pragma unroll
+    for (int j = kBwdWin - 1; j >= 0; --j) {
+      const int t = tw + j;
+      if (t >= t1) {  // past the end of the sequence (the last window may be partial)
+        du_w[j] = 0.0f; dd_w[j] = 0.0f; dz_w[j] = 0.0f;
+        continue;
+      }
+      float dsp, a[kN];
+      const float dt = bwd_dt(dl[j], r.bias, p.softplus, dsp);
+      bwd_decay<STRUCT>(dt, r, a);
+      const float* br = bc[t - t0];
+      const float* cr = br + 16;
+      float gy = go_[j];
+      if constexpr (HAS_Z) {
+        float yv = 0.0f;
+#pragma unroll
+        for (int n = 0; n < kN; ++n) yv = fmaf(cr[n], hs[j + 1][n], yv);
+        yv = fmaf(r.Dd, uu[j], yv);
+        float sv, ds;
+        bwd_silu(zz[j], sv, ds);
+        dz_w[j] = go_[j] * yv * ds;
+        gy = go_[j] * sv;
+      }
+      float du = gy * r.Dd;
+      dDacc = fmaf(gy, uu[j], dDacc);
+      float ddt = 0.0f;
+      float red[32];  // dB (0..15) and dC (16..31) of this row and step
+#pragma unroll
+      for (int n = 0; n < kN; ++n) {
+        g[n] = fmaf(gy, cr[n], g[n]);
+        red[16 + n] = row_ok ? gy * hs[j + 1][n] : 0.0f;
+        const float gah = g[n] * a[n] * hs[j][n];
+        ddt = fmaf(g[n], br[n] * uu[j], fmaf(r.A[n], gah, ddt));
+        dA[n] = fmaf(gah, dt, dA[n]);
+        const float gdt = g[n] * dt;
+        red[n] = row_ok ? gdt * uu[j] : 0.0f;
+        du = fmaf(gdt, br[n], du);
+        g[n] *= a[n];
+      }
+      const float draw = ddt * dsp;
+      dbacc += draw;
+      du_w[j] = du;
+      dd_w[j] = draw;
+      const float tot = warp_transpose_sum(red);
+      float* dst = tid < 16 ? p.dB + (int64_t(b) * kN + tid) * p.L + t
+                            : p.dC + (int64_t(b) * kN + (tid - 16)) * p.L + t;
+      atomicAdd(dst, tot);
+    }
+    if (row_ok) {
+      const bool vout = p.vec_rows != 0;
+      bwd_store_win<T>(p.du, duo, tw, t1, vout, du_w);
+      bwd_store_win<T>(p.ddelta, ddo, tw, t1, vout, dd_w);
+      if constexpr (HAS_Z) bwd_store_win<T>(p.dz, dzo, tw, t1, vout, dz_w);
+    }
+  }
+}
+
 template <typename T, bool HAS_Z>
 __global__ void __launch_bounds__(kBwdRows) scan_bwd_kernel(const BwdArgs p) {
   __shared__ __align__(16) float bc_s[kBwdChunk][32];
-  __shared__ __align__(16) float hsub[kBwdChunk / kBwdSub][kN][kBwdRows];  // sub-chunk start states
-  __shared__ __align__(16) float hbuf[kBwdSub][kN][kBwdRows];              // states of one sub-chunk
+  __shared__ __align__(16) float hwin[kBwdChunk / kBwdWin][kN][kBwdRows];  // window start states
   const int tid = threadIdx.x;
   const int tile = blockIdx.x;
   const int c = blockIdx.y;
@@ -246,16 +435,14 @@ __global__ void __launch_bounds__(kBwdRows) scan_bwd_kernel(const BwdArgs p) {
   const int64_t rowg = int64_t(tile) * kBwdRows + tid;
   BwdRow r;
   bwd_row(p, dc, r);
+  bool st = true;
+#pragma unroll
+  for (int n = 1; n < kN; ++n) st = st && (r.A[n] == float(n + 1) * r.A[0]);
+  const bool structured = __syncthreads_and(st) && !p.force_general;
   bwd_stage_bc<T>(p, b, t0, bc_s);
   __syncthreads();
 
-  const int64_t uo = int64_t(b) * p.u_sb + int64_t(dc) * p.u_sd;
-  const int64_t ro = int64_t(b) * p.dl_sb + int64_t(dc) * p.dl_sd;
-  const int64_t go = int64_t(b) * p.g_sb + int64_t(dc) * p.g_sd;
-  const int64_t zo = int64_t(b) * p.z_sb + int64_t(dc) * p.z_sd;
-
-  // forward from the chunk's start state, keeping the start state of every sub-chunk
-  float h[kN];
+  float h[kN], g[kN], dA[kN];
   if (c == 0) {
 #pragma unroll
     for (int n = 0; n < kN; ++n) h[n] = 0.0f;
@@ -267,24 +454,6 @@ __global__ void __launch_bounds__(kBwdRows) scan_bwd_kernel(const BwdArgs p) {
       h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
     }
   }
-  auto step_fwd = [&](int t) {
-    float dsp;
-    const float dt = bwd_dt(bwd_ld<T>(p.delta, ro + t), r.bias, p.softplus, dsp);
-    const float w = dt * bwd_ld<T>(p.u, uo + t);
-    const float* br = bc_s[t - t0];
-#pragma unroll
-    for (int n = 0; n < kN; ++n) h[n] = fmaf(ex2f(dt * r.A2[n]), h[n], w * br[n]);
-  };
-  const int nsub = (t1 - t0 + kBwdSub - 1) / kBwdSub;
-  for (int k = 0; k < nsub; ++k) {
-#pragma unroll
-    for (int n = 0; n < kN; ++n) hsub[k][n][tid] = h[n];
-    if (k + 1 < nsub)
-      for (int t = t0 + k * kBwdSub; t < t0 + (k + 1) * kBwdSub; ++t) step_fwd(t);
-  }
-
-  // backward from the incoming gradient
-  float g[kN], dA[kN];
   {
     const float4* src = reinterpret_cast<const float4*>(p.ws_Q + (int64_t(c) * rows_total + rowg) * kN);
 #pragma unroll
@@ -296,69 +465,10 @@ __global__ void __launch_bounds__(kBwdRows) scan_bwd_kernel(const BwdArgs p) {
 #pragma unroll
   for (int n = 0; n < kN; ++n) dA[n] = 0.0f;
   float dDacc = 0.0f, dbacc = 0.0f;
-  for (int k = nsub - 1; k >= 0; --k) {
-    const int ts = t0 + k * kBwdSub;
-    const int te = min(t1, ts + kBwdSub);
-    // recompute this sub-chunk's states into hbuf
-#pragma unroll
-    for (int n = 0; n < kN; ++n) h[n] = hsub[k][n][tid];
-    for (int t = ts; t < te; ++t) {
-      step_fwd(t);
-#pragma unroll
-      for (int n = 0; n < kN; ++n) hbuf[t - ts][n][tid] = h[n];
-    }
-    // sweep it backwards
-    for (int t = te - 1; t >= ts; --t) {
-      float dsp;
-      const float raw = bwd_ld<T>(p.delta, ro + t);
-      const float dt = bwd_dt(raw, r.bias, p.softplus, dsp);
-      const float uu = bwd_ld<T>(p.u, uo + t);
-      const float gout = bwd_ld<T>(p.dout, go + t);
-      float gy = gout;
-      float yv = 0.0f;
-      const float* br = bc_s[t - t0];
-      const float* cr = br + 16;
-      float red[32];  // dB (0..15) and dC (16..31) partials of this row
-#pragma unroll
-      for (int n = 0; n < kN; ++n) yv = fmaf(cr[n], hbuf[t - ts][n][tid], yv);
-      yv = fmaf(r.Dd, uu, yv);
-      if constexpr (HAS_Z) {
-        float s, ds;
-        const float zz = bwd_ld<T>(p.z, zo + t);
-        bwd_silu(zz, s, ds);
-        if (row_ok) bwd_st<T>(p.dz, int64_t(b) * p.dz_sb + int64_t(d) * p.dz_sd + t, gout * yv * ds);
-        gy = gout * s;
-      }
-      float du = gy * r.Dd;
-      dDacc = fmaf(gy, uu, dDacc);
-      float ddt = 0.0f;
-#pragma unroll
-      for (int n = 0; n < kN; ++n) {
-        const float ht = hbuf[t - ts][n][tid];
-        const float hp = t > ts ? hbuf[t - ts - 1][n][tid] : hsub[k][n][tid];
-        g[n] = fmaf(gy, cr[n], g[n]);
-        red[16 + n] = row_ok ? gy * ht : 0.0f;
-        const float a = ex2f(dt * r.A2[n]);
-        const float gah = g[n] * a * hp;
-        ddt = fmaf(g[n], br[n] * uu, fmaf(r.A[n], gah, ddt));
-        dA[n] = fmaf(gah, dt, dA[n]);
-        red[n] = row_ok ? g[n] * dt * uu : 0.0f;
-        du = fmaf(g[n] * dt, br[n], du);
-        g[n] *= a;
-      }
-      const float draw = ddt * dsp;
-      dbacc += draw;
-      if (row_ok) {
-        bwd_st<T>(p.du, int64_t(b) * p.du_sb + int64_t(d) * p.du_sd + t, du);
-        bwd_st<T>(p.ddelta, int64_t(b) * p.dd_sb + int64_t(d) * p.dd_sd + t, draw);
-      }
-      const float tot = warp_transpose_sum(red);
-      // lane i holds dB (i < 16) or dC (i >= 16) of state i % 16 summed over the 32 rows
-      float* dst = tid < 16 ? p.dB + (int64_t(b) * kN + tid) * p.L + t
-                            : p.dC + (int64_t(b) * kN + (tid - 16)) * p.L + t;
-      atomicAdd(dst, tot);
-    }
-  }
+  if (structured)
+    bwd_chunk<T, HAS_Z, true>(p, r, bc_s, hwin, b, d, row_ok, dc, t0, t1, h, g, dA, dDacc, dbacc);
+  else
+    bwd_chunk<T, HAS_Z, false>(p, r, bc_s, hwin, b, d, row_ok, dc, t0, t1, h, g, dA, dDacc, dbacc);
   if (row_ok) {
 #pragma unroll
     for (int n = 0; n < kN; ++n) atomicAdd(p.dA + int64_t(d) * kN + n, dA[n]);
