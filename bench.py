@@ -10,10 +10,14 @@ the timed region starts.  The timed steps rotate through enough copies of the
 workload's buffers to cover 4x the L2 (one copy when a single set is that
 large), so no step finds its inputs in L2 and the write-back of one step's
 dirty lines is paid inside the steps that follow; only a workload too small for
-that (over 16 copies) flushes the L2 (a 256 MiB write) before each step
+that (over 32 copies) flushes the L2 (a 256 MiB write) before each step
 instead, outside the step's event bracket.  The K timed steps are captured into
-one CUDA graph (start event, step, end event per step) so host launch overhead
-cannot leak into a step's device time.
+one CUDA graph so host launch overhead cannot leak into device time: one event
+pair brackets the K back-to-back steps (an event between steps drains the GPU
+and costs several microseconds, a third of a 10 us step), or, with the L2
+flushed between steps, one pair per step.  For the roofline the dominant kernel
+is timed on its own, with events around each launch; a step that is a single
+launch of it takes the step time instead, which those events would inflate.
 
 Multi-GPU (``torchrun --nproc-per-node N bench.py --gpus N``): rows of the scan
 are independent, so every rank runs its own batch of the same shape (weak
@@ -120,7 +124,7 @@ def binding_roofline(alg_bytes: float, alg_flops: float, ms: float, hbm_gbs: flo
     return {"bound": "hbm", **hbm, "other": {"bound": "alu", **alu}}
 
 
-def ring_size(set_bytes: int, l2_bytes: int, max_sets: int = 16) -> int:
+def ring_size(set_bytes: int, l2_bytes: int, max_sets: int = 32) -> int:
     """Number of input/output buffer sets the timed steps rotate through so that no
     step finds its data in L2: one set when a set alone is 4x the L2, else enough sets
     to cover 4x the L2; 0 (flush the L2 between steps instead) if that needs more than
@@ -540,17 +544,24 @@ def run_mssm(args):
 
     # ---- capture the K timed steps into one graph
     # external=True: the records become event nodes of the graph, so every replay re-records them
-    starts = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(args.steps)]
+    # one event pair per step only when the L2 flush must stay outside the bracket
+    npairs = args.steps if flush_between else 1
+    starts = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(npairs)]
+    ends = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(npairs)]
     before = m.mssm_kernel_stats()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
+        if not flush_between:
+            starts[0].record()
         for k in range(args.steps):
             if flush_between:
                 flush.zero_()
-            starts[k].record()
+                starts[k].record()
             step(k)
-            ends[k].record()
+            if flush_between:
+                ends[k].record()
+        if not flush_between:
+            ends[0].record()
     after = m.mssm_kernel_stats()
     launches = sum(after[k]["launches"] - before[k]["launches"] for k in after)
 
@@ -591,6 +602,13 @@ def run_mssm(args):
     dom = kern.get(dom_kernel)
     peak, peak_kind = measured_peaks()
     dom_ms = dom["ms_per_launch"] if dom else None
+    # a step that is exactly one launch of the dominant kernel: its back-to-back step time
+    single = (dom is not None and launches == args.steps and
+              all(v["launches_per_step"] == (1.0 if k == dom_kernel else 0.0) for k, v in kern.items()))
+    dom_timing = "events around each launch"
+    if single and not flush_between:
+        dom_ms = ms_per_step
+        dom_timing = "step time of back-to-back single-launch steps"
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     alu_peak = fp32_peak_tflops(sms, max_sm_mhz())
     # the conv: K FMAs per element (its SiLU runs on the SFU); the backward: BWD_FLOP_PER_STATE
@@ -604,7 +622,7 @@ def run_mssm(args):
                 f"decode_path={args.decode_path}" if kind == "decode" else None)
     traffic, traffic_src = recorded_traffic(dom_kernel, args.workload, plan_key)
     roofline = binding_roofline(alg_bytes, alg_flops, dom_ms, peak, alu_peak) if dom_ms else {"bound": None}
-    roofline.update({"kernel": dom_kernel, "ms_per_launch": dom_ms,
+    roofline.update({"kernel": dom_kernel, "ms_per_launch": dom_ms, "timing": dom_timing,
                      "peak_source": f"HBM: {peak_kind} copy rate; FP32: {sms} SMs x 128 lanes x 2 x "
                                     f"{max_sm_mhz():.0f} MHz",
                      "algorithmic_bytes_per_launch": alg_bytes, "algorithmic_flops_per_launch": alg_flops,
@@ -622,7 +640,8 @@ def run_mssm(args):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; no datasets or weights)",
         "config": {**config, "l2": l2_note,
                    "parallelism": f"replicas x{world} (independent rows, no collective)",
-                   "timing": "CUDA events per step inside one captured graph"},
+                   "timing": ("CUDA events per step inside one captured graph" if flush_between else
+                              "one CUDA event pair around the K back-to-back steps of one captured graph")},
         "hbm_gbs": step_gbs * world, "hbm_gbs_per_gpu": step_gbs,
         "hbm_frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS, "hbm_frac_of_measured": step_gbs / peak,
         "kernels": kern, "roofline": roofline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,

@@ -6,7 +6,9 @@
 //   out[b,d,t] = act(bias[d] + sum_{k<K} w[d,k] x[b,d,t-(K-1)+k]),  x = 0 before the start
 //
 // The work is HBM-bound: 2 + 2 bytes per element in bf16 against K FMAs and one
-// SFU operation.  A warp item is one row (b, d) over kConvPieces pieces of 32
+// SFU operation; the taps and the SiLU run on packed f32x2 pairs of outputs, so a
+// warp spends few enough issue slots per element for its compute to hide under the
+// loads of the other warps.  A warp item is one row (b, d) over kConvPieces pieces of 32
 // lanes x one 16-byte block.  Each lane issues the loads of all its blocks up
 // front, then per piece takes the K - 1 inputs before its block from the lane
 // below by shuffle (lane 0: from the previous piece, or loaded for the first)
@@ -26,7 +28,7 @@ namespace mssm {
 
 constexpr int kConvMaxK = 4;
 constexpr int kConvWarps = 4;   // rows per CTA
-constexpr int kConvPieces = 4;  // pieces of 32 blocks per warp item
+constexpr int kConvPieces = 8;  // pieces of 32 blocks per warp item
 
 struct ConvArgs {
   const void* x;
@@ -98,10 +100,15 @@ __global__ void __launch_bounds__(32 * kConvWarps) causal_conv1d_kernel(const Co
     raw[q] = (p.vec && tl >= tb && tl + S <= te) ? __ldg(reinterpret_cast<const uint4*>(xr + tl))
                                                  : make_uint4(0u, 0u, 0u, 0u);
   }
-  float w[K];
+  f2_t w2[K];  // tap weights, broadcast to both lanes of a pair
 #pragma unroll
-  for (int k = 0; k < K; ++k) w[k] = p.w[int64_t(d) * p.w_sd + int64_t(k) * p.w_sk];
+  for (int k = 0; k < K; ++k) {
+    const float wk = p.w[int64_t(d) * p.w_sd + int64_t(k) * p.w_sk];
+    w2[k] = f2(wk, wk);
+  }
   const float bias = p.bias ? p.bias[int64_t(d) * p.bias_s] : 0.0f;
+  const f2_t bias2 = f2(bias, bias);
+  const f2_t half2 = f2(0.5f, 0.5f);
   // lane 0's halo for the first piece: the K - 1 inputs before ta
   float carry[kConvMaxK - 1];
 #pragma unroll
@@ -112,7 +119,9 @@ __global__ void __launch_bounds__(32 * kConvWarps) causal_conv1d_kernel(const Co
     const int tp = ta + q * P;
     if (tp >= t1) break;  // warp-uniform
     const int tl = tp + lane * S;  // this lane's block
-    float xv[S];
+    // xe[0 .. K-2]: the K - 1 inputs before the block (halo), xe[K-1 ..]: the block
+    float xe[S + kConvMaxK - 1];
+    float* xv = xe + (K - 1);
     if (p.vec && tl >= tb && tl + S <= te) {
       conv_unpack<T>(raw[q], xv);
     } else {  // a block cut by the sequence's edges, or an unaligned row
@@ -120,26 +129,37 @@ __global__ void __launch_bounds__(32 * kConvWarps) causal_conv1d_kernel(const Co
       for (int j = 0; j < S; ++j) xv[j] = x_at(tl + j);
     }
     // halo: the last K - 1 inputs of the lane below; lane 0 takes the carried ones
-    float halo[kConvMaxK - 1];
 #pragma unroll
     for (int k = 0; k < K - 1; ++k) {
       const float up = __shfl_up_sync(0xffffffffu, xv[S - (K - 1) + k], 1);
-      halo[k] = lane == 0 ? carry[k] : up;
+      xe[k] = lane == 0 ? carry[k] : up;
     }
 #pragma unroll
     for (int k = 0; k < K - 1; ++k) carry[k] = __shfl_sync(0xffffffffu, xv[S - (K - 1) + k], 31);
 
+    // outputs in pairs (y_j, y_j+1) on the packed f32x2 pipe: tap k reads the input
+    // pair (xe[j + k], xe[j + k + 1])
     float y[S];
 #pragma unroll
-    for (int j = 0; j < S; ++j) {
-      float acc = bias;
+    for (int j = 0; j < S; j += 2) {
+      f2_t acc = bias2;
 #pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const int i = j - (K - 1) + k;  // input index relative to the block
-        const float xin = i >= 0 ? xv[i] : halo[K - 1 + i];
-        acc = fmaf(w[k], xin, acc);
+      for (int k = 0; k < K; ++k) acc = fma2(w2[k], f2(xe[j + k], xe[j + k + 1]), acc);
+      if constexpr (SILU && sizeof(T) == 2) {
+        // silu(a) = h (1 + tanh h), h = a / 2, on both lanes of the pair
+        const f2_t h = mul2(acc, half2);
+        float hlo, hhi;
+        f2split(h, hlo, hhi);
+        float tlo, thi;
+        asm("tanh.approx.f32 %0, %1;" : "=f"(tlo) : "f"(hlo));
+        asm("tanh.approx.f32 %0, %1;" : "=f"(thi) : "f"(hhi));
+        acc = fma2(h, f2(tlo, thi), h);
       }
-      y[j] = SILU ? gate_f<T>(acc) : acc;  // silu: SFU tanh form for bf16 output, exact for fp32
+      f2split(acc, y[j], y[j + 1]);
+      if constexpr (SILU && sizeof(T) == 4) {
+        y[j] = gate_f<T>(y[j]);  // exact form for fp32 outputs
+        y[j + 1] = gate_f<T>(y[j + 1]);
+      }
     }
     // store the outputs in [t0, t1)
     if (p.vec && tl >= t0 && tl + S <= t1) {

@@ -164,15 +164,23 @@ __device__ __forceinline__ float blk_at(const uint4& v, int j) {
 
 // softplus in base 2: returns softplus(v) / ln2 given v2 = v * log2(e).
 //  * v > 20: v (remainder below 2.1e-9, PyTorch's softplus threshold).
-//  * e = e^v < 2^-6: the series e - e^2/2 + e^3/3 (scaled by log2 e), whose
-//    truncation error is below e^4/4 (relative < 2^-20); avoids forming 1 + e.
-//  * otherwise log2(1 + e), within the SFU's 2^-22 absolute error of a result
-//    >= log2(1 + 2^-6), i.e. < 2e-5 relative.
+//  * PRECISE (fp32 I/O), e = e^v < 2^-6: the series e - e^2/2 + e^3/3 (scaled by
+//    log2 e), whose truncation error is below e^4/4 (relative < 2^-20); avoids
+//    forming 1 + e.
+//  * otherwise log2(1 + e), within the SFU's 2^-22 absolute error: < 2e-5 relative
+//    for a result >= log2(1 + 2^-6).  Without PRECISE (bf16 I/O) this form is used
+//    for small e too: the rounding of 1 + e and the SFU add up to an absolute error
+//    below 3.3e-7 in the result (2.3e-7 in the step), whose effect on an output is
+//    far below the rounding of a bf16 value.
+template <bool PRECISE = true>
 __device__ __forceinline__ float softplus2(float v2) {
   const float e = ex2f(v2);
   const float big = lg2f(1.0f + e);
-  const float small = e * fmaf(e, fmaf(e, 0.48089834696298783f, -0.72134752044448170f), 1.4426950408889634f);
-  const float r = (e < 0.015625f) ? small : big;
+  float r = big;
+  if constexpr (PRECISE) {
+    const float small = e * fmaf(e, fmaf(e, 0.48089834696298783f, -0.72134752044448170f), 1.4426950408889634f);
+    r = (e < 0.015625f) ? small : big;
+  }
   return (v2 > 28.853900817779268f) ? v2 : r;
 }
 
@@ -355,7 +363,7 @@ __device__ __forceinline__ void block_scalars(const uint4& ru, const uint4& rd, 
 #pragma unroll
   for (int j = 0; j < S; ++j) {
     const float v2 = fmaf(blk_at<T>(rd, j), kLog2e, rp.bias2);
-    float s = SOFTPLUS ? softplus2(v2) : v2;
+    float s = SOFTPLUS ? softplus2<sizeof(T) == 4>(v2) : v2;
     float uu = blk_at<T>(ru, j);
     if constexpr (PARTIAL) {
       const bool in = j >= lo && j < valid;
@@ -803,7 +811,7 @@ __device__ __forceinline__ void block_scalars_bwd(const uint4& ru, const uint4& 
 #pragma unroll
   for (int j = 0; j < S; ++j) {
     const float v2 = fmaf(blk_at<T>(rd, j), kLog2e, rp.bias2);
-    const float s = SOFTPLUS ? softplus2(v2) : v2;
+    const float s = SOFTPLUS ? softplus2<sizeof(T) == 4>(v2) : v2;
     sv[j] = s;
     wv[j] = s * blk_at<T>(ru, j);
   }

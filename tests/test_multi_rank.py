@@ -94,4 +94,5 @@ def test_ring_size_covers_four_l2():
     assert bench.ring_size(1347 << 20, l2) == 1                   # one set is already > 4x L2
     r = bench.ring_size(50_900_000, l2)
     assert r == 11 and r * 50_900_000 >= 4 * l2 and (r - 1) * 50_900_000 < 4 * l2
+    assert 0 < bench.ring_size(25_190_400, l2) <= 32               # the conv workload still rotates
     assert bench.ring_size(240_000, l2) == 0                      # tiny: flush instead

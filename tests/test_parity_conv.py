@@ -41,7 +41,7 @@ def test_conv_matches_oracle(cuda_device, K, io, silu, with_bias):
     check_close(to_f64(out), ref_conv(x, w, b, io, silu), io, "conv out")
 
 
-@pytest.mark.parametrize("L", [1, 3, 7, 255, 256, 257, 2049])
+@pytest.mark.parametrize("L", [1, 3, 7, 255, 256, 257, 2049, 4100])
 @pytest.mark.parametrize("io", ["bf16", "f32"])
 def test_conv_ragged_lengths(cuda_device, L, io):
     import selective_state_space_46_b200 as m
