@@ -20,8 +20,8 @@
 //     state, window by window (kBwdWin steps held in registers, the windows' start
 //     states in shared memory), and sweeps them backwards from Q_c, writing du,
 //     ddelta, dz and accumulating dA, dD, dbias (per row, then one atomic add per
-//     CTA) and dB, dC (a warp transpose-reduction over the 32 rows, then one atomic
-//     add per lane and step).
+//     CTA) and dB, dC (a transpose-reduction over the warp's 32 rows through shared
+//     memory, then one atomic add per lane and step).
 #pragma once
 
 #include <cstdint>
@@ -141,22 +141,33 @@ __device__ __forceinline__ void bwd_stage_bc(const BwdArgs& p, int b, int t0, fl
   }
 }
 
-// Reduce 32 per-lane quantities v[0..31] over the warp: lane i returns the sum of v[i]
-// over all lanes (31 shuffles, the recursive-halving transpose).
-__device__ __forceinline__ float warp_transpose_sum(float (&v)[32]) {
+// Reduce 32 per-lane quantities v[0..31] over the warp through a 4 KB shared buffer
+// s[32][32]: lane i writes v[q] to s[q][i] (one bank per lane), then sums row i with
+// eight 16-byte loads, taken in the order chunk ^ (i % 8) so that the eight lanes of a
+// quarter-warp read eight different chunks, and packed adds.  Lane i returns the sum of
+// v[i] over all lanes.  The buffer must be free on entry; it is free again on return.
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[32], float* s) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int w = 16; w >= 1; w >>= 1) {
-    const bool upper = (lane & w) != 0;
+  for (int q = 0; q < 32; ++q) s[q * 32 + lane] = v[q];
+  __syncwarp();
+  const ulonglong2* row = reinterpret_cast<const ulonglong2*>(s + lane * 32);
+  f2_t acc[4];
 #pragma unroll
-    for (int i = 0; i < w; ++i) {
-      // keep the half this lane is responsible for, send the other half to lane ^ w
-      const float keep = upper ? v[i + w] : v[i];
-      const float send = upper ? v[i] : v[i + w];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+  for (int c = 0; c < 8; ++c) {
+    const ulonglong2 x = row[c ^ (lane & 7)];
+    if (c < 2) {
+      acc[2 * c] = x.x;
+      acc[2 * c + 1] = x.y;
+    } else {
+      acc[2 * (c & 1)] = add2(acc[2 * (c & 1)], x.x);
+      acc[2 * (c & 1) + 1] = add2(acc[2 * (c & 1) + 1], x.y);
     }
   }
-  return v[0];
+  __syncwarp();
+  float lo, hi;
+  f2split(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), lo, hi);
+  return lo + hi;
 }
 
 // ---------------------------------------------------------------------------
@@ -454,6 +465,10 @@ __device__ __forceinline__ void bwd_chunk(const BwdArgs& p, const BwdRow& r, con
     f2_t hs[kBwdWin + 1][kN / 2];  // hs[0]: the window's start state, hs[j + 1]: after step j
 #pragma unroll
     for (int k = 0; k < kN / 2; ++k) hs[0][k] = hwin[w][k][tid];
+    // slots w (just read) and w + 1 (read for the window before) are free: the 4 KB buffer
+    // of the dB/dC reduction
+    __syncwarp();
+    float* red_s = reinterpret_cast<float*>(&hwin[w][0][0]);
 #pragma unroll
     for (int j = 0; j < kBwdWin; ++j) {
       float dsp;  // unused here
@@ -521,7 +536,7 @@ __device__ __forceinline__ void bwd_chunk(const BwdArgs& p, const BwdRow& r, con
       dbacc += draw;
       du_w[j] = fmaf(gy, r.Dd, u0v + u1v);
       dd_w[j] = draw;
-      const float tot = warp_transpose_sum(red);
+      const float tot = warp_transpose_sum(red, red_s);
       float* dst = tid < 16 ? p.dB + (int64_t(b) * kN + tid) * p.L + t
                             : p.dC + (int64_t(b) * kN + (tid - 16)) * p.L + t;
       atomicAdd(dst, tot);
@@ -538,7 +553,8 @@ __device__ __forceinline__ void bwd_chunk(const BwdArgs& p, const BwdRow& r, con
 template <typename T, bool HAS_Z>
 __global__ void __launch_bounds__(kBwdRows) scan_bwd_kernel(const BwdArgs p) {
   __shared__ __align__(16) float bc_s[kBwdChunk][32];
-  __shared__ __align__(16) f2_t hwin[kBwdChunk / kBwdWin][kN / 2][kBwdRows];  // window start states
+  // window start states, and one spare slot so that two free slots always follow window w
+  __shared__ __align__(16) f2_t hwin[kBwdChunk / kBwdWin + 1][kN / 2][kBwdRows];
   const int tid = threadIdx.x;
   const int tile = blockIdx.x;
   const int c = blockIdx.y;
