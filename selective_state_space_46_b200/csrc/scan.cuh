@@ -127,6 +127,15 @@ __device__ __forceinline__ SeqRange seq_range(const ScanArgs& p, int v) {
 // ---------------------------------------------------------------------------
 // small device helpers
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: a grid launched with programmatic stream serialization may
+// start while the grid before it in the stream still runs; griddep_wait() returns once that
+// grid has completed and its writes are visible (at once for a grid launched without it).
+// griddep_launch_dependents() lets the next such grid start before this one ends.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -457,7 +466,7 @@ template <typename T, int ROWS, bool HAS_Z, bool SOFTPLUS, bool STRUCT, bool ZOH
 __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[kTC * 32], uint4* slots,
                                               int b, int t0, int t1, const T* urow, const T* dlrow,
                                               const T* zrow, T* orow, bool row_ok, const RowParams& rp,
-                                              f2_t (&h2)[8], float* ssum = nullptr) {
+                                              f2_t (&h2)[8], float* ssum = nullptr, const float* carry = nullptr) {
   constexpr int S = 16 / int(sizeof(T));
   constexpr bool LOAD_Z = HAS_Z && READOUT;
   const int bmode = !ZOH ? 0 : STRUCT ? 1 : 2;
@@ -474,7 +483,21 @@ __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[k
   constexpr int kBlkPerChunk = kTC / S;
   const int tid = threadIdx.x;
   const bool vec = p.vec_rows != 0;
-  if (t1 <= t0) return;
+  auto take_carry = [&]() {
+    if (!carry) return;
+    griddep_wait();
+    const float4* src = reinterpret_cast<const float4*>(carry);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = __ldcg(src + i);
+      h2[2 * i] = f2(v.x, v.y);
+      h2[2 * i + 1] = f2(v.z, v.w);
+    }
+  };
+  if (t1 <= t0) {
+    take_carry();
+    return;
+  }
   // blocks are aligned to S-step boundaries of the row; a chunk that starts inside a block
   // (packed sequences) runs its first `head` steps as identity steps and stores nothing there
   const int ta = t0 - t0 % S;
@@ -520,6 +543,9 @@ __device__ __forceinline__ void forward_chunk(const ScanArgs& p, float (*bc_s)[k
   float xc[S], wc[S];
   scalars(0, ru, *slot(0, 1), xc, wc);
   __syncthreads();
+  // the carried start state is the previous kernel's output: everything above (row
+  // constants, B/C staging, the first input fetches) may overlap that kernel's tail
+  take_carry();
 
   int k = 0;
   for (int c = 0; c < nchunks; ++c) {
@@ -610,13 +636,14 @@ __device__ __forceinline__ void load_h0(const ScanArgs& p, int b, int d, f2_t (&
 template <typename T, int ROWS, bool HAS_Z, bool SOFTPLUS, bool ZOH>
 __device__ __forceinline__ void forward_any(const ScanArgs& p, float (*bc_s)[kTC * 32], uint4* slots, int b,
                                             int t0, int t1, const T* urow, const T* dlrow, const T* zrow, T* orow,
-                                            bool row_ok, const RowParams& rp, bool structured, f2_t (&h2)[8]) {
+                                            bool row_ok, const RowParams& rp, bool structured, f2_t (&h2)[8],
+                                            const float* carry = nullptr) {
   if (structured)
     forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, true, ZOH>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
-                                                       row_ok, rp, h2);
+                                                       row_ok, rp, h2, nullptr, carry);
   else
     forward_chunk<T, ROWS, HAS_Z, SOFTPLUS, false, ZOH>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow,
-                                                        row_ok, rp, h2);
+                                                        row_ok, rp, h2, nullptr, carry);
 }
 
 // 64-row CTAs are used when the grid must fill 16 warps per SM (128 registers);
@@ -647,23 +674,23 @@ __global__ void __launch_bounds__(ROWS, ROWS == 32 ? 9 : 8) scan_out_kernel(cons
   const bool st = load_row_params<ROWS>(p, dc, rp);
   const bool structured = __syncthreads_and(st) && !p.force_general;
 
+  // chunk 0 starts from h0 (an input); a later chunk from the carry the summary kernel
+  // folded, read inside forward_chunk once that kernel has completed (this grid may be
+  // launched while it still runs)
   f2_t h2[8];
+  const float* carry = nullptr;
   if (seg > 0) {
     const int64_t rows_total = int64_t(p.Bt) * p.tiles_per_batch * ROWS;
     const int64_t rowg = int64_t(tile) * ROWS + tid;
-    const float4* src = reinterpret_cast<const float4*>(p.ws_H + (int64_t(seg - 1) * rows_total + rowg) * kN);
+    carry = p.ws_H + (int64_t(seg - 1) * rows_total + rowg) * kN;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 v = __ldcg(src + i);
-      h2[2 * i] = f2(v.x, v.y);
-      h2[2 * i + 1] = f2(v.z, v.w);
-    }
+    for (int k = 0; k < 8; ++k) h2[k] = 0ull;
   } else {
     load_h0(p, vb, dc, h2);
   }
 
   forward_any<T, ROWS, HAS_Z, SOFTPLUS, ZOH>(p, bc_s, slots, b, t0, t1, urow, dlrow, zrow, orow, row_ok, rp,
-                                             structured, h2);
+                                             structured, h2, carry);
 
   if (seg == sr.last_seg && row_ok && p.last_state) {
     float* dst = p.last_state + int64_t(vb) * p.ls_sb + int64_t(d) * p.ls_sd;
@@ -877,17 +904,18 @@ __device__ __forceinline__ void backward_chunk(const ScanArgs& p, float (*bc_s)[
         const float w = wc[j];
         f2_t v[8];
         if constexpr (STRUCT) {
-          // v_n = w pi^(n+1), pi = 2^(A_0 T_j) = prod_{r>t} A_bar_r,0
+          // v_n = w pi^(n+1), pi = 2^(A_0 T_j) = prod_{r>t} A_bar_r,0: pairs by a tree of
+          // depth 3 over the broadcast powers pi^2, pi^4, pi^8
           const float pi = ex2f(rp.A0 * Tj[j]);
-          const float pi2 = pi * pi;
-          float c0 = w * pi, c1 = w * pi2;
-          v[0] = f2(c0, c1);
+          const float pi2 = pi * pi, pi4 = pi2 * pi2, pi8 = pi4 * pi4;
+          v[0] = f2(w * pi, w * pi2);
+          v[1] = mul2(v[0], f2(pi2, pi2));
+          const f2_t q4 = f2(pi4, pi4);
+          v[2] = mul2(v[0], q4);
+          v[3] = mul2(v[1], q4);
+          const f2_t q8 = f2(pi8, pi8);
 #pragma unroll
-          for (int kk = 1; kk < 8; ++kk) {
-            c0 *= pi2;
-            c1 *= pi2;
-            v[kk] = f2(c0, c1);
-          }
+          for (int kk = 0; kk < 4; ++kk) v[4 + kk] = mul2(v[kk], q8);
         } else {
           const f2_t T2 = f2(Tj[j], Tj[j]);
           const f2_t w2 = f2(w, w);
@@ -975,6 +1003,12 @@ __global__ void __launch_bounds__(ROWS, 512 / ROWS) scan_chunk_state_kernel(cons
     }
     __stcg(p.ws_S + int64_t(seg) * rows_total + rowg, Ssum);
   }
+  // The forward kernel that follows may start once every CTA has got here: its CTAs then
+  // take the places of the CTAs that exit and run their prologue during the folds below.
+  // (Triggering earlier would let them hold registers beside this kernel's CTAs and push
+  // part of their grid into a second wave.)  They read the folded carries only after
+  // griddep_wait(), which waits for this whole grid.
+  griddep_launch_dependents();
 
   // The last kernel-1 CTA of this row tile folds the chunk summaries, in chunk
   // order, into carried states: prefix_k = 2^(A S_k) prefix_(k-1) + H_k, stored

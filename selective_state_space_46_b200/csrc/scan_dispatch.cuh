@@ -27,6 +27,24 @@ struct ScanDispatch {
   template <typename T, int ROWS, bool HAS_Z, bool SP>
   static cudaError_t out_t(const ScanArgs& a, cudaStream_t s) {
     dim3 g(a.Bt * a.tiles_per_batch, a.nseg);
+    if (a.nseg > 1 && a.cu_seqlens) {
+      // Packed sequences, right after the chunk-summary kernel: a programmatic dependent
+      // launch, so that the CTAs' prologue overlaps that kernel's long carry folds (they
+      // read the carries after griddep_wait).  Measured on B200: 387 -> 364 us for 32
+      // packed sequences; on plain batches whose forward grid fits one wave it cost 6%
+      // (the early CTAs are placed unevenly over the SMs), so they launch normally.
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = g;
+      cfg.blockDim = dim3(ROWS);
+      cfg.dynamicSmemBytes = 0;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      return cudaLaunchKernelEx(&cfg, scan_out_kernel<T, ROWS, HAS_Z, SP, ZOH>, a);
+    }
     scan_out_kernel<T, ROWS, HAS_Z, SP, ZOH><<<g, ROWS, 0, s>>>(a);
     return cudaGetLastError();
   }
