@@ -169,6 +169,7 @@ KERNEL_SOURCES = {
     "scan_chunk_state": ("device_common.cuh", "scan.cuh", "scan.cu", "scan_zoh.cu", "scan_dispatch.cuh"),
     "state_update": ("device_common.cuh", "decode.cuh", "decode.cu"),
     "conv": ("device_common.cuh", "conv.cuh", "conv.cu"),
+    "scan_bwd": ("device_common.cuh", "bwd.cuh", "bwd.cu"),
 }
 
 
@@ -618,7 +619,7 @@ def run_mssm(args):
         alg_flops = units * N_STATE * BWD_FLOP_PER_STATE
     else:
         alg_flops = algorithmic_flops(units)
-    plan_key = (plan_string(config.get("plan")) if kind == "scan" else
+    plan_key = (plan_string(config.get("plan")) if kind == "scan" and not args.backward else
                 f"decode_path={args.decode_path}" if kind == "decode" else None)
     traffic, traffic_src = recorded_traffic(dom_kernel, args.workload, plan_key)
     roofline = binding_roofline(alg_bytes, alg_flops, dom_ms, peak, alu_peak) if dom_ms else {"bound": None}
