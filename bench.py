@@ -409,6 +409,7 @@ def run_mssm(args):
 
     seed = rank_seed(rank)
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, args.chunk_len)
+    m.mssm_set_option(m.MSSM_OPT_ROWS_PER_CTA, args.rows_per_cta)
     m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 1 if args.general_a else 0)
     m.mssm_set_option(m.MSSM_OPT_DECODE_PATH, m.DECODE_PATHS.get(args.decode_path, 0))
     m.mssm_set_option(m.MSSM_OPT_SCHEDULE, m.SCHEDULES.get(args.schedule, 0))
@@ -784,6 +785,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--chunk-len", type=int, default=0, help="length split (0: automatic; multiple of 64)")
+    ap.add_argument("--rows-per-cta", type=int, default=0, choices=[0, 32, 64],
+                    help="channels per row tile of the scan (0: automatic)")
     ap.add_argument("--decode-path", choices=["auto", "stream", "bulk_tile", "per_row"], default="auto",
                     help="decode kernel (MSSM_OPT_DECODE_PATH)")
     ap.add_argument("--zoh", action="store_true", help="zero-order-hold discretisation (scan workloads)")

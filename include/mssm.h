@@ -340,6 +340,9 @@ mssm_status mssm_get_error(void *stream);
  *     aligned batch rows.  2 one bulk-copied tile of 256 rows per CTA; needs the
  *     contiguous state.  3 one thread per row, any layout.  A forced path whose
  *     conditions fail falls back to the next one that holds.
+ *   MSSM_OPT_ROWS_PER_CTA (value 0, 32 or 64): channels per row tile (CTA) of the
+ *     scan plan, one channel per thread; 0 automatic.  64-channel tiles take the
+ *     forward or summaries + forward schedule only.
  *   MSSM_OPT_TEST_HOOKS (value 0/1, for testing failure detection only): when 1,
  *     the chained scan schedule publishes no carried states, so every chunk after
  *     the first gives up its bounded wait (about 0.5 s), runs from a zero state
@@ -353,7 +356,8 @@ typedef enum {
     MSSM_OPT_KERNEL_TIMING = 3,
     MSSM_OPT_SCHEDULE = 4,
     MSSM_OPT_DECODE_PATH = 5,
-    MSSM_OPT_TEST_HOOKS = 6
+    MSSM_OPT_TEST_HOOKS = 6,
+    MSSM_OPT_ROWS_PER_CTA = 7
 } mssm_option;
 mssm_status mssm_set_option(int option, int64_t value);
 

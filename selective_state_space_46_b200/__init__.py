@@ -22,7 +22,7 @@ __all__ = [
     "mssm_get_error", "mssm_set_option", "mssm_shutdown", "mssm_version", "mssm_status_string",
     "mssm_last_error", "selective_scan_fwd", "state_update", "lib_path",
     "MSSM_OPT_FORCE_GENERAL_A", "MSSM_OPT_CHUNK_LEN", "MSSM_OPT_KERNEL_TIMING", "MSSM_OPT_SCHEDULE", "SCHEDULES",
-    "MSSM_OPT_DECODE_PATH", "DECODE_PATHS", "MSSM_OPT_TEST_HOOKS", "MSSM_ERR_TIMEOUT", "mssm_kernel_stats", "mssm_scan_plan",
+    "MSSM_OPT_DECODE_PATH", "DECODE_PATHS", "MSSM_OPT_TEST_HOOKS", "MSSM_OPT_ROWS_PER_CTA", "MSSM_ERR_TIMEOUT", "mssm_kernel_stats", "mssm_scan_plan",
     "mssm_selective_scan_fwd_ex", "MSSM_DISC_EULER", "MSSM_DISC_ZOH",
     "mssm_causal_conv1d_fwd", "mssm_causal_conv1d_update", "causal_conv1d", "causal_conv1d_update",
     "mssm_selective_scan_bwd", "selective_scan_bwd",
@@ -41,6 +41,7 @@ MSSM_OK, MSSM_ERR_INVALID_ARG, MSSM_ERR_UNSUPPORTED, MSSM_ERR_CUDA, MSSM_ERR_TIM
 MSSM_OPT_FORCE_GENERAL_A, MSSM_OPT_CHUNK_LEN, MSSM_OPT_KERNEL_TIMING, MSSM_OPT_SCHEDULE = 1, 2, 3, 4
 MSSM_OPT_DECODE_PATH = 5
 MSSM_OPT_TEST_HOOKS = 6
+MSSM_OPT_ROWS_PER_CTA = 7
 MSSM_DISC_EULER, MSSM_DISC_ZOH = 0, 1
 SCHEDULES = {"forward": 1, "summaries+forward": 2, "chained": 3, "fused": 4}
 DECODE_PATHS = {"stream": 1, "bulk_tile": 2, "per_row": 3}

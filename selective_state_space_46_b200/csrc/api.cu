@@ -36,6 +36,7 @@ std::mutex g_mu;
 int g_force_general = 0;
 int64_t g_chunk_len = 0;
 int g_schedule = -1;
+int g_rows_per_cta = 0;  // 0 automatic, else 32 or 64
 int g_decode_path = 0;  // MSSM_OPT_DECODE_PATH
 int g_test_hooks = 0;   // MSSM_OPT_TEST_HOOKS  // -1 automatic, else the forced LaunchShape mode
 
@@ -173,7 +174,7 @@ int64_t round_seg(int64_t v) {
 // another, so the chained schedule costs at least nseg items, which is what rules it out
 // for a few long sequences among short ones.
 LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forced_seg, int forced_mode,
-                         int64_t total_len = -1) {
+                         int forced_rows, int64_t total_len = -1) {
   constexpr double kOut = 96.0, kSum = 55.0, kSumFwd = 70.0, kIpc1 = 0.6, kIpc2 = 0.7;
   constexpr double kStart = 4000.0, kLaunch = 6000.0, kItem = 4000.0, kFold = 200.0;
   auto ipc = [&](int64_t k) { return k <= 1 ? kIpc1 : kIpc2; };
@@ -185,9 +186,9 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
     const int64_t k = (resident * (rows / 32) + 3) / 4;
     return double(waves) * (double(k) * steps * instr / ipc(k) + kStart) + kLaunch;
   };
-  LaunchShape best{0, 32, L > 0 ? L : 1, 1, 0};
+  LaunchShape best{0, forced_rows ? forced_rows : 32, L > 0 ? L : 1, 1, 0};
   double best_cost = -1.0;
-  if (forced_mode == 0) return LaunchShape{0, 32, L > 0 ? L : 1, 1, 0};
+  if (forced_mode == 0) return LaunchShape{0, forced_rows ? forced_rows : 32, L > 0 ? L : 1, 1, 0};
   auto consider = [&](const LaunchShape& sh, double cost) {
     if (forced_mode > 0 && sh.mode != forced_mode) return;
     if (best_cost < 0.0 || cost < best_cost * 0.999) {
@@ -197,6 +198,7 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
   };
   const bool packed = total_len >= 0;
   for (int rows : {32, 64}) {
+    if (forced_rows && rows != forced_rows) continue;
     const int64_t tpb = (D + rows - 1) / rows;
     const int64_t tiles = Bt * tpb;
     for (int64_t want = 1; want <= 64; ++want) {
@@ -275,6 +277,10 @@ mssm_status mssm_set_option(int option, int64_t value) {
     case MSSM_OPT_SCHEDULE:
       if (value < 0 || value > 4) return fail(MSSM_ERR_INVALID_ARG, "SCHEDULE takes 0 (automatic) to 4");
       g_schedule = int(value) - 1;
+      return MSSM_OK;
+    case MSSM_OPT_ROWS_PER_CTA:
+      if (value != 0 && value != 32 && value != 64) return fail(MSSM_ERR_INVALID_ARG, "ROWS_PER_CTA takes 0, 32 or 64");
+      g_rows_per_cta = int(value);
       return MSSM_OK;
     case MSSM_OPT_TEST_HOOKS:
       if (value < 0 || value > 1) return fail(MSSM_ERR_INVALID_ARG, "TEST_HOOKS takes 0 or 1");
@@ -452,7 +458,7 @@ ScanPlan scan_plan(ScanCall& call, int sm_count) {
   a.force_general = g_force_general;
   a.test_no_publish = g_test_hooks & 1;
   const LaunchShape shape =
-      choose_shape(call.Bt, call.D, call.L, sm_count, g_chunk_len, g_schedule, call.total_len);
+      choose_shape(call.Bt, call.D, call.L, sm_count, g_chunk_len, g_schedule, g_rows_per_cta, call.total_len);
   ScanPlan plan;
   plan.mode = shape.mode;
   plan.rows_per_cta = shape.rows;
@@ -1061,12 +1067,13 @@ mssm_status mssm_scan_plan_packed(int64_t S, int64_t D, int64_t max_seqlen, int6
     std::lock_guard<std::mutex> lk(g_mu);
     forced = g_chunk_len;
   }
-  int forced_mode;
+  int forced_mode, forced_rows;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     forced_mode = g_schedule;
+    forced_rows = g_rows_per_cta;
   }
-  const LaunchShape sh = choose_shape(Bt, D, L, sm_count, forced, forced_mode, total_len);
+  const LaunchShape sh = choose_shape(Bt, D, L, sm_count, forced, forced_mode, forced_rows, total_len);
   if (rows_per_cta) *rows_per_cta = sh.rows;
   if (chunk_len) *chunk_len = sh.seg;
   if (n_chunks) *n_chunks = sh.nseg;

@@ -268,6 +268,10 @@ def test_options_and_strings(lib):
     assert lib.mssm_set_option(6, 1) == 0 and lib.mssm_set_option(6, 0) == 0
     assert lib.mssm_set_option(2, 128) == 0
     assert lib.mssm_set_option(2, 0) == 0
+    for v in (16, 48, -32, 128):
+        assert lib.mssm_set_option(7, v) == INVALID
+    for v in (64, 32, 0):
+        assert lib.mssm_set_option(7, v) == 0
     lib.mssm_status_string.restype = ctypes.c_char_p
     assert lib.mssm_status_string(2) == b"MSSM_ERR_UNSUPPORTED"
     lib.mssm_version.restype = ctypes.c_char_p

@@ -20,6 +20,7 @@ def _reset_options():
     m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 0)
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
     m.mssm_set_option(m.MSSM_OPT_SCHEDULE, 0)
+    m.mssm_set_option(m.MSSM_OPT_ROWS_PER_CTA, 0)
 
 
 @pytest.fixture(autouse=True)
@@ -153,6 +154,49 @@ def test_chunked_carry(chunk, structured, io, schedule):
     inp = synth.make_scan_inputs(2, 80, 1000, io_dtype=io, seed=chunk, delta_range=(1e-4, 1e-2))
     if not structured:
         inp.A = random_A(80, chunk)
+    compare_full(inp)
+
+
+@pytest.mark.parametrize("Bt,D,L", [(1, 1, 1), (2, 5, 7), (1, 64, 15), (1, 65, 100), (2, 130, 257),
+                                    (3, 129, 1000), (1, 200, 777)])
+@pytest.mark.parametrize("schedule,chunk", [("forward", 0), ("summaries+forward", 64),
+                                            ("summaries+forward", 192)])
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_64_row_tiles(Bt, D, L, schedule, chunk, io):
+    """Plans forced to 64-channel row tiles (two warps per CTA)."""
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_ROWS_PER_CTA, 64)
+    m.mssm_set_option(m.MSSM_OPT_SCHEDULE, m.SCHEDULES[schedule])
+    if chunk:
+        m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, chunk)
+    plan = m.mssm_scan_plan(Bt, D, L)
+    assert plan["rows_per_cta"] == 64
+    inp = synth.make_scan_inputs(Bt, D, L, io_dtype=io, seed=D * 3 + L)
+    compare_full(inp)
+
+
+@pytest.mark.parametrize("with_z,with_D,with_bias,softplus", [
+    (False, False, False, False), (True, True, False, True), (False, True, True, True)])
+@pytest.mark.parametrize("structured", [True, False])
+def test_64_row_tiles_options(with_z, with_D, with_bias, softplus, structured):
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_ROWS_PER_CTA, 64)
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 128)
+    inp = synth.make_scan_inputs(2, 100, 600, io_dtype="bf16", seed=11, with_z=with_z, with_D=with_D,
+                                 with_bias=with_bias, softplus=softplus)
+    if not softplus:  # a positive, small step without softplus (a negative one makes the states grow)
+        pos = np.abs(synth.bf16_bits_to_f32(inp.delta)) * 0.05
+        inp.delta = synth.f32_to_bf16_bits(pos)
+        inp.delta_bias = None
+    if not structured:
+        inp.A = random_A(100, 5)
+    compare_full(inp)
+
+
+def test_64_row_tiles_default_workload():
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_ROWS_PER_CTA, 64)
+    inp = synth.workload_inputs("scan_bf16_2x1536x2048", seed=0)
     compare_full(inp)
 
 

@@ -20,6 +20,7 @@ def _reset():
     m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 0)
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
     m.mssm_set_option(m.MSSM_OPT_SCHEDULE, 0)
+    m.mssm_set_option(m.MSSM_OPT_ROWS_PER_CTA, 0)
 
 
 @pytest.fixture(autouse=True)
@@ -74,6 +75,26 @@ def test_varlen_each_schedule(schedule, chunk, structured, io):
         inp.A = random_A(70, 3)
     out, last = run_varlen(inp, cu)
     y_ref, h_ref = oracle_varlen(inp, cu)
+    check_close(to_f64(out), y_ref, io, "y")
+    check_close(to_f64(last), h_ref, io, "last_state")
+
+
+@pytest.mark.parametrize("schedule,chunk", [("forward", 0), ("summaries+forward", 64),
+                                            ("summaries+forward", 128)])
+@pytest.mark.parametrize("structured", [True, False])
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_varlen_64_row_tiles(schedule, chunk, structured, io):
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_ROWS_PER_CTA, 64)
+    m.mssm_set_option(m.MSSM_OPT_SCHEDULE, m.SCHEDULES[schedule])
+    if chunk:
+        m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, chunk)
+    inp, cu = packed(LENGTHS, 100, io, seed=4)
+    if not structured:
+        inp.A = random_A(100, 4)
+    h0 = np.random.default_rng(4).standard_normal((len(LENGTHS), 100, 16)).astype(np.float32) * 0.3
+    out, last = run_varlen(inp, cu, h0=h0)
+    y_ref, h_ref = oracle_varlen(inp, cu, h0=h0)
     check_close(to_f64(out), y_ref, io, "y")
     check_close(to_f64(last), h_ref, io, "last_state")
 
