@@ -661,9 +661,13 @@ def run_mssm(args):
 
 
 def run_e2e(args, kind, inp, d, dev, m, units, world):
+    """The same metric end to end through the public API: every step copies its inputs from
+    pinned host memory to the device, makes the C-ABI call and copies its results back.  Two
+    device buffer sets and three streams pipeline the steps: the uploads of step k + 1 overlap
+    the call and the downloads of step k (PCIe is full duplex, with a copy engine each way)."""
     import torch
     import torch.distributed as dist
-    steps = max(1, min(args.steps, 20))
+    steps = max(2, min(args.steps, 20))
 
     def pin(a):
         if a is None:
@@ -674,103 +678,132 @@ def run_e2e(args, kind, inp, d, dev, m, units, world):
             t = torch.from_numpy(np.ascontiguousarray(a, np.float32))
         return t.pin_memory()
 
-    if kind == "conv":
-        hx = pin(inp.x)
-        xd = torch.empty(hx.shape, dtype=hx.dtype, device=dev)
-        w_d, b_d = pin(inp.weight).to(dev), pin(inp.bias).to(dev)
-        out = torch.empty_like(xd)
-        y_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h2d = hx.numel() * hx.element_size()
-        d2h = y_host.numel() * y_host.element_size()
+    def dev_like(v):
+        return None if v is None else torch.empty(v.shape, dtype=v.dtype, device=dev)
 
-        def one():
-            xd.copy_(hx, non_blocking=True)
-            m.mssm_causal_conv1d_fwd(xd, w_d, b_d, out, None, 0, True)
-            y_host.copy_(out, non_blocking=True)
+    def host_like(v):
+        return None if v is None else torch.empty(v.shape, dtype=v.dtype).pin_memory()
+
+    def upload(h, dd):
+        for k, v in h.items():
+            if v is not None:
+                dd[k].copy_(v, non_blocking=True)
+
+    def download(dd, hh):
+        for k, v in dd.items():
+            if v is not None:
+                hh[k].copy_(v, non_blocking=True)
+
+    # per kind: host inputs h, and make_set() -> (device inputs, device results, host results, call)
+    if kind == "conv":
+        h = {"x": pin(inp.x)}
+        w_d, b_d = pin(inp.weight).to(dev), pin(inp.bias).to(dev)
+
+        def make_set():
+            di = {"x": dev_like(h["x"])}
+            do = {"y": torch.empty_like(di["x"])}
+            return di, do, {"y": host_like(do["y"])}, (
+                lambda: m.mssm_causal_conv1d_fwd(di["x"], w_d, b_d, do["y"], None, 0, True))
+        path_out = "y"
     elif kind == "scan" and args.backward:
         names = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
         h = {k: pin(getattr(inp, k)) for k in names}
         rng = np.random.default_rng(7)
         dout_h = rng.standard_normal(inp.u.shape).astype(np.float32)
         h["dout"] = pin(synth.f32_to_bf16_bits(dout_h) if inp.io_dtype == "bf16" else dout_h)
-        dd = {k: (None if v is None else torch.empty(v.shape, dtype=v.dtype, device=dev)) for k, v in h.items()}
-        for k in h:
-            if h[k] is not None:
-                dd[k].copy_(h[k])
-        g = m.selective_scan_bwd(dd["u"], dd["delta"], dd["A"], dd["B"], dd["C"], dd["D"], dd["z"],
-                                 dd["delta_bias"], inp.softplus, dd["dout"])
-        g_host = {k: (None if v is None else torch.empty(v.shape, dtype=v.dtype).pin_memory()) for k, v in g.items()}
-        h2d = sum(v.numel() * v.element_size() for v in h.values() if v is not None)
-        d2h = sum(v.numel() * v.element_size() for v in g_host.values() if v is not None)
 
-        def one():
-            for k in h:
-                if h[k] is not None:
-                    dd[k].copy_(h[k], non_blocking=True)
-            m.mssm_selective_scan_bwd(dd["u"], dd["delta"], dd["A"], dd["B"], dd["C"], dd["D"], dd["z"],
-                                      dd["delta_bias"], inp.softplus, dd["dout"], g["du"], g["ddelta"], g["dA"],
-                                      g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"])
-            for k, v in g.items():
-                if v is not None:
-                    g_host[k].copy_(v, non_blocking=True)
+        def make_set():
+            di = {k: dev_like(v) for k, v in h.items()}
+            upload(h, di)
+            torch.cuda.synchronize(dev)
+            g = m.selective_scan_bwd(di["u"], di["delta"], di["A"], di["B"], di["C"], di["D"], di["z"],
+                                     di["delta_bias"], inp.softplus, di["dout"])
+            do = {k: v for k, v in g.items() if v is not None}
+            return di, do, {k: host_like(v) for k, v in do.items()}, (
+                lambda: m.mssm_selective_scan_bwd(di["u"], di["delta"], di["A"], di["B"], di["C"], di["D"], di["z"],
+                                                  di["delta_bias"], inp.softplus, di["dout"], g["du"], g["ddelta"],
+                                                  g["dA"], g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"]))
+        path_out = "every gradient"
     elif kind == "scan":
         names = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
         h = {k: pin(getattr(inp, k)) for k in names}
         varlen = inp.cu_seqlens is not None
         if varlen:
             h["cu_seqlens"] = torch.from_numpy(inp.cu_seqlens).pin_memory()
-        dd = {k: (None if v is None else torch.empty(v.shape, dtype=v.dtype, device=dev)) for k, v in h.items()}
-        out = torch.empty_like(dd["u"])
         nstate = len(inp.cu_seqlens) - 1 if varlen else inp.batch
         max_seqlen = int(np.diff(inp.cu_seqlens).max()) if varlen else 0
-        last = torch.empty(nstate, inp.dim, N_STATE, device=dev)
-        y_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        s_host = torch.empty(last.shape, dtype=last.dtype).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in h.values() if v is not None)
-        d2h = y_host.numel() * y_host.element_size() + s_host.numel() * s_host.element_size()
         disc = m.MSSM_DISC_ZOH if args.zoh else m.MSSM_DISC_EULER
 
-        def one():
-            for k in h:
-                if h[k] is not None:
-                    dd[k].copy_(h[k], non_blocking=True)
-            m.mssm_selective_scan_fwd_ex(dd["u"], dd["delta"], dd["A"], dd["B"], dd["C"], dd["D"], dd["z"],
-                                         dd["delta_bias"], inp.softplus, out, last, discretization=disc,
-                                         cu_seqlens=dd.get("cu_seqlens"), max_seqlen=max_seqlen)
-            y_host.copy_(out, non_blocking=True)
-            s_host.copy_(last, non_blocking=True)
+        def make_set():
+            di = {k: dev_like(v) for k, v in h.items()}
+            do = {"y": torch.empty_like(di["u"]), "last": torch.empty(nstate, inp.dim, N_STATE, device=dev)}
+            return di, do, {k: host_like(v) for k, v in do.items()}, (
+                lambda: m.mssm_selective_scan_fwd_ex(di["u"], di["delta"], di["A"], di["B"], di["C"], di["D"],
+                                                     di["z"], di["delta_bias"], inp.softplus, do["y"], do["last"],
+                                                     discretization=disc, cu_seqlens=di.get("cu_seqlens"),
+                                                     max_seqlen=max_seqlen))
+        path_out = "y and the final state"
     else:
         names = ("state", "x", "dt", "A", "B", "C", "D", "z")
         h = {k: pin(getattr(inp, k)) for k in names}
-        dd = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in h.items()}
-        out = torch.empty_like(dd["x"])
-        y_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        s_host = torch.empty(dd["state"].shape, dtype=torch.float32).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in h.values())
-        d2h = y_host.numel() * y_host.element_size() + s_host.numel() * s_host.element_size()
 
-        def one():
-            for k in names:
-                dd[k].copy_(h[k], non_blocking=True)
-            m.mssm_state_update(dd["state"], dd["x"], dd["dt"], dd["A"], dd["B"], dd["C"], dd["D"], dd["z"], out)
-            y_host.copy_(out, non_blocking=True)
-            s_host.copy_(dd["state"], non_blocking=True)
+        def make_set():
+            di = {k: dev_like(v) for k, v in h.items()}
+            do = {"y": torch.empty_like(di["x"]), "state": di["state"]}
+            return di, do, {k: host_like(v) for k, v in do.items()}, (
+                lambda: m.mssm_state_update(di["state"], di["x"], di["dt"], di["A"], di["B"], di["C"], di["D"],
+                                            di["z"], do["y"]))
+        path_out = "y and the updated state"
 
-    one()
+    sets = [make_set() for _ in range(2)]
+    h2d = sum(v.numel() * v.element_size() for v in h.values() if v is not None)
+    d2h = sum(v.numel() * v.element_size() for v in sets[0][2].values() if v is not None)
+    s_in, s_call, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = {name: [torch.cuda.Event() for _ in sets] for name in ("in", "call", "out")}
+
+    def run(n):
+        for k in range(n):
+            j = k % len(sets)
+            di, do, ho, call = sets[j]
+            with torch.cuda.stream(s_in):
+                if k >= len(sets):
+                    # the step before that has read this set's inputs and copied out its results
+                    # (the decode state is both)
+                    s_in.wait_event(ev["out"][j])
+                upload(h, di)
+                ev["in"][j].record(s_in)
+            with torch.cuda.stream(s_call):
+                s_call.wait_event(ev["in"][j])
+                if k >= len(sets):
+                    s_call.wait_event(ev["out"][j])  # this set's results were copied out
+                call()
+                ev["call"][j].record(s_call)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev["call"][j])
+                download(do, ho)
+                ev["out"][j].record(s_out)
+
+    main = torch.cuda.current_stream(dev)
+    run(len(sets))
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(steps):
-        one()
-    t1.record()
+    t0.record(main)
+    for s in (s_in, s_call, s_out):
+        s.wait_stream(main)
+    run(steps)
+    for s in (s_in, s_call, s_out):
+        main.wait_stream(s)
+    t1.record(main)
     torch.cuda.synchronize(dev)
     ms = reduce_max(t0.elapsed_time(t1), dist if world > 1 else None) / steps
     return {"value": units * world / (ms / 1e3), "unit": "elems/s" if kind in ("scan", "conv") else "rows/s",
             "ms_per_step": ms, "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "path": "pinned host buffers -> H2D copies -> C-ABI call -> D2H of y and final state"}
+            "path": (f"pinned host buffers -> H2D copies -> C-ABI call -> D2H of {path_out}, every step; "
+                     "two buffer sets on three streams, the uploads of one step overlapping the call and "
+                     "downloads of the one before")}
 
 
 def main(argv=None):
