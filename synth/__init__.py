@@ -207,6 +207,8 @@ WORKLOADS = {
                                     io_dtype="bf16", delta_range=(1e-4, 1e-2), with_z=True),
     # the causal conv1d (K = 4) + SiLU that produces u, at the Mamba-130M prefill shape
     "conv_bf16_2x1536x2048": dict(kind="conv", batch=2, dim=1536, length=2048, io_dtype="bf16", K=4),
+    # the same conv at the Mamba-2.8B prefill shape (671 MB of traffic per call)
+    "conv_bf16_8x5120x4096": dict(kind="conv", batch=8, dim=5120, length=4096, io_dtype="bf16", K=4),
     # packed variable-length prefill: 32 sequences of 64..4096 steps (log-uniform) over
     # Mamba-130M's 1536 channels, concatenated along L without padding
     "scan_varlen_bf16_1536x32seq": dict(kind="scan", batch=1, dim=1536, nseq=32, len_range=(64, 4096),
