@@ -70,19 +70,6 @@ struct BwdArgs {
   unsigned* ws_count;   // [tiles]: pass B arrivals, reset by the folding CTA
 };
 
-template <typename T>
-__device__ __forceinline__ float bwd_ld(const void* base, int64_t off) {
-  return Elem<T>::load(static_cast<const T*>(base) + off);
-}
-template <typename T>
-__device__ __forceinline__ void bwd_st(void* base, int64_t off, float v) {
-  if constexpr (sizeof(T) == 2) {
-    static_cast<uint16_t*>(base)[off] = f_to_bf16(v);
-  } else {
-    static_cast<float*>(base)[off] = v;
-  }
-}
-
 // dt of one step: softplus(delta + bias) or delta + bias; also sigmoid(delta + bias), the
 // derivative of softplus (1 without softplus)
 __device__ __forceinline__ float bwd_dt(float raw, float bias, bool softplus, float& dsp) {
