@@ -278,6 +278,24 @@ def test_options_and_strings(lib):
     assert re.match(rb"^\d+\.\d+\.\d+$", lib.mssm_version())
 
 
+def test_scan_plan_measured_best():
+    """The automatic plans of the benchmark workloads are the ones measured fastest on B200
+    (sweeps of chunk length, rows per CTA and schedule): a change to the cost model that moves
+    one of them must be measured again."""
+    import selective_state_space_46_b200 as m
+    for opt in (m.MSSM_OPT_CHUNK_LEN, m.MSSM_OPT_SCHEDULE, m.MSSM_OPT_ROWS_PER_CTA):
+        m.mssm_set_option(opt, 0)
+    expect = {
+        (2, 1536, 2048, -1): ("summaries+forward", 32, 192),   # 65 us; 128: 65.6, 256: 74.8, 64 rows: 67-89
+        (8, 5120, 4096, -1): ("chained", 32, 512),             # 773 us; summaries+forward: 1089
+        (1, 2048, 131072, -1): ("summaries+forward", 64, 3584),  # 1683 us; 32 rows: 1838
+        (32, 1536, 4096, 27048): ("summaries+forward", 64, 128),  # packed: 365 us; 32 rows: 391
+    }
+    for (S, D, L, total), (sched, rows, chunk) in expect.items():
+        plan = m.mssm_scan_plan(S, D, L, sm_count=148, total_len=total)
+        assert (plan["schedule"], plan["rows_per_cta"], plan["chunk_len"]) == (sched, rows, chunk), (S, D, L, plan)
+
+
 def test_scan_plan_host_only(lib):
     """The launch plan is host logic: check its invariants without a GPU."""
     f = lib.mssm_scan_plan
