@@ -52,7 +52,7 @@ DECODE_METRIC = "selective state update rows/s and achieved HBM GB/s vs ~8 TB/s 
 CONV_METRIC = "causal conv1d + SiLU B·D·L elems/s and achieved HBM GB/s vs ~8 TB/s B200 peak"
 BWD_METRIC = "selective-scan backward B·D·L elems/s and achieved HBM GB/s vs ~8 TB/s B200 peak"
 BWD_FLOP_PER_STATE = 22  # the forward recomputed (6) and the reverse step (16) per (element, state)
-DEFAULT_WORKLOAD = "scan_bf16_2x1536x2048"
+DEFAULT_WORKLOAD = "scan_bf16_1x2048x131072"
 L2_FLUSH_BYTES = 256 << 20
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0

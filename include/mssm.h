@@ -403,7 +403,13 @@ typedef enum {
  */
 mssm_status mssm_kernel_stats(int64_t *launches, int64_t *timed, double *ms, int reset);
 
-/* Frees the library's per-device workspaces (call with no work in flight). */
+/*
+ * Frees the library's per-device workspaces and forgets the device addresses it
+ * cached (of the no-allocation scratch array and of the error word).  Call it
+ * with no work in flight, and before any cudaDeviceReset: a reset unloads the
+ * library's device module, and addresses cached from before it would be stale.
+ * The library may be used again afterwards; it looks the addresses up anew.
+ */
 mssm_status mssm_shutdown(void);
 
 /* Library version, "major.minor.patch". */

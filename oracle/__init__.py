@@ -238,6 +238,24 @@ def scan_rows(inp, rows: Sequence[Tuple[int, int]]):
     return np.stack(ys), np.stack(hs)
 
 
+def scan_block(inp, b: int, d0: int, d1: int, h0=None, zoh: bool = False):
+    """Oracle scan of channels ``d0 .. d1 - 1`` of batch ``b`` of a ``synth.ScanInputs`` problem
+    (``h0`` [1, d1 - d0, N] or None).  Returns ``(y [1, d1 - d0, L], last_state [1, d1 - d0, N])``.
+    Lets full-size outputs be checked on every row with bounded host memory."""
+    from synth import to_f64  # input widening only (bit manipulation)
+
+    def sl(name):
+        a = getattr(inp, name)
+        return None if a is None else to_f64(a[b:b + 1, d0:d1], inp.io_dtype)
+
+    def ch(name):
+        a = getattr(inp, name)
+        return None if a is None else np.asarray(a[d0:d1], np.float64)
+
+    return scan(sl("u"), sl("delta"), ch("A"), _widen_batch(inp, "B", b), _widen_batch(inp, "C", b),
+                ch("D"), sl("z"), ch("delta_bias"), inp.softplus, h0=h0, zoh=zoh)
+
+
 def _widen_slice(inp, name, b, d):
     a = getattr(inp, name)
     if a is None:

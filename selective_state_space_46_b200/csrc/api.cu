@@ -1154,6 +1154,13 @@ mssm_status mssm_shutdown(void) {
     g_dev[i].bwd_ws = nullptr;
     g_dev[i].bwd_bytes = 0;
   }
+  // Cached addresses of module symbols (the no-allocation scratch, the error word) are only
+  // valid while the module stays loaded; look them up again after a device reset.
+  for (int i = 0; i < 64; ++i) {
+    g_noalloc_ptr[i] = nullptr;
+    g_noalloc_sms[i] = 0;
+  }
+  mssm::forget_device_addresses();
   if (prev >= 0) cudaSetDevice(prev);
   return st;
 }

@@ -5,10 +5,19 @@ namespace mssm {
 
 __device__ unsigned int g_device_error = 0u;
 
-// Address of this device's copy of the error word, looked up once per device
+// Address of each device's copy of the error word, looked up once per device
 // (the caller serialises launches, so the cache needs no lock of its own).
+static void* g_error_word_cache[64] = {};
+// per device: SM count once the streaming kernels' shared-memory opt-in is set (0: not yet)
+static int g_stream_sms[64] = {};
+
+void forget_device_addresses() {
+  for (void*& p : g_error_word_cache) p = nullptr;
+  for (int& v : g_stream_sms) v = 0;  // a reset also drops the kernels' attributes
+}
+
 cudaError_t device_error_word(unsigned int** out) {
-  static void* cache[64] = {};
+  void** cache = g_error_word_cache;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -23,7 +32,7 @@ cudaError_t device_error_word(unsigned int** out) {
 
 // SM count and the streaming kernels' shared-memory opt-in, once per device
 static cudaError_t stream_setup(int* sms) {
-  static int sm_cache[64] = {};
+  int* sm_cache = g_stream_sms;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

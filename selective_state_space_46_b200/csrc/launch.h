@@ -20,6 +20,9 @@ cudaError_t launch_scan_chained(const ScanArgs& a, int grid, int dtype, bool has
 cudaError_t launch_scan_fused(const ScanArgs& a, int grid, int dtype, bool has_z, bool softplus, cudaStream_t s);
 // Device address of this device's error word (cached per device).
 cudaError_t device_error_word(unsigned int** out);
+// Drops every cached device address of a module symbol (after this, the next call looks
+// them up again: a device reset may load the module at another address).
+void forget_device_addresses();
 // bulk: the state is one contiguous [rows][16] range (bulk-copy kernel), else one thread per row.
 enum class DecodePath { kStream, kBulkTile, kPerRow };
 cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, DecodePath path, cudaStream_t s);

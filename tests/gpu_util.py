@@ -50,3 +50,26 @@ def run_scan(inp, dev=None, **kw):
                                      dev["z"], dev["delta_bias"], inp.softplus, **kw)
     torch.cuda.synchronize()
     return out, last
+
+
+def check_scan_every_row(inp, out, last, zoh=False, h0=None, elems_per_block=1 << 23):
+    """Compare a whole GPU scan output with the oracle on every row, element by element.
+
+    The oracle runs on blocks of channels of one batch at a time (``oracle.scan_block``), so the
+    host holds only one block's fp64 inputs and outputs: a full-size problem costs its oracle time
+    (a few seconds on the host cores) and little memory.  Returns the worst scaled error of y and
+    of the final state."""
+    import oracle
+    block = max(1, min(inp.dim, elems_per_block // max(1, inp.length)))
+    worst_y = worst_h = 0.0
+    for b in range(inp.batch):
+        for d0 in range(0, inp.dim, block):
+            d1 = min(inp.dim, d0 + block)
+            hb = None if h0 is None else np.asarray(h0[b:b + 1, d0:d1], np.float64)
+            y_ref, h_ref = oracle.scan_block(inp, b, d0, d1, h0=hb, zoh=zoh)
+            worst_y = max(worst_y, check_close(to_f64(out[b:b + 1, d0:d1]), y_ref, inp.io_dtype,
+                                               f"y (batch {b}, channels {d0}..{d1 - 1})"))
+            if last is not None:
+                worst_h = max(worst_h, check_close(to_f64(last[b:b + 1, d0:d1]), h_ref, inp.io_dtype,
+                                                   f"last_state (batch {b}, channels {d0}..{d1 - 1})"))
+    return worst_y, worst_h

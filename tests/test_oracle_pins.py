@@ -82,21 +82,25 @@ def test_A_zero_is_prefix_sum():
 # 2. LTI case: constant dt, B, C -> causal convolution with K_k = sum_n C_n a_n^k dt B_n
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("softplus", [True, False])
-def test_lti_equals_convolution(softplus):
+@pytest.mark.parametrize("softplus,with_bias", [(True, False), (False, False), (True, True), (False, True)])
+def test_lti_equals_convolution(softplus, with_bias):
     rng = np.random.default_rng(2)
     D, L = 3, 50
     u = rng.standard_normal((1, D, L))
     A = -np.exp(rng.uniform(-2.0, 1.0, size=(D, N)))
     raw = rng.uniform(-3.0, 0.5, size=D)
+    bias = rng.uniform(0.5, 1.5, size=D) if with_bias else None
+    if with_bias and not softplus:
+        raw = raw * 0.01       # keep raw + bias positive: a stable step
     delta = np.repeat(raw[None, :, None], L, axis=2)
     b = rng.standard_normal(N)
     c = rng.standard_normal(N)
     B = np.repeat(b[None, :, None], L, axis=2)
     C = np.repeat(c[None, :, None], L, axis=2)
     Dv = rng.standard_normal(D)
-    y, _ = oracle.scan(u, delta, A, B, C, Dv, None, None, softplus)
-    dt = softplus_ref(raw) if softplus else raw
+    y, _ = oracle.scan(u, delta, A, B, C, Dv, None, bias, softplus)
+    pre = raw + (bias if with_bias else 0.0)
+    dt = softplus_ref(pre) if softplus else pre
     for d in range(D):
         k = np.arange(L)
         a = np.exp(dt[d] * A[d])                       # [N]
@@ -196,17 +200,47 @@ def test_large_delta_resets_state():
 #    composition of the per-step affine maps h -> A_bar h + B_bar x)
 # ---------------------------------------------------------------------------
 
-def test_decode_steps_reproduce_scan():
+@pytest.mark.parametrize("softplus", [True, False])
+def test_decode_steps_reproduce_scan(softplus):
     rng = np.random.default_rng(8)
     p = rand_problem(rng, 2, 5, 20)
-    y, last = oracle.scan(**p, softplus=True)
+    if not softplus:
+        # without softplus the step is raw + bias itself: keep it positive (a stable decay)
+        p["delta"] = np.abs(p["delta"]) * 0.05
+        p["delta_bias"] = rng.uniform(0.01, 0.1, size=5)
+    y, last = oracle.scan(**p, softplus=softplus)
     state = np.zeros((2, 5, N))
     for t in range(20):
         state, yt = oracle.state_update(state, p["u"][..., t], p["delta"][..., t], p["A"],
                                         p["B"][..., t], p["C"][..., t], p["D"], p["z"][..., t],
-                                        p["delta_bias"], True)
+                                        p["delta_bias"], softplus)
         np.testing.assert_allclose(yt, y[..., t], rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(state, last, rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_scan_rows_and_blocks_equal_the_whole_problem(io):
+    """oracle.scan_rows and oracle.scan_block (which slice rows' inputs and their batch's B/C and
+    widen them) give
+    exactly the rows of the whole-problem oracle: a wrong batch of B/C, a wrong channel of A, D
+    or bias, or a wrong widening would show here."""
+    import synth
+    inp = synth.make_scan_inputs(3, 9, 37, io_dtype=io, seed=41)
+    y, last = oracle.scan_inputs(inp)
+    rows = [(0, 0), (0, 8), (1, 3), (2, 0), (2, 5), (2, 8), (1, 3)]
+    ys, hs = oracle.scan_rows(inp, rows)
+    for i, (b, d) in enumerate(rows):
+        np.testing.assert_array_equal(ys[i], y[b, d])
+        np.testing.assert_array_equal(hs[i], last[b, d])
+    # oracle.scan_block: channel blocks of one batch, the same way
+    for b, d0, d1 in [(0, 0, 9), (1, 2, 7), (2, 8, 9)]:
+        yb, hb = oracle.scan_block(inp, b, d0, d1)
+        np.testing.assert_array_equal(yb[0], y[b, d0:d1])
+        np.testing.assert_array_equal(hb[0], last[b, d0:d1])
+    y_z, last_z = oracle.scan_inputs(inp, zoh=True)
+    yb, hb = oracle.scan_block(inp, 2, 1, 6, zoh=True)
+    np.testing.assert_array_equal(yb[0], y_z[2, 1:6])
+    np.testing.assert_array_equal(hb[0], last_z[2, 1:6])
 
 
 @pytest.mark.parametrize("split", [1, 7, 19])
@@ -569,19 +603,25 @@ MUTANTS = {
     "conv_window_off_by_one": ("int64_t src = t + j - (K - 1);", "int64_t src = t + j - K;"),
     "conv_bias_dropped": ("double acc = bias ? bias[d] : 0.0;", "double acc = 0.0;"),
     "conv_silu_dropped": ("silu_flag ? silu(acc) : acc;", "acc;"),
+    "decode_bias_only_with_softplus": ("double dt = dt_in[r] + (bias ? bias[d] : 0.0);\n        if (softplus_flag)\n            dt = sp_exact(dt);",
+                                       "double dt = dt_in[r];\n        if (softplus_flag)\n            dt = sp_exact(dt + (bias ? bias[d] : 0.0));"),
+    "scan_bias_only_with_softplus": ("double dt = dr[t] + (bias ? bias[d] : 0.0);",
+                                     "double dt = dr[t] + (bias && softplus_flag ? bias[d] : 0.0);"),
     "decode_bias_dropped": ("double dt = dt_in[r] + (bias ? bias[d] : 0.0);", "double dt = dt_in[r];"),
     "decode_gate_dropped": ("            y *= silu(z[r]);\n        out[r] = y;", "        out[r] = y;"),
 }
 
 PIN_CALLS = [
     test_A_zero_is_prefix_sum,
-    lambda: test_lti_equals_convolution(True),
-    lambda: test_lti_equals_convolution(False),
+    lambda: test_lti_equals_convolution(True, False),
+    lambda: test_lti_equals_convolution(False, False),
+    lambda: test_lti_equals_convolution(False, True),
     test_lti_step_input_closed_form,
     lambda: test_tiny_unrolled_sum(4, 5, 2),
     test_delta_to_zero_preserves_state,
     test_large_delta_resets_state,
-    test_decode_steps_reproduce_scan,
+    lambda: test_decode_steps_reproduce_scan(True),
+    lambda: test_decode_steps_reproduce_scan(False),
     lambda: test_split_scan_equals_scan(7),
     test_affine_composition_is_associative,
     test_linear_in_u,

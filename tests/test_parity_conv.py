@@ -59,17 +59,16 @@ def test_conv_workload_size(cuda_device):
     check_close(to_f64(out), ref_conv(x, w, b, "bf16"), "bf16", "conv out")
 
 
-def test_conv_large_workload_sampled(cuda_device):
-    """8 x 5120 x 4096 in the benchmark's launch configuration, checked on sampled rows."""
+def test_conv_large_workload_every_row(cuda_device):
+    """8 x 5120 x 4096 in the benchmark's launch configuration, every element against the
+    oracle (batch by batch, to bound host memory)."""
     import selective_state_space_46_b200 as m
     inp = synth.workload_inputs("conv_bf16_8x5120x4096", seed=0)
     out = m.causal_conv1d(to_dev(inp.x), to_dev(inp.weight), to_dev(inp.bias))
     torch.cuda.synchronize()
-    rng = np.random.default_rng(1)
-    for b, d in zip(rng.integers(0, inp.batch, 12), rng.integers(0, inp.dim, 12)):
-        got = to_f64(out[b:b + 1, d:d + 1])
-        ref = ref_conv(inp.x[b:b + 1, d:d + 1], inp.weight[d:d + 1], inp.bias[d:d + 1], "bf16")
-        check_close(got, ref, "bf16", f"conv row ({b}, {d})")
+    for b in range(inp.batch):
+        check_close(to_f64(out[b:b + 1]), ref_conv(inp.x[b:b + 1], inp.weight, inp.bias, "bf16"), "bf16",
+                    f"conv batch {b}")
 
 
 def test_conv_unaligned_rows(cuda_device):

@@ -136,3 +136,31 @@ def test_decode_steps_reproduce_scan(cuda_device, io):
     y_ref, h_ref = oracle.scan_inputs(inp)
     check_close(to_f64(y_dec), y_ref, io, "decode-chain y")
     check_close(to_f64(state), h_ref, "f32", "decode-chain state")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("decode_path", ["auto"], indirect=True)
+def test_decode_1000_successive_steps_downscaled(cuda_device, decode_path):
+    """The decode workload is timed over 1000 successive in-place steps whose per-token inputs
+    cycle through a ring of 8 draws.  The same 1000 steps on a copy with batch 4 (every channel
+    and state of the full shape): the final state against the oracle's after the same 1000
+    steps, and the outputs of the last ring's worth of steps."""
+    import selective_state_space_46_b200 as m
+    ring = [synth.workload_inputs("decode_bf16_256x5120", batch=4, step_stream=k) for k in range(8)]
+    state = to_dev(ring[0].state)
+    dring = [dev_decode(r) for r in ring]
+    st_ref = ring[0].state.astype(np.float64)
+    outs, refs = [], []
+    for k in range(1000):
+        r, dv = ring[k % 8], dring[k % 8]
+        out = torch.empty_like(dv["x"])
+        m.mssm_state_update(state, dv["x"], dv["dt"], dv["A"], dv["B"], dv["C"], dv["D"], dv["z"], out)
+        st_ref, y_ref = oracle.state_update_inputs(r, state=st_ref)
+        if k >= 992:
+            outs.append(out)
+            refs.append(y_ref)
+    torch.cuda.synchronize()
+    m.mssm_get_error()
+    for k, (o, y_ref) in enumerate(zip(outs, refs)):
+        check_close(to_f64(o), y_ref, "bf16", f"y step {992 + k}")
+    check_close(to_f64(state), st_ref, "f32", "state after 1000 steps")

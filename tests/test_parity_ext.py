@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from gpu_util import check_close, dev_scan_inputs, to_dev, to_f64
+from gpu_util import check_close, check_scan_every_row, dev_scan_inputs, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -140,29 +140,11 @@ def test_zoh_zero_A(schedule):
         check_close(to_f64(last), h_ref, "f32", "last_state")
 
 
-def test_zoh_sampled_full_size():
-    """The 8 x 5120 x 4096 workload with the zero-order hold, checked on sampled rows."""
-    import selective_state_space_46_b200 as m
+def test_zoh_full_size_every_row():
+    """The 8 x 5120 x 4096 workload with the zero-order hold, every element against the oracle."""
     inp = synth.workload_inputs("scan_bf16_8x5120x4096")
     out, last = _run_ex(inp, zoh=True)
-    rng = np.random.default_rng(1)
-    rows = [(b, int(d)) for b in range(inp.batch) for d in rng.choice(inp.dim, 3, replace=False)]
-    ys, hs = [], []
-    from synth import to_f64 as widen
-    for b, d in rows:
-        sl = lambda name: None if getattr(inp, name) is None else widen(getattr(inp, name)[b:b + 1, d:d + 1],
-                                                                          inp.io_dtype)
-        y, h = oracle.scan(sl("u"), sl("delta"), inp.A[d:d + 1].astype(np.float64),
-                           widen(inp.B[b:b + 1], inp.io_dtype), widen(inp.C[b:b + 1], inp.io_dtype),
-                           None if inp.D is None else inp.D[d:d + 1].astype(np.float64), sl("z"),
-                           None if inp.delta_bias is None else inp.delta_bias[d:d + 1].astype(np.float64),
-                           inp.softplus, zoh=True)
-        ys.append(y[0, 0])
-        hs.append(h[0, 0])
-    got_y = np.stack([to_f64(out[b, d]) for b, d in rows])
-    got_h = np.stack([to_f64(last[b, d]) for b, d in rows])
-    check_close(got_y, np.stack(ys), "bf16", "y")
-    check_close(got_h, np.stack(hs), "bf16", "last_state")
+    check_scan_every_row(inp, out, last, zoh=True)
 
 
 @pytest.mark.parametrize("path", ["stream", "bulk_tile", "per_row"])

@@ -1,8 +1,8 @@
 """GPU parity of mssm_selective_scan_fwd against the fp64 oracle.
 
-Small and medium problems are compared element by element; the full-size
-prefill shapes are run whole on the GPU in the launch configuration the
-benchmark uses and checked on sampled rows that the oracle computes one by one.
+Every problem, the full-size prefill shapes included, is compared element by
+element; the full-size shapes run whole on the GPU in the launch configuration
+the benchmark uses, and the oracle checks them block by block of channels.
 """
 import numpy as np
 import pytest
@@ -10,7 +10,7 @@ import torch
 
 import oracle
 import synth
-from gpu_util import check_close, dev_scan_inputs, run_scan, to_dev, to_f64
+from gpu_util import check_close, check_scan_every_row, dev_scan_inputs, run_scan, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -71,30 +71,21 @@ def test_workload_bf16_2x1536x2048_each_schedule(schedule):
     m.mssm_get_error()
 
 
-def _sampled(name, rows_per_batch=6, seed=0):
-    inp = synth.workload_inputs(name)
+@pytest.mark.slow
+def test_workload_bf16_8x5120x4096_every_row():
+    """The Mamba-2.8B-shaped prefill in the benchmark's launch configuration, every element of y
+    and of the final state against the oracle."""
+    inp = synth.workload_inputs("scan_bf16_8x5120x4096")
     out, last = run_scan(inp)
-    rng = np.random.default_rng(seed)
-    rows = []
-    for b in range(inp.batch):
-        ds = set(rng.choice(inp.dim, size=rows_per_batch, replace=False).tolist())
-        ds |= {0, inp.dim - 1}
-        rows += [(b, int(d)) for d in sorted(ds)]
-    y_ref, h_ref = oracle.scan_rows(inp, rows)
-    bi = torch.tensor([r[0] for r in rows], device=out.device)
-    di = torch.tensor([r[1] for r in rows], device=out.device)
-    check_close(to_f64(out[bi, di]), y_ref, inp.io_dtype, "y")
-    check_close(to_f64(last[bi, di]), h_ref, inp.io_dtype, "last_state")
+    check_scan_every_row(inp, out, last)
 
 
 @pytest.mark.slow
-def test_workload_bf16_8x5120x4096_sampled():
-    _sampled("scan_bf16_8x5120x4096", rows_per_batch=4)
-
-
-@pytest.mark.slow
-def test_workload_bf16_1x2048x131072_sampled():
-    _sampled("scan_bf16_1x2048x131072", rows_per_batch=10)
+def test_workload_bf16_1x2048x131072_every_row():
+    """The long-context workload (the benchmark's default), every element against the oracle."""
+    inp = synth.workload_inputs("scan_bf16_1x2048x131072")
+    out, last = run_scan(inp)
+    check_scan_every_row(inp, out, last)
 
 
 # ---------------------------------------------------------------------------

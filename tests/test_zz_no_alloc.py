@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from gpu_util import TOL, dev_scan_inputs
 
@@ -38,6 +39,19 @@ def _close(got, ref, io_dtype):
     assert float(err.max()) <= tol, float(err.max())
 
 
+def _check(inp, m, calls=2):
+    """`calls` no-allocation scans in a row of one problem: each against the allocating scan and
+    against the fp64 oracle (so a fault shared by both entry points, such as in the launch
+    planning or the workspace layout, is caught too)."""
+    y_o, h_o = oracle.scan_inputs(inp)
+    for _ in range(calls):
+        (y_ref, h_ref), (y_na, h_na) = _scan_both(inp, m)
+        _close(y_na, y_ref, inp.io_dtype)
+        _close(h_na, h_ref, inp.io_dtype)
+        _close(y_na, y_o, inp.io_dtype)
+        _close(h_na, h_o, inp.io_dtype)
+
+
 def test_noalloc_matches_the_allocating_scan_on_two_calls_in_a_row(cuda_device):
     import selective_state_space_46_b200 as m
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
@@ -51,9 +65,7 @@ def test_noalloc_matches_the_allocating_scan_on_two_calls_in_a_row(cuda_device):
         for inp in (first, second):
             if inp is second:
                 m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 128)
-            (y_ref, h_ref), (y_na, h_na) = _scan_both(inp, m)
-            _close(y_na, y_ref, inp.io_dtype)
-            _close(h_na, h_ref, inp.io_dtype)
+            _check(inp, m, calls=1)
     finally:
         m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
 
@@ -81,7 +93,22 @@ def test_noalloc_chained_schedule_matches(cuda_device):
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
     inp = synth.make_scan_inputs(2, 9600, 1000, io_dtype="bf16", seed=6)
     assert m.mssm_scan_plan(inp.batch, inp.dim, inp.length)["schedule"] == "chained"
-    for _ in range(2):
-        (y_ref, h_ref), (y_na, h_na) = _scan_both(inp, m)
-        _close(y_na, y_ref, inp.io_dtype)
-        _close(h_na, h_ref, inp.io_dtype)
+    _check(inp, m, calls=2)
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_noalloc_fused_schedule_two_calls(cuda_device, io):
+    """The fused look-back schedule keeps the most in the fixed array: per-chunk flags, chunk
+    sums, summaries and end states.  Forced, with short chunks, twice in a row: the second call
+    finds the first call's published flags in the array and must clear them first."""
+    import selective_state_space_46_b200 as m
+    m.mssm_set_option(m.MSSM_OPT_SCHEDULE, m.SCHEDULES["fused"])
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 64)
+    try:
+        inp = synth.make_scan_inputs(2, 100, 700, io_dtype=io, seed=8, delta_range=(1e-4, 1e-2))
+        assert m.mssm_scan_plan(inp.batch, inp.dim, inp.length)["schedule"] == "fused"
+        _check(inp, m, calls=2)
+        m.mssm_get_error()   # no bounded look-back wait gave up
+    finally:
+        m.mssm_set_option(m.MSSM_OPT_SCHEDULE, 0)
+        m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 0)
