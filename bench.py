@@ -209,8 +209,8 @@ def recorded_traffic(kernel: str, workload: str, plan: str | None = None):
 def plan_string(plan: dict | None) -> str | None:
     if not plan:
         return None
-    return (f"{plan['schedule']} rows_per_cta={plan['rows_per_cta']} chunk_len={plan['chunk_len']} "
-            f"n_chunks={plan['n_chunks']}")
+    return (f"{plan['schedule']} rows_per_cta={plan['rows_per_cta']} rows_per_thread={plan.get('rows_per_thread', 1)} "
+            f"chunk_len={plan['chunk_len']} n_chunks={plan['n_chunks']}")
 
 
 class ClockSampler:
@@ -410,6 +410,7 @@ def run_mssm(args):
     seed = rank_seed(rank)
     m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, args.chunk_len)
     m.mssm_set_option(m.MSSM_OPT_ROWS_PER_CTA, args.rows_per_cta)
+    m.mssm_set_option(m.MSSM_OPT_ROWS_PER_THREAD, args.rows_per_thread)
     m.mssm_set_option(m.MSSM_OPT_FORCE_GENERAL_A, 1 if args.general_a else 0)
     m.mssm_set_option(m.MSSM_OPT_DECODE_PATH, m.DECODE_PATHS.get(args.decode_path, 0))
     m.mssm_set_option(m.MSSM_OPT_SCHEDULE, m.SCHEDULES.get(args.schedule, 0))
@@ -454,7 +455,7 @@ def run_mssm(args):
                   "discretization": "zero-order hold" if args.zoh else "euler",
                   "chunk_len": args.chunk_len or "auto",
                   "plan": m.mssm_scan_plan(nstate, inp.dim, max_seqlen,
-                                           total_len=inp.length if varlen else -1)}
+                                           total_len=inp.length if varlen else -1, io_dtype=inp.io_dtype)}
         if varlen:
             config.update({"sequences": nstate, "max_seqlen": max_seqlen, "packed_length": inp.length})
         metric, unit = METRIC, "elems/s"
@@ -818,12 +819,14 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--chunk-len", type=int, default=0, help="length split (0: automatic; multiple of 64)")
-    ap.add_argument("--rows-per-cta", type=int, default=0, choices=[0, 32, 64],
+    ap.add_argument("--rows-per-cta", type=int, default=0, choices=[0, 32, 64, 128],
                     help="channels per row tile of the scan (0: automatic)")
+    ap.add_argument("--rows-per-thread", type=int, default=0, choices=[0, 1, 2],
+                    help="channels per thread of the scan kernels (0: automatic; 2: bf16 I/O only)")
     ap.add_argument("--decode-path", choices=["auto", "stream", "bulk_tile", "per_row"], default="auto",
                     help="decode kernel (MSSM_OPT_DECODE_PATH)")
     ap.add_argument("--zoh", action="store_true", help="zero-order-hold discretisation (scan workloads)")
-    ap.add_argument("--schedule", choices=["auto", "forward", "summaries+forward", "chained", "fused"],
+    ap.add_argument("--schedule", choices=["auto", "forward", "summaries+forward", "chained", "fused", "split"],
                     default="auto", help="force a scan schedule (MSSM_OPT_SCHEDULE)")
     ap.add_argument("--backward", action="store_true", help="time the backward scan instead (scan workloads)")
     ap.add_argument("--general-a", action="store_true",

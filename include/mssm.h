@@ -324,25 +324,34 @@ mssm_status mssm_get_error(void *stream);
  *   MSSM_OPT_CHUNK_LEN (value 0, or a positive multiple of 64): length of the
  *     chunks a sequence is split into (a value >= L means no split); 0 restores
  *     the automatic choice.
- *   MSSM_OPT_SCHEDULE (value 0..4): 0 automatic; otherwise force a schedule of
+ *   MSSM_OPT_SCHEDULE (value 0..5): 0 automatic; otherwise force a schedule of
  *     mssm_scan_plan (value = schedule + 1: 1 forward only, no split; 2 summaries
- *     + forward; 3 chained; 4 fused single pass).  A forced split schedule needs
- *     L > 64; otherwise the plan falls back to forward only.  The fused schedule
- *     takes plain batches only (packed sequences fall back to the automatic plan).
+ *     + forward; 3 chained; 4 fused single pass; 5 split chunks).  A forced split
+ *     schedule needs L > 64; otherwise the plan falls back to forward only.  The
+ *     fused and split-chunk schedules take plain batches only, and the split-chunk
+ *     schedule chunk lengths that are multiples of 256 (4 sub-segments of whole
+ *     64-step blocks); otherwise the plan falls back to forward only.
  *   MSSM_OPT_KERNEL_TIMING (value 0/1): when 1, every kernel launch is bracketed
  *     by two CUDA events recorded on the caller's stream (see mssm_kernel_stats).
  *   MSSM_OPT_DECODE_PATH (value 0..3): the state-update kernel.  0 automatic:
  *     the first of 1, 2, 3 whose layout conditions hold.  1 persistent streaming
- *     kernel (per CTA a block of 128 channels and a ring of bulk-copied tiles);
+ *     kernel (per warp a block of 32 channels and a ring of bulk-copied tiles);
  *     needs the state as one contiguous, 16-byte aligned [Bt, D, 16] range, x,
  *     dt and z with unit channel stride and 16-byte aligned batch rows, D a
  *     multiple of 8 (bf16) or 4 (f32), and B, C with unit n stride and 16-byte
  *     aligned batch rows.  2 one bulk-copied tile of 256 rows per CTA; needs the
  *     contiguous state.  3 one thread per row, any layout.  A forced path whose
  *     conditions fail falls back to the next one that holds.
- *   MSSM_OPT_ROWS_PER_CTA (value 0, 32 or 64): channels per row tile (CTA) of the
- *     scan plan, one channel per thread; 0 automatic.  64-channel tiles take the
- *     forward or summaries + forward schedule only.
+ *   MSSM_OPT_ROWS_PER_CTA (value 0, 32, 64 or 128): channels per row tile of the
+ *     scan plan; 0 automatic.  With one channel per thread a tile is one CTA of
+ *     32 or 64 threads; with two channels per thread (bf16 I/O only) a 64- or
+ *     128-channel tile is a CTA of 32 or 64 threads.  The chained, fused and
+ *     split-chunk schedules take tiles of one warp (32 channels, or 64 with two
+ *     per thread).
+ *   MSSM_OPT_ROWS_PER_THREAD (value 0, 1 or 2): channels each thread of the scan
+ *     kernels keeps in registers (each step's B and C are then read once for
+ *     all of them); 0 automatic.  Two per thread exist for bf16 I/O only; for
+ *     fp32 I/O a forced 2 means 1.
  *   MSSM_OPT_TEST_HOOKS (value 0/1, for testing failure detection only): when 1,
  *     the chained scan schedule publishes no carried states, so every chunk after
  *     the first gives up its bounded wait (about 0.5 s), runs from a zero state
@@ -357,20 +366,26 @@ typedef enum {
     MSSM_OPT_SCHEDULE = 4,
     MSSM_OPT_DECODE_PATH = 5,
     MSSM_OPT_TEST_HOOKS = 6,
-    MSSM_OPT_ROWS_PER_CTA = 7
+    MSSM_OPT_ROWS_PER_CTA = 7,
+    MSSM_OPT_ROWS_PER_THREAD = 8
 } mssm_option;
 mssm_status mssm_set_option(int option, int64_t value);
 
 /*
  * Host-only query of the launch plan mssm_selective_scan_fwd would use for a
- * [Bt, D, L] problem on a GPU with sm_count SMs (sm_count <= 0: the current
- * device, or 148 when there is none): channels per CTA (32 or 64), chunk length,
+ * [Bt, D, L] problem with bf16 I/O on a GPU with sm_count SMs (sm_count <= 0:
+ * the current device, or 148 when there is none): channels per row tile (32, 64
+ * or 128), chunk length,
  * number of chunks (1 = no split) and schedule: 0 = one forward kernel,
  * 1 = chunk-summary kernel + forward kernel, 2 = persistent chained forward
  * kernel (chunks of a tile run in order, each starting from the state the
  * previous one published), 3 = fused single pass (one persistent kernel: every
  * chunk summarises itself, looks back over the published summaries of the
- * chunks before it for its start state, then runs forward).  Honours MSSM_OPT_CHUNK_LEN.  Launches nothing; any
+ * chunks before it for its start state, then runs forward), 4 = split chunks
+ * (one persistent kernel of 4-warp CTAs: the warps summarise the 4 sub-segments
+ * of a chunk, combine the summaries in shared memory with the chunk's incoming
+ * state, which the previous chunk hands over, and sweep their sub-segments
+ * forward).  Honours MSSM_OPT_CHUNK_LEN.  Launches nothing; any
  * output pointer may be NULL.
  */
 mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int *rows_per_cta,
@@ -382,6 +397,30 @@ mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int *
  */
 mssm_status mssm_scan_plan_packed(int64_t S, int64_t D, int64_t max_seqlen, int64_t total_len, int sm_count,
                                   int *rows_per_cta, int64_t *chunk_len, int64_t *n_chunks, int *schedule);
+
+/* The full launch plan of a scan (mssm_scan_plan_query). */
+typedef struct {
+    int32_t struct_size;      /* sizeof(mssm_scan_plan_info), set by the caller */
+    int32_t schedule;         /* 0..4, as mssm_scan_plan reports it */
+    int32_t rows_per_cta;     /* channels per row tile: 32, 64 or 128 */
+    int32_t rows_per_thread;  /* channels per thread: 1 or 2 (2: bf16 I/O only) */
+    int64_t chunk_len;        /* steps per chunk of the length split */
+    int64_t n_chunks;         /* chunks per sequence (1 = no split) */
+    int32_t grid;             /* persistent CTAs of the chained and fused schedules, else 0 */
+    int32_t reserved;
+} mssm_scan_plan_info;
+
+/*
+ * The plan mssm_selective_scan_fwd (and _ex) would use for S sequences of at
+ * most max_seqlen steps (total_len: their summed length for packed sequences,
+ * < 0 for S full sequences) of D channels with I/O dtype io_dtype (MSSM_F32 or
+ * MSSM_BF16) on a GPU with sm_count SMs (<= 0: the current device, or 148).
+ * Honours the tuning options below.  Host only; launches nothing.  Returns
+ * MSSM_ERR_INVALID_ARG for a null info, a struct_size below this version's
+ * size, negative sizes or another dtype.
+ */
+mssm_status mssm_scan_plan_query(int64_t S, int64_t D, int64_t max_seqlen, int64_t total_len, int io_dtype,
+                                 int sm_count, mssm_scan_plan_info *info);
 
 /* Kernel kinds counted by mssm_kernel_stats. */
 typedef enum {

@@ -22,7 +22,7 @@ __all__ = [
     "mssm_get_error", "mssm_set_option", "mssm_shutdown", "mssm_version", "mssm_status_string",
     "mssm_last_error", "selective_scan_fwd", "state_update", "lib_path",
     "MSSM_OPT_FORCE_GENERAL_A", "MSSM_OPT_CHUNK_LEN", "MSSM_OPT_KERNEL_TIMING", "MSSM_OPT_SCHEDULE", "SCHEDULES",
-    "MSSM_OPT_DECODE_PATH", "DECODE_PATHS", "MSSM_OPT_TEST_HOOKS", "MSSM_OPT_ROWS_PER_CTA", "MSSM_ERR_TIMEOUT", "mssm_kernel_stats", "mssm_scan_plan",
+    "MSSM_OPT_DECODE_PATH", "DECODE_PATHS", "MSSM_OPT_TEST_HOOKS", "MSSM_OPT_ROWS_PER_CTA", "MSSM_OPT_ROWS_PER_THREAD", "MSSM_ERR_TIMEOUT", "mssm_kernel_stats", "mssm_scan_plan",
     "mssm_selective_scan_fwd_ex", "MSSM_DISC_EULER", "MSSM_DISC_ZOH",
     "mssm_causal_conv1d_fwd", "mssm_causal_conv1d_update", "causal_conv1d", "causal_conv1d_update",
     "mssm_selective_scan_bwd", "selective_scan_bwd",
@@ -42,8 +42,9 @@ MSSM_OPT_FORCE_GENERAL_A, MSSM_OPT_CHUNK_LEN, MSSM_OPT_KERNEL_TIMING, MSSM_OPT_S
 MSSM_OPT_DECODE_PATH = 5
 MSSM_OPT_TEST_HOOKS = 6
 MSSM_OPT_ROWS_PER_CTA = 7
+MSSM_OPT_ROWS_PER_THREAD = 8
 MSSM_DISC_EULER, MSSM_DISC_ZOH = 0, 1
-SCHEDULES = {"forward": 1, "summaries+forward": 2, "chained": 3, "fused": 4}
+SCHEDULES = {"forward": 1, "summaries+forward": 2, "chained": 3, "fused": 4, "split": 5}
 DECODE_PATHS = {"stream": 1, "bulk_tile": 2, "per_row": 3}
 KERNEL_KINDS = ("scan_chunk_state", "scan_out", "state_update", "conv", "scan_bwd")
 
@@ -98,6 +99,17 @@ _lib.mssm_scan_plan_packed.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_
                                        ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int64),
                                        ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int)]
 _lib.mssm_scan_plan_packed.restype = ctypes.c_int
+
+
+class mssm_scan_plan_info(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_int32), ("schedule", ctypes.c_int32), ("rows_per_cta", ctypes.c_int32),
+                ("rows_per_thread", ctypes.c_int32), ("chunk_len", ctypes.c_int64), ("n_chunks", ctypes.c_int64),
+                ("grid", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_lib.mssm_scan_plan_query.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                      ctypes.c_int, ctypes.POINTER(mssm_scan_plan_info)]
+_lib.mssm_scan_plan_query.restype = ctypes.c_int
 
 
 class MssmError(RuntimeError):
@@ -172,14 +184,17 @@ def mssm_kernel_stats(reset: bool = False) -> dict:
     return {k: {"launches": launches[i], "timed": timed[i], "ms": ms[i]} for i, k in enumerate(KERNEL_KINDS)}
 
 
-def mssm_scan_plan(Bt: int, D: int, L: int, sm_count: int = 0, total_len: int = -1) -> dict:
+def mssm_scan_plan(Bt: int, D: int, L: int, sm_count: int = 0, total_len: int = -1, io_dtype: str = "bf16") -> dict:
     """Launch plan of the scan for a [Bt, D, L] problem, or for Bt packed sequences of at most
-    L steps summing to ``total_len`` (host only, launches nothing)."""
-    rows, seg, nseg, sched = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int()
-    _check(_lib.mssm_scan_plan_packed(Bt, D, L, total_len, sm_count, ctypes.byref(rows), ctypes.byref(seg),
-                                      ctypes.byref(nseg), ctypes.byref(sched)))
-    return {"rows_per_cta": rows.value, "chunk_len": seg.value, "n_chunks": nseg.value,
-            "schedule": ("forward", "summaries+forward", "chained", "fused")[sched.value]}
+    L steps summing to ``total_len``, with ``io_dtype`` ('bf16' or 'f32') I/O (mssm_scan_plan_query;
+    host only, launches nothing)."""
+    info = mssm_scan_plan_info()
+    info.struct_size = ctypes.sizeof(mssm_scan_plan_info)
+    dt = {"bf16": MSSM_BF16, "f32": MSSM_F32}[io_dtype]
+    _check(_lib.mssm_scan_plan_query(Bt, D, L, total_len, dt, sm_count, ctypes.byref(info)))
+    return {"rows_per_cta": info.rows_per_cta, "rows_per_thread": info.rows_per_thread,
+            "chunk_len": info.chunk_len, "n_chunks": info.n_chunks, "grid": info.grid,
+            "schedule": ("forward", "summaries+forward", "chained", "fused", "split")[info.schedule]}
 
 
 def mssm_get_error(stream=None) -> None:

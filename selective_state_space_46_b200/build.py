@@ -72,8 +72,21 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         return obj
 
     srcs = sources()
-    with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
-        objs = list(ex.map(compile_one, srcs))
+    headers = [p for p in _inputs() if not p.endswith(".cu")]
+    newest_header = max((os.path.getmtime(p) for p in headers), default=0.0)
+
+    def stale(src):
+        # an object is rebuilt when its source, any header or this script is newer than it,
+        # or when extra flags are given (they may change the code)
+        obj = os.path.join(BUILD_DIR, os.path.basename(src).replace(".cu", ".o"))
+        if force or extra_flags or not os.path.exists(obj):
+            return True
+        return os.path.getmtime(obj) < max(os.path.getmtime(src), newest_header)
+
+    todo = [src for src in srcs if stale(src)]
+    with ThreadPoolExecutor(max_workers=max(1, min(len(todo), os.cpu_count() or 1))) as ex:
+        list(ex.map(compile_one, todo))
+    objs = [os.path.join(BUILD_DIR, os.path.basename(src).replace(".cu", ".o")) for src in srcs]
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     if verbose:

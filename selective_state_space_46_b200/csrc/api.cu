@@ -36,7 +36,8 @@ std::mutex g_mu;
 int g_force_general = 0;
 int64_t g_chunk_len = 0;
 int g_schedule = -1;
-int g_rows_per_cta = 0;  // 0 automatic, else 32 or 64
+int g_rows_per_cta = 0;     // 0 automatic, else 32, 64 or 128
+int g_rows_per_thread = 0;  // 0 automatic, else 1 or 2
 int g_decode_path = 0;  // MSSM_OPT_DECODE_PATH
 int g_test_hooks = 0;   // MSSM_OPT_TEST_HOOKS  // -1 automatic, else the forced LaunchShape mode
 
@@ -146,10 +147,15 @@ bool same_ptr(const mssm_tensor* a, const mssm_tensor* b) {
 // Launch shape of the scan.
 //   mode 0: one forward kernel over whole sequences (nseg == 1)
 //   mode 1: chunk-summary kernel + forward kernel over nseg chunks
-//   mode 2: persistent chained forward kernel (32-row tiles, `grid` CTAs)
+//   mode 2: persistent chained forward kernel (`grid` one-warp CTAs)
+//   mode 3: fused single pass (`grid` one-warp CTAs)
+//   mode 4: split chunks (`grid` persistent CTAs of kSplitWarps warps; a chunk of seg steps is
+//           kSplitWarps sub-segments summarised, combined and swept by one warp each)
+// rows: channels per row tile; rpt: rows per thread (rows / rpt threads per CTA).
 struct LaunchShape {
   int mode;
   int rows;
+  int rpt;
   int64_t seg, nseg;
   int grid;
 };
@@ -159,48 +165,91 @@ int64_t round_seg(int64_t v) {
   return v < mssm::kSegQuant ? mssm::kSegQuant : v;
 }
 
-// Cost model, in cycles of the busiest SM sub-partition (SMSP).  Measured on
-// B200: a warp-step of the forward kernel issues about kOut instructions and
-// of the summary kernel kSum; an SMSP sustains kIpc1 instructions per cycle
-// with one warp and kIpc2 with two or more (more warps do not raise it).  A
-// CTA costs kStart cycles of start-up latency per wave, a launch kLaunch, a
-// chained work item kItem, and the carry fold kFold per chunk.  Grid kernels
-// run their CTAs in waves of at most kMaxCta per SM (register limited) and
-// put ceil(warps / 4) warps on the busiest SMSP.
+// Cost model, in cycles of the busiest SM sub-partition (SMSP).  Measured on B200:
+// cycles per 32 elements one SMSP spends on the forward sweep (cyc_out) and on the
+// chunk summaries (cyc_sum), by rows per thread and by the warps resident on the SMSP
+// (one warp cannot hide its own latencies; two or more reach the same rate).  A CTA
+// costs kStart cycles of start-up latency per wave, a launch kLaunch, a chained work
+// item kItem, and the carry fold kFold per chunk.  Grid kernels run their CTAs in waves
+// of at most out_ctas per SM (register and shared-memory limited) and put
+// ceil(warps / 4) warps on the busiest SMSP.
 //
 // Packed sequences (total_len >= 0: the sum of the Bt sequence lengths, each at most L)
 // count only the chunks that hold steps, about total_len / seg + Bt per row tile column,
-// and pay the forward-sweep summary (kSumFwd).  A chained tile runs its chunks one after
-// another, so the chained schedule costs at least nseg items, which is what rules it out
-// for a few long sequences among short ones.
+// and pay the forward-sweep summary.  A chained tile runs its chunks one after another,
+// so the chained schedule costs at least nseg items, which is what rules it out for a
+// few long sequences among short ones.
+struct TileKind {
+  int rows, rpt;
+};
+// Measured on B200 (bf16 I/O, gate, softplus + bias, structured A), SMSP cycles per 32
+// elements by the warps resident on the busiest SMSP: forward sweep, one row per thread,
+// about 160 with two warps (the chained kernel at 8 per SM), 147 with four (64-row CTAs at
+// 16 per SM); two rows per thread 150 with three or more but 221 with one (half the warps
+// for the same rows); chunk summaries 86 (one row per thread) and 95 (two).  One warp per
+// SMSP is extrapolated.  The split-chunk schedule costs a forward sweep, a summary and about 14
+// cycles of composition and hand-over per 32 elements.
+double cyc_out(int rpt, int64_t k) {
+  if (rpt == 1) return k <= 1 ? 190.0 : k == 2 ? 160.0 : k == 3 ? 155.0 : 147.0;
+  return k <= 1 ? 221.0 : k == 2 ? 185.0 : 150.0;
+}
+double cyc_sum(int rpt, int64_t k, bool fwd_sweep) {
+  if (fwd_sweep) return cyc_out(rpt, k) * 0.8;
+  if (rpt == 1) return k <= 1 ? 110.0 : k == 2 ? 95.0 : 86.0;
+  return k <= 1 ? 120.0 : k == 2 ? 105.0 : 95.0;
+}
+constexpr double kSplitCombine = 14.0;
+int out_ctas(int rows, int rpt) {  // resident CTAs per SM of the grid kernels
+  if (rpt == 1) return rows == 32 ? 9 : 8;
+  return rows == 64 ? 12 : 6;
+}
+
 LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forced_seg, int forced_mode,
-                         int forced_rows, int64_t total_len = -1) {
-  constexpr double kOut = 96.0, kSum = 55.0, kSumFwd = 70.0, kIpc1 = 0.6, kIpc2 = 0.7;
-  constexpr double kStart = 4000.0, kLaunch = 6000.0, kItem = 4000.0, kFold = 200.0;
-  auto ipc = [&](int64_t k) { return k <= 1 ? kIpc1 : kIpc2; };
-  auto grid_time = [&](int64_t ctas, int rows, double steps, double instr) {
-    const int64_t max_cta = rows == 32 ? 12 : 8;
+                         int forced_rows, int forced_rpt, int dtype, int64_t total_len = -1) {
+  // kCta: each CTA's own start (its first B/C stage and input blocks arriving), paid by every
+  // warp of the busiest SMSP in turn
+  constexpr double kStart = 4000.0, kLaunch = 6000.0, kItem = 4000.0, kFold = 200.0, kCta = 3000.0;
+  const bool packed = total_len >= 0;
+  // forced tile shapes that do not exist fall back to the nearest that does
+  if (dtype != MSSM_BF16) {
+    if (forced_rpt == 2) forced_rpt = 1;
+    if (forced_rows == 128) forced_rows = 64;
+  }
+  if ((forced_rows == 32 && forced_rpt == 2) || (forced_rows == 128 && forced_rpt == 1)) forced_rpt = 0;
+  // row tile kinds: two rows per thread are built for bf16 I/O only, and are planned only
+  // when forced (measured no faster than one row per thread on any benchmark shape)
+  std::vector<TileKind> kinds = {{32, 1}, {64, 1}};
+  if (dtype == MSSM_BF16 && (forced_rpt == 2 || forced_rows == 128)) {
+    kinds.push_back({64, 2});
+    kinds.push_back({128, 2});
+  }
+  auto grid_time = [&](int64_t ctas, const TileKind& tk, double steps, bool sum) {
+    const int nt = tk.rows / tk.rpt;
+    const int64_t max_cta = out_ctas(tk.rows, tk.rpt);
     const int64_t on_sm = (ctas + sms - 1) / sms;
     const int64_t waves = (on_sm + max_cta - 1) / max_cta;
     const int64_t resident = on_sm < max_cta ? on_sm : max_cta;
-    const int64_t k = (resident * (rows / 32) + 3) / 4;
-    return double(waves) * (double(k) * steps * instr / ipc(k) + kStart) + kLaunch;
+    const int64_t k = (resident * (nt / 32) + 3) / 4;
+    const double cyc = sum ? cyc_sum(tk.rpt, k, packed) : cyc_out(tk.rpt, k);
+    return double(waves) * (double(k) * (steps * tk.rpt * cyc + kCta) + kStart) + kLaunch;
   };
-  LaunchShape best{0, forced_rows ? forced_rows : 32, L > 0 ? L : 1, 1, 0};
+  const int def_rows = forced_rows ? forced_rows : (forced_rpt == 2 ? 64 : 32);
+  const int def_rpt = forced_rpt ? forced_rpt : (def_rows == 128 ? 2 : 1);
+  LaunchShape best{0, def_rows, def_rpt, L > 0 ? L : 1, 1, 0};
   double best_cost = -1.0;
-  if (forced_mode == 0) return LaunchShape{0, forced_rows ? forced_rows : 32, L > 0 ? L : 1, 1, 0};
   auto consider = [&](const LaunchShape& sh, double cost) {
-    if (forced_mode > 0 && sh.mode != forced_mode) return;
+    if (forced_mode >= 0 && sh.mode != forced_mode) return;
     if (best_cost < 0.0 || cost < best_cost * 0.999) {
       best_cost = cost;
       best = sh;
     }
   };
-  const bool packed = total_len >= 0;
-  for (int rows : {32, 64}) {
-    if (forced_rows && rows != forced_rows) continue;
-    const int64_t tpb = (D + rows - 1) / rows;
+  for (const TileKind& tk : kinds) {
+    if (forced_rows && tk.rows != forced_rows) continue;
+    if (forced_rpt && tk.rpt != forced_rpt) continue;
+    const int64_t tpb = (D + tk.rows - 1) / tk.rows;
     const int64_t tiles = Bt * tpb;
+    const bool one_warp = tk.rows / tk.rpt == 32;  // tile kinds of the persistent kernels
     for (int64_t want = 1; want <= 64; ++want) {
       int64_t seg = forced_seg > 0 ? forced_seg : round_seg((L + want - 1) / want);
       int64_t nseg = L > 0 ? (L + seg - 1) / seg : 1;
@@ -208,36 +257,47 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
         seg *= 2;
         nseg = (L + seg - 1) / seg;
       }
+      if (forced_mode == 0) nseg = 1, seg = L > 0 ? L : 1;
       // CTAs (items) that hold steps; the rest of a packed grid exits at once
       int64_t out_items = tiles * nseg, sum_items = tiles * (nseg - 1);
       if (packed) {
         out_items = std::min<int64_t>(out_items, tpb * ((total_len + seg - 1) / seg + Bt));
         sum_items = std::min<int64_t>(sum_items, tpb * (total_len / seg));
       }
-      double cost = grid_time(out_items, rows, double(seg), kOut);
-      if (nseg > 1)
-        cost += grid_time(sum_items, rows, double(seg), packed ? kSumFwd : kSum) + kFold * double(nseg);
-      consider(LaunchShape{nseg > 1 ? 1 : 0, rows, seg, nseg, 0}, cost);
-      // fused single pass (forced only, until measured): 32-row tiles, persistent one-warp CTAs
-      if (rows == 32 && nseg > 1 && forced_mode == 3 && !packed) {
-        consider(LaunchShape{3, 32, seg, nseg, int(std::min<int64_t>(tiles * nseg, 8 * int64_t(sms)))}, 0.0);
-      }
-      // chained: 32-row tiles, at most 8 one-warp CTAs per SM and never more CTAs than tiles
-      if (rows == 32 && nseg > 1 && forced_mode == 2 && tiles < 4 * int64_t(sms)) {
-        consider(LaunchShape{2, 32, seg, nseg, int(std::min<int64_t>(tiles, 8 * int64_t(sms)))}, 0.0);
-      }
-      if (rows == 32 && nseg > 1) {
-        const int64_t per_sm = tiles / sms < 8 ? tiles / sms : 8;
+      double cost = grid_time(out_items, tk, double(seg), false);
+      if (nseg > 1) cost += grid_time(sum_items, tk, double(seg), true) + kFold * double(nseg);
+      consider(LaunchShape{nseg > 1 ? 1 : 0, tk.rows, tk.rpt, seg, nseg, 0}, cost);
+      if (one_warp && nseg > 1) {
+        const int64_t cap = int64_t(tk.rpt == 1 ? 8 : 12) * sms;  // resident one-warp CTAs
+        // fused single pass (forced only): persistent one-warp CTAs
+        if (forced_mode == 3 && !packed)
+          consider(LaunchShape{3, tk.rows, tk.rpt, seg, nseg, int(std::min<int64_t>(tiles * nseg, cap))}, 0.0);
+        // chained, forced: never more CTAs than tiles
+        if (forced_mode == 2 && tiles < cap)
+          consider(LaunchShape{2, tk.rows, tk.rpt, seg, nseg, int(std::min<int64_t>(tiles, cap))}, 0.0);
+        // split chunks (forced only: measured slower than summaries + forward on every
+        // benchmark shape): a chunk is kSplitWarps sub-segments of whole summary blocks
+        if (forced_mode == 4 && !packed && seg % (mssm::kSplitWarps * mssm::kSegQuant) == 0) {
+          const int64_t grid = std::min<int64_t>(tiles * nseg, int64_t(3) * sms);
+          const int64_t k = 3;  // warps per SMSP (3 CTAs of 4 warps per SM)
+          const int64_t rounds = (tiles * nseg + grid - 1) / grid;
+          const double sub = double(seg) / mssm::kSplitWarps;
+          const double item =
+              sub * tk.rpt * (cyc_out(tk.rpt, k) + cyc_sum(tk.rpt, k, false) + kSplitCombine) * double(k) + kItem;
+          consider(LaunchShape{4, tk.rows, tk.rpt, seg, nseg, int(grid)},
+                   double(rounds) * item + kLaunch + kStart * double(nseg));
+        }
+        const int64_t per_sm = std::min<int64_t>(tiles / sms, tk.rpt == 1 ? 8 : 12);
         if (per_sm >= 4) {
-          // each CTA takes whole items; k warps share an SMSP's issue
+          // each CTA takes whole items; k warps share an SMSP
           const int64_t grid = per_sm * sms;
           const int64_t k = (per_sm + 3) / 4;
           const int64_t rounds = std::max<int64_t>((out_items + grid - 1) / grid, nseg);
-          const double item = double(seg) * kOut * double(k) / ipc(k) + kItem;
-          consider(LaunchShape{2, 32, seg, nseg, int(grid)}, double(rounds) * item + kLaunch);
+          const double item = double(seg) * tk.rpt * cyc_out(tk.rpt, k) * double(k) + kItem;
+          consider(LaunchShape{2, tk.rows, tk.rpt, seg, nseg, int(grid)}, double(rounds) * item + kLaunch);
         }
       }
-      if (forced_seg > 0 || L <= mssm::kSegQuant) break;
+      if (forced_mode == 0 || forced_seg > 0 || L <= mssm::kSegQuant) break;
     }
   }
   return best;
@@ -275,12 +335,17 @@ mssm_status mssm_set_option(int option, int64_t value) {
       g_chunk_len = value;
       return MSSM_OK;
     case MSSM_OPT_SCHEDULE:
-      if (value < 0 || value > 4) return fail(MSSM_ERR_INVALID_ARG, "SCHEDULE takes 0 (automatic) to 4");
+      if (value < 0 || value > 5) return fail(MSSM_ERR_INVALID_ARG, "SCHEDULE takes 0 (automatic) to 5");
       g_schedule = int(value) - 1;
       return MSSM_OK;
     case MSSM_OPT_ROWS_PER_CTA:
-      if (value != 0 && value != 32 && value != 64) return fail(MSSM_ERR_INVALID_ARG, "ROWS_PER_CTA takes 0, 32 or 64");
+      if (value != 0 && value != 32 && value != 64 && value != 128)
+        return fail(MSSM_ERR_INVALID_ARG, "ROWS_PER_CTA takes 0, 32, 64 or 128");
       g_rows_per_cta = int(value);
+      return MSSM_OK;
+    case MSSM_OPT_ROWS_PER_THREAD:
+      if (value < 0 || value > 2) return fail(MSSM_ERR_INVALID_ARG, "ROWS_PER_THREAD takes 0, 1 or 2");
+      g_rows_per_thread = int(value);
       return MSSM_OK;
     case MSSM_OPT_TEST_HOOKS:
       if (value < 0 || value > 1) return fail(MSSM_ERR_INVALID_ARG, "TEST_HOOKS takes 0 or 1");
@@ -445,6 +510,7 @@ mssm_status scan_prepare_ext(const mssm_scan_ext* ext, const mssm_tensor* out, c
 struct ScanPlan {
   int mode = 0;
   int rows_per_cta = 64;
+  int rpt = 1;            // rows per thread
   int grid = 0;
   int64_t nseg = 1;
   // mode 1: arrival counters, chunk sums, chunk end states
@@ -457,11 +523,12 @@ ScanPlan scan_plan(ScanCall& call, int sm_count) {
   mssm::ScanArgs& a = call.a;
   a.force_general = g_force_general;
   a.test_no_publish = g_test_hooks & 1;
-  const LaunchShape shape =
-      choose_shape(call.Bt, call.D, call.L, sm_count, g_chunk_len, g_schedule, g_rows_per_cta, call.total_len);
+  const LaunchShape shape = choose_shape(call.Bt, call.D, call.L, sm_count, g_chunk_len, g_schedule, g_rows_per_cta,
+                                         g_rows_per_thread, call.dtype, call.total_len);
   ScanPlan plan;
   plan.mode = shape.mode;
   plan.rows_per_cta = shape.rows;
+  plan.rpt = shape.rpt;
   plan.grid = shape.grid;
   plan.nseg = shape.nseg;
   a.tiles_per_batch = int((call.D + shape.rows - 1) / shape.rows);
@@ -473,21 +540,21 @@ ScanPlan scan_plan(ScanCall& call, int sm_count) {
     plan.count_bytes = ((size_t(tiles) * 4 + 255) / 256) * 256;
     plan.s_bytes = ((size_t(shape.nseg - 1) * rows_total * 4 + 255) / 256) * 256;
     plan.h_bytes = size_t(shape.nseg - 1) * rows_total * mssm::kN * 4;
-  } else if (shape.mode == 2) {
+  } else if (shape.mode == 2 || shape.mode == 4) {
     plan.count_bytes = ((size_t(tiles + 1) * 4 + 255) / 256) * 256;
-    plan.h_bytes = size_t(tiles) * 32 * mssm::kN * 4;
+    plan.h_bytes = size_t(tiles) * shape.rows * mssm::kN * 4;
   } else if (shape.mode == 3) {
     const size_t recs = size_t(tiles) * size_t(shape.nseg);
     plan.count_bytes = ((size_t(recs + 1) * 4 + 255) / 256) * 256;
-    plan.s_bytes = ((recs * 32 * 4 + 255) / 256) * 256;
-    plan.h_bytes = 2 * recs * 32 * mssm::kN * 4;  // summaries and end states
+    plan.s_bytes = ((recs * shape.rows * 4 + 255) / 256) * 256;
+    plan.h_bytes = 2 * recs * shape.rows * mssm::kN * 4;  // summaries and end states
   }
   return plan;
 }
 
 void scan_bind_workspace(mssm::ScanArgs& a, const ScanPlan& plan, void* ws) {
   char* base = static_cast<char*>(ws);
-  if (plan.mode == 2) {
+  if (plan.mode == 2 || plan.mode == 4) {
     a.ch_ticket = reinterpret_cast<unsigned*>(base);
     a.ch_flags = reinterpret_cast<unsigned*>(base) + 1;
     a.ch_carry = reinterpret_cast<float*>(base + plan.count_bytes);
@@ -516,28 +583,37 @@ mssm_status scan_launch(ScanCall& call, const ScanPlan& plan, void* ws, cudaStre
     e = cudaMemsetAsync(ws, 0, plan.count_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(fused schedule flags)");
     e = tracked(MSSM_KERNEL_SCAN_OUT, s, [&] {
-      return mssm::launch_scan_fused(call.a, plan.grid, call.dtype, call.has_z, call.softplus, s);
+      return mssm::launch_scan_fused(call.a, plan.grid, plan.rpt, call.dtype, call.has_z, call.softplus, s);
     });
     if (e != cudaSuccess) return cuda_fail(e, "fused scan kernel launch");
+    return MSSM_OK;
+  }
+  if (plan.mode == 4) {
+    e = cudaMemsetAsync(ws, 0, plan.count_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(split schedule flags)");
+    e = tracked(MSSM_KERNEL_SCAN_OUT, s, [&] {
+      return mssm::launch_scan_split(call.a, plan.grid, plan.rpt, call.dtype, call.has_z, call.softplus, s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "split scan kernel launch");
     return MSSM_OK;
   }
   if (plan.mode == 2) {
     e = cudaMemsetAsync(ws, 0, plan.count_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(chained schedule flags)");
     e = tracked(MSSM_KERNEL_SCAN_OUT, s, [&] {
-      return mssm::launch_scan_chained(call.a, plan.grid, call.dtype, call.has_z, call.softplus, s);
+      return mssm::launch_scan_chained(call.a, plan.grid, plan.rpt, call.dtype, call.has_z, call.softplus, s);
     });
     if (e != cudaSuccess) return cuda_fail(e, "chained scan kernel launch");
     return MSSM_OK;
   }
   if (plan.nseg > 1) {
     e = tracked(MSSM_KERNEL_SCAN_CHUNK_STATE, s, [&] {
-      return mssm::launch_scan_chunk_state(call.a, plan.rows_per_cta, call.dtype, call.softplus, s);
+      return mssm::launch_scan_chunk_state(call.a, plan.rows_per_cta, plan.rpt, call.dtype, call.softplus, s);
     });
     if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel launch");
   }
   e = tracked(MSSM_KERNEL_SCAN_OUT, s, [&] {
-    return mssm::launch_scan_out(call.a, plan.rows_per_cta, call.dtype, call.has_z, call.softplus, s);
+    return mssm::launch_scan_out(call.a, plan.rows_per_cta, plan.rpt, call.dtype, call.has_z, call.softplus, s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
   return MSSM_OK;
@@ -553,7 +629,7 @@ mssm_status scan_fwd_impl(ScanCall& call, void* stream) {
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceState* ds = device_state(dev);
   const ScanPlan plan = scan_plan(call, ds->sm_count);
-  if (plan.mode == 2 || plan.mode == 3) {
+  if (plan.mode >= 2) {
     // ticket, flags and carried states: zeroed by scan_launch where they must be
     const size_t need = plan.need() + size_t(ds->count_cap) * 4;
     if (ds->ws_bytes < need) {
@@ -919,7 +995,7 @@ mssm_status mssm_selective_scan_bwd(const mssm_tensor* u, const mssm_tensor* del
     a.cu_seqlens = nullptr;
     if ((e = mssm::device_error_word(&a.err)) != cudaSuccess) return cuda_fail(e, "device error word");
     e = tracked(MSSM_KERNEL_SCAN_CHUNK_STATE, s,
-                [&] { return mssm::launch_scan_chunk_state(a, mssm::kBwdRows, dt, softplus_flag != 0, s); });
+                [&] { return mssm::launch_scan_chunk_state(a, mssm::kBwdRows, 1, dt, softplus_flag != 0, s); });
     if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel launch (backward pass A)");
   }
   // passes B and C
@@ -1053,8 +1129,26 @@ mssm_status mssm_scan_plan(int64_t Bt, int64_t D, int64_t L, int sm_count, int* 
 
 mssm_status mssm_scan_plan_packed(int64_t S, int64_t D, int64_t max_seqlen, int64_t total_len, int sm_count,
                                   int* rows_per_cta, int64_t* chunk_len, int64_t* n_chunks, int* schedule) {
+  mssm_scan_plan_info info;
+  info.struct_size = int32_t(sizeof(info));
+  mssm_status st = mssm_scan_plan_query(S, D, max_seqlen, total_len, MSSM_BF16, sm_count, &info);
+  if (st != MSSM_OK) return st;
+  if (rows_per_cta) *rows_per_cta = info.rows_per_cta;
+  if (chunk_len) *chunk_len = info.chunk_len;
+  if (n_chunks) *n_chunks = info.n_chunks;
+  if (schedule) *schedule = info.schedule;
+  return MSSM_OK;
+}
+
+mssm_status mssm_scan_plan_query(int64_t S, int64_t D, int64_t max_seqlen, int64_t total_len, int io_dtype,
+                                 int sm_count, mssm_scan_plan_info* info) {
   const int64_t Bt = S, L = max_seqlen;
+  if (!info) return fail(MSSM_ERR_INVALID_ARG, "info: null pointer");
+  if (info->struct_size < int32_t(sizeof(mssm_scan_plan_info)))
+    return fail(MSSM_ERR_INVALID_ARG, "info->struct_size = %d; expected at least %d", int(info->struct_size),
+                int(sizeof(mssm_scan_plan_info)));
   if (Bt < 0 || D < 0 || L < 0) return fail(MSSM_ERR_INVALID_ARG, "negative size");
+  if (io_dtype != MSSM_F32 && io_dtype != MSSM_BF16) return fail(MSSM_ERR_INVALID_ARG, "io_dtype must be f32 or bf16");
   if (sm_count <= 0) {
     int dev = 0, v = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -1063,21 +1157,22 @@ mssm_status mssm_scan_plan_packed(int64_t S, int64_t D, int64_t max_seqlen, int6
     sm_count = v;
   }
   int64_t forced;
+  int forced_mode, forced_rows, forced_rpt;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     forced = g_chunk_len;
-  }
-  int forced_mode, forced_rows;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
     forced_mode = g_schedule;
     forced_rows = g_rows_per_cta;
+    forced_rpt = g_rows_per_thread;
   }
-  const LaunchShape sh = choose_shape(Bt, D, L, sm_count, forced, forced_mode, forced_rows, total_len);
-  if (rows_per_cta) *rows_per_cta = sh.rows;
-  if (chunk_len) *chunk_len = sh.seg;
-  if (n_chunks) *n_chunks = sh.nseg;
-  if (schedule) *schedule = sh.mode;
+  const LaunchShape sh =
+      choose_shape(Bt, D, L, sm_count, forced, forced_mode, forced_rows, forced_rpt, io_dtype, total_len);
+  info->schedule = sh.mode;
+  info->rows_per_cta = sh.rows;
+  info->rows_per_thread = sh.rpt;
+  info->chunk_len = sh.seg;
+  info->n_chunks = sh.nseg;
+  info->grid = sh.grid;
   return MSSM_OK;
 }
 

@@ -11,10 +11,15 @@ static void* g_error_word_cache[64] = {};
 // per device: SM count once the streaming kernels' shared-memory opt-in is set (0: not yet)
 static int g_stream_sms[64] = {};
 
+static int g_address_generation = 0;
+
 void forget_device_addresses() {
   for (void*& p : g_error_word_cache) p = nullptr;
   for (int& v : g_stream_sms) v = 0;  // a reset also drops the kernels' attributes
+  ++g_address_generation;
 }
+
+int device_address_generation() { return g_address_generation; }
 
 cudaError_t device_error_word(unsigned int** out) {
   void** cache = g_error_word_cache;
@@ -41,8 +46,8 @@ static cudaError_t stream_setup(int* sms) {
     int v = 0;
     e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const int b16 = kStreamBufs * int(StreamSlot<uint16_t>::kBytes);
-    const int b32 = kStreamBufs * int(StreamSlot<float>::kBytes);
+    const int b16 = kWsWarps * kWsBufs * int(StreamSlot<uint16_t>::kBytes);
+    const int b32 = kWsWarps * kWsBufs * int(StreamSlot<float>::kBytes);
     if ((e = cudaFuncSetAttribute(state_update_stream_kernel<uint16_t, true>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, b16)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(state_update_stream_kernel<uint16_t, false>,
@@ -61,8 +66,8 @@ static cudaError_t stream_setup(int* sms) {
 // Batch groups of the streaming kernel: as many CTAs per channel block as fill the
 // resident slots, but no more groups than batches.
 int stream_groups(int Bt, int D, int sms) {
-  const int nblk = (D + kStreamRows - 1) / kStreamRows;
-  int groups = (sms * kStreamCtasPerSm) / nblk;
+  const int nblk = (D + kWsRows - 1) / kWsRows;
+  int groups = (sms * kStreamCtasPerSm * kWsWarps) / nblk;
   if (groups < 1) groups = 1;
   if (groups > Bt) groups = Bt;
   // same number of batches per CTA with as few groups as that needs
@@ -80,9 +85,9 @@ static cudaError_t launch_decode_t(DecodeArgs a, DecodePath path, cudaStream_t s
     int sms = 0;
     if ((e = stream_setup(&sms)) != cudaSuccess) return e;
     a.groups = stream_groups(a.Bt, a.D, sms);
-    const int64_t nblk = (a.D + kStreamRows - 1) / kStreamRows;
-    state_update_stream_kernel<T, HAS_Z>
-        <<<unsigned(nblk * a.groups), kStreamRows, kStreamBufs * StreamSlot<T>::kBytes, s>>>(a);
+    const int64_t warps = int64_t((a.D + kWsRows - 1) / kWsRows) * a.groups;
+    state_update_stream_kernel<T, HAS_Z><<<unsigned((warps + kWsWarps - 1) / kWsWarps), kWsWarps * 32,
+                                           kWsWarps * kWsBufs * StreamSlot<T>::kBytes, s>>>(a);
   } else if (path == DecodePath::kBulkTile) {
     state_update_bulk_kernel<T, HAS_Z><<<unsigned(blocks), kDecodeThreads, 0, s>>>(a);
   } else {

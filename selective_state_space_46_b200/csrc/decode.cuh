@@ -205,37 +205,42 @@ __global__ void __launch_bounds__(kDecodeThreads) state_update_bulk_kernel(const
 }
 
 // ---------------------------------------------------------------------------
-// persistent streaming form.  A CTA owns one block of kStreamRows channels and
-// walks the batches b = g, g + G, g + 2G, ... of that block (g, G: its batch
-// group and the group count).  Per (batch, channel block) tile, one thread
-// issues bulk copies of everything the tile reads -- the contiguous 8 KB of
-// state, the x / dt / z runs of the block and the batch's B and C rows -- into
-// one slot of a shared-memory ring, all counted on the slot's mbarrier;
-// kStreamBufs - 1 tiles are in flight ahead of the one being updated, and the
-// updated state leaves by a bulk store that overlaps the following tiles.  The
-// block's A rows, skip weights and biases are loaded once per CTA into
-// registers.  So no thread waits on a global load inside the loop: the only
-// waits are the (bounded) mbarrier waits the ring hides.
+// persistent streaming form.  Every warp owns one block of 32 channels and walks
+// the batches b = g, g + G, g + 2G, ... of that block (g, G: its batch group and
+// the group count), independently of the other warps of its CTA.  Per (batch,
+// channel block) tile, lane 0 issues bulk copies of everything the tile reads --
+// the contiguous 2 KB of state, the x / dt / z runs of the block and the batch's
+// B and C rows -- into one slot of the warp's own shared-memory ring, all counted
+// on the slot's mbarrier; kWsAhead tiles are in flight ahead of the one being
+// updated, and the updated state leaves by a bulk store that overlaps the
+// following tiles.  A, the skip weight and the bias of a lane's channel are
+// loaded once into registers.  The only waits in the loop are the (bounded)
+// mbarrier waits the ring hides and warp-level syncs: no warp waits for another
+// (a CTA-wide tile synchronised all 128 threads twice per tile, which was the
+// kernel's largest stall).
 //
 // Needs: contiguous 16-byte-aligned state; x, dt (and z) with unit channel
 // stride, 16-byte-aligned batch rows and D a multiple of 16 / sizeof(T); B and
 // C with unit n stride and 16-byte-aligned batch rows (the host checks all).
 // ---------------------------------------------------------------------------
-constexpr int kStreamRows = 128;      // channels per CTA, one thread each
-constexpr int kStreamBufs = 8;        // ring slots per CTA (swept: 3..8 slots x 3..6 CTAs; 8 x 3 best)
-constexpr int kStreamAhead = kStreamBufs - 1;
-constexpr int kStreamCtasPerSm = 3;   // 3 x (8 x <= 9.9 KB) shared memory, 384 threads
+constexpr int kWsRows = 32;          // channels per warp, one lane each
+constexpr int kWsWarps = 4;          // warps per CTA
+constexpr int kWsBufs = 6;           // ring slots per warp
+constexpr int kWsAhead = kWsBufs - 1;
+constexpr int kStreamCtasPerSm = 3;  // 3 x 4 warps x 6 slots of <= 2.5 KB of shared memory
 
 template <typename T>
 struct StreamSlot {
   static constexpr uint32_t kState = 0;
-  static constexpr uint32_t kX = kStreamRows * kN * 4;
-  static constexpr uint32_t kDt = kX + kStreamRows * sizeof(T);
-  static constexpr uint32_t kZ = kDt + kStreamRows * sizeof(T);
-  static constexpr uint32_t kB = kZ + kStreamRows * sizeof(T);
+  static constexpr uint32_t kX = kWsRows * kN * 4;
+  static constexpr uint32_t kDt = kX + kWsRows * sizeof(T);
+  static constexpr uint32_t kZ = kDt + kWsRows * sizeof(T);
+  static constexpr uint32_t kB = kZ + kWsRows * sizeof(T);
   static constexpr uint32_t kC = kB + kN * sizeof(T);
   static constexpr uint32_t kBytes = kC + kN * sizeof(T);
-  static_assert(kBytes % 16 == 0 && kX % 16 == 0 && kB % 16 == 0, "slot layout must keep 16-byte alignment");
+  static_assert(kBytes % 16 == 0 && kX % 16 == 0 && kDt % 16 == 0 && kZ % 16 == 0 && kB % 16 == 0 &&
+                    kC % 16 == 0,
+                "slot layout must keep 16-byte alignment");
 };
 
 __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t mb, uint32_t parity) {
@@ -257,30 +262,34 @@ __device__ __forceinline__ float smem_elem(const unsigned char* base, int j) {
 }
 
 template <typename T, bool HAS_Z>
-__global__ void __launch_bounds__(kStreamRows, kStreamCtasPerSm) state_update_stream_kernel(const DecodeArgs p) {
+__global__ void __launch_bounds__(kWsWarps * 32, kStreamCtasPerSm) state_update_stream_kernel(const DecodeArgs p) {
   using L = StreamSlot<T>;
-  extern __shared__ __align__(128) unsigned char ring_s[];  // kStreamBufs slots of L::kBytes
-  __shared__ __align__(8) unsigned long long mbar[kStreamBufs];
-  const int tid = threadIdx.x;
-  const int nblk = (p.D + kStreamRows - 1) / kStreamRows;
-  const int cb = int(blockIdx.x % uint32_t(nblk));
-  const int g = int(blockIdx.x / uint32_t(nblk));
+  extern __shared__ __align__(128) unsigned char ring_s[];  // kWsWarps x kWsBufs slots of L::kBytes
+  __shared__ __align__(8) unsigned long long mbar[kWsWarps][kWsBufs];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nblk = (p.D + kWsRows - 1) / kWsRows;
+  const int gw = int(blockIdx.x) * kWsWarps + warp;
+  const int cb = gw % nblk;
+  const int g = gw / nblk;
+  // a whole warp leaves here (nothing below synchronises more than one warp)
   if (g >= p.Bt || g >= p.groups) return;
-  const int c0 = cb * kStreamRows;
-  const int nrows = p.D - c0 < kStreamRows ? p.D - c0 : kStreamRows;
-  const uint32_t mine = uint32_t(p.Bt - 1 - g) / uint32_t(p.groups) + 1;  // batches of this CTA
-  const bool live = tid < nrows;
-  const int d = c0 + (live ? tid : nrows - 1);
-  const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(ring_s));
-  const uint32_t mb0 = static_cast<uint32_t>(__cvta_generic_to_shared(&mbar[0]));
+  const int c0 = cb * kWsRows;
+  const int nrows = p.D - c0 < kWsRows ? p.D - c0 : kWsRows;
+  const uint32_t mine = uint32_t(p.Bt - 1 - g) / uint32_t(p.groups) + 1;  // batches of this warp
+  const bool live = lane < nrows;
+  const int d = c0 + (live ? lane : nrows - 1);
+  unsigned char* wring = ring_s + warp * (kWsBufs * L::kBytes);
+  const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(wring));
+  const uint32_t mb0 = static_cast<uint32_t>(__cvta_generic_to_shared(&mbar[warp][0]));
   constexpr uint32_t ES = sizeof(T);
   const uint32_t run_bytes = uint32_t(nrows) * ES;  // a multiple of 16 (D % (16 / ES) == 0)
   const uint32_t tile_bytes = uint32_t(nrows) * kN * 4 + (HAS_Z ? 3u : 2u) * run_bytes + 2u * kN * ES;
 
-  auto issue = [&](uint32_t i) {  // one thread
+  auto issue = [&](uint32_t i) {  // lane 0
     const int64_t b = int64_t(g) + int64_t(i) * p.groups;
-    const uint32_t slot = ring + (i % kStreamBufs) * L::kBytes;
-    const uint32_t mb = mb0 + (i % kStreamBufs) * 8;
+    const uint32_t slot = ring + (i % kWsBufs) * L::kBytes;
+    const uint32_t mb = mb0 + (i % kWsBufs) * 8;
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(tile_bytes) : "memory");
     bulk_load(slot + L::kState, p.state + (b * p.D + c0) * kN, uint32_t(nrows) * kN * 4, mb);
     bulk_load(slot + L::kX, static_cast<const T*>(p.x) + b * p.x_sb + c0, run_bytes, mb);
@@ -290,20 +299,19 @@ __global__ void __launch_bounds__(kStreamRows, kStreamCtasPerSm) state_update_st
     bulk_load(slot + L::kC, static_cast<const T*>(p.C) + b * p.C_sb, kN * ES, mb);
   };
 
-  if (tid == 0) {
+  if (lane == 0) {
 #pragma unroll
-    for (int k = 0; k < kStreamBufs; ++k)
+    for (int k = 0; k < kWsBufs; ++k)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mb0 + 8 * k) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (uint32_t j = 0; j < uint32_t(kWsAhead) && j < mine; ++j) issue(j);
   }
-  __syncthreads();
-  if (tid == 0)
-    for (uint32_t j = 0; j < uint32_t(kStreamAhead) && j < mine; ++j) issue(j);
+  __syncwarp();
 
-  // per-channel constants, once per CTA.  The state row is visited in the lane-rotated
+  // per-channel constants, once per warp.  The state row is visited in the lane-rotated
   // quarter order q = (kq + rot) & 3 (bank-conflict free), so A is stored pre-rotated:
   // a2r[4 kq + e] = A[d, 4 q + e] * log2(e), and the loop indexes it with constants.
-  const int rot = (tid >> 1) & 3;
+  const int rot = (lane >> 1) & 3;
   float a2r[kN];
   {
     const float* Ar = p.A + int64_t(d) * p.A_sd;
@@ -318,21 +326,21 @@ __global__ void __launch_bounds__(kStreamRows, kStreamCtasPerSm) state_update_st
   uint32_t i = 0;
   bool ok = true;
   for (; i < mine; ++i) {
-    const uint32_t k = i % kStreamBufs;
-    const unsigned char* slot = ring_s + k * L::kBytes;
+    const uint32_t k = i % kWsBufs;
+    unsigned char* slot = wring + k * L::kBytes;
     uint32_t done = 0;
-    for (int it = 0; it < kDecodeSpinLimit && !done; ++it) done = mbar_try_wait(mb0 + k * 8, (i / kStreamBufs) & 1u);
-    if (!__syncthreads_and(done)) {
+    for (int it = 0; it < kDecodeSpinLimit && !done; ++it) done = mbar_try_wait(mb0 + k * 8, (i / kWsBufs) & 1u);
+    if (!__all_sync(0xffffffffu, done)) {
       ok = false;
       break;
     }
     if (live) {
       const int64_t b = int64_t(g) + int64_t(i) * p.groups;
-      const float x = smem_elem<T>(slot + L::kX, tid);
-      float dt = smem_elem<T>(slot + L::kDt, tid) + bias;
+      const float x = smem_elem<T>(slot + L::kX, lane);
+      float dt = smem_elem<T>(slot + L::kDt, lane) + bias;
       if (p.softplus) dt = softplus_f(dt);
       const float w = dt * x;
-      float4* hs = reinterpret_cast<float4*>(const_cast<unsigned char*>(slot) + L::kState + tid * (kN * 4));
+      float4* hs = reinterpret_cast<float4*>(slot + L::kState + lane * (kN * 4));
       float y = 0.0f;
 #pragma unroll
       for (int kq = 0; kq < 4; ++kq) {
@@ -343,18 +351,18 @@ __global__ void __launch_bounds__(kStreamRows, kStreamCtasPerSm) state_update_st
         for (int e = 0; e < 4; ++e) {
           const int n = 4 * q + e;
           const float ed = ex2f(dt * a2r[4 * kq + e]);
-          float g = w;
+          float gn = w;
           if (p.zoh) {
             const float an = a2r[4 * kq + e] * kLn2;
-            g = zoh_gain_f(ed, dt, an, an != 0.0f ? rcpf(an) : 0.0f) * x;
+            gn = zoh_gain_f(ed, dt, an, an != 0.0f ? rcpf(an) : 0.0f) * x;
           }
-          hv[e] = fmaf(ed, hv[e], g * smem_elem<T>(slot + L::kB, n));
+          hv[e] = fmaf(ed, hv[e], gn * smem_elem<T>(slot + L::kB, n));
           y = fmaf(smem_elem<T>(slot + L::kC, n), hv[e], y);
         }
         hs[q] = make_float4(hv[0], hv[1], hv[2], hv[3]);
       }
       y = fmaf(Dd, x, y);
-      if constexpr (HAS_Z) y *= gate_f<T>(smem_elem<T>(slot + L::kZ, tid));
+      if constexpr (HAS_Z) y *= gate_f<T>(smem_elem<T>(slot + L::kZ, lane));
       T* o = static_cast<T*>(p.out) + b * p.o_sb + int64_t(d) * p.o_sd;
       if constexpr (sizeof(T) == 2) {
         *o = f_to_bf16(y);
@@ -364,32 +372,32 @@ __global__ void __launch_bounds__(kStreamRows, kStreamCtasPerSm) state_update_st
     }
     // generic-proxy accesses of this slot -> ordered before the bulk store and the next bulk load
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-    if (tid == 0) {
+    __syncwarp();
+    if (lane == 0) {
       const int64_t b = int64_t(g) + int64_t(i) * p.groups;
       asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
                    ::"l"(p.state + (b * p.D + c0) * kN), "r"(ring + k * L::kBytes + L::kState),
                    "r"(uint32_t(nrows) * kN * 4) : "memory");
       asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-      if (i + kStreamAhead < mine) {
-        // tile i + kStreamAhead takes the slot of tile i - 1, whose store is the older of
+      if (i + kWsAhead < mine) {
+        // tile i + kWsAhead takes the slot of tile i - 1, whose store is the older of
         // the (at most) two stores in flight
         asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-        issue(i + kStreamAhead);
+        issue(i + kWsAhead);
       }
     }
   }
-  if (!ok && tid == 0) {
-    // record the error; give the loads still in flight (tiles i .. i + kStreamAhead - 1) a
-    // bounded time to land before the CTA's shared memory is released
+  if (!ok && lane == 0) {
+    // record the error; give the loads still in flight (tiles i .. i + kWsAhead - 1) a
+    // bounded time to land before the warp's slots can be released
     atomicOr(p.err, 1u);
-    for (uint32_t j = i; j < i + kStreamAhead && j < mine; ++j) {
+    for (uint32_t j = i; j < i + kWsAhead && j < mine; ++j) {
       uint32_t done = 0;
       for (int it = 0; it < kDecodeSpinLimit && !done; ++it)
-        done = mbar_try_wait(mb0 + (j % kStreamBufs) * 8, (j / kStreamBufs) & 1u);
+        done = mbar_try_wait(mb0 + (j % kWsBufs) * 8, (j / kWsBufs) & 1u);
     }
   }
-  if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------

@@ -205,6 +205,10 @@ WORKLOADS = {
     # long context, slow decay spanning many chunks
     "scan_bf16_1x2048x131072": dict(kind="scan", batch=1, dim=2048, length=131072,
                                     io_dtype="bf16", delta_range=(1e-4, 1e-2), with_z=True),
+    # the long-context shape cut to 16384 steps (inputs still larger than the L2): the case
+    # the full ncu captures of the scan kernels run on
+    "scan_bf16_1x2048x16384": dict(kind="scan", batch=1, dim=2048, length=16384,
+                                   io_dtype="bf16", delta_range=(1e-4, 1e-2), with_z=True),
     # the causal conv1d (K = 4) + SiLU that produces u, at the Mamba-130M prefill shape
     "conv_bf16_2x1536x2048": dict(kind="conv", batch=2, dim=1536, length=2048, io_dtype="bf16", K=4),
     # the same conv at the Mamba-2.8B prefill shape (671 MB of traffic per call)

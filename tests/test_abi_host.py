@@ -259,8 +259,9 @@ def test_options_and_strings(lib):
     assert lib.mssm_set_option(1, 2) == INVALID
     assert lib.mssm_set_option(2, 100) == INVALID      # not a multiple of 64
     assert lib.mssm_set_option(99, 0) == INVALID
-    assert lib.mssm_set_option(4, 5) == INVALID
-    assert lib.mssm_set_option(4, 4) == 0 and lib.mssm_set_option(4, 3) == 0 and lib.mssm_set_option(4, 0) == 0
+    assert lib.mssm_set_option(4, 6) == INVALID
+    for v in (5, 4, 3, 0):
+        assert lib.mssm_set_option(4, v) == 0
     assert lib.mssm_set_option(5, 4) == INVALID and lib.mssm_set_option(5, -1) == INVALID
     for v in (1, 2, 3, 0):
         assert lib.mssm_set_option(5, v) == 0
@@ -268,10 +269,14 @@ def test_options_and_strings(lib):
     assert lib.mssm_set_option(6, 1) == 0 and lib.mssm_set_option(6, 0) == 0
     assert lib.mssm_set_option(2, 128) == 0
     assert lib.mssm_set_option(2, 0) == 0
-    for v in (16, 48, -32, 128):
+    for v in (16, 48, -32, 256):
         assert lib.mssm_set_option(7, v) == INVALID
-    for v in (64, 32, 0):
+    for v in (128, 64, 32, 0):
         assert lib.mssm_set_option(7, v) == 0
+    for v in (-1, 3, 4):
+        assert lib.mssm_set_option(8, v) == INVALID
+    for v in (2, 1, 0):
+        assert lib.mssm_set_option(8, v) == 0
     lib.mssm_status_string.restype = ctypes.c_char_p
     assert lib.mssm_status_string(2) == b"MSSM_ERR_UNSUPPORTED"
     lib.mssm_version.restype = ctypes.c_char_p
@@ -280,20 +285,26 @@ def test_options_and_strings(lib):
 
 def test_scan_plan_measured_best():
     """The automatic plans of the benchmark workloads are the ones measured fastest on B200
-    (sweeps of chunk length, rows per CTA and schedule): a change to the cost model that moves
-    one of them must be measured again."""
+    (sweeps of chunk length, rows per tile, rows per thread and schedule): a change to the cost
+    model that moves one of them must be measured again."""
     import selective_state_space_46_b200 as m
-    for opt in (m.MSSM_OPT_CHUNK_LEN, m.MSSM_OPT_SCHEDULE, m.MSSM_OPT_ROWS_PER_CTA):
+    for opt in (m.MSSM_OPT_CHUNK_LEN, m.MSSM_OPT_SCHEDULE, m.MSSM_OPT_ROWS_PER_CTA, m.MSSM_OPT_ROWS_PER_THREAD):
         m.mssm_set_option(opt, 0)
     expect = {
-        (2, 1536, 2048, -1): ("summaries+forward", 32, 192),   # 65 us; 128: 65.6, 256: 74.8, 64 rows: 67-89
-        (8, 5120, 4096, -1): ("chained", 32, 512),             # 773 us; summaries+forward: 1089
-        (1, 2048, 131072, -1): ("summaries+forward", 64, 3584),  # 1683 us; 32 rows: 1838
-        (32, 1536, 4096, 27048): ("summaries+forward", 64, 128),  # packed: 365 us; 32 rows: 391
+        # 63.1 us; 32 rows chunk 128: 63.8, 64 rows chunk 128: 65.3, chunk 192: 66.2, split: 73.5
+        (2, 1536, 2048, -1): ("summaries+forward", 32, 1, 192),
+        # 746 us; chunk 256: 761, 1024: 752; two rows per thread: 1096-1107; forward only: 1139
+        (8, 5120, 4096, -1): ("chained", 32, 1, 512),
+        # 1662-1674 us; chunk 2560: 1759, 4608: 2031; 32 rows: 1737; split: 1780-1818;
+        # two rows per thread: 1680-1769; fused: 1815
+        (1, 2048, 131072, -1): ("summaries+forward", 64, 1, 3584),
+        # packed sequences
+        (32, 1536, 4096, 27048): ("summaries+forward", 64, 1, 192),
     }
-    for (S, D, L, total), (sched, rows, chunk) in expect.items():
+    for (S, D, L, total), want in expect.items():
         plan = m.mssm_scan_plan(S, D, L, sm_count=148, total_len=total)
-        assert (plan["schedule"], plan["rows_per_cta"], plan["chunk_len"]) == (sched, rows, chunk), (S, D, L, plan)
+        got = (plan["schedule"], plan["rows_per_cta"], plan["rows_per_thread"], plan["chunk_len"])
+        assert got == want, (S, D, L, plan)
 
 
 def test_scan_plan_host_only(lib):
