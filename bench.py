@@ -206,6 +206,15 @@ def recorded_traffic(kernel: str, workload: str, plan: str | None = None):
     return val, os.path.relpath(p, ROOT)
 
 
+def recorded_step_traffic(kernel: str, workload: str, plan: str | None = None):
+    """DRAM bytes of a whole step (every kernel of it), when the same summary recorded them."""
+    val, src = recorded_traffic(kernel, workload, plan)
+    if val is None:
+        return None
+    m_s = re.search(r"step_dram_bytes\s*=\s*([0-9.eE+]+)", open(os.path.join(ROOT, src)).read())
+    return float(m_s.group(1)) if m_s else None
+
+
 def plan_string(plan: dict | None) -> str | None:
     if not plan:
         return None
@@ -629,7 +638,8 @@ def run_mssm(args):
                      "peak_source": f"HBM: {peak_kind} copy rate; FP32: {sms} SMs x 128 lanes x 2 x "
                                     f"{max_sm_mhz():.0f} MHz",
                      "algorithmic_bytes_per_launch": alg_bytes, "algorithmic_flops_per_launch": alg_flops,
-                     "traffic": traffic, "traffic_source": traffic_src})
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "traffic_step": recorded_step_traffic(dom_kernel, args.workload, plan_key)})
 
     # ---- end to end: host buffers in pinned memory, copies inside the timed region
     e2e = None

@@ -194,7 +194,7 @@ double cyc_out(int rpt, int64_t k) {
   return k <= 1 ? 221.0 : k == 2 ? 185.0 : 150.0;
 }
 double cyc_sum(int rpt, int64_t k, bool fwd_sweep) {
-  if (fwd_sweep) return cyc_out(rpt, k) * 0.8;
+  if (fwd_sweep) return cyc_out(rpt, k) * 0.7;  // measured 0.67-0.73 of the forward kernel
   if (rpt == 1) return k <= 1 ? 110.0 : k == 2 ? 95.0 : 86.0;
   return k <= 1 ? 120.0 : k == 2 ? 105.0 : 95.0;
 }
@@ -266,6 +266,25 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
       }
       double cost = grid_time(out_items, tk, double(seg), false);
       if (nseg > 1) cost += grid_time(sum_items, tk, double(seg), true) + kFold * double(nseg);
+      if (packed) {
+        // packed sequences: most CTAs hold fewer than seg steps, so count the work itself
+        // (every tile sweeps and summarises total_len steps, each CTA's warps pay their
+        // start) at the SMSP rate of a full SM of this kind, plus a tail of kPackedTail of
+        // one item's duration (the last items run on a draining GPU), and no less than
+        // that duration (a chunk of the longest sequence is swept by one warp).  Fitted to the
+        // chunk-length sweep of 32 sequences of up to 4096 steps (27048 in all) x 1536
+        // channels: 4-6% above the measured times at chunks of 128 to 512, in their order.
+        constexpr double kPackedTail = 0.15;
+        const double smsps = 4.0 * double(sms), wpt = double(tk.rows / tk.rpt) / 32.0;
+        const int64_t kf = (int64_t(out_ctas(tk.rows, tk.rpt)) * (tk.rows / tk.rpt / 32) + 3) / 4;
+        const double c_out = tk.rpt * cyc_out(tk.rpt, kf), c_sum = tk.rpt * cyc_sum(tk.rpt, kf, true);
+        const double per_step = double(tpb) * wpt * double(total_len) / smsps;
+        cost = per_step * c_out + double(out_items) * wpt * kCta / smsps + kStart + kLaunch;
+        if (nseg > 1)
+          cost += per_step * c_sum + double(sum_items) * wpt * kCta / smsps + kStart + kLaunch + kFold * double(nseg);
+        const double item = double(seg) * double(kf) * (c_out + (nseg > 1 ? c_sum : 0.0));
+        cost = std::max(cost + kPackedTail * item, item);  // ... and never below one item's own sweep
+      }
       consider(LaunchShape{nseg > 1 ? 1 : 0, tk.rows, tk.rpt, seg, nseg, 0}, cost);
       if (one_warp && nseg > 1) {
         const int64_t cap = int64_t(tk.rpt == 1 ? 8 : 12) * sms;  // resident one-warp CTAs
