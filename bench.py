@@ -493,7 +493,7 @@ def run_mssm(args):
                                           gk["dA"], gk["dB"], gk["dC"], gk["dD"], gk["dz"], gk["ddelta_bias"])
             metric = BWD_METRIC
             dom_kernel = "scan_bwd"
-            config["pass"] = "backward (passes A, B, C)"
+            config["pass"] = "backward (chunk summaries both ways, then the per-chunk recompute and sweep)"
     elif kind == "conv":
         inp = synth.workload_inputs(args.workload, seed=seed)
         units = inp.batch * inp.dim * inp.length

@@ -240,11 +240,11 @@ mssm_status mssm_state_update_ex(mssm_tensor *state, const mssm_tensor *x,
 /*
  * Backward of mssm_selective_scan_fwd (Euler discretisation, zero initial state,
  * no packed sequences): the gradients of Loss with respect to every input, given
- * dout = dLoss/dout.  The states are recomputed, never stored: the forward's
- * chunk summaries give every 64-step chunk's start state, a reverse pass of chunk
- * summaries gives every chunk's incoming dLoss/dh, and every chunk then sweeps its
- * recomputed states backwards ("Mamba selective state space", the hardware-aware
- * scan: intermediates are recomputed in the backward pass).
+ * dout = dLoss/dout.  The states are recomputed, never stored: one pass of chunk
+ * summaries, both ways, gives every 64-step chunk's start state and incoming
+ * dLoss/dh, and every chunk then sweeps its recomputed states backwards ("Mamba
+ * selective state space", the hardware-aware scan: intermediates are recomputed in
+ * the backward pass).
  *   inputs     as for mssm_selective_scan_fwd, plus dout [Bt, D, L] dtype of u
  *   du, ddelta [Bt, D, L] dtype of u, written (ddelta: with respect to delta before
  *              the bias and softplus)
@@ -428,7 +428,7 @@ typedef enum {
     MSSM_KERNEL_SCAN_OUT = 1,         /* forward sweep with fused epilogue */
     MSSM_KERNEL_STATE_UPDATE = 2,     /* decode step */
     MSSM_KERNEL_CONV = 3,             /* causal conv1d (prefill and decode step) */
-    MSSM_KERNEL_SCAN_BWD = 4,         /* backward scan (passes B and C; pass A counts as CHUNK_STATE) */
+    MSSM_KERNEL_SCAN_BWD = 4,         /* backward scan (both of its passes) */
     MSSM_KERNEL_KINDS = 5
 } mssm_kernel_kind;
 

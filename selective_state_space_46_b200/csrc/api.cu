@@ -963,16 +963,17 @@ mssm_status mssm_selective_scan_bwd(const mssm_tensor* u, const mssm_tensor* del
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(gradients)");
   if (L == 0) return MSSM_OK;
 
-  // workspace: pass A's chunk states (H, S, counters) and pass B's (G, S, Q, counters)
+  // workspace: the chunk summaries (H then the start states, G, S), the incoming gradients Q,
+  // and the arrival counters
   const int64_t tpb = (Dd + mssm::kBwdRows - 1) / mssm::kBwdRows;
   const int64_t tiles = Bt * tpb, rows_total = tiles * mssm::kBwdRows;
   const int64_t nseg = (L + mssm::kBwdChunk - 1) / mssm::kBwdChunk;
   if (nseg > 65535 || tiles > INT32_MAX) return fail(MSSM_ERR_UNSUPPORTED, "problem too large for the backward grid");
   auto al = [](size_t v) { return (v + 255) / 256 * 256; };
   const size_t cnt_b = al(size_t(tiles) * 4);
-  const size_t hA_b = al(size_t(nseg - 1) * rows_total * mssm::kN * 4), sA_b = al(size_t(nseg - 1) * rows_total * 4);
-  const size_t g_b = al(size_t(nseg) * rows_total * mssm::kN * 4), sB_b = al(size_t(nseg) * rows_total * 4);
-  const size_t need = 2 * cnt_b + hA_b + sA_b + 2 * g_b + sB_b;
+  const size_t h_b = al(size_t(nseg - 1) * rows_total * mssm::kN * 4);
+  const size_t g_b = al(size_t(nseg) * rows_total * mssm::kN * 4), s_b = al(size_t(nseg) * rows_total * 4);
+  const size_t need = cnt_b + h_b + 2 * g_b + s_b;
   int dev = -1;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   DeviceState* ds = device_state(dev);
@@ -990,34 +991,13 @@ mssm_status mssm_selective_scan_bwd(const mssm_tensor* u, const mssm_tensor* del
     ds->bwd_bytes = need;
   }
   char* base = static_cast<char*>(ds->bwd_ws);
-  unsigned* cntA = reinterpret_cast<unsigned*>(base);
-  unsigned* cntB = reinterpret_cast<unsigned*>(base + cnt_b);
-  float* hA = reinterpret_cast<float*>(base + 2 * cnt_b);
-  float* sA = reinterpret_cast<float*>(base + 2 * cnt_b + hA_b);
-  float* gB = reinterpret_cast<float*>(base + 2 * cnt_b + hA_b + sA_b);
-  float* qB = reinterpret_cast<float*>(base + 2 * cnt_b + hA_b + sA_b + g_b);
-  float* sB = reinterpret_cast<float*>(base + 2 * cnt_b + hA_b + sA_b + 2 * g_b);
-  if ((e = cudaMemsetAsync(base, 0, 2 * cnt_b, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(counters)");
+  unsigned* cnt = reinterpret_cast<unsigned*>(base);
+  float* hA = reinterpret_cast<float*>(base + cnt_b);
+  float* gB = reinterpret_cast<float*>(base + cnt_b + h_b);
+  float* qB = reinterpret_cast<float*>(base + cnt_b + h_b + g_b);
+  float* sB = reinterpret_cast<float*>(base + cnt_b + h_b + 2 * g_b);
+  if ((e = cudaMemsetAsync(base, 0, cnt_b, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(counters)");
 
-  // pass A: the forward chunk summaries and their fold give every chunk's start state
-  if (nseg > 1) {
-    mssm::ScanArgs a = call.a;
-    a.force_general = g_force_general;
-    a.tiles_per_batch = int(tpb);
-    a.seg_len = mssm::kBwdChunk;
-    a.nseg = int(nseg);
-    a.ws_H = hA;
-    a.ws_S = sA;
-    a.ws_count = cntA;
-    a.h0 = nullptr;
-    a.zoh = 0;
-    a.cu_seqlens = nullptr;
-    if ((e = mssm::device_error_word(&a.err)) != cudaSuccess) return cuda_fail(e, "device error word");
-    e = tracked(MSSM_KERNEL_SCAN_CHUNK_STATE, s,
-                [&] { return mssm::launch_scan_chunk_state(a, mssm::kBwdRows, 1, dt, softplus_flag != 0, s); });
-    if (e != cudaSuccess) return cuda_fail(e, "chunk-state kernel launch (backward pass A)");
-  }
-  // passes B and C
   mssm::BwdArgs b{};
   b.u = u->data; b.delta = delta->data; b.z = z ? z->data : nullptr; b.dout = dout->data;
   b.u_sb = u->stride[0]; b.u_sd = u->stride[1]; b.dl_sb = delta->stride[0]; b.dl_sd = delta->stride[1];
@@ -1038,7 +1018,7 @@ mssm_status mssm_selective_scan_bwd(const mssm_tensor* u, const mssm_tensor* del
   b.Bt = int(Bt); b.D = int(Dd); b.L = int(L);
   b.softplus = softplus_flag != 0;
   b.nseg = int(nseg); b.tiles_per_batch = int(tpb);
-  b.hstart = hA; b.ws_G = gB; b.ws_S = sB; b.ws_Q = qB; b.ws_count = cntB;
+  b.hstart = hA; b.ws_G = gB; b.ws_S = sB; b.ws_Q = qB; b.ws_count = cnt;
   b.vec_rows = rows_vec(u) && rows_vec(delta) && rows_vec(dout) && rows_vec(du) && rows_vec(ddelta) &&
                (!z || (rows_vec(z) && rows_vec(dz)));
   b.force_general = g_force_general;

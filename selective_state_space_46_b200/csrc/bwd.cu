@@ -1,5 +1,5 @@
-// Instantiation and launch of the backward scan kernels (passes B and C; pass A is the
-// forward chunk-summary kernel of scan.cu).
+// Instantiation and launch of the backward scan kernels: pass A (the chunk summaries both
+// ways and their folds) and pass B (the per-chunk recompute and backward sweep).
 #include "launch.h"
 
 namespace mssm {
@@ -8,7 +8,7 @@ template <typename T, bool HAS_Z>
 static cudaError_t bwd_t(const BwdArgs& a, cudaStream_t s) {
   const unsigned tiles = unsigned(a.Bt * a.tiles_per_batch);
   if (a.nseg > 1) {
-    scan_bwd_summary_kernel<T, HAS_Z><<<dim3(tiles, a.nseg - 1), kBwdRows, 0, s>>>(a);
+    scan_bwd_summary_kernel<T, HAS_Z><<<dim3(tiles, a.nseg), kBwdRows, 0, s>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

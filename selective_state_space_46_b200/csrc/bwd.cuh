@@ -9,19 +9,20 @@
 // ("Mamba selective state space", the hardware-aware scan: intermediates are
 // recomputed in the backward pass instead of being written).
 //
-// Three chunk-parallel passes over chunks of kBwdChunk steps, one thread per row:
-//  A. the forward chunk summaries and their fold (scan_chunk_state_kernel) give
-//     every chunk's start state;
-//  B. scan_bwd_summary_kernel: every chunk but the first runs the g recurrence
-//     from a zero incoming gradient, giving G_c (what it sends to the chunk
-//     before) and S_c (its summed step); the last CTA of a row tile folds them
-//     backwards, Q_(c-1) = exp(A S_c) Q_c + G_c, into each chunk's incoming Q_c;
-//  C. scan_bwd_kernel: every chunk recomputes its states forward from its start
-//     state, window by window (kBwdWin steps held in registers, the windows' start
-//     states in shared memory), and sweeps them backwards from Q_c, writing du,
-//     ddelta, dz and accumulating dA, dD, dbias (per row, then one atomic add per
-//     CTA) and dB, dC (a transpose-reduction over the warp's 32 rows through shared
-//     memory, then one atomic add per lane and step).
+// Two chunk-parallel passes over chunks of kBwdChunk steps, one thread per row:
+//  A. scan_bwd_summary_kernel: one backward sweep over every chunk gives its forward
+//     summary H_c (the state it leaves from a zero start), its reverse summary G_c
+//     (the gradient it sends to the chunk before from a zero incoming gradient) and
+//     S_c (its summed step); the last CTA of a row tile folds them forwards into
+//     every chunk's start state and backwards, Q_(c-1) = exp(A S_c) Q_c + G_c, into
+//     every chunk's incoming gradient Q_c;
+//  B. scan_bwd_kernel: every chunk recomputes its states forward from its start
+//     state, window by window (the states after a window's even steps held in
+//     registers, the windows' start states in shared memory),
+//     and sweeps them backwards from Q_c, writing du, ddelta, dz and accumulating
+//     dA, dD, dbias (per row, then one atomic add per CTA) and dB, dC (a
+//     transpose-reduction over the warp's 32 rows through shared memory, then one
+//     atomic add per lane and step).
 #pragma once
 
 #include <cstdint>
@@ -31,7 +32,7 @@
 
 namespace mssm {
 
-constexpr int kBwdChunk = 64;  // steps per chunk (the forward summaries' quantum)
+constexpr int kBwdChunk = 64;  // steps per chunk
 constexpr int kBwdRows = 32;   // rows per CTA (one warp)
 
 struct BwdArgs {
@@ -63,11 +64,11 @@ struct BwdArgs {
   int nseg, tiles_per_batch;
   int vec_rows;       // u, delta, dout, z, du, ddelta, dz rows start 16-byte aligned
   int force_general;  // never take the structured-A powers
-  const float* hstart;  // [nseg-1][rows][16]: start state of chunk k+1 at k (pass A)
-  float* ws_G;          // [nseg][rows][16]: pass B outgoing gradient of chunk c
-  float* ws_S;          // [nseg][rows]: pass B summed step of chunk c
-  float* ws_Q;          // [nseg][rows][16]: incoming gradient of chunk c (pass B fold)
-  unsigned* ws_count;   // [tiles]: pass B arrivals, reset by the folding CTA
+  float* hstart;    // [nseg-1][rows][16]: chunk k's summary H_k, then (folded) chunk k+1's start state
+  float* ws_G;      // [nseg][rows][16]: outgoing gradient summary G_c of chunk c
+  float* ws_S;      // [nseg][rows]: summed step S_c of chunk c
+  float* ws_Q;      // [nseg][rows][16]: incoming gradient of chunk c (the fold)
+  unsigned* ws_count;  // [tiles]: pass A arrivals, reset by the folding CTA
 };
 
 // dt of one step: softplus(delta + bias) or delta + bias; also sigmoid(delta + bias), the
@@ -116,12 +117,35 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& p, int d, BwdRow& r) {
 }
 
 // B and C of steps [t0, t0 + kBwdChunk) of batch b into shared memory, fp32 [t][32]
-// (B in 0..15, C in 16..31); zero past L.  Each of the 32 threads loads one row of B or C.
+// (B in 0..15, C in 16..31); zero past L.  Each of the 32 threads loads one row of B or C,
+// as 16-byte blocks where the row's chunk is whole and aligned.
 template <typename T>
 __device__ __forceinline__ void bwd_stage_bc(const BwdArgs& p, int b, int t0, float (*bc)[32]) {
   const int r = threadIdx.x;
   const T* base = r < 16 ? static_cast<const T*>(p.B) + int64_t(b) * p.B_sb + int64_t(r) * p.B_sn
                          : static_cast<const T*>(p.C) + int64_t(b) * p.C_sb + int64_t(r - 16) * p.C_sn;
+  constexpr int kPer = 16 / int(sizeof(T));  // elements per 16-byte block
+  if (t0 + kBwdChunk <= p.L && (reinterpret_cast<uintptr_t>(base + t0) & 15) == 0) {
+    const uint4* src = reinterpret_cast<const uint4*>(base + t0);
+    uint4 v[kBwdChunk / kPer];
+#pragma unroll
+    for (int i = 0; i < kBwdChunk / kPer; ++i) v[i] = __ldg(src + i);
+#pragma unroll
+    for (int i = 0; i < kBwdChunk / kPer; ++i) {
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          bc[i * 8 + 2 * e][r] = bf16lo(w[e]);
+          bc[i * 8 + 2 * e + 1][r] = bf16hi(w[e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) bc[i * 4 + e][r] = __uint_as_float(w[e]);
+      }
+    }
+    return;
+  }
   for (int j = 0; j < kBwdChunk; ++j) {
     const int t = t0 + j;
     bc[j][r] = t < p.L ? Elem<T>::load(base + t) : 0.0f;
@@ -158,12 +182,12 @@ __device__ __forceinline__ float warp_transpose_sum(float (&v)[32], float* s) {
 }
 
 // ---------------------------------------------------------------------------
-// pass C: recompute the chunk's states and sweep them backwards.  The chunk is
+// pass B: recompute the chunk's states and sweep them backwards.  The chunk is
 // walked in windows of kBwdWin steps: a first forward sweep leaves each window's
 // start state in shared memory (2 KB per window for the warp); then, window by
-// window from the last, the window's kBwdWin states are recomputed into
-// registers and swept backwards.  The window's inputs are read once, as 16-byte
-// blocks where the rows allow.
+// window from the last, the window's states are recomputed into registers and
+// swept backwards.  The window's inputs are read once, as 16-byte blocks where the
+// rows allow.
 // ---------------------------------------------------------------------------
 constexpr int kBwdWin = 8;
 
@@ -187,6 +211,51 @@ __device__ __forceinline__ void bwd_load_win(const void* base, int64_t off, int 
       v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
     }
   } else {
+#pragma unroll
+    for (int j = 0; j < kBwdWin; ++j) v[j] = t + j < t_end ? Elem<T>::load(row + t + j) : 0.0f;
+  }
+}
+
+// A window's raw 16-byte blocks of one row (kBwdWin steps), fetched ahead of their use.
+template <typename T>
+struct WinBuf {
+  uint4 q[kBwdWin * sizeof(T) / 16];
+};
+
+template <typename T>
+__device__ __forceinline__ void bwd_fetch_win(const void* base, int64_t off, int t, int t_end, bool vec,
+                                              WinBuf<T>& wb) {
+  if (vec && t + kBwdWin <= t_end) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(base) + off + t);
+#pragma unroll
+    for (int i = 0; i < int(kBwdWin * sizeof(T) / 16); ++i) wb.q[i] = __ldg(src + i);
+  }
+}
+
+// the window's values from its fetched blocks (or, for a partial window or an unaligned row,
+// by plain loads now)
+template <typename T>
+__device__ __forceinline__ void bwd_unpack_win(const void* base, int64_t off, int t, int t_end, bool vec,
+                                               const WinBuf<T>& wb, float (&v)[kBwdWin]) {
+  if (vec && t + kBwdWin <= t_end) {
+    if constexpr (sizeof(T) == 2) {
+      const uint32_t ws[4] = {wb.q[0].x, wb.q[0].y, wb.q[0].z, wb.q[0].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = bf16lo(ws[i]);
+        v[2 * i + 1] = bf16hi(ws[i]);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        v[4 * i] = __uint_as_float(wb.q[i].x);
+        v[4 * i + 1] = __uint_as_float(wb.q[i].y);
+        v[4 * i + 2] = __uint_as_float(wb.q[i].z);
+        v[4 * i + 3] = __uint_as_float(wb.q[i].w);
+      }
+    }
+  } else {
+    const T* row = static_cast<const T*>(base) + off;
 #pragma unroll
     for (int j = 0; j < kBwdWin; ++j) v[j] = t + j < t_end ? Elem<T>::load(row + t + j) : 0.0f;
   }
@@ -247,40 +316,53 @@ __device__ __forceinline__ void bwd_decay(float dt, const BwdRow& r, f2_t (&a)[k
 }
 
 // ---------------------------------------------------------------------------
-// pass B: the g recurrence of chunk c >= 1 from a zero incoming gradient, walked
-// backwards in windows of kBwdWin steps (16-byte loads of delta, dout and z where
-// the rows allow) with the 16 states as 8 packed pairs; then the fold, by the last
-// CTA of the row tile to arrive.
+// pass A: one backward sweep over chunk c gives both of its summaries, sharing the
+// step's dt and decay powers: the forward one, H_c = sum_t (prod_(s>t) a_s) dt_t u_t B_t
+// (the state the chunk leaves from a zero start, accumulated with the running product
+// P of the later steps' decays), and the reverse one, G_c (the gradient the chunk sends
+// to the one before from a zero incoming gradient: g = a (g + gy C) from the last step
+// to the first), plus S_c = sum_t dt_t.  The last CTA of a row tile to arrive folds
+// them: forwards, start_(c+1) = exp(A S_c) start_c + H_c from start_0 = 0, and
+// backwards, Q_(c-1) = exp(A S_c) Q_c + G_c from Q_(nseg-1) = 0.  Windows of kBwdWin
+// steps, 16-byte loads of u, delta, dout and z where the rows allow, the 16 states as 8
+// packed pairs.
 // ---------------------------------------------------------------------------
-
-// C of steps [t0, t0 + kBwdChunk) of batch b into shared memory, fp32 [t][16]; zero past L.
-// Thread i loads row i % 16 over one half of the steps.
-template <typename T>
-__device__ __forceinline__ void bwd_stage_c(const BwdArgs& p, int b, int t0, float (*cs)[kN]) {
-  const int n = threadIdx.x & (kN - 1);
-  const int j0 = (threadIdx.x / kN) * (kBwdChunk / 2);
-  const T* base = static_cast<const T*>(p.C) + int64_t(b) * p.C_sb + int64_t(n) * p.C_sn;
-#pragma unroll 8
-  for (int j = j0; j < j0 + kBwdChunk / 2; ++j) {
-    const int t = t0 + j;
-    cs[j][n] = t < p.L ? Elem<T>::load(base + t) : 0.0f;
-  }
-}
-
 template <typename T, bool HAS_Z, bool STRUCT>
-__device__ __forceinline__ void bwd_summary_chunk(const BwdArgs& p, const BwdRow& r, const float (*cs)[kN], int b,
-                                                  int dc, int t0, int t1, f2_t (&g2)[8], float& ssum) {
+__device__ __forceinline__ void bwd_summary_chunk(const BwdArgs& p, const BwdRow& r, const float (*bc)[32], int b,
+                                                  int dc, int t0, int t1, f2_t (&H)[kN / 2], f2_t (&g2)[kN / 2],
+                                                  float& ssum) {
+  const int64_t uo = int64_t(b) * p.u_sb + int64_t(dc) * p.u_sd;
   const int64_t ro = int64_t(b) * p.dl_sb + int64_t(dc) * p.dl_sd;
   const int64_t go = int64_t(b) * p.g_sb + int64_t(dc) * p.g_sd;
   const int64_t zo = int64_t(b) * p.z_sb + int64_t(dc) * p.z_sd;
   const bool vin = p.vec_rows != 0;
+  f2_t P[kN / 2];
+#pragma unroll
+  for (int k = 0; k < kN / 2; ++k) P[k] = f2(1.0f, 1.0f);
   const int nwin = (t1 - t0 + kBwdWin - 1) / kBwdWin;
+  // the inputs of window w are fetched while window w + 1 is swept
+  WinBuf<T> nu, nd, ng, nz;
+  {
+    const int tw = t0 + (nwin - 1) * kBwdWin;
+    bwd_fetch_win<T>(p.u, uo, tw, t1, vin, nu);
+    bwd_fetch_win<T>(p.delta, ro, tw, t1, vin, nd);
+    bwd_fetch_win<T>(p.dout, go, tw, t1, vin, ng);
+    if constexpr (HAS_Z) bwd_fetch_win<T>(p.z, zo, tw, t1, vin, nz);
+  }
   for (int w = nwin - 1; w >= 0; --w) {
     const int tw = t0 + w * kBwdWin;
-    float dl[kBwdWin], gd[kBwdWin], zz[kBwdWin];
-    bwd_load_win<T>(p.delta, ro, tw, t1, vin, dl);
-    bwd_load_win<T>(p.dout, go, tw, t1, vin, gd);
-    if constexpr (HAS_Z) bwd_load_win<T>(p.z, zo, tw, t1, vin, zz);
+    const WinBuf<T> cu = nu, cd = nd, cg = ng, cz = nz;
+    if (w > 0) {
+      bwd_fetch_win<T>(p.u, uo, tw - kBwdWin, t1, vin, nu);
+      bwd_fetch_win<T>(p.delta, ro, tw - kBwdWin, t1, vin, nd);
+      bwd_fetch_win<T>(p.dout, go, tw - kBwdWin, t1, vin, ng);
+      if constexpr (HAS_Z) bwd_fetch_win<T>(p.z, zo, tw - kBwdWin, t1, vin, nz);
+    }
+    float uu[kBwdWin], dl[kBwdWin], gd[kBwdWin], zz[kBwdWin];
+    bwd_unpack_win<T>(p.u, uo, tw, t1, vin, cu, uu);
+    bwd_unpack_win<T>(p.delta, ro, tw, t1, vin, cd, dl);
+    bwd_unpack_win<T>(p.dout, go, tw, t1, vin, cg, gd);
+    if constexpr (HAS_Z) bwd_unpack_win<T>(p.z, zo, tw, t1, vin, cz, zz);
 #pragma unroll
     for (int j = kBwdWin - 1; j >= 0; --j) {
       if (tw + j >= t1) continue;  // past the end of the sequence (a partial last window)
@@ -294,11 +376,15 @@ __device__ __forceinline__ void bwd_summary_chunk(const BwdArgs& p, const BwdRow
       }
       f2_t a[kN / 2];
       bwd_decay<STRUCT>(dt, r, a);
-      const f2_t gy2 = f2(gy, gy);
-      const ulonglong2* cq = reinterpret_cast<const ulonglong2*>(cs[tw - t0 + j]);
+      const f2_t gy2 = f2(gy, gy), w2 = f2(dt * uu[j], dt * uu[j]);
+      const ulonglong2* q = reinterpret_cast<const ulonglong2*>(bc[tw - t0 + j]);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const ulonglong2 cc = cq[k];  // C pairs (4k, 4k+1), (4k+2, 4k+3)
+        const ulonglong2 bb = q[k], cc = q[4 + k];  // B and C pairs (4k, 4k+1), (4k+2, 4k+3)
+        H[2 * k] = fma2(P[2 * k], mul2(w2, bb.x), H[2 * k]);
+        H[2 * k + 1] = fma2(P[2 * k + 1], mul2(w2, bb.y), H[2 * k + 1]);
+        P[2 * k] = mul2(P[2 * k], a[2 * k]);
+        P[2 * k + 1] = mul2(P[2 * k + 1], a[2 * k + 1]);
         g2[2 * k] = mul2(a[2 * k], fma2(gy2, cc.x, g2[2 * k]));
         g2[2 * k + 1] = mul2(a[2 * k + 1], fma2(gy2, cc.y, g2[2 * k + 1]));
       }
@@ -307,13 +393,30 @@ __device__ __forceinline__ void bwd_summary_chunk(const BwdArgs& p, const BwdRow
   }
 }
 
+__device__ __forceinline__ void bwd_store16(float* dst, const f2_t (&v)[kN / 2]) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float x0, x1, x2, x3;
+    f2split(v[2 * i], x0, x1);
+    f2split(v[2 * i + 1], x2, x3);
+    __stcg(d4 + i, make_float4(x0, x1, x2, x3));
+  }
+}
+
+__device__ __forceinline__ void bwd_load16(const float* src, float4 (&v)[4]) {
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __ldcg(s4 + i);
+}
+
 template <typename T, bool HAS_Z>
 __global__ void __launch_bounds__(kBwdRows) scan_bwd_summary_kernel(const BwdArgs p) {
-  __shared__ __align__(16) float cs[kBwdChunk][kN];
+  __shared__ __align__(16) float bc_s[kBwdChunk][32];
   __shared__ int s_last;
   const int tid = threadIdx.x;
   const int tile = blockIdx.x;
-  const int c = blockIdx.y + 1;
+  const int c = blockIdx.y;
   const int b = tile / p.tiles_per_batch;
   const int d = (tile - b * p.tiles_per_batch) * kBwdRows + tid;
   const int dc = d < p.D ? d : p.D - 1;
@@ -322,74 +425,93 @@ __global__ void __launch_bounds__(kBwdRows) scan_bwd_summary_kernel(const BwdArg
   BwdRow r;
   bwd_row(p, dc, r);
   const bool structured = __syncthreads_and(r.structured) && !p.force_general;
-  bwd_stage_c<T>(p, b, t0, cs);
+  bwd_stage_bc<T>(p, b, t0, bc_s);
   __syncthreads();
 
-  f2_t g2[8];
+  f2_t H[kN / 2], g2[kN / 2];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) g2[k] = f2(0.0f, 0.0f);
+  for (int k = 0; k < kN / 2; ++k) H[k] = g2[k] = f2(0.0f, 0.0f);
   float ssum = 0.0f;
   if (structured)
-    bwd_summary_chunk<T, HAS_Z, true>(p, r, cs, b, dc, t0, t1, g2, ssum);
+    bwd_summary_chunk<T, HAS_Z, true>(p, r, bc_s, b, dc, t0, t1, H, g2, ssum);
   else
-    bwd_summary_chunk<T, HAS_Z, false>(p, r, cs, b, dc, t0, t1, g2, ssum);
+    bwd_summary_chunk<T, HAS_Z, false>(p, r, bc_s, b, dc, t0, t1, H, g2, ssum);
   const int64_t rows_total = int64_t(p.Bt) * p.tiles_per_batch * kBwdRows;
   const int64_t rowg = int64_t(tile) * kBwdRows + tid;
-  {
-    float gv[kN];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) f2split(g2[k], gv[2 * k], gv[2 * k + 1]);
-    float4* dst = reinterpret_cast<float4*>(p.ws_G + (int64_t(c) * rows_total + rowg) * kN);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) __stcg(dst + i, make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]));
-    __stcg(p.ws_S + int64_t(c) * rows_total + rowg, ssum);
-  }
-  // the last CTA of the row tile folds backwards: Q_(nseg-1) = 0, Q_(c-1) = exp(A S_c) Q_c + G_c,
-  // with chunk c-1's summary fetched while chunk c's is applied
+  // the first chunk sends no gradient back, and the last one's end state starts nothing
+  if (c + 1 < p.nseg) bwd_store16(p.hstart + (int64_t(c) * rows_total + rowg) * kN, H);
+  if (c > 0) bwd_store16(p.ws_G + (int64_t(c) * rows_total + rowg) * kN, g2);
+  __stcg(p.ws_S + int64_t(c) * rows_total + rowg, ssum);
+
+  // the last CTA of the row tile to arrive folds both ways
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&p.ws_count[tile], 1u) == unsigned(p.nseg - 2));
+  if (tid == 0) s_last = (atomicAdd(&p.ws_count[tile], 1u) == unsigned(p.nseg - 1));
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  auto fetch = [&](int k, float& sk, float4 (&gk)[4]) {
-    sk = __ldcg(p.ws_S + int64_t(k) * rows_total + rowg);
-    const float4* gs = reinterpret_cast<const float4*>(p.ws_G + (int64_t(k) * rows_total + rowg) * kN);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) gk[i] = __ldcg(gs + i);
-  };
-  f2_t q[kN / 2];
-#pragma unroll
-  for (int k = 0; k < kN / 2; ++k) q[k] = f2(0.0f, 0.0f);
-  float s_cur = 0.0f;
-  float4 g_cur[4];
-  fetch(p.nseg - 1, s_cur, g_cur);
-  for (int k = p.nseg - 1; k >= 0; --k) {
-    float4* qd = reinterpret_cast<float4*>(p.ws_Q + (int64_t(k) * rows_total + rowg) * kN);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float q0, q1, q2, q3;
-      f2split(q[2 * i], q0, q1);
-      f2split(q[2 * i + 1], q2, q3);
-      __stcg(qd + i, make_float4(q0, q1, q2, q3));
-    }
-    if (k == 0) break;
-    float s_nx = 0.0f;
-    float4 g_nx[4] = {};
-    if (k > 1) fetch(k - 1, s_nx, g_nx);
-    f2_t a[kN / 2];
+  auto decay_of = [&](float sk, f2_t (&a)[kN / 2]) {
     if (structured)
-      bwd_decay<true>(s_cur, r, a);
+      bwd_decay<true>(sk, r, a);
     else
-      bwd_decay<false>(s_cur, r, a);
+      bwd_decay<false>(sk, r, a);
+  };
+  // forwards: hstart[k] (the start state of chunk k + 1) = exp(A S_k) hstart[k - 1] + H_k, in place
+  {
+    f2_t h[kN / 2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      q[2 * i] = fma2(a[2 * i], q[2 * i], f2(g_cur[i].x, g_cur[i].y));
-      q[2 * i + 1] = fma2(a[2 * i + 1], q[2 * i + 1], f2(g_cur[i].z, g_cur[i].w));
+    for (int k = 0; k < kN / 2; ++k) h[k] = f2(0.0f, 0.0f);
+    float s_cur = __ldcg(p.ws_S + rowg);
+    float4 h_cur[4];
+    bwd_load16(p.hstart + rowg * kN, h_cur);
+    for (int k = 0; k + 1 < p.nseg; ++k) {
+      float s_nx = 0.0f;
+      float4 h_nx[4] = {};
+      if (k + 2 < p.nseg) {  // the next chunk's summary, fetched while this one is applied
+        s_nx = __ldcg(p.ws_S + int64_t(k + 1) * rows_total + rowg);
+        bwd_load16(p.hstart + (int64_t(k + 1) * rows_total + rowg) * kN, h_nx);
+      }
+      f2_t a[kN / 2];
+      decay_of(s_cur, a);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        h[2 * i] = fma2(a[2 * i], h[2 * i], f2(h_cur[i].x, h_cur[i].y));
+        h[2 * i + 1] = fma2(a[2 * i + 1], h[2 * i + 1], f2(h_cur[i].z, h_cur[i].w));
+      }
+      bwd_store16(p.hstart + (int64_t(k) * rows_total + rowg) * kN, h);
+      s_cur = s_nx;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) h_cur[i] = h_nx[i];
     }
-    s_cur = s_nx;
+  }
+  // backwards: Q_(nseg-1) = 0, Q_(k-1) = exp(A S_k) Q_k + G_k
+  {
+    f2_t q[kN / 2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) g_cur[i] = g_nx[i];
+    for (int k = 0; k < kN / 2; ++k) q[k] = f2(0.0f, 0.0f);
+    float s_cur = __ldcg(p.ws_S + int64_t(p.nseg - 1) * rows_total + rowg);
+    float4 g_cur[4];
+    bwd_load16(p.ws_G + (int64_t(p.nseg - 1) * rows_total + rowg) * kN, g_cur);
+    for (int k = p.nseg - 1; k >= 0; --k) {
+      bwd_store16(p.ws_Q + (int64_t(k) * rows_total + rowg) * kN, q);
+      if (k == 0) break;
+      float s_nx = 0.0f;
+      float4 g_nx[4] = {};
+      if (k > 1) {
+        s_nx = __ldcg(p.ws_S + int64_t(k - 1) * rows_total + rowg);
+        bwd_load16(p.ws_G + (int64_t(k - 1) * rows_total + rowg) * kN, g_nx);
+      }
+      f2_t a[kN / 2];
+      decay_of(s_cur, a);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        q[2 * i] = fma2(a[2 * i], q[2 * i], f2(g_cur[i].x, g_cur[i].y));
+        q[2 * i + 1] = fma2(a[2 * i + 1], q[2 * i + 1], f2(g_cur[i].z, g_cur[i].w));
+      }
+      s_cur = s_nx;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) g_cur[i] = g_nx[i];
+    }
   }
   if (tid == 0) p.ws_count[tile] = 0u;
 }
@@ -407,10 +529,15 @@ __device__ __forceinline__ void bwd_fwd_step(const f2_t (&a)[kN / 2], float wv, 
   }
 }
 
+// The backward sweep of one chunk.  Registers hold a window's states after its even steps
+// only (he[i] = h after 2i of its steps, he[0] its start); the chain rule needs, at step
+// j, the state after the step (h_post) and a_j h_pre, which is h_post - (dt u)_j B_j, so
+// a state after an odd step is never needed before the step itself recomputes it.  The
+// window start states live in shared memory, [window][pair][lane] (2 KB per window).
 template <typename T, bool HAS_Z, bool STRUCT>
 __device__ __forceinline__ void bwd_chunk(const BwdArgs& p, const BwdRow& r, const float (*bc)[32],
-                                          f2_t (*hwin)[kN / 2][kBwdRows], int b, bool row_ok, int dc, int t0,
-                                          int t1, f2_t (&h)[kN / 2], f2_t (&g)[kN / 2], f2_t (&dA)[kN / 2],
+                                          f2_t (*hwin)[kN / 2][kBwdRows], int b, bool row_ok, int dc, int t0, int t1,
+                                          f2_t (&h)[kN / 2], f2_t (&g)[kN / 2], f2_t (&dA)[kN / 2],
                                           float& dDacc, float& dbacc) {
   const int tid = threadIdx.x;
   const int64_t uo = int64_t(b) * p.u_sb + int64_t(dc) * p.u_sd;
@@ -422,11 +549,11 @@ __device__ __forceinline__ void bwd_chunk(const BwdArgs& p, const BwdRow& r, con
   const int64_t dzo = int64_t(b) * p.dz_sb + int64_t(dc) * p.dz_sd;
   const bool vin = p.vec_rows != 0;
   const int nwin = (t1 - t0 + kBwdWin - 1) / kBwdWin;
-  // forward: every window's start state
-  for (int w = 0; w < nwin; ++w) {
+  // forward: every window's start state but the last one's to the scratch; h ends as the
+  // last window's start state
+  for (int w = 0; w + 1 < nwin; ++w) {
 #pragma unroll
     for (int k = 0; k < kN / 2; ++k) hwin[w][k][tid] = h[k];
-    if (w + 1 == nwin) break;
     const int tw = t0 + w * kBwdWin;
     float uu[kBwdWin], dl[kBwdWin];
     bwd_load_win<T>(p.u, uo, tw, t1, vin, uu);
@@ -443,26 +570,37 @@ __device__ __forceinline__ void bwd_chunk(const BwdArgs& p, const BwdRow& r, con
   // backward, window by window
   for (int w = nwin - 1; w >= 0; --w) {
     const int tw = t0 + w * kBwdWin;
+    f2_t he[kBwdWin / 2 + 1][kN / 2];
+    if (w + 1 == nwin) {
+#pragma unroll
+      for (int k = 0; k < kN / 2; ++k) he[0][k] = h[k];
+    } else {
+#pragma unroll
+      for (int k = 0; k < kN / 2; ++k) he[0][k] = hwin[w][k][tid];
+    }
+    // slots w (just read, or never written for the last window) and w + 1 (read for the
+    // window before) are free: the 4 KB buffer of the dB/dC reduction
+    __syncwarp();
+    float* red_s = reinterpret_cast<float*>(&hwin[w][0][0]);
     float uu[kBwdWin], dl[kBwdWin], go_[kBwdWin], zz[kBwdWin];
     bwd_load_win<T>(p.u, uo, tw, t1, vin, uu);
     bwd_load_win<T>(p.delta, ro, tw, t1, vin, dl);
     bwd_load_win<T>(p.dout, go, tw, t1, vin, go_);
     if constexpr (HAS_Z) bwd_load_win<T>(p.z, zo, tw, t1, vin, zz);
-    // recompute the window's states into registers
-    f2_t hs[kBwdWin + 1][kN / 2];  // hs[0]: the window's start state, hs[j + 1]: after step j
+    // recompute the window's states; keep those after its even steps
+    {
+      f2_t odd[kN / 2];
 #pragma unroll
-    for (int k = 0; k < kN / 2; ++k) hs[0][k] = hwin[w][k][tid];
-    // slots w (just read) and w + 1 (read for the window before) are free: the 4 KB buffer
-    // of the dB/dC reduction
-    __syncwarp();
-    float* red_s = reinterpret_cast<float*>(&hwin[w][0][0]);
-#pragma unroll
-    for (int j = 0; j < kBwdWin; ++j) {
-      float dsp;  // unused here
-      const float dt = bwd_dt(dl[j], r.bias, p.softplus, dsp);
-      f2_t a[kN / 2];
-      bwd_decay<STRUCT>(dt, r, a);
-      bwd_fwd_step(a, dt * uu[j], bc[tw - t0 + j], hs[j], hs[j + 1]);
+      for (int j = 0; j < kBwdWin; ++j) {
+        float dsp;  // unused here
+        const float dt = bwd_dt(dl[j], r.bias, p.softplus, dsp);
+        f2_t a[kN / 2];
+        bwd_decay<STRUCT>(dt, r, a);
+        if (j % 2 == 0)
+          bwd_fwd_step(a, dt * uu[j], bc[tw - t0 + j], he[j / 2], odd);
+        else
+          bwd_fwd_step(a, dt * uu[j], bc[tw - t0 + j], odd, he[j / 2 + 1]);
+      }
     }
     float du_w[kBwdWin], dd_w[kBwdWin], dz_w[kBwdWin];
 #pragma unroll
@@ -478,14 +616,29 @@ __device__ __forceinline__ void bwd_chunk(const BwdArgs& p, const BwdRow& r, con
       bwd_decay<STRUCT>(dt, r, a);
       // B pairs at q[0..3], C pairs at q[4..7], read where they are used
       const ulonglong2* q = reinterpret_cast<const ulonglong2*>(bc[t - t0]);
+      const float wv = dt * uu[j];
+      // post: the state after step j; ah: a_j times the state before it
+      f2_t post[kN / 2], ah[kN / 2];
+#pragma unroll
+      for (int k = 0; k < kN / 2; ++k) {
+        const ulonglong2 bb = q[k >> 1];
+        const f2_t Bk = (k & 1) ? bb.y : bb.x;
+        if (j % 2 == 0) {
+          ah[k] = mul2(a[k], he[j / 2][k]);
+          post[k] = fma2(f2(wv, wv), Bk, ah[k]);
+        } else {
+          post[k] = he[j / 2 + 1][k];
+          ah[k] = fma2(f2(-wv, -wv), Bk, post[k]);
+        }
+      }
       float gy = go_[j];
       if constexpr (HAS_Z) {
         f2_t ya = f2(0.0f, 0.0f);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const ulonglong2 cc = q[4 + k];
-          ya = fma2(cc.x, hs[j + 1][2 * k], ya);
-          ya = fma2(cc.y, hs[j + 1][2 * k + 1], ya);
+          ya = fma2(cc.x, post[2 * k], ya);
+          ya = fma2(cc.y, post[2 * k + 1], ya);
         }
         float y0, y1;
         f2split(ya, y0, y1);
@@ -507,8 +660,8 @@ __device__ __forceinline__ void bwd_chunk(const BwdArgs& p, const BwdRow& r, con
         const ulonglong2 bb = q[k >> 1], cc = q[4 + (k >> 1)];
         const f2_t Bk = (k & 1) ? bb.y : bb.x, Ck = (k & 1) ? cc.y : cc.x;
         g[k] = fma2(gy2, Ck, g[k]);
-        f2split(mul2(gym2, hs[j + 1][k]), red[16 + 2 * k], red[17 + 2 * k]);
-        const f2_t gah = mul2(mul2(g[k], a[k]), hs[j][k]);
+        f2split(mul2(gym2, post[k]), red[16 + 2 * k], red[17 + 2 * k]);
+        const f2_t gah = mul2(g[k], ah[k]);
         ddt2 = fma2(g[k], mul2(Bk, u2), fma2(r.A[k], gah, ddt2));
         dA[k] = fma2(gah, dt2, dA[k]);
         const f2_t gdt = mul2(g[k], dt2);
@@ -537,8 +690,13 @@ __device__ __forceinline__ void bwd_chunk(const BwdArgs& p, const BwdRow& r, con
   }
 }
 
+// pass B's register cap per thread, which sets its occupancy (one-warp CTAs, 65536 registers
+// per SM)
+#ifndef MSSM_BWD_MAXNREG
+#define MSSM_BWD_MAXNREG 255
+#endif
 template <typename T, bool HAS_Z>
-__global__ void __launch_bounds__(kBwdRows) scan_bwd_kernel(const BwdArgs p) {
+__global__ void __maxnreg__(MSSM_BWD_MAXNREG) scan_bwd_kernel(const BwdArgs p) {
   __shared__ __align__(16) float bc_s[kBwdChunk][32];
   // window start states, and one spare slot so that two free slots always follow window w
   __shared__ __align__(16) f2_t hwin[kBwdChunk / kBwdWin + 1][kN / 2][kBwdRows];

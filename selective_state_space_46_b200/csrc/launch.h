@@ -39,8 +39,8 @@ cudaError_t launch_state_update(const DecodeArgs& a, int dtype, bool has_z, Deco
 // Causal conv1d + SiLU: grid (ceil(rows / kConvWarps), items); one decode step of it.
 cudaError_t launch_causal_conv1d(const ConvArgs& a, int items, int dtype, bool silu, cudaStream_t s);
 cudaError_t launch_causal_conv1d_update(const ConvUpdateArgs& a, int dtype, cudaStream_t s);
-// Backward scan, passes B and C (pass A: launch_scan_chunk_state with 32-row tiles and
-// chunks of kBwdChunk steps, into the same workspace rows).
+// Backward scan: pass A (chunk summaries both ways and their folds, when there is more than
+// one chunk) and pass B (recompute and backward sweep per chunk).
 cudaError_t launch_scan_bwd(const BwdArgs& a, int dtype, bool has_z, cudaStream_t s);
 // Reads (and optionally clears) the current device's error word.
 cudaError_t read_device_error(unsigned int* value, bool clear);
