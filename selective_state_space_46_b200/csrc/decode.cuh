@@ -261,6 +261,18 @@ __device__ __forceinline__ float smem_elem(const unsigned char* base, int j) {
   return Elem<T>::load(reinterpret_cast<const T*>(base) + j);
 }
 
+// values 4q .. 4q+3 of a 16-value run of T in shared memory (16-byte aligned), one load
+template <typename T>
+__device__ __forceinline__ void smem_quarter(const unsigned char* base, int q, float (&v)[4]) {
+  if constexpr (sizeof(T) == 2) {
+    const uint2 w = *reinterpret_cast<const uint2*>(base + q * 8);
+    v[0] = bf16lo(w.x); v[1] = bf16hi(w.x); v[2] = bf16lo(w.y); v[3] = bf16hi(w.y);
+  } else {
+    const float4 w = *reinterpret_cast<const float4*>(base + q * 16);
+    v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
+  }
+}
+
 template <typename T, bool HAS_Z>
 __global__ void __launch_bounds__(kWsWarps * 32, kStreamCtasPerSm) state_update_stream_kernel(const DecodeArgs p) {
   using L = StreamSlot<T>;
@@ -347,17 +359,19 @@ __global__ void __launch_bounds__(kWsWarps * 32, kStreamCtasPerSm) state_update_
         const int q = (kq + rot) & 3;
         float4 h = hs[q];
         float hv[4] = {h.x, h.y, h.z, h.w};
+        float bq[4], cq[4];  // B and C of states 4q .. 4q+3, one shared load each
+        smem_quarter<T>(slot + L::kB, q, bq);
+        smem_quarter<T>(slot + L::kC, q, cq);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int n = 4 * q + e;
           const float ed = ex2f(dt * a2r[4 * kq + e]);
           float gn = w;
           if (p.zoh) {
             const float an = a2r[4 * kq + e] * kLn2;
             gn = zoh_gain_f(ed, dt, an, an != 0.0f ? rcpf(an) : 0.0f) * x;
           }
-          hv[e] = fmaf(ed, hv[e], gn * smem_elem<T>(slot + L::kB, n));
-          y = fmaf(smem_elem<T>(slot + L::kC, n), hv[e], y);
+          hv[e] = fmaf(ed, hv[e], gn * bq[e]);
+          y = fmaf(cq[e], hv[e], y);
         }
         hs[q] = make_float4(hv[0], hv[1], hv[2], hv[3]);
       }
