@@ -820,7 +820,8 @@ def run_e2e(args, kind, inp, d, dev, m, units, world):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 50; 1000 successive steps for the decode workload)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mssm", "reference"], default="mssm")
     ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default=DEFAULT_WORKLOAD)
@@ -844,6 +845,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.steps is None:
+        decode = synth.WORKLOADS[args.workload]["kind"] == "decode"
+        args.steps = 1000 if decode and args.impl == "mssm" else 50
     if args.impl == "reference":
         return run_reference(args)
     return run_mssm(args)
