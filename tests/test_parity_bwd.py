@@ -72,6 +72,15 @@ def test_bwd_optional_inputs(cuda_device, with_z, with_D, with_bias, softplus):
     compare(g, ref, "f32")
 
 
+@pytest.mark.parametrize("Bt,D,L", [(1, 40, 1000), (2, 33, 1096), (1, 40, 8192)])
+def test_bwd_aligned_rows_ragged_chunks(cuda_device, Bt, D, L):
+    """bf16 rows that start 16-byte aligned (the vector loads and the 16-byte B/C staging)
+    with a last chunk of 40 or 8 steps, and 128 chunks folded both ways."""
+    inp = synth.make_scan_inputs(Bt, D, L, io_dtype="bf16", seed=L + D)
+    g, ref = run_bwd(inp, seed=L)
+    compare(g, ref, "bf16")
+
+
 def test_bwd_default_workload_shape(cuda_device):
     """2 x 512 x 2048 (a quarter of the default prefill's channels), bf16."""
     inp = synth.make_scan_inputs(2, 512, 2048, io_dtype="bf16", seed=9)
