@@ -347,6 +347,45 @@ __device__ __forceinline__ void store_block(T* row, int t, int t_lo, int t_end, 
   }
 }
 
+// 2^x for a pair of exponents on the FP32 pipe, for the general-A path, whose 16
+// exponentials per element make the SFU its busiest unit: kExpFmaPairs of the 8 pairs take
+// this form, the rest ex2 (measured on B200, one pair of eight: 2552 -> 2418 us on
+// 1 x 2048 x 131072, 88.6 -> 86.2 us on 2 x 1536 x 2048; two or three pairs load the FP32
+// pipe more than they relieve the SFU).  Cody and Waite's reduction x = j + f, with j the integer nearest
+// x (adding and subtracting 1.5 * 2^23 rounds it) and f = x - j in [-1/2, 1/2] exactly; 2^f by
+// a degree-5 polynomial whose coefficients are a minimax fit of the relative error
+// (fit_exp2.py: at most 1.9e-7 relative in fp32 Horner evaluation, as accurate as ex2.approx);
+// 2^j by adding j to the exponent field.  x is clamped to [-125, 127] first, so the result
+// stays a normal number (decay factors below 2^-125 act as zero, as ex2.approx.ftz's do below
+// 2^-126).
+constexpr int kExpFmaPairs = 1;
+constexpr float kExp2C0 = 1.0000001192092896f;
+constexpr float kExp2C1 = 0.6931470036506653f;
+constexpr float kExp2C2 = 0.24022118747234344f;
+constexpr float kExp2C3 = 0.05550695210695267f;
+constexpr float kExp2C4 = 0.009675589390099049f;
+constexpr float kExp2C5 = 0.0013282300205901265f;
+constexpr float kRoundShift = 12582912.0f;  // 1.5 * 2^23
+__device__ __forceinline__ f2_t exp2_fma2(f2_t x) {
+  float x0, x1;
+  f2split(x, x0, x1);
+  const f2_t xc = f2(fminf(fmaxf(x0, -125.0f), 127.0f), fminf(fmaxf(x1, -125.0f), 127.0f));
+  const f2_t t = add2(xc, f2(kRoundShift, kRoundShift));
+  const f2_t j = add2(t, f2(-kRoundShift, -kRoundShift));
+  const f2_t fr = fma2(j, f2(-1.0f, -1.0f), xc);
+  f2_t p = fma2(f2(kExp2C5, kExp2C5), fr, f2(kExp2C4, kExp2C4));
+  p = fma2(p, fr, f2(kExp2C3, kExp2C3));
+  p = fma2(p, fr, f2(kExp2C2, kExp2C2));
+  p = fma2(p, fr, f2(kExp2C1, kExp2C1));
+  p = fma2(p, fr, f2(kExp2C0, kExp2C0));
+  float t0, t1, p0, p1;
+  f2split(t, t0, t1);
+  f2split(p, p0, p1);
+  const int j0 = __float_as_int(t0) - __float_as_int(kRoundShift);
+  const int j1 = __float_as_int(t1) - __float_as_int(kRoundShift);
+  return f2(__int_as_float(__float_as_int(p0) + (j0 << 23)), __int_as_float(__float_as_int(p1) + (j1 << 23)));
+}
+
 // Powers a^1 .. a^16 as eight pairs (a^(2k+1), a^(2k+2)); 15 multiplies, depth 4.
 __device__ __forceinline__ void powers16(float a, f2_t (&dA)[8]) {
   const float a2 = a * a;
@@ -450,8 +489,14 @@ __device__ __forceinline__ float step_recurrence(const ulonglong2 (&bb)[4], cons
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       float lo, hi;
-      f2split(mul2(s2, rp.Ap[k]), lo, hi);
-      const float elo = ex2f(lo), ehi = ex2f(hi);
+      float elo, ehi;
+      if (k < kExpFmaPairs) {
+        f2split(exp2_fma2(mul2(s2, rp.Ap[k])), elo, ehi);
+      } else {
+        f2split(mul2(s2, rp.Ap[k]), lo, hi);
+        elo = ex2f(lo);
+        ehi = ex2f(hi);
+      }
       dA[k] = f2(elo, ehi);
       if constexpr (ZOH) {
         float alo, ahi, ilo, ihi;
@@ -589,7 +634,7 @@ __device__ __forceinline__ void forward_rows(const ScanArgs& p, float (*bc_s)[kT
   auto run_block = [&](auto partial_tag, int k, int lo, int valid, const float* bcrow, const uint4 (&ru)[R],
                        const uint4 (&rd)[R], const uint4 (&rz)[R]) {
     constexpr bool PARTIAL = decltype(partial_tag)::value;
-    float y[R][S];
+    [[maybe_unused]] float y[R][S];  // written and stored when READOUT
     if constexpr (!ZOH && READOUT && sizeof(T) == 2 && R == 1) {
       // steps in pairs: the per-step scalar arithmetic of two steps runs as f32x2 operations
       // (one row per thread only: with two, the extra pairs cost spills)
@@ -1103,9 +1148,13 @@ __device__ __forceinline__ void backward_rows(const ScanArgs& p, float (*bc_s)[k
             const f2_t w2 = f2(w, w);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-              float lo, hi;
-              f2split(mul2(T2, rp[i].Ap[kk]), lo, hi);
-              v[kk] = mul2(w2, f2(ex2f(lo), ex2f(hi)));
+              if (kk < kExpFmaPairs) {
+                v[kk] = mul2(w2, exp2_fma2(mul2(T2, rp[i].Ap[kk])));
+              } else {
+                float lo, hi;
+                f2split(mul2(T2, rp[i].Ap[kk]), lo, hi);
+                v[kk] = mul2(w2, f2(ex2f(lo), ex2f(hi)));
+              }
             }
           }
 #pragma unroll
