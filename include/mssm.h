@@ -253,8 +253,8 @@ mssm_status mssm_state_update_ex(mssm_tensor *state, const mssm_tensor *x,
  *   dD, ddelta_bias [D] f32, given exactly when D / delta_bias are
  * The f32 gradients must be dense; they are zeroed and accumulated with atomic
  * adds, so their rounding order is not fixed.  Uses a per-device workspace of
- * about (2 x 68 x L / 64) bytes per row, grown with cudaMalloc on demand (which
- * synchronises the device) and freed by mssm_shutdown().
+ * about 196 x L / 64 bytes per row (49 floats per 64-step chunk), grown with
+ * cudaMalloc on demand (which synchronises the device) and freed by mssm_shutdown().
  */
 mssm_status mssm_selective_scan_bwd(const mssm_tensor *u, const mssm_tensor *delta, const mssm_tensor *A,
                                     const mssm_tensor *B, const mssm_tensor *C, const mssm_tensor *D,
