@@ -353,18 +353,19 @@ __device__ __forceinline__ void store_block(T* row, int t, int t_lo, int t_end, 
 // 1 x 2048 x 131072, 88.6 -> 86.2 us on 2 x 1536 x 2048; two or three pairs load the FP32
 // pipe more than they relieve the SFU).  Cody and Waite's reduction x = j + f, with j the integer nearest
 // x (adding and subtracting 1.5 * 2^23 rounds it) and f = x - j in [-1/2, 1/2] exactly; 2^f by
-// a degree-5 polynomial whose coefficients are a minimax fit of the relative error
-// (fit_exp2.py: at most 1.9e-7 relative in fp32 Horner evaluation, as accurate as ex2.approx);
-// 2^j by adding j to the exponent field.  x is clamped to [-125, 127] first, so the result
+// a degree-5 polynomial 1 + f q(f) whose coefficients are a minimax fit of the relative error
+// made here (fit_exp2.py: at most 1.7e-7 relative in fp32 Horner evaluation; exact constant
+// term, so the decay factors near 1 that compound over long memories carry no bias); 2^j by
+// adding j to the exponent field.  x is clamped to [-125, 127] first, so the result
 // stays a normal number (decay factors below 2^-125 act as zero, as ex2.approx.ftz's do below
 // 2^-126).
 constexpr int kExpFmaPairs = 1;
-constexpr float kExp2C0 = 1.0000001192092896f;
+constexpr float kExp2C0 = 1.0f;
 constexpr float kExp2C1 = 0.6931470036506653f;
-constexpr float kExp2C2 = 0.24022118747234344f;
-constexpr float kExp2C3 = 0.05550695210695267f;
-constexpr float kExp2C4 = 0.009675589390099049f;
-constexpr float kExp2C5 = 0.0013282300205901265f;
+constexpr float kExp2C2 = 0.24022242426872253f;
+constexpr float kExp2C3 = 0.05550733953714371f;
+constexpr float kExp2C4 = 0.009671513922512531f;
+constexpr float kExp2C5 = 0.001326472032815218f;
 constexpr float kRoundShift = 12582912.0f;  // 1.5 * 2^23
 __device__ __forceinline__ f2_t exp2_fma2(f2_t x) {
   float x0, x1;

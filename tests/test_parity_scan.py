@@ -129,6 +129,27 @@ def test_general_A_values(io):
     compare_full(inp)
 
 
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+@pytest.mark.parametrize("chunk", [0, 128])
+def test_general_A_extreme_decay(io, chunk):
+    """General A whose per-step decay exponents reach far below 2^-125 (steps up to about 5
+    times A down to -60): the exponentials computed on the FP32 pipe clamp there, the SFU ones
+    flush to zero; both must agree with the oracle as a decay factor of zero would,
+    whole-sequence and across chunk summaries.  A stays below -0.3, so no state keeps a long
+    memory: with steps this large, a decay factor within 1% of 1 held for hundreds of steps
+    compounds the SFU exponential's own error past the fp32 tolerance."""
+    import selective_state_space_46_b200 as m
+    Bt, D, L = 2, 70, 600
+    inp = synth.make_scan_inputs(Bt, D, L, io_dtype=io, seed=41)
+    rng = np.random.default_rng(41)
+    A = -np.exp(rng.uniform(np.log(0.3), np.log(60.0), size=(D, 16)))
+    inp.A = A.astype(np.float32)
+    inp.delta_bias = rng.uniform(-1.0, 4.0, size=D).astype(np.float32)
+    if chunk:
+        m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, chunk)
+    compare_full(inp)
+
+
 # ---------------------------------------------------------------------------
 # the length split and its carry
 # ---------------------------------------------------------------------------
