@@ -308,12 +308,16 @@ LaunchShape choose_shape(int64_t Bt, int64_t D, int64_t L, int sms, int64_t forc
         }
         const int64_t per_sm = std::min<int64_t>(tiles / sms, tk.rpt == 1 ? 8 : 12);
         if (per_sm >= 4) {
-          // each CTA takes whole items; k warps share an SMSP
+          // each CTA takes whole items from a ticket, so the items run in about items / grid
+          // rounds plus a tail of a quarter round (fitted to the measured chunk-length choices
+          // of 8 x 5120 x 1024, 64 x 1536 x 512, 8 x 5120 x 4096 and 8 x 5120 x 16384), and in
+          // no fewer rounds than the tile's chain of chunks; k warps share an SMSP
+          constexpr double kChainTail = 0.25;
           const int64_t grid = per_sm * sms;
           const int64_t k = (per_sm + 3) / 4;
-          const int64_t rounds = std::max<int64_t>((out_items + grid - 1) / grid, nseg);
+          const double rounds = std::max(double(out_items) / double(grid) + kChainTail, double(nseg));
           const double item = double(seg) * tk.rpt * cyc_out(tk.rpt, k) * double(k) + kItem;
-          consider(LaunchShape{2, tk.rows, tk.rpt, seg, nseg, int(grid)}, double(rounds) * item + kLaunch);
+          consider(LaunchShape{2, tk.rows, tk.rpt, seg, nseg, int(grid)}, rounds * item + kLaunch);
         }
       }
       if (forced_mode == 0 || forced_seg > 0 || L <= mssm::kSegQuant) break;

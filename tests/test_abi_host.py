@@ -298,6 +298,10 @@ def test_scan_plan_measured_best():
         # 1662-1674 us; chunk 2560: 1759, 4608: 2031; 32 rows: 1737; split: 1780-1818;
         # two rows per thread: 1680-1769; fused: 1815
         (1, 2048, 131072, -1): ("summaries+forward", 64, 1, 3584),
+        # many rows, short sequences, chained: chunk 256 211.0 us, 128: 223.6, 64: 247.9
+        (8, 5120, 1024, -1): ("chained", 32, 1, 256),
+        # 251.2 us; chunk 128: 258.4, 64: 289.2
+        (64, 1536, 512, -1): ("chained", 32, 1, 256),
         # packed sequences (32 of up to 4096 steps): 64 rows chunk 256: 320.4 us, 384: 323.2,
         # 512: 332.7, 192: 327.8, 128: 343.2; 32 rows chunk 256: 343.4, 384: 351.7
         (32, 1536, 4096, 27048): ("summaries+forward", 64, 1, 320),
