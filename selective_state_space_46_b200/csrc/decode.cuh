@@ -243,10 +243,15 @@ struct StreamSlot {
                 "slot layout must keep 16-byte alignment");
 };
 
+// One wait on a ring slot's mbarrier: the warp sleeps until the phase completes or about
+// kStreamWaitHintNs pass (instead of re-polling), so warps that wait for their data take no
+// issue slots from the warps that have theirs.
+constexpr uint32_t kStreamWaitHintNs = 2000;
+constexpr int kStreamWaitLimit = 1 << 19;  // bounded: at most about a second of waiting
 __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t mb, uint32_t parity) {
   uint32_t done;
-  asm volatile("{\n .reg .pred pr;\n mbarrier.try_wait.parity.shared::cta.b64 pr, [%1], %2;\n selp.u32 %0, 1, 0, pr;\n}"
-               : "=r"(done) : "r"(mb), "r"(parity) : "memory");
+  asm volatile("{\n .reg .pred pr;\n mbarrier.try_wait.parity.shared::cta.b64 pr, [%1], %2, %3;\n selp.u32 %0, 1, 0, pr;\n}"
+               : "=r"(done) : "r"(mb), "r"(parity), "r"(kStreamWaitHintNs) : "memory");
   return done;
 }
 
@@ -341,7 +346,7 @@ __global__ void __launch_bounds__(kWsWarps * 32, kStreamCtasPerSm) state_update_
     const uint32_t k = i % kWsBufs;
     unsigned char* slot = wring + k * L::kBytes;
     uint32_t done = 0;
-    for (int it = 0; it < kDecodeSpinLimit && !done; ++it) done = mbar_try_wait(mb0 + k * 8, (i / kWsBufs) & 1u);
+    for (int it = 0; it < kStreamWaitLimit && !done; ++it) done = mbar_try_wait(mb0 + k * 8, (i / kWsBufs) & 1u);
     if (!__all_sync(0xffffffffu, done)) {
       ok = false;
       break;
@@ -407,7 +412,7 @@ __global__ void __launch_bounds__(kWsWarps * 32, kStreamCtasPerSm) state_update_
     atomicOr(p.err, 1u);
     for (uint32_t j = i; j < i + kWsAhead && j < mine; ++j) {
       uint32_t done = 0;
-      for (int it = 0; it < kDecodeSpinLimit && !done; ++it)
+      for (int it = 0; it < kStreamWaitLimit && !done; ++it)
         done = mbar_try_wait(mb0 + (j % kWsBufs) * 8, (j / kWsBufs) & 1u);
     }
   }
