@@ -36,6 +36,9 @@
  *  - Supported dtype mixes: everything fp32; or bf16 for u/delta/B/C/z/out
  *    (x/dt/B/C/z/out for decode) with fp32 A, D, bias and state.
  *  - The state size N must be 16 (MSSM_ERR_UNSUPPORTED otherwise).
+ *  - Sizes: Bt, D and L each below 2^31, and the number of rows (Bt * D, or the
+ *    sequence count * D for packed sequences) below 2^31 (MSSM_ERR_UNSUPPORTED
+ *    otherwise).
  *  - The innermost (length) dimension of u/delta/z/out/B/C must have stride 1.
  *  - All calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream).  Argument errors are reported synchronously, before

@@ -431,6 +431,8 @@ mssm_status scan_prepare(const mssm_tensor* u, const mssm_tensor* delta, const m
   if (last_state && (st = check(last_state, "last_state", 3, s_bdn, MSSM_F32, true)) != MSSM_OK) return st;
   if (Bt > INT32_MAX || Dd > INT32_MAX || L > INT32_MAX - 2 * mssm::kSegQuant)
     return fail(MSSM_ERR_UNSUPPORTED, "Bt, D and L must each fit in 31 bits");
+  if (Bt * Dd > int64_t(INT32_MAX) || (state_batches >= 0 && state_batches * Dd > int64_t(INT32_MAX)))
+    return fail(MSSM_ERR_UNSUPPORTED, "Bt * D (or the sequence count * D) must fit in 31 bits");
   const mssm_tensor* ins[] = {u, delta, B, C, z, A, D, delta_bias};
   for (const mssm_tensor* t : ins)
     if (same_ptr(out, t)) return fail(MSSM_ERR_INVALID_ARG, "out must not alias an input");

@@ -143,6 +143,15 @@ class Ext(ctypes.Structure):
                 ("h0", ctypes.POINTER(T)), ("cu_seqlens", ctypes.POINTER(T)), ("max_seqlen", ctypes.c_int64)]
 
 
+def test_scan_rejects_rows_beyond_31_bits(lib):
+    """2^31 rows (Bt * D) at L = 1 would fit in device memory, but the kernels index rows
+    with 32-bit integers: the call is refused on the host, before any CUDA call (so this
+    runs without a GPU; the descriptors' pointers are never dereferenced)."""
+    a = scan_args(Bt=1 << 16, D=1 << 15, L=1)
+    assert call_scan(lib, a) == UNSUPPORTED
+    assert "31 bits" in last_error(lib)
+
+
 @pytest.mark.parametrize("case", ["short_struct", "bad_disc", "h0_shape", "h0_dtype", "h0_inner_stride",
                                   "h0_aliases_last_state"])
 def test_scan_ext_validation(lib, case):
