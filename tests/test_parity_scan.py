@@ -261,6 +261,22 @@ def test_long_slow_decay_many_chunks():
     compare_full(inp)
 
 
+@pytest.mark.parametrize("schedule", ["summaries+forward", "chained"])
+def test_chunk_count_past_the_grid_limit(schedule):
+    """4.2 M steps (8 channels) forced into 64-step chunks would need 65 553 chunks, past the 65 535 a grid
+    dimension holds: the plan doubles the chunk length instead; every row against the oracle."""
+    import selective_state_space_46_b200 as m
+    Bt, D, L = 1, 8, (1 << 22) + 777
+    m.mssm_set_option(m.MSSM_OPT_CHUNK_LEN, 64)
+    m.mssm_set_option(m.MSSM_OPT_SCHEDULE, m.SCHEDULES[schedule])
+    plan = m.mssm_scan_plan(Bt, D, L)
+    assert plan["n_chunks"] <= 65535 and plan["chunk_len"] == 128 and plan["schedule"] == schedule, plan
+    inp = synth.make_scan_inputs(Bt, D, L, io_dtype="bf16", seed=13, delta_range=(1e-4, 1e-2))
+    out, last = run_scan(inp)
+    m.mssm_get_error()
+    check_scan_every_row(inp, out, last)
+
+
 # ---------------------------------------------------------------------------
 # layouts: strided and unaligned rows take the scalar path
 # ---------------------------------------------------------------------------
