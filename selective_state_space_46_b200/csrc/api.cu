@@ -953,6 +953,11 @@ mssm_status mssm_selective_scan_bwd(const mssm_tensor* u, const mssm_tensor* del
     for (const mssm_tensor* o2 : outs)
       if (o2 != o && same_ptr(o, o2)) return fail(MSSM_ERR_INVALID_ARG, "gradients must not alias each other");
   }
+  // the grid limits, checked before anything is launched
+  const int64_t tpb = (Dd + mssm::kBwdRows - 1) / mssm::kBwdRows;
+  const int64_t tiles = Bt * tpb, rows_total = tiles * mssm::kBwdRows;
+  const int64_t nseg = (L + mssm::kBwdChunk - 1) / mssm::kBwdChunk;
+  if (nseg > 65535 || tiles > INT32_MAX) return fail(MSSM_ERR_UNSUPPORTED, "problem too large for the backward grid");
   if (call.noop) return MSSM_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lk(g_mu);
@@ -971,10 +976,6 @@ mssm_status mssm_selective_scan_bwd(const mssm_tensor* u, const mssm_tensor* del
 
   // workspace: the chunk summaries (H then the start states, G, S), the incoming gradients Q,
   // and the arrival counters
-  const int64_t tpb = (Dd + mssm::kBwdRows - 1) / mssm::kBwdRows;
-  const int64_t tiles = Bt * tpb, rows_total = tiles * mssm::kBwdRows;
-  const int64_t nseg = (L + mssm::kBwdChunk - 1) / mssm::kBwdChunk;
-  if (nseg > 65535 || tiles > INT32_MAX) return fail(MSSM_ERR_UNSUPPORTED, "problem too large for the backward grid");
   auto al = [](size_t v) { return (v + 255) / 256 * 256; };
   const size_t cnt_b = al(size_t(tiles) * 4);
   const size_t h_b = al(size_t(nseg - 1) * rows_total * mssm::kN * 4);

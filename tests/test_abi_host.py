@@ -248,6 +248,21 @@ def test_empty_problem_is_noop(lib):
     assert call_scan(lib, a) == 0
 
 
+def test_bwd_refuses_too_many_chunks_before_launching(lib):
+    """More than 65 535 chunks of 64 steps cannot be gridded: refused with UNSUPPORTED before the
+    gradients are zeroed or anything else reaches the device (without a GPU a CUDA call would
+    fail with MSSM_ERR_CUDA instead; the descriptors' pointers are never dereferenced)."""
+    Bt, D, L, N = 1, 8, 65535 * 64 + 1, 16
+    t = lambda shape, dt=1: ctypes.byref(mk(shape, dt))  # noqa: E731
+    f = lib.mssm_selective_scan_bwd
+    f.restype = ctypes.c_int
+    st = f(t([Bt, D, L]), t([Bt, D, L]), t([D, N], 0), t([Bt, N, L]), t([Bt, N, L]), t([D], 0), t([Bt, D, L]),
+           t([D], 0), 1, t([Bt, D, L]), t([Bt, D, L]), t([Bt, D, L]), t([D, N], 0), t([Bt, N, L], 0),
+           t([Bt, N, L], 0), t([D], 0), t([Bt, D, L]), t([D], 0), None)
+    assert st == UNSUPPORTED, (st, last_error(lib))
+    assert "too large" in last_error(lib)
+
+
 def test_decode_validation(lib):
     P = ctypes.byref
     f = lib.mssm_state_update
