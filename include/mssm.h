@@ -244,8 +244,9 @@ mssm_status mssm_state_update_ex(mssm_tensor *state, const mssm_tensor *x,
  * Backward of mssm_selective_scan_fwd (Euler discretisation, zero initial state,
  * no packed sequences): the gradients of Loss with respect to every input, given
  * dout = dLoss/dout.  The states are recomputed, never stored: one pass of chunk
- * summaries, both ways, gives every 64-step chunk's start state and incoming
- * dLoss/dh, and every chunk then sweeps its recomputed states backwards ("Mamba
+ * summaries, both ways, gives every chunk's start state and incoming dLoss/dh
+ * (chunks of 64 steps, or 32 from 1024 row tiles of 32 channels on), and every
+ * chunk then sweeps its recomputed states backwards ("Mamba
  * selective state space", the hardware-aware scan: intermediates are recomputed in
  * the backward pass).
  *   inputs     as for mssm_selective_scan_fwd, plus dout [Bt, D, L] dtype of u
@@ -256,8 +257,9 @@ mssm_status mssm_state_update_ex(mssm_tensor *state, const mssm_tensor *x,
  *   dD, ddelta_bias [D] f32, given exactly when D / delta_bias are
  * The f32 gradients must be dense; they are zeroed and accumulated with atomic
  * adds, so their rounding order is not fixed.  Uses a per-device workspace of
- * about 196 x L / 64 bytes per row (49 floats per 64-step chunk), grown with
- * cudaMalloc on demand (which synchronises the device) and freed by mssm_shutdown().
+ * 49 floats per chunk and row (about 196 x L / 64 bytes per row, twice that with
+ * 32-step chunks), grown with cudaMalloc on demand (which synchronises the device)
+ * and freed by mssm_shutdown().  L may reach 65535 x 64 steps.
  */
 mssm_status mssm_selective_scan_bwd(const mssm_tensor *u, const mssm_tensor *delta, const mssm_tensor *A,
                                     const mssm_tensor *B, const mssm_tensor *C, const mssm_tensor *D,

@@ -9,7 +9,8 @@
 // ("Mamba selective state space", the hardware-aware scan: intermediates are
 // recomputed in the backward pass instead of being written).
 //
-// Two chunk-parallel passes over chunks of kBwdChunk steps, one thread per row:
+// Two chunk-parallel passes over chunks of kBwdChunk steps (kBwdChunkShort when there are
+// many row tiles), one thread per row:
 //  A. scan_bwd_summary_kernel: one backward sweep over every chunk gives its forward
 //     summary H_c (the state it leaves from a zero start), its reverse summary G_c
 //     (the gradient it sends to the chunk before from a zero incoming gradient) and
@@ -32,7 +33,9 @@
 
 namespace mssm {
 
-constexpr int kBwdChunk = 64;  // steps per chunk
+constexpr int kBwdChunk = 64;       // steps per chunk
+constexpr int kBwdChunkShort = 32;  // steps per chunk when there are many row tiles
+constexpr int kBwdShortChunkTiles = 1024;  // from this many row tiles on, 32-step chunks
 constexpr int kBwdRows = 32;   // rows per CTA (one warp)
 
 struct BwdArgs {
@@ -62,6 +65,7 @@ struct BwdArgs {
   int Bt, D, L;
   int softplus;
   int nseg, tiles_per_batch;
+  int chunk;          // steps per chunk: kBwdChunk or kBwdChunkShort
   int vec_rows;       // u, delta, dout, z, du, ddelta, dz rows start 16-byte aligned
   int force_general;  // never take the structured-A powers
   float* hstart;    // [nseg-1][rows][16]: chunk k's summary H_k, then (folded) chunk k+1's start state
@@ -116,22 +120,22 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& p, int d, BwdRow& r) {
   r.bias = p.bias ? p.bias[int64_t(d) * p.bias_s] : 0.0f;
 }
 
-// B and C of steps [t0, t0 + kBwdChunk) of batch b into shared memory, fp32 [t][32]
+// B and C of steps [t0, t0 + CHUNK) of batch b into shared memory, fp32 [t][32]
 // (B in 0..15, C in 16..31); zero past L.  Each of the 32 threads loads one row of B or C,
 // as 16-byte blocks where the row's chunk is whole and aligned.
-template <typename T>
+template <typename T, int CHUNK>
 __device__ __forceinline__ void bwd_stage_bc(const BwdArgs& p, int b, int t0, float (*bc)[32]) {
   const int r = threadIdx.x;
   const T* base = r < 16 ? static_cast<const T*>(p.B) + int64_t(b) * p.B_sb + int64_t(r) * p.B_sn
                          : static_cast<const T*>(p.C) + int64_t(b) * p.C_sb + int64_t(r - 16) * p.C_sn;
   constexpr int kPer = 16 / int(sizeof(T));  // elements per 16-byte block
-  if (t0 + kBwdChunk <= p.L && (reinterpret_cast<uintptr_t>(base + t0) & 15) == 0) {
+  if (t0 + CHUNK <= p.L && (reinterpret_cast<uintptr_t>(base + t0) & 15) == 0) {
     const uint4* src = reinterpret_cast<const uint4*>(base + t0);
-    uint4 v[kBwdChunk / kPer];
+    uint4 v[CHUNK / kPer];
 #pragma unroll
-    for (int i = 0; i < kBwdChunk / kPer; ++i) v[i] = __ldg(src + i);
+    for (int i = 0; i < CHUNK / kPer; ++i) v[i] = __ldg(src + i);
 #pragma unroll
-    for (int i = 0; i < kBwdChunk / kPer; ++i) {
+    for (int i = 0; i < CHUNK / kPer; ++i) {
       const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
       if constexpr (sizeof(T) == 2) {
 #pragma unroll
@@ -146,7 +150,7 @@ __device__ __forceinline__ void bwd_stage_bc(const BwdArgs& p, int b, int t0, fl
     }
     return;
   }
-  for (int j = 0; j < kBwdChunk; ++j) {
+  for (int j = 0; j < CHUNK; ++j) {
     const int t = t0 + j;
     bc[j][r] = t < p.L ? Elem<T>::load(base + t) : 0.0f;
   }
@@ -410,9 +414,9 @@ __device__ __forceinline__ void bwd_load16(const float* src, float4 (&v)[4]) {
   for (int i = 0; i < 4; ++i) v[i] = __ldcg(s4 + i);
 }
 
-template <typename T, bool HAS_Z>
+template <typename T, bool HAS_Z, int CHUNK>
 __global__ void __launch_bounds__(kBwdRows) scan_bwd_summary_kernel(const BwdArgs p) {
-  __shared__ __align__(16) float bc_s[kBwdChunk][32];
+  __shared__ __align__(16) float bc_s[CHUNK][32];
   __shared__ int s_last;
   const int tid = threadIdx.x;
   const int tile = blockIdx.x;
@@ -420,12 +424,12 @@ __global__ void __launch_bounds__(kBwdRows) scan_bwd_summary_kernel(const BwdArg
   const int b = tile / p.tiles_per_batch;
   const int d = (tile - b * p.tiles_per_batch) * kBwdRows + tid;
   const int dc = d < p.D ? d : p.D - 1;
-  const int t0 = c * kBwdChunk;
-  const int t1 = min(p.L, t0 + kBwdChunk);
+  const int t0 = c * CHUNK;
+  const int t1 = min(p.L, t0 + CHUNK);
   BwdRow r;
   bwd_row(p, dc, r);
   const bool structured = __syncthreads_and(r.structured) && !p.force_general;
-  bwd_stage_bc<T>(p, b, t0, bc_s);
+  bwd_stage_bc<T, CHUNK>(p, b, t0, bc_s);
   __syncthreads();
 
   f2_t H[kN / 2], g2[kN / 2];
@@ -695,11 +699,11 @@ __device__ __forceinline__ void bwd_chunk(const BwdArgs& p, const BwdRow& r, con
 #ifndef MSSM_BWD_MAXNREG
 #define MSSM_BWD_MAXNREG 255
 #endif
-template <typename T, bool HAS_Z>
+template <typename T, bool HAS_Z, int CHUNK>
 __global__ void __maxnreg__(MSSM_BWD_MAXNREG) scan_bwd_kernel(const BwdArgs p) {
-  __shared__ __align__(16) float bc_s[kBwdChunk][32];
+  __shared__ __align__(16) float bc_s[CHUNK][32];
   // window start states, and one spare slot so that two free slots always follow window w
-  __shared__ __align__(16) f2_t hwin[kBwdChunk / kBwdWin + 1][kN / 2][kBwdRows];
+  __shared__ __align__(16) f2_t hwin[CHUNK / kBwdWin + 1][kN / 2][kBwdRows];
   const int tid = threadIdx.x;
   const int tile = blockIdx.x;
   const int c = blockIdx.y;
@@ -707,14 +711,14 @@ __global__ void __maxnreg__(MSSM_BWD_MAXNREG) scan_bwd_kernel(const BwdArgs p) {
   const int d = (tile - b * p.tiles_per_batch) * kBwdRows + tid;
   const bool row_ok = d < p.D;
   const int dc = row_ok ? d : p.D - 1;
-  const int t0 = c * kBwdChunk;
-  const int t1 = min(p.L, t0 + kBwdChunk);
+  const int t0 = c * CHUNK;
+  const int t1 = min(p.L, t0 + CHUNK);
   const int64_t rows_total = int64_t(p.Bt) * p.tiles_per_batch * kBwdRows;
   const int64_t rowg = int64_t(tile) * kBwdRows + tid;
   BwdRow r;
   bwd_row(p, dc, r);
   const bool structured = __syncthreads_and(r.structured) && !p.force_general;
-  bwd_stage_bc<T>(p, b, t0, bc_s);
+  bwd_stage_bc<T, CHUNK>(p, b, t0, bc_s);
   __syncthreads();
 
   f2_t h[kN / 2], g[kN / 2], dA[kN / 2];

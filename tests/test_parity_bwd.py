@@ -81,6 +81,15 @@ def test_bwd_aligned_rows_ragged_chunks(cuda_device, Bt, D, L):
     compare(g, ref, "bf16")
 
 
+@pytest.mark.parametrize("Bt,D,L", [(32, 1024, 300), (16, 2050, 97)])
+def test_bwd_short_chunks_many_tiles(cuda_device, Bt, D, L):
+    """From 1024 row tiles of 32 channels on, the backward runs in 32-step chunks: ragged
+    lengths and a partial last tile per batch."""
+    inp = synth.make_scan_inputs(Bt, D, L, io_dtype="bf16", seed=Bt + L)
+    g, ref = run_bwd(inp, seed=L)
+    compare(g, ref, "bf16")
+
+
 def test_bwd_default_workload_shape(cuda_device):
     """2 x 512 x 2048 (a quarter of the default prefill's channels), bf16."""
     inp = synth.make_scan_inputs(2, 512, 2048, io_dtype="bf16", seed=9)
