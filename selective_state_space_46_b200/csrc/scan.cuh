@@ -358,7 +358,7 @@ __device__ __forceinline__ void store_block(T* row, int t, int t_lo, int t_end, 
 // term, so the decay factors near 1 that compound over long memories carry no bias); 2^j by
 // adding j to the exponent field.  x is clamped to [-125, 127] first, so the result
 // stays a normal number (decay factors below 2^-125 act as zero, as ex2.approx.ftz's do below
-// 2^-126).
+// 2^-126); a NaN exponent gives NaN.
 constexpr int kExpFmaPairs = 1;
 constexpr float kExp2C0 = 1.0f;
 constexpr float kExp2C1 = 0.6931470036506653f;
@@ -384,7 +384,9 @@ __device__ __forceinline__ f2_t exp2_fma2(f2_t x) {
   f2split(p, p0, p1);
   const int j0 = __float_as_int(t0) - __float_as_int(kRoundShift);
   const int j1 = __float_as_int(t1) - __float_as_int(kRoundShift);
-  return f2(__int_as_float(__float_as_int(p0) + (j0 << 23)), __int_as_float(__float_as_int(p1) + (j1 << 23)));
+  const float r0 = __int_as_float(__float_as_int(p0) + (j0 << 23));
+  const float r1 = __int_as_float(__float_as_int(p1) + (j1 << 23));
+  return f2(x0 != x0 ? x0 : r0, x1 != x1 ? x1 : r1);  // a NaN exponent stays NaN, as with ex2
 }
 
 // Powers a^1 .. a^16 as eight pairs (a^(2k+1), a^(2k+2)); 15 multiplies, depth 4.

@@ -44,7 +44,9 @@ def emulate(x, c):
     for k in (3, 2, 1, 0):
         p = _f32(p.astype(np.float64) * f + c[k])
     jint = t.view(np.int32) - shift.view(np.int32)
-    return (p.view(np.int32) + (jint << 23)).view(np.float32)
+    r = (p.view(np.int32) + (jint << 23)).view(np.float32)
+    xs = _f32(x)
+    return np.where(np.isnan(xs), xs, r)
 
 
 def test_constants_are_the_fit():
@@ -93,3 +95,9 @@ def test_clamped_inputs():
     low = np.exp2(-125.0)
     assert np.all(got[:4] > 0) and np.allclose(got[:4], low, rtol=2e-7)
     assert np.allclose(got[4:], np.exp2(127.0), rtol=2e-7) and np.all(np.isfinite(got))
+
+
+def test_nan_propagates():
+    c = _header_constants()
+    got = emulate(_f32([np.nan, -1.0, np.nan]), c)
+    assert np.isnan(got[0]) and np.isnan(got[2]) and np.isfinite(got[1])

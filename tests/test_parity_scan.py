@@ -150,6 +150,23 @@ def test_general_A_extreme_decay(io, chunk):
     compare_full(inp)
 
 
+@pytest.mark.parametrize("n", [0, 5])
+def test_general_A_nan_propagates(n):
+    """A NaN in A reaches the outputs of its channel whichever unit computes that state's decay
+    (state 0 is in the pair computed on the FP32 pipe, state 5 on the SFU); other channels stay
+    finite."""
+    inp = synth.make_scan_inputs(2, 40, 300, io_dtype="f32", seed=3)
+    A = random_A(40, 3)
+    A[7, n] = np.nan
+    inp.A = A
+    out, last = run_scan(inp)
+    y, h = to_f64(out), to_f64(last)
+    assert np.isnan(y[:, 7, :]).all() and np.isnan(h[:, 7, n]).all()
+    others = np.ones(40, bool)
+    others[7] = False
+    assert np.isfinite(y[:, others, :]).all() and np.isfinite(h[:, others, :]).all()
+
+
 # ---------------------------------------------------------------------------
 # the length split and its carry
 # ---------------------------------------------------------------------------
